@@ -1,0 +1,329 @@
+"""GPU parity of the CUDA path (through the C ABI) against the CPU oracle.
+
+Every case feeds the same seeded inputs to libloopkv and to the oracle and checks:
+  * packed history bytes (codes, fp16 scales and zeros, hi/lo planes) bit-exact;
+  * the refine set S bit-exact except within 1e-6 of tau (tie band);
+  * outputs within 2e-3 absolute, row max and row sum within 1e-4 relative.
+"""
+import numpy as np
+import pytest
+import torch
+
+from lkv_helpers import bits_of, check_row, f32
+from mixed_precision_kv_append_b200 import loopkv as L
+from mixed_precision_kv_append_b200 import synth
+from oracle import oracle as O
+
+pytestmark = pytest.mark.gpu
+
+BITS = {L.CELL_4B: 4, L.CELL_2B: 2}
+
+
+def _plan(n_layers, n_loops, H, D, B, max_blocks, modes, tau, tau_mode=L.TAU_REL_MAX, dtype=torch.bfloat16):
+    return L.Plan(n_layers, n_loops, H, D, B, max_blocks, modes, tau, tau_mode, dtype)
+
+
+class Model:
+    """A small cache plus the raw token history of every (cell, request), as the oracle sees it."""
+
+    def __init__(self, w: synth.Workload, max_blocks=None, tau=None, tau_mode=None):
+        self.w = w
+        self.tau = w.tau if tau is None else tau
+        self.tau_mode = w.tau_mode if tau_mode is None else tau_mode
+        self.plan = _plan(w.n_layers, w.n_loops, w.H, w.D, w.B, max_blocks or w.max_blocks, w.modes, self.tau,
+                          self.tau_mode, w.dtype)
+        self.cache = L.Cache(self.plan)
+        self.tokens = {}  # (cell, req) -> (K [n, H, D] float32, V)
+        self._hist_cache = {}
+
+    def cell(self, loop, layer):
+        return loop * self.w.n_layers + layer
+
+    def src(self, loop, layer):
+        c = self.cell(loop, layer)
+        if self.w.modes[c] == L.CELL_SHARE:
+            return self.cell(self.w.n_loops - 1, layer)
+        return c
+
+    def ingest(self, T_override=None):
+        w = self.w
+        for layer in range(w.n_layers):
+            for req in range(w.B):
+                T = w.lengths[req] if T_override is None else T_override[req]
+                ks, vs = synth.layer_history(w, layer, req, T=T, device="cuda")
+                for lp in range(w.n_loops):
+                    self.cache.ingest(lp, layer, req, ks[lp].contiguous(), vs[lp].contiguous())
+                    self.tokens[(self.cell(lp, layer), req)] = (f32(ks[lp]), f32(vs[lp]))
+        self.cache.check("ingest")
+
+    def append_step(self, step):
+        w = self.w
+        self.cache.flush()
+        for layer in range(w.n_layers):
+            _, ks, vs = synth.step_tokens(w, step, layer, device="cuda")
+            for lp in range(w.n_loops):
+                self.cache.append(lp, layer, ks[lp].contiguous(), vs[lp].contiguous())
+                c = self.cell(lp, layer)
+                for req in range(w.B):
+                    K, V = self.tokens[(c, req)]
+                    self.tokens[(c, req)] = (np.concatenate([K, f32(ks[lp][req:req + 1])]),
+                                             np.concatenate([V, f32(vs[lp][req:req + 1])]))
+        self._hist_cache.clear()
+
+    def head_history(self, cell, req, h, n_hist):
+        key = (cell, req, h, n_hist)
+        if key not in self._hist_cache:
+            K, V = self.tokens[(cell, req)]
+            self._hist_cache[key] = O.HeadHistory(K[:n_hist, h], V[:n_hist, h], BITS[self.w.modes[cell]]) \
+                if n_hist else None
+        return self._hist_cache[key]
+
+    def check_cell(self, loop, layer, q, rows=None, where=""):
+        """Decode cell (loop, layer) on the GPU and compare the given (req, head) rows."""
+        w = self.w
+        out, bm, rm, rs = self.cache.decode_debug(loop, layer, q)
+        self.cache.check(f"decode {where}")
+        hist, tail = self.cache.lengths(loop, layer)
+        c, s = self.cell(loop, layer), self.src(loop, layer)
+        out, bm, rm, rs = f32(out), bm.cpu().numpy().view(np.uint32), f32(rm), f32(rs)
+        qn = f32(q)
+        rows = rows if rows is not None else [(r, h) for r in range(w.B) for h in range(w.H)]
+        worst, ties = 0.0, 0
+        for req, h in rows:
+            n_hist, n_tail = int(hist[req]), int(tail[req])
+            K, V = self.tokens[(c, req)]
+            n_own = K.shape[0]
+            assert n_own == n_hist + n_tail, (n_own, n_hist, n_tail)
+            hh = self.head_history(s, req, h, n_hist)
+            err, nt = check_row(out[req, h], bm[req, h], rm[req, h], rs[req, h], qn[req, h].astype(np.float64),
+                                hh, K[n_hist:, h], V[n_hist:, h], self.tau, self.tau_mode,
+                                where=f"{where} cell ({loop},{layer}) req {req} head {h}")
+            worst, ties = max(worst, err), ties + nt
+        return worst, ties
+
+    def check_bytes(self, loop, layer, reqs=None, heads=None):
+        """Packed bytes of the cell's own pages against the oracle's packing."""
+        w = self.w
+        c = self.cell(loop, layer)
+        assert w.modes[c] != L.CELL_SHARE
+        hist, _ = self.cache.lengths(loop, layer)
+        for req in (reqs if reqs is not None else range(w.B)):
+            main, lo = self.cache.head_blocks(loop, layer, req)
+            n_hist = int(hist[req])
+            assert main.shape[0] == n_hist // 16
+            for h in (heads if heads is not None else range(w.H)):
+                hh = self.head_history(c, req, h, n_hist)
+                if hh is None:
+                    continue
+                om, ol = hh.packed_blocks()
+                assert np.array_equal(main[:, h].numpy(), om), f"main bytes differ: cell {c} req {req} head {h}"
+                if BITS[w.modes[c]] == 4:
+                    assert np.array_equal(lo[:, h].numpy(), ol), f"lo bytes differ: cell {c} req {req} head {h}"
+
+
+def _q(w, step, layer, loop):
+    qs, _, _ = synth.step_tokens(w, step, layer, device="cuda")
+    return qs[loop].contiguous()
+
+
+def test_tiny_config_bytes_and_decode():
+    w = synth.workload("tiny")
+    m = Model(w)
+    m.ingest()
+    for lp in range(2):
+        m.check_bytes(lp, 0)
+        m.check_cell(lp, 0, _q(w, 0, 0, lp), where="tiny")
+
+
+@pytest.mark.parametrize("tau,tau_mode", [(0.0, 0), (0.01, 0), (0.3, 0), (1.5, 0), (0.002, 1), (0.05, 1)])
+def test_ragged_rows_tails_and_share_cells(tau, tau_mode):
+    # loop 0: [share of a 4-bit cell, 4-bit]; loop 1: [2-bit, share of a 2-bit cell]; loop 2 (final): [4b, 2b]
+    modes = [L.CELL_SHARE, L.CELL_4B, L.CELL_2B, L.CELL_SHARE, L.CELL_4B, L.CELL_2B]
+    w = synth.Workload("ragged_small", 2, 3, 4, 128, 5, [5, 37, 300, 1000, 64], torch.bfloat16, modes, tau,
+                       tau_mode=tau_mode, seed=3)
+    m = Model(w)
+    m.ingest()
+    for layer in range(2):
+        for lp in range(3):
+            if modes[m.cell(lp, layer)] != L.CELL_SHARE:
+                m.check_bytes(lp, layer)
+            m.check_cell(lp, layer, _q(w, 1, layer, lp), where=f"tau={tau} mode={tau_mode}")
+
+
+def test_head_dim_64_bf16_and_fp32_tails():
+    for dtype in (torch.float32, torch.bfloat16):
+        w = synth.Workload("d64", 1, 2, 2, 64, 2, [100, 257], dtype, [L.CELL_2B, L.CELL_4B], 0.05, seed=5)
+        m = Model(w)
+        m.ingest()
+        for lp in range(2):
+            m.check_bytes(lp, 0)
+            m.check_cell(lp, 0, _q(w, 0, 0, lp), where=f"d64 {dtype}")
+
+
+def test_append_flush_sequence():
+    modes = [L.CELL_4B, L.CELL_SHARE, L.CELL_2B, L.CELL_4B]  # 2 layers x 2 loops
+    w = synth.Workload("append", 2, 2, 4, 128, 3, [20, 64, 95], torch.bfloat16, modes, 0.02, append_steps=70,
+                       seed=7)
+    m = Model(w)
+    m.ingest()
+    for step in range(70):
+        m.append_step(step)
+        if step % 9 == 0 or step in (11, 12, 43, 44, 69):
+            for layer in range(2):
+                for lp in range(2):
+                    m.check_cell(lp, layer, _q(w, step, layer, lp), where=f"step {step}")
+    m.cache.check("append sequence")
+    for layer in range(2):
+        for lp in range(2):
+            if modes[m.cell(lp, layer)] != L.CELL_SHARE:
+                m.check_bytes(lp, layer)
+            hist, tail = m.cache.lengths(lp, layer)
+            for req in range(w.B):
+                n = w.lengths[req] + 70
+                assert int(tail[req]) >= 1 and int(hist[req]) % 32 == 0 and int(hist[req]) + int(tail[req]) == n
+
+
+def test_share_cell_with_final_loop_query_is_bit_identical():
+    modes = [L.CELL_SHARE, L.CELL_4B]
+    w = synth.Workload("share", 1, 2, 4, 128, 2, [512, 1024], torch.bfloat16, modes, 0.01, seed=9)
+    m = Model(w)
+    m.ingest()  # multiples of 32: every tail is empty
+    q = _q(w, 0, 0, 1)
+    a = m.cache.decode(0, 0, q)
+    b = m.cache.decode(1, 0, q)
+    m.cache.check("share")
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("name,B,T,modes,tau,steps", [
+    ("kivi4_8k", 8, [8192] * 8, [0, 0, 0, 0], 0.0, 0),
+    ("mixed_8k", 32, [8192] * 32, [0, 1, 2, 0], 0.01, 0),
+    ("long_16k", 32, [16384] * 32, [0, 2, 1, 0], 0.005, 2),
+    ("ragged_2p6b", 8, None, [1, 2, 0, 0], 0.01, 0),
+])
+def test_full_size_sampled_rows(name, B, T, modes, tau, steps):
+    """Benchmark shapes (one layer of four loops): the launch configuration the benchmark times,
+    checked on sampled rows of every cell and on the packed bytes of sampled heads."""
+    base = synth.workload(name)
+    lengths = T if T is not None else base.lengths
+    w = synth.Workload(name, 1, 4, 16, 128, B, lengths, torch.bfloat16, modes, tau, append_steps=steps, seed=1)
+    m = Model(w, max_blocks=base.max_blocks)
+    m.ingest()
+    for s in range(steps):
+        m.append_step(s)
+    rng = np.random.default_rng(0)
+    for lp in range(4):
+        rows = [(int(rng.integers(B)), int(rng.integers(16))) for _ in range(5)] + [(B - 1, 15), (0, 0)]
+        m.check_cell(lp, 0, _q(w, steps, 0, lp), rows=rows, where=name)
+        if modes[lp] != L.CELL_SHARE:
+            m.check_bytes(lp, 0, reqs=[0, B - 1], heads=[0, 7])
+
+
+def test_graph_replay_matches_eager():
+    modes = [L.CELL_4B, L.CELL_2B, L.CELL_SHARE, L.CELL_4B]
+    w = synth.Workload("graph", 2, 2, 4, 128, 3, [33, 64, 200], torch.bfloat16, modes, 0.01, append_steps=40,
+                       seed=11)
+    m = Model(w)
+    m.ingest()
+    qs = [[_q(w, 0, layer, lp) for lp in range(2)] for layer in range(2)]
+    _, ks, vs = synth.step_tokens(w, 0, 0, device="cuda")
+    outs = [[torch.empty_like(qs[0][0], dtype=torch.float32) for _ in range(2)] for _ in range(2)]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        m.cache.flush(stream=s)  # warm the launch attributes outside the capture
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            m.cache.flush(stream=s)
+            for layer in range(2):
+                for lp in range(2):
+                    m.cache.append(lp, layer, ks[lp], vs[lp], stream=s)
+                    L.loopkv_decode(m.plan.handle, lp, layer, qs[layer][lp], m.cache.handle, outs[layer][lp],
+                                    stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    for rep in range(35):
+        g.replay()
+        torch.cuda.synchronize()
+        for layer in range(2):
+            for lp in range(2):
+                c = m.cell(lp, layer)
+                for req in range(w.B):
+                    K, V = m.tokens[(c, req)]
+                    m.tokens[(c, req)] = (np.concatenate([K, f32(ks[lp][req:req + 1])]),
+                                          np.concatenate([V, f32(vs[lp][req:req + 1])]))
+        m._hist_cache.clear()
+        if rep in (0, 30, 34):
+            for layer in range(2):
+                for lp in range(2):
+                    ref = outs[layer][lp].clone()
+                    eager = m.cache.decode(lp, layer, qs[layer][lp])
+                    assert torch.equal(ref, eager)
+                    m.check_cell(lp, layer, qs[layer][lp], where=f"graph replay {rep}")
+    m.cache.check("graph")
+
+
+def test_device_errors_are_reported():
+    modes = [L.CELL_4B, L.CELL_4B]
+    w = synth.Workload("err", 1, 2, 2, 64, 2, [64, 64], torch.float32, modes, 0.01, seed=13)
+    m = Model(w, max_blocks=8)
+    m.ingest()
+    # ingest into a non-empty (cell, request)
+    k = torch.zeros((32, 2, 64), device="cuda")
+    m.cache.ingest(0, 0, 0, k, k)
+    assert m.cache.status() == (-10, L.DEV_STATE)
+    # a 33rd token in a tail without flush
+    for _ in range(33):
+        m.cache.append(0, 0, torch.zeros((2, 2, 64), device="cuda"), torch.zeros((2, 2, 64), device="cuda"))
+    rc, bits = m.cache.status()
+    assert rc == -9 and bits & L.DEV_TAIL_FULL
+    # non-finite and out-of-range groups
+    m.cache.reset_request(1)
+    bad = torch.randn((32, 2, 64), device="cuda")
+    bad[3, 1, 7] = float("nan")
+    m.cache.ingest(1, 0, 1, bad, torch.randn((32, 2, 64), device="cuda"))
+    rc, bits = m.cache.status()
+    assert rc == -5 and bits & L.DEV_NONFINITE
+    m.cache.reset_request(1)
+    big = torch.randn((32, 2, 64), device="cuda")
+    big[0, 0, 0] = -1e6
+    m.cache.ingest(1, 0, 1, big, torch.randn((32, 2, 64), device="cuda"))
+    rc, bits = m.cache.status()
+    assert rc == -6 and bits & L.DEV_RANGE
+    # host-side argument errors come back before any launch
+    with pytest.raises(L.LoopKVError):
+        m.cache.ingest(5, 0, 0, k, k)
+    with pytest.raises(L.LoopKVError):
+        m.cache.ingest(0, 0, 0, torch.zeros((10 * 32, 2, 64), device="cuda"), torch.zeros((320, 2, 64),
+                                                                                          device="cuda"))
+
+
+def test_pool_exhaustion_and_reset():
+    modes = [L.CELL_4B]
+    w = synth.Workload("pool", 1, 1, 2, 64, 4, [64] * 4, torch.float32, modes, 0.0, seed=17)
+    plan = _plan(1, 1, 2, 64, 4, 8, modes, 0.0, dtype=torch.float32)
+    need = plan.required_bytes()
+    per_block = 2 * (1024 + 256)
+    cache = L.Cache(plan, nbytes=need - 20 * per_block)  # room for fewer than 16 blocks
+    ks, vs = synth.layer_history(w, 0, 0, T=64, device="cuda")
+    for req in range(4):
+        cache.ingest(0, 0, req, ks[0], vs[0])
+    rc, bits = cache.status()
+    assert rc == -4 and bits & L.DEV_POOL_EXHAUSTED
+    hist, _ = cache.lengths(0, 0)
+    full = [r for r in range(4) if int(hist[r]) == 64]
+    assert len(full) >= 1
+    cache.reset_request(full[0])
+    hist, _ = cache.lengths(0, 0)
+    assert int(hist[full[0]]) == 0
+    missing = [r for r in range(4) if int(hist[r]) == 0 and r != full[0]][0]
+    cache.ingest(0, 0, missing, ks[0], vs[0])
+    assert cache.status() == (0, 0)
+
+
+def test_empty_row_is_reported():
+    plan = _plan(1, 1, 2, 64, 1, 4, [L.CELL_4B], 0.0, dtype=torch.float32)
+    cache = L.Cache(plan)
+    out = cache.decode(0, 0, torch.randn((1, 2, 64), device="cuda"))
+    rc, bits = cache.status()
+    assert rc == -11 and bits & L.DEV_EMPTY_ROW
+    assert torch.all(out == 0)
