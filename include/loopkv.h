@@ -227,8 +227,8 @@ int loopkv_status(loopkv_cache *cache, void *stream, int *device_status);
 /* Device addresses of cell (loop, layer). */
 int loopkv_cell_view_get(const loopkv_cache *cache, int loop, int layer, loopkv_cell_view *out);
 
-/* Decode launch shape chosen for a batch of B rows (cluster size, stages), for
- * reporting.  Host-only. */
+/* Decode launch shape chosen for a batch of B requests (cluster size, CTAs, shared
+ * memory per CTA), for reporting.  Queries the occupancy of the current device. */
 int loopkv_decode_shape(const loopkv_plan *plan, int B, int *cluster_size, int *ctas, int *smem_bytes);
 
 const char *loopkv_strerror(int code);

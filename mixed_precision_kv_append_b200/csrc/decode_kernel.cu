@@ -1,9 +1,10 @@
 // decode_kernel.cu -- fused, plan-driven decode attention over the LoopKV cache.
 //
-// One launch per cell (LoopKV paper, §3.4 "One launch per cell").  A thread-block
-// cluster of C CTAs serves one (request, head) row; CTA r of the cluster owns the
-// 32-token groups r, r+C, r+2C, ... of the row's history, and CTA C-1 also the
-// unquantized tail.  Each CTA:
+// One launch per cell (LoopKV paper, §3.4 "One launch per cell").  The grid is a set
+// of persistent thread-block clusters of C CTAs; cluster c serves the (request, head)
+// rows c, c + NC, c + 2NC, ... one after another.  Inside a row, CTA k of the cluster
+// owns the 32-token groups k, k+C, k+2C, ... of the history, and CTA C-1 also the
+// unquantized tail.  For each row a CTA:
 //   1. K pass: streams the key codes and per-channel key scale/zero of its groups
 //      into shared memory with bulk asynchronous copies (a producer warp, an
 //      mbarrier ring), and computes every score from the full 4-bit (or 2-bit) keys
@@ -21,6 +22,11 @@
 //      scale and zero are folded into the weight and a running sum.
 //   4. Merge: since all CTAs used the same m, their partial sums add directly; the
 //      CTAs reduce them through distributed shared memory and write out = o / l.
+// Rows are software-pipelined: while the cluster barrier that publishes row r's
+// maxima completes, the CTA already streams and scores the keys of row r+1, so the
+// memory pipe never drains at a row boundary.  One cluster barrier per row carries
+// both the per-warp maxima (with their partial exponential sums, for the normalised
+// rule) of row r and the partial outputs of row r-1.
 //
 // Code extraction: a field masked out of a packed word, read as an fp32 bit pattern
 // x < 2^24, has the value x * 2^-149 exactly (subnormal or smallest-exponent normal
@@ -33,11 +39,15 @@
 #include "lkv_device.cuh"
 #include "lkv_internal.h"
 
+#include <algorithm>
+#include <cstdlib>
+
 namespace lkv {
 namespace {
 
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kMinCtasPerSm = 4;
 constexpr int kVScaleExp = 40; // V accumulators hold code * w * s * 2^(p - 40)
 
 template <int BITS, int D> struct Geo {
@@ -139,84 +149,108 @@ __device__ __forceinline__ int value_channel(int e, int n) { return 8 * (n & 1) 
 __device__ __forceinline__ int value_pos(int n) { return n < 6 ? 4 * n : (n == 6 ? 8 : 12); }
 
 struct Smem {
-    uint8_t *ring;
-    uint64_t *full;
-    uint64_t *empty;
-    float *scores; // [cap * 32] history scores, then [32] tail scores
-    float *aw;     // [kConsumerWarps][D] key factors
-    float *qs;     // [D] pre-scaled query (tail scoring)
-    float *wmax;   // [kConsumerWarps]
-    float *wsum;   // [kConsumerWarps]
-    float *red;    // [kConsumerWarps][D + 1]
-    float *po;     // [D + 1] CTA partial o and l, read by the other CTAs
+    uint8_t *ring;     // [stages][STAGE]
+    uint64_t *full;    // [stages]
+    uint64_t *empty;   // [stages]
+    float *scores;     // [2][cap * 32 + 32] scores of a row (history, then tail), by row parity
+    float *stat;       // [3][kConsumerWarps][2] per-warp (max, sum exp(s - max)), by row index mod 3
+    float *part;       // [2][D + 1] CTA partial o and l of a row, by row parity
+    float *aw;         // [kConsumerWarps][D] key factors
+    float *wv;         // [kConsumerWarps][32] weights of the group a warp reads
+    float *red;        // [kConsumerWarps][D + 1]
+    int32_t *ids;      // [2][2 * cap] block ids of a row's groups (even, odd block), by row parity
 };
+
+// Byte offsets of the shared-memory regions; every region starts on a 16-byte boundary
+// (the key factors and the stage data are read with 16-byte vector loads).
+struct SmemLayout {
+    int full, empty, scores, stat, part, aw, wv, red, ids, total;
+};
+
+__host__ __device__ constexpr int align16(int x) { return (x + 15) & ~15; }
+
+template <int BITS, int D> __host__ __device__ constexpr SmemLayout smem_layout(int stages, int cap)
+{
+    SmemLayout L{};
+    int o = stages * Geo<BITS, D>::STAGE; // ring, 128-byte aligned slots
+    L.full = o;
+    o = align16(o + stages * 8);
+    L.empty = o;
+    o = align16(o + stages * 8);
+    L.scores = o;
+    o = align16(o + 2 * (cap * 32 + 32) * 4);
+    L.aw = o;
+    o = align16(o + kConsumerWarps * D * 4);
+    L.stat = o;
+    o = align16(o + 3 * kConsumerWarps * 2 * 4);
+    L.part = o;
+    o = align16(o + 2 * (D + 1) * 4);
+    L.wv = o;
+    o = align16(o + kConsumerWarps * 32 * 4);
+    L.red = o;
+    o = align16(o + kConsumerWarps * (D + 1) * 4);
+    L.ids = o;
+    o = align16(o + 2 * 2 * cap * 4);
+    L.total = o;
+    return L;
+}
 
 template <int BITS, int D> __host__ __device__ constexpr int smem_bytes(int stages, int cap)
 {
-    using G = Geo<BITS, D>;
-    return stages * G::STAGE + 2 * stages * 8 + (cap * 32 + 32) * 4 + kConsumerWarps * D * 4 + D * 4 +
-           2 * kConsumerWarps * 4 + kConsumerWarps * (D + 1) * 4 + (D + 1) * 4 + 128;
+    return smem_layout<BITS, D>(stages, cap).total;
+}
+
+template <int BITS, int D> __host__ __device__ constexpr int smem_fixed(int cap)
+{
+    return smem_layout<BITS, D>(0, cap).total;
 }
 
 template <int BITS, int D> __device__ Smem carve(uint8_t *base, int stages, int cap)
 {
-    using G = Geo<BITS, D>;
+    const SmemLayout L = smem_layout<BITS, D>(stages, cap);
     Smem s;
-    uint8_t *p = base;
-    s.ring = p;
-    p += stages * G::STAGE;
-    s.full = reinterpret_cast<uint64_t *>(p);
-    p += stages * 8;
-    s.empty = reinterpret_cast<uint64_t *>(p);
-    p += stages * 8;
-    s.scores = reinterpret_cast<float *>(p);
-    p += (cap * 32 + 32) * 4;
-    s.aw = reinterpret_cast<float *>(p);
-    p += kConsumerWarps * D * 4;
-    s.qs = reinterpret_cast<float *>(p);
-    p += D * 4;
-    s.wmax = reinterpret_cast<float *>(p);
-    p += kConsumerWarps * 4;
-    s.wsum = reinterpret_cast<float *>(p);
-    p += kConsumerWarps * 4;
-    s.red = reinterpret_cast<float *>(p);
-    p += kConsumerWarps * (D + 1) * 4;
-    s.po = reinterpret_cast<float *>(p);
+    s.ring = base;
+    s.full = reinterpret_cast<uint64_t *>(base + L.full);
+    s.empty = reinterpret_cast<uint64_t *>(base + L.empty);
+    s.scores = reinterpret_cast<float *>(base + L.scores);
+    s.aw = reinterpret_cast<float *>(base + L.aw);
+    s.stat = reinterpret_cast<float *>(base + L.stat);
+    s.part = reinterpret_cast<float *>(base + L.part);
+    s.wv = reinterpret_cast<float *>(base + L.wv);
+    s.red = reinterpret_cast<float *>(base + L.red);
+    s.ids = reinterpret_cast<int32_t *>(base + L.ids);
     return s;
 }
 
-// Maximum over all CTAs of the cluster of the per-warp values v[kConsumerWarps].
-__device__ __forceinline__ float cluster_max(const float *v, uint32_t C, int lane)
+// Host check of a layout: every region 16-byte aligned and inside the allocation.
+template <int BITS, int D> bool layout_ok(int stages, int cap)
 {
-    float m = -INFINITY;
-    for (uint32_t k = lane; k < C * kConsumerWarps; k += 32)
-        m = fmaxf(m, ld_dsmem_f32(v + (k % kConsumerWarps), k / kConsumerWarps));
-    return warp_max(m);
+    const SmemLayout L = smem_layout<BITS, D>(stages, cap);
+    const int offs[] = {L.full, L.empty, L.scores, L.aw, L.stat, L.part, L.wv, L.red, L.ids};
+    int prev = stages * Geo<BITS, D>::STAGE;
+    for (int o : offs) {
+        if (o % 16 || o < prev)
+            return false;
+        prev = o;
+    }
+    return (Geo<BITS, D>::STAGE % 128) == 0 && L.total >= prev;
 }
 
-// Sum over all CTAs in a fixed order (rank-major, then warp), identical in every warp.
-__device__ __forceinline__ float cluster_sum_fixed(const float *v, uint32_t C)
-{
-    float s = 0.f;
-    for (uint32_t r = 0; r < C; ++r)
-        for (int w = 0; w < kConsumerWarps; ++w)
-            s += ld_dsmem_f32(v + w, r);
-    return s;
-}
+// One (request, head) row as seen by one CTA of its cluster.
+struct RowCtx {
+    int row, b, h;
+    int hist, tail;   // validated lengths
+    int nmy;          // 32-token groups of the history owned by this CTA
+    bool tail_cta;    // this CTA also reads the tail
+};
 
-template <int BITS, int D, typename DT>
-__global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeArgs a, const int stages)
+__device__ __forceinline__ RowCtx row_ctx(const DecodeArgs &a, int row, uint32_t crank, uint32_t C)
 {
-    using G = Geo<BITS, D>;
-    extern __shared__ __align__(128) uint8_t smem_raw[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int row = blockIdx.y;
-    const int b = row / a.H, h = row % a.H;
-    const uint32_t crank = cluster_ctarank(), C = cluster_nctarank();
-    Smem sm = carve<BITS, D>(smem_raw, stages, a.cap_groups);
-
-    // Row lengths (history of the source cell, tail of this cell), validated.
-    int hist = a.hist_len[b], tail = a.tail_len[b];
+    RowCtx r;
+    r.row = row;
+    r.b = row / a.H;
+    r.h = row % a.H;
+    int hist = a.hist_len[r.b], tail = a.tail_len[r.b];
     bool bad = false;
     if (hist < 0 || hist > a.max_blocks * 16 || (hist & 31)) {
         bad = true;
@@ -232,15 +266,61 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeArgs a, co
         bad = true;
         nmy = a.cap_groups;
     }
-    const bool tail_cta = (crank == C - 1) && tail > 0;
     if (bad && threadIdx.x == 0)
         atomicOr(a.status, LOOPKV_DEV_STATE);
+    r.hist = hist;
+    r.tail = tail;
+    r.nmy = nmy;
+    r.tail_cta = (crank == C - 1) && tail > 0;
+    return r;
+}
 
+// Row max m (log2 units) and, for the normalised rule, l = sum_t 2^(s_t - m), from the
+// per-warp pairs of every CTA of the cluster (fixed order: every caller gets the same).
+__device__ __forceinline__ void cluster_row_stats(const float *stat, uint32_t C, float &m, float &l)
+{
+    m = -INFINITY;
+    for (uint32_t r = 0; r < C; ++r)
+        for (int w = 0; w < kConsumerWarps; ++w)
+            m = fmaxf(m, ld_dsmem_f32(stat + 2 * w, r));
+    l = 0.f;
+    if (m == -INFINITY)
+        return;
+    for (uint32_t r = 0; r < C; ++r)
+        for (int w = 0; w < kConsumerWarps; ++w) {
+            const float mw = ld_dsmem_f32(stat + 2 * w, r);
+            if (mw != -INFINITY)
+                l += ld_dsmem_f32(stat + 2 * w + 1, r) * exp2f(mw - m);
+        }
+}
+
+__device__ __forceinline__ float row_threshold(const DecodeArgs &a, float m, float l, bool decide)
+{
+    if (!decide)
+        return -INFINITY;
+    return a.tau_mode == LOOPKV_TAU_ABS_PROB ? m + log2f(a.tau * l) : m + log2f(a.tau);
+}
+
+// First stage index >= base in [base, base + n) owned by warp w (stage s -> warp s % NW).
+__device__ __forceinline__ int first_owned(int base, int w)
+{
+    return ((w - base) % kConsumerWarps + kConsumerWarps) % kConsumerWarps;
+}
+
+template <int BITS, int D, typename DT>
+__global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const DecodeArgs a, const int stages)
+{
+    using G = Geo<BITS, D>;
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t crank = cluster_ctarank(), C = cluster_nctarank();
+    const int cid = blockIdx.x / (int)C, ncl = gridDim.x / (int)C;
+    const int rows = a.rows;
+    const int nrows = cid < rows ? (rows - 1 - cid) / ncl + 1 : 0; // rows cid, cid + ncl, ...
+    Smem sm = carve<BITS, D>(smem_raw, stages, a.cap_groups);
+    const int SC = a.cap_groups * 32 + 32; // score buffer stride
     const bool all_hot = (BITS == 4) && !(a.tau > 0.f);
     const bool decide = (BITS == 4) && (a.tau > 0.f); // lo planes depend on the row max
-    const int32_t *bt = a.block_table + (int64_t)b * a.max_blocks;
-    const DT *tailk = reinterpret_cast<const DT *>(a.tail) + ((int64_t)b * 2 * a.H + h) * 32 * D;
-    const DT *tailv = reinterpret_cast<const DT *>(a.tail) + ((int64_t)(b * 2 + 1) * a.H + h) * 32 * D;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < stages; ++i) {
@@ -249,356 +329,425 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeArgs a, co
         }
         fence_mbar_init();
     }
-    // pre-scaled query (log2(e)/sqrt(D) folded in) for the tail
-    const DT *qrow = reinterpret_cast<const DT *>(a.q) + (int64_t)row * D;
-    for (int c = threadIdx.x; c < D; c += kThreads)
-        sm.qs[c] = to_f32(qrow[c]) * a.qscale;
     __syncthreads();
-
-    float m2 = -INFINITY, thr2 = -INFINITY;
 
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------------ producer
-        auto block_id = [&](int idx) -> int64_t {
-            int64_t id = bt[idx];
-            if (id < 0 || id >= a.pool_blocks) {
-                atomicOr(a.status, LOOPKV_DEV_STATE);
-                id = 0;
-            }
-            return id;
-        };
-        auto wait_empty = [&](int i) {
-            if (i >= stages)
-                mbar_wait(&sm.empty[i % stages], ((i / stages) - 1) & 1, a.status);
-        };
-        for (int i = 0; i < nmy; ++i) { // K stages
-            wait_empty(i);
-            if (lane == 0) {
-                const int g = (int)crank + i * (int)C;
-                uint8_t *st = sm.ring + (i % stages) * G::STAGE;
-                uint64_t *fb = &sm.full[i % stages];
-                mbar_arrive_expect_tx(fb, 2 * G::KB);
-                bulk_g2s(st, a.main + (block_id(2 * g) * a.H + h) * G::HM, G::KB, fb);
-                bulk_g2s(st + G::KB, a.main + (block_id(2 * g + 1) * a.H + h) * G::HM, G::KB, fb);
-            }
-            __syncwarp();
-        }
-        cluster_arrive(); // barrier 1: the producer contributes no score
-
-        auto issue_main = [&](int j) { // V meta + hi of group j, without arriving
-            const int i = nmy + j;
-            wait_empty(i);
-            if (lane == 0) {
-                const int g = (int)crank + j * (int)C;
-                uint8_t *st = sm.ring + (i % stages) * G::STAGE;
-                uint64_t *fb = &sm.full[i % stages];
-                mbar_expect_tx(fb, 2 * G::VB);
-                bulk_g2s(st, a.main + (block_id(2 * g) * a.H + h) * G::HM + G::KB, G::VB, fb);
-                bulk_g2s(st + G::VB, a.main + (block_id(2 * g + 1) * a.H + h) * G::HM + G::KB, G::VB, fb);
+        auto load_ids = [&](const RowCtx &rc, int par) {
+            const int32_t *bt = a.block_table + (int64_t)rc.b * a.max_blocks;
+            int32_t *ids = sm.ids + par * 2 * a.cap_groups;
+            for (int k = lane; k < 2 * rc.nmy; k += 32) {
+                int id = bt[2 * ((int)crank + (k >> 1) * (int)C) + (k & 1)];
+                if (id < 0 || id >= a.pool_blocks) {
+                    atomicOr(a.status, LOOPKV_DEV_STATE);
+                    id = 0;
+                }
+                ids[k] = id;
             }
             __syncwarp();
         };
-        auto issue_lo = [&](int j) { // lo planes of the hot tokens of group j, then arrive
-            const int i = nmy + j;
-            const int g = (int)crank + j * (int)C;
-            uint8_t *st = sm.ring + (i % stages) * G::STAGE;
-            uint64_t *fb = &sm.full[i % stages];
-            uint32_t mask = 0;
-            if (BITS == 4)
-                mask = all_hot ? 0xFFFFFFFFu : __ballot_sync(0xFFFFFFFFu, sm.scores[j * 32 + lane] >= thr2);
-            if (a.s_bitmap && lane == 0)
-                a.s_bitmap[(int64_t)row * a.bitmap_words + g] = mask;
-            if (BITS == 4 && mask == 0xFFFFFFFFu) {
+        auto wait_empty = [&](int s) {
+            if (s >= stages)
+                mbar_wait(&sm.empty[s % stages], ((s / stages) - 1) & 1, a.status);
+        };
+        auto issue_k = [&](const RowCtx &rc, int par, int base) {
+            const int32_t *ids = sm.ids + par * 2 * a.cap_groups;
+            for (int i = 0; i < rc.nmy; ++i) {
+                const int s = base + i;
+                wait_empty(s);
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(fb, 2 * G::LOB);
-                    bulk_g2s(st + 2 * G::VB, a.lo + (block_id(2 * g) * a.H + h) * G::LOB, G::LOB, fb);
-                    bulk_g2s(st + 2 * G::VB + G::LOB, a.lo + (block_id(2 * g + 1) * a.H + h) * G::LOB, G::LOB, fb);
+                    uint8_t *st = sm.ring + (s % stages) * G::STAGE;
+                    uint64_t *fb = &sm.full[s % stages];
+                    mbar_arrive_expect_tx(fb, 2 * G::KB);
+                    bulk_g2s(st, a.main + ((int64_t)ids[2 * i] * a.H + rc.h) * G::HM, G::KB, fb);
+                    bulk_g2s(st + G::KB, a.main + ((int64_t)ids[2 * i + 1] * a.H + rc.h) * G::HM, G::KB, fb);
                 }
-            } else {
-                if (lane == 0)
-                    mbar_arrive_expect_tx(fb, (uint32_t)__popc(mask) * G::ROWV);
                 __syncwarp();
-                if (BITS == 4 && ((mask >> lane) & 1u)) {
-                    const int blk = lane >> 4, r = lane & 15;
-                    bulk_g2s(st + 2 * G::VB + blk * G::LOB + r * G::ROWV,
-                             a.lo + (block_id(2 * g + blk) * a.H + h) * G::LOB + r * G::ROWV, G::ROWV, fb);
-                }
             }
-            __syncwarp();
+        };
+        auto issue_v = [&](const RowCtx &rc, int par, int base, float thr2) {
+            const int32_t *ids = sm.ids + par * 2 * a.cap_groups;
+            const float *sc = sm.scores + par * SC;
+            for (int i = 0; i < rc.nmy; ++i) {
+                const int s = base + i;
+                const int g = (int)crank + i * (int)C;
+                uint32_t mask = 0;
+                if (BITS == 4)
+                    mask = all_hot ? 0xFFFFFFFFu : __ballot_sync(0xFFFFFFFFu, sc[i * 32 + lane] >= thr2);
+                if (a.s_bitmap && lane == 0)
+                    a.s_bitmap[(int64_t)rc.row * a.bitmap_words + g] = mask;
+                wait_empty(s);
+                uint8_t *st = sm.ring + (s % stages) * G::STAGE;
+                uint64_t *fb = &sm.full[s % stages];
+                const int64_t b0 = ids[2 * i], b1 = ids[2 * i + 1];
+                const bool full_lo = BITS == 4 && mask == 0xFFFFFFFFu;
+                if (lane == 0) {
+                    const uint32_t lo_bytes = full_lo ? 2 * G::LOB : (uint32_t)__popc(mask) * G::ROWV;
+                    mbar_arrive_expect_tx(fb, 2 * G::VB + lo_bytes);
+                    bulk_g2s(st, a.main + (b0 * a.H + rc.h) * G::HM + G::KB, G::VB, fb);
+                    bulk_g2s(st + G::VB, a.main + (b1 * a.H + rc.h) * G::HM + G::KB, G::VB, fb);
+                    if (full_lo) {
+                        bulk_g2s(st + 2 * G::VB, a.lo + (b0 * a.H + rc.h) * G::LOB, G::LOB, fb);
+                        bulk_g2s(st + 2 * G::VB + G::LOB, a.lo + (b1 * a.H + rc.h) * G::LOB, G::LOB, fb);
+                    }
+                }
+                __syncwarp();
+                if (BITS == 4 && !full_lo && ((mask >> lane) & 1u)) {
+                    const int blk = lane >> 4, r = lane & 15;
+                    const int64_t bb = blk ? b1 : b0;
+                    bulk_g2s(st + 2 * G::VB + blk * G::LOB + r * G::ROWV,
+                             a.lo + (bb * a.H + rc.h) * G::LOB + r * G::ROWV, G::ROWV, fb);
+                }
+                __syncwarp();
+            }
         };
 
-        if (decide) {
-            const int npre = nmy < stages ? nmy : stages;
-            for (int j = 0; j < npre; ++j)
-                issue_main(j);
-            cluster_wait();
-            m2 = cluster_max(sm.wmax, C, lane);
-            float lt = 1.f;
-            if (a.tau_mode == LOOPKV_TAU_ABS_PROB) {
-                cluster_arrive();
-                cluster_wait();
-                lt = cluster_sum_fixed(sm.wsum, C);
-            }
-            thr2 = m2 + log2f(a.tau * lt);
-            for (int j = 0; j < npre; ++j)
-                issue_lo(j);
-            for (int j = npre; j < nmy; ++j) {
-                issue_main(j);
-                issue_lo(j);
-            }
-        } else {
-            for (int j = 0; j < nmy; ++j) {
-                issue_main(j);
-                issue_lo(j);
-            }
-            cluster_wait();
-            if (a.tau_mode == LOOPKV_TAU_ABS_PROB) {
-                cluster_arrive();
-                cluster_wait();
-            }
+        int pos = 0;
+        RowCtx prev{};
+        if (nrows > 0) {
+            prev = row_ctx(a, cid, crank, C);
+            load_ids(prev, 0);
+            issue_k(prev, 0, pos);
+            pos += prev.nmy;
         }
-        cluster_arrive(); // barrier 3: partial sums ready
+        cluster_arrive(); // row 0
+        for (int i = 1; i < nrows; ++i) {
+            const RowCtx cur = row_ctx(a, cid + i * ncl, crank, C);
+            load_ids(cur, i & 1);
+            issue_k(cur, i & 1, pos);
+            pos += cur.nmy;
+            cluster_wait(); // row i - 1
+            float m2, l2;
+            cluster_row_stats(sm.stat + ((i - 1) % 3) * kConsumerWarps * 2, C, m2, l2);
+            issue_v(prev, (i - 1) & 1, pos, row_threshold(a, m2, l2, decide));
+            pos += prev.nmy;
+            prev = cur;
+            cluster_arrive(); // row i
+        }
+        cluster_wait(); // last row
+        if (nrows > 0) {
+            float m2, l2;
+            cluster_row_stats(sm.stat + ((nrows - 1) % 3) * kConsumerWarps * 2, C, m2, l2);
+            issue_v(prev, (nrows - 1) & 1, pos, row_threshold(a, m2, l2, decide));
+        }
+        cluster_arrive(); // partials of the last row
         cluster_wait();
-        cluster_arrive(); // barrier 4: remote reads done
+        cluster_arrive(); // remote reads done
         cluster_wait();
         return;
     }
 
     // ---------------------------------------------------------------- consumers
-    float qreg[D / 32];
-#pragma unroll
-    for (int i = 0; i < D / 32; ++i)
-        qreg[i] = sm.qs[lane + 32 * i];
     float *aw = sm.aw + warp * D;
-    float mx = -INFINITY;
-
-    for (int i = warp; i < nmy; i += kConsumerWarps) { // K pass
-        const int slot = i % stages;
-        mbar_wait(&sm.full[slot], (i / stages) & 1, a.status);
-        const uint8_t *st = sm.ring + slot * G::STAGE;
-        const __half *ksc = reinterpret_cast<const __half *>(st + G::KCODES);        // even block: scales
-        const __half *kzp = reinterpret_cast<const __half *>(st + G::KB + G::KCODES); // odd block: zeros
-        float av[D / 32];
-        float zs = 0.f, amax = 0.f;
+    float *wv = sm.wv + warp * 32;
+    int kslot[D / 32];
+    float kpow[D / 32];
 #pragma unroll
-        for (int k = 0; k < D / 32; ++k) {
-            const int c = lane + 32 * k;
-            av[k] = qreg[k] * __half2float(ksc[c]);
-            zs = fmaf(qreg[k], __half2float(kzp[c]), zs);
-            amax = fmaxf(amax, fabsf(av[k]));
-        }
-        zs = warp_sum(zs);
-        amax = warp_max(amax);
-        const int E = amax > 0.f ? ilogbf(amax) : 0;
-#pragma unroll
-        for (int k = 0; k < D / 32; ++k) {
-            int slot_c, pos;
-            key_slot<BITS>(lane + 32 * k, slot_c, pos);
-            aw[slot_c] = mul_pow2(av[k], 126 - E - pos);
-        }
-        __syncwarp();
-        const uint32_t *kr = reinterpret_cast<const uint32_t *>(st + (lane >> 4) * G::KB + (lane & 15) * G::ROWK);
-        float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int w4 = 0; w4 < G::WORDSK / 4; ++w4) {
-            const uint4 cw = reinterpret_cast<const uint4 *>(kr)[w4];
-            if (BITS == 4) {
-                key_word4(cw.x, aw + 8 * (4 * w4 + 0), acc);
-                key_word4(cw.y, aw + 8 * (4 * w4 + 1), acc);
-                key_word4(cw.z, aw + 8 * (4 * w4 + 2), acc);
-                key_word4(cw.w, aw + 8 * (4 * w4 + 3), acc);
-            } else {
-                key_word2(cw.x, aw + 16 * (4 * w4 + 0), acc);
-                key_word2(cw.y, aw + 16 * (4 * w4 + 1), acc);
-                key_word2(cw.z, aw + 16 * (4 * w4 + 2), acc);
-                key_word2(cw.w, aw + 16 * (4 * w4 + 3), acc);
-            }
-        }
-        const float s2 = mul_pow2(acc.x + acc.y, E + 23) + zs;
-        sm.scores[i * 32 + lane] = s2;
-        mx = fmaxf(mx, s2);
-        __syncwarp();
-        if (lane == 0)
-            mbar_arrive(&sm.empty[slot]);
+    for (int k = 0; k < D / 32; ++k) {
+        int pos;
+        key_slot<BITS>(lane + 32 * k, kslot[k], pos);
+        kpow[k] = __int_as_float((24 - pos + 127) << 23);
     }
-    float *tsc = sm.scores + a.cap_groups * 32;
-    if (tail_cta && warp == kConsumerWarps - 1 && lane < tail) { // tail keys, exact
-        const DT *kt = tailk + (int64_t)lane * D;
-        float s2 = 0.f;
-        for (int c = 0; c < D; ++c)
-            s2 = fmaf(sm.qs[c], to_f32(kt[c]), s2);
-        tsc[lane] = s2;
-        mx = fmaxf(mx, s2);
-    }
-    mx = warp_max(mx);
-    if (lane == 0)
-        sm.wmax[warp] = mx;
-    cluster_arrive(); // barrier 1
-    cluster_wait();
-    m2 = cluster_max(sm.wmax, C, lane);
-
-    float lt = 1.f;
-    if (a.tau_mode == LOOPKV_TAU_ABS_PROB) {
-        float ps = 0.f;
-        for (int i = warp; i < nmy; i += kConsumerWarps)
-            ps += exp2f(sm.scores[i * 32 + lane] - m2);
-        if (tail_cta && warp == kConsumerWarps - 1 && lane < tail)
-            ps += exp2f(tsc[lane] - m2);
-        ps = warp_sum(ps);
-        if (lane == 0)
-            sm.wsum[warp] = ps;
-        cluster_arrive(); // barrier 2
-        cluster_wait();
-        lt = cluster_sum_fixed(sm.wsum, C);
-    }
-    thr2 = decide ? m2 + log2f(a.tau * lt) : -INFINITY;
-
-    // V pass: lane = (token slot ts, 32-channel group cg)
-    const int cg = lane % G::NCG, ts = lane / G::NCG;
-    float2 acc[2][2][4];
-#pragma unroll
-    for (int k = 0; k < 2; ++k)
-#pragma unroll
-        for (int e = 0; e < 2; ++e)
-#pragma unroll
-            for (int n = 0; n < 4; ++n)
-                acc[k][e][n] = make_float2(0.f, 0.f);
-    float zacc = 0.f, lsum = 0.f;
     const float vscale = 6.490371073168535e32f; // 2^(149 - kVScaleExp) = 2^109
-    const int first_v = ((warp - nmy) % kConsumerWarps + kConsumerWarps) % kConsumerWarps;
-    for (int j = first_v; j < nmy; j += kConsumerWarps) {
-        const int i = nmy + j;
-        const int slot = i % stages;
-        mbar_wait(&sm.full[slot], (i / stages) & 1, a.status);
-        const uint8_t *st = sm.ring + slot * G::STAGE;
-#pragma unroll
-        for (int u = 0; u < 32 / G::TPI; ++u) {
-            const int t = u * G::TPI + ts;
-            const float s2 = sm.scores[j * 32 + t];
-            const float w = exp2f(s2 - m2);
-            const bool hot = all_hot || (BITS == 4 && s2 >= thr2);
-            const int blk = t >> 4, r = t & 15;
-            const uint8_t *vb = st + blk * G::VB;
-            const __half2 meta = *reinterpret_cast<const __half2 *>(vb + r * G::NCG * 4 + cg * 4);
-            const float vs = __low2float(meta), vz = __high2float(meta);
-            const uint2 hw = *reinterpret_cast<const uint2 *>(vb + G::VMETA + r * G::ROWV + cg * 8);
-            uint2 lw = make_uint2(0u, 0u);
-            float W;
-            if (BITS == 4) {
-                if (hot)
-                    lw = *reinterpret_cast<const uint2 *>(st + 2 * G::VB + blk * G::LOB + r * G::ROWV + cg * 8);
-                W = w * vs;
-                zacc = fmaf(w, hot ? vz : fmaf(1.5f, vs, vz), zacc);
-            } else {
-                W = w * vs * 0.25f;
-                zacc = fmaf(w, vz, zacc);
-            }
-            if (cg == 0)
-                lsum += w;
-            const float Wp = W * vscale;
-            value_word(hw.x, lw.x, Wp, acc[0]);
-            value_word(hw.y, lw.y, Wp, acc[1]);
-        }
-        __syncwarp();
-        if (lane == 0)
-            mbar_arrive(&sm.empty[slot]);
-    }
 
-    // Reduce over the token slots of the warp (lanes with the same cg).
+    // K pass of one row: scores into the row's buffer, per-warp (max, sum) into stat.
+    auto consume_k = [&](const RowCtx &rc, int idx, int base) {
+        const int par = idx & 1;
+        float *sc = sm.scores + par * SC;
+        const DT *qrow = reinterpret_cast<const DT *>(a.q) + (int64_t)rc.row * D;
+        float qreg[D / 32];
 #pragma unroll
-    for (int off = G::NCG; off < 32; off <<= 1) {
+        for (int k = 0; k < D / 32; ++k)
+            qreg[k] = to_f32(qrow[lane + 32 * k]) * a.qscale;
+        float mx = -INFINITY;
+        for (int i = first_owned(base, warp); i < rc.nmy; i += kConsumerWarps) {
+            const int s = base + i;
+            const int slot = s % stages;
+            mbar_wait(&sm.full[slot], (s / stages) & 1, a.status);
+            const uint8_t *st = sm.ring + slot * G::STAGE;
+            const __half *ksc = reinterpret_cast<const __half *>(st + G::KCODES);        // even block: scales
+            const __half *kzp = reinterpret_cast<const __half *>(st + G::KB + G::KCODES); // odd block: zeros
+            float av[D / 32];
+            float zs = 0.f, amax = 0.f;
 #pragma unroll
-        for (int k = 0; k < 2; ++k)
+            for (int k = 0; k < D / 32; ++k) {
+                const int c = lane + 32 * k;
+                av[k] = qreg[k] * __half2float(ksc[c]);
+                zs = fmaf(qreg[k], __half2float(kzp[c]), zs);
+                amax = fmaxf(amax, fabsf(av[k]));
+            }
+            zs = warp_sum(zs);
+            amax = warp_max(amax);
+            // Factor of channel c: a_c * 2^(149 - pos - K), K = E + 23, E = exponent of amax,
+            // so |factor| < 2^127 and every product code * factor is exact up to one rounding.
+            const uint32_t abits = __float_as_uint(amax);
+            const int E = abits >= 0x00800000u ? (int)(abits >> 23) - 127 : 0;
+            if (E >= -25 && E <= 100 && abits >= 0x00800000u) { // warp-uniform fast path
+                const float f = __int_as_float((102 - E + 127) << 23); // 2^(102 - E)
 #pragma unroll
-            for (int e = 0; e < 2; ++e)
+                for (int k = 0; k < D / 32; ++k)
+                    aw[kslot[k]] = (av[k] * f) * kpow[k];
+            } else {
 #pragma unroll
-                for (int n = 0; n < 4; ++n) {
-                    acc[k][e][n].x += __shfl_xor_sync(0xFFFFFFFFu, acc[k][e][n].x, off);
-                    acc[k][e][n].y += __shfl_xor_sync(0xFFFFFFFFu, acc[k][e][n].y, off);
+                for (int k = 0; k < D / 32; ++k) {
+                    int slot_c, pos;
+                    key_slot<BITS>(lane + 32 * k, slot_c, pos);
+                    aw[slot_c] = mul_pow2(av[k], 126 - E - pos);
                 }
-        zacc += __shfl_xor_sync(0xFFFFFFFFu, zacc, off);
-    }
-    lsum = warp_sum(lsum);
-    float *red = sm.red + warp * (D + 1);
-    if (lane < G::NCG) {
+            }
+            __syncwarp();
+            const uint32_t *kr =
+                reinterpret_cast<const uint32_t *>(st + (lane >> 4) * G::KB + (lane & 15) * G::ROWK);
+            float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int k = 0; k < 2; ++k)
-#pragma unroll
-            for (int e = 0; e < 2; ++e)
-#pragma unroll
-                for (int n = 0; n < 8; ++n) {
-                    const float v = (n & 1) ? acc[k][e][n >> 1].y : acc[k][e][n >> 1].x;
-                    const int ch = 32 * cg + 16 * k + value_channel(e, n);
-                    red[ch] = mul_pow2(v, kVScaleExp - value_pos(n)) + zacc;
+            for (int w4 = 0; w4 < G::WORDSK / 4; ++w4) {
+                const uint4 cw = reinterpret_cast<const uint4 *>(kr)[w4];
+                if (BITS == 4) {
+                    key_word4(cw.x, aw + 8 * (4 * w4 + 0), acc);
+                    key_word4(cw.y, aw + 8 * (4 * w4 + 1), acc);
+                    key_word4(cw.z, aw + 8 * (4 * w4 + 2), acc);
+                    key_word4(cw.w, aw + 8 * (4 * w4 + 3), acc);
+                } else {
+                    key_word2(cw.x, aw + 16 * (4 * w4 + 0), acc);
+                    key_word2(cw.y, aw + 16 * (4 * w4 + 1), acc);
+                    key_word2(cw.z, aw + 16 * (4 * w4 + 2), acc);
+                    key_word2(cw.w, aw + 16 * (4 * w4 + 3), acc);
                 }
-    }
-    if (lane == 0)
-        red[D] = lsum;
-    __syncwarp();
-    if (tail_cta && warp == kConsumerWarps - 1) { // tail values, exact
-        float tl = 0.f;
-        for (int t = 0; t < tail; ++t) {
-            const float w = exp2f(tsc[t] - m2);
-            tl += w;
-            const DT *vt = tailv + (int64_t)t * D;
+            }
+            const float accs = acc.x + acc.y;
+            const float s2 = (E <= 100 ? accs * __int_as_float((E + 150) << 23) : mul_pow2(accs, E + 23)) + zs;
+            sc[i * 32 + lane] = s2;
+            mx = fmaxf(mx, s2);
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&sm.empty[slot]);
+        }
+        if (rc.tail_cta && warp == kConsumerWarps - 1) { // tail keys, exact; lane = tail token
+            const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)rc.b * 2 * a.H + rc.h) * 32 * D;
+            float s2 = 0.f;
 #pragma unroll
             for (int k = 0; k < D / 32; ++k)
-                red[lane + 32 * k] = fmaf(w, to_f32(vt[lane + 32 * k]), red[lane + 32 * k]);
+                for (int c = 0; c < 32; ++c) {
+                    const float qc = __shfl_sync(0xFFFFFFFFu, qreg[k], c);
+                    if (lane < rc.tail)
+                        s2 = fmaf(qc, to_f32(kt[(int64_t)lane * D + 32 * k + c]), s2);
+                }
+            if (lane < rc.tail) {
+                sc[a.cap_groups * 32 + lane] = s2;
+                mx = fmaxf(mx, s2);
+            }
         }
-        __syncwarp();
-        if (lane == 0)
-            red[D] += tl;
-    }
-    named_sync(1, kConsumerWarps * 32);
-    for (int c = threadIdx.x; c <= D; c += kConsumerWarps * 32) {
-        float s = 0.f;
+        mx = warp_max(mx);
+        float ls = 0.f;
+        if (a.tau_mode == LOOPKV_TAU_ABS_PROB && mx != -INFINITY) {
+            for (int i = first_owned(base, warp); i < rc.nmy; i += kConsumerWarps)
+                ls += exp2f(sc[i * 32 + lane] - mx);
+            if (rc.tail_cta && warp == kConsumerWarps - 1 && lane < rc.tail)
+                ls += exp2f(sc[a.cap_groups * 32 + lane] - mx);
+            ls = warp_sum(ls);
+        }
+        if (lane == 0) {
+            float *st = sm.stat + (idx % 3) * kConsumerWarps * 2;
+            st[2 * warp] = mx;
+            st[2 * warp + 1] = ls;
+        }
+    };
+
+    // V pass of one row, then the CTA partial (o, l) into part[row parity].
+    auto consume_v = [&](const RowCtx &rc, int idx, int base, float m2, float thr2) {
+        const int par = idx & 1;
+        const float *sc = sm.scores + par * SC;
+        const int cg = lane % G::NCG, ts = lane / G::NCG;
+        float2 acc[2][2][4];
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w)
-            s += sm.red[w * (D + 1) + c];
-        sm.po[c] = s;
+        for (int k = 0; k < 2; ++k)
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+#pragma unroll
+                for (int n = 0; n < 4; ++n)
+                    acc[k][e][n] = make_float2(0.f, 0.f);
+        float zacc = 0.f, lsum = 0.f;
+        for (int i = first_owned(base, warp); i < rc.nmy; i += kConsumerWarps) {
+            const int s = base + i;
+            const int slot = s % stages;
+            const float s2l = sc[i * 32 + lane];
+            const float wl = exp2f(s2l - m2);
+            const uint32_t hotmask =
+                all_hot ? 0xFFFFFFFFu : (BITS == 4 ? __ballot_sync(0xFFFFFFFFu, s2l >= thr2) : 0u);
+            lsum += wl;
+            wv[lane] = wl;
+            __syncwarp();
+            mbar_wait(&sm.full[slot], (s / stages) & 1, a.status);
+            const uint8_t *st = sm.ring + slot * G::STAGE;
+#pragma unroll
+            for (int u = 0; u < 32 / G::TPI; ++u) {
+                const int t = u * G::TPI + ts;
+                const float w = wv[t];
+                const bool hot = (hotmask >> t) & 1u;
+                const int blk = t >> 4, r = t & 15;
+                const uint8_t *vb = st + blk * G::VB;
+                const __half2 meta = *reinterpret_cast<const __half2 *>(vb + r * G::NCG * 4 + cg * 4);
+                const float vs = __low2float(meta), vz = __high2float(meta);
+                const uint2 hw = *reinterpret_cast<const uint2 *>(vb + G::VMETA + r * G::ROWV + cg * 8);
+                uint2 lw = make_uint2(0u, 0u);
+                float W;
+                if (BITS == 4) {
+                    if (hot)
+                        lw = *reinterpret_cast<const uint2 *>(st + 2 * G::VB + blk * G::LOB + r * G::ROWV + cg * 8);
+                    W = w * vs;
+                    zacc = fmaf(w, hot ? vz : fmaf(1.5f, vs, vz), zacc);
+                } else {
+                    W = w * vs * 0.25f;
+                    zacc = fmaf(w, vz, zacc);
+                }
+                const float Wp = W * vscale;
+                value_word(hw.x, lw.x, Wp, acc[0]);
+                value_word(hw.y, lw.y, Wp, acc[1]);
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&sm.empty[slot]);
+        }
+        // reduce over the token slots of the warp (lanes with the same cg)
+#pragma unroll
+        for (int off = G::NCG; off < 32; off <<= 1) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+#pragma unroll
+                for (int e = 0; e < 2; ++e)
+#pragma unroll
+                    for (int n = 0; n < 4; ++n) {
+                        acc[k][e][n].x += __shfl_xor_sync(0xFFFFFFFFu, acc[k][e][n].x, off);
+                        acc[k][e][n].y += __shfl_xor_sync(0xFFFFFFFFu, acc[k][e][n].y, off);
+                    }
+            zacc += __shfl_xor_sync(0xFFFFFFFFu, zacc, off);
+        }
+        lsum = warp_sum(lsum);
+        float *red = sm.red + warp * (D + 1);
+        if (lane < G::NCG) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+#pragma unroll
+                for (int e = 0; e < 2; ++e)
+#pragma unroll
+                    for (int n = 0; n < 8; ++n) {
+                        const float v = (n & 1) ? acc[k][e][n >> 1].y : acc[k][e][n >> 1].x;
+                        const int ch = 32 * cg + 16 * k + value_channel(e, n);
+                        red[ch] = mul_pow2(v, kVScaleExp - value_pos(n)) + zacc;
+                    }
+        }
+        if (lane == 0)
+            red[D] = lsum;
+        __syncwarp();
+        if (rc.tail_cta && warp == kConsumerWarps - 1) { // tail values, exact
+            const DT *vt0 = reinterpret_cast<const DT *>(a.tail) + ((int64_t)(rc.b * 2 + 1) * a.H + rc.h) * 32 * D;
+            float tl = 0.f;
+            for (int t = 0; t < rc.tail; ++t) {
+                const float w = exp2f(sc[a.cap_groups * 32 + t] - m2);
+                tl += w;
+                const DT *vt = vt0 + (int64_t)t * D;
+#pragma unroll
+                for (int k = 0; k < D / 32; ++k)
+                    red[lane + 32 * k] = fmaf(w, to_f32(vt[lane + 32 * k]), red[lane + 32 * k]);
+            }
+            __syncwarp();
+            if (lane == 0)
+                red[D] += tl;
+        }
+        named_sync(1, kConsumerWarps * 32);
+        float *part = sm.part + par * (D + 1);
+        for (int c = threadIdx.x; c <= D; c += kConsumerWarps * 32) {
+            float sum = 0.f;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w)
+                sum += sm.red[w * (D + 1) + c];
+            part[c] = sum;
+        }
+    };
+
+    // CTA `crank` writes channels [crank*D/C, (crank+1)*D/C) of a row, summing the
+    // partials of every CTA of the cluster.
+    auto merge = [&](const RowCtx &rc, int idx, float m2) {
+        const float *part = sm.part + (idx & 1) * (D + 1);
+        const int per = D / (int)C;
+        if ((int)threadIdx.x < per) {
+            const int c = (int)crank * per + (int)threadIdx.x;
+            float o = 0.f, l = 0.f;
+            for (uint32_t r = 0; r < C; ++r) {
+                o += ld_dsmem_f32(part + c, r);
+                l += ld_dsmem_f32(part + D, r);
+            }
+            float out = 0.f;
+            if (l > 0.f)
+                out = o / l;
+            else if (c == 0)
+                atomicOr(a.status, LOOPKV_DEV_EMPTY_ROW);
+            a.out[(int64_t)rc.row * D + c] = out;
+            if (c == 0) {
+                if (a.row_max)
+                    a.row_max[rc.row] = m2 * 0.6931471805599453f;
+                if (a.row_sum)
+                    a.row_sum[rc.row] = l;
+            }
+        }
+    };
+
+    int pos = 0;
+    RowCtx prev{}, prev2{};
+    float m_prev = 0.f, m_prev2 = 0.f;
+    if (nrows > 0) {
+        prev = row_ctx(a, cid, crank, C);
+        consume_k(prev, 0, pos);
+        pos += prev.nmy;
     }
-    cluster_arrive(); // barrier 3
+    cluster_arrive(); // row 0
+    for (int i = 1; i < nrows; ++i) {
+        named_sync(1, kConsumerWarps * 32); // every consumer warp is done with row i - 2
+        const RowCtx cur = row_ctx(a, cid + i * ncl, crank, C);
+        consume_k(cur, i, pos);
+        pos += cur.nmy;
+        cluster_wait(); // row i - 1: maxima of row i - 1, partials of row i - 2
+        if (i >= 2)
+            merge(prev2, i - 2, m_prev2);
+        float m2, l2;
+        cluster_row_stats(sm.stat + ((i - 1) % 3) * kConsumerWarps * 2, C, m2, l2);
+        consume_v(prev, i - 1, pos, m2, row_threshold(a, m2, l2, decide));
+        pos += prev.nmy;
+        prev2 = prev;
+        m_prev2 = m2;
+        prev = cur;
+        cluster_arrive(); // row i
+    }
+    cluster_wait(); // last row
+    if (nrows >= 2)
+        merge(prev2, nrows - 2, m_prev2);
+    if (nrows > 0) {
+        float m2, l2;
+        cluster_row_stats(sm.stat + ((nrows - 1) % 3) * kConsumerWarps * 2, C, m2, l2);
+        consume_v(prev, nrows - 1, pos, m2, row_threshold(a, m2, l2, decide));
+        m_prev = m2;
+    }
+    cluster_arrive(); // partials of the last row
     cluster_wait();
-    // CTA `crank` reduces channels [crank*D/C, (crank+1)*D/C) over the cluster.
-    const int per = D / (int)C;
-    if ((int)threadIdx.x < per) {
-        const int c = (int)crank * per + (int)threadIdx.x;
-        float s = 0.f, l = 0.f;
-        for (uint32_t r = 0; r < C; ++r) {
-            s += ld_dsmem_f32(sm.po + c, r);
-            l += ld_dsmem_f32(sm.po + D, r);
-        }
-        float o = 0.f;
-        if (l > 0.f)
-            o = s / l;
-        else if (c == 0)
-            atomicOr(a.status, LOOPKV_DEV_EMPTY_ROW);
-        a.out[(int64_t)row * D + c] = o;
-        if (c == 0) {
-            if (a.row_max)
-                a.row_max[row] = m2 * 0.6931471805599453f;
-            if (a.row_sum)
-                a.row_sum[row] = l;
-        }
-    }
-    cluster_arrive(); // barrier 4
+    if (nrows > 0)
+        merge(prev, nrows - 1, m_prev);
+    cluster_arrive(); // remote reads done
     cluster_wait();
 }
 
 template <int BITS, int D, typename DT>
-int launch_t(const DecodeArgs &a, int B, const DecodeShape &shp, cudaStream_t s)
+int launch_t(const DecodeArgs &a, const DecodeShape &shp, cudaStream_t s)
 {
     auto kern = decode_kernel<BITS, D, DT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, shp.smem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e == cudaSuccess && shp.cluster > 8)
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess)
         return LOOPKV_ERR_CUDA;
-    if (shp.cluster > 8) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess)
-            return LOOPKV_ERR_CUDA;
-    }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(shp.cluster, B * a.H, 1);
+    cfg.gridDim = dim3(shp.cluster * shp.clusters, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = shp.smem;
     cfg.stream = s;
@@ -613,40 +762,119 @@ int launch_t(const DecodeArgs &a, int B, const DecodeShape &shp, cudaStream_t s)
     return e == cudaSuccess ? LOOPKV_OK : LOOPKV_ERR_CUDA;
 }
 
-}  // namespace
-
-DecodeShape decode_shape(int bits, int D, int rows, int max_blocks)
+// Clusters of size C that can be resident at once for this kernel and shared memory.
+template <int BITS, int D, typename DT> int max_active_clusters(int C, int smem)
 {
-    DecodeShape shp;
-    shp.threads = kThreads;
-    shp.stages = 8;
-    const int max_groups = max_blocks / 2;
-    // Cluster size: enough CTAs to cover the GPU several times, at most 8 (portable).
-    int C = 1;
-    while (C < 8 && rows * C < 4 * 148)
-        C *= 2;
-    while (C > 1 && (max_groups + C - 1) / C < 1)
-        C /= 2;
-    shp.cluster = C;
-    const int cap = (max_groups + C - 1) / C;
-    if (bits == 4)
-        shp.smem = D == 128 ? smem_bytes<4, 128>(shp.stages, cap) : smem_bytes<4, 64>(shp.stages, cap);
-    else
-        shp.smem = D == 128 ? smem_bytes<2, 128>(shp.stages, cap) : smem_bytes<2, 64>(shp.stages, cap);
-    return shp;
+    auto kern = decode_kernel<BITS, D, DT>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return 0;
+    cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (C > 8)
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(C, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
 }
 
-int launch_decode(const DecodeArgs &a, int bits, int D, int dtype, int B, const DecodeShape &shp, cudaStream_t s)
+template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_blocks)
+{
+    using G = Geo<BITS, D>;
+    DecodeShape best = {};
+    double best_eff = -1.0;
+    const int max_groups = max_blocks / 2;
+    int sm_count = 148;
+    {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            sm_count = 148;
+    }
+    const int smem_per_sm = 228 * 1024;
+    const char *env_c = getenv("LOOPKV_DECODE_CLUSTER");
+    const char *env_s = getenv("LOOPKV_DECODE_STAGES");
+    const char *env_o = getenv("LOOPKV_DECODE_CTAS_PER_SM");
+    const int want_ctas = env_o ? atoi(env_o) : 4;
+    for (int C = 1; C <= 16; C *= 2) {
+        if (env_c && atoi(env_c) != C)
+            continue;
+        if (D / C < 4)
+            continue;
+        const int cap = (max_groups + C - 1) / C;
+        // stages: fill the shared memory of `want_ctas` CTAs per SM (1 KB reserved per CTA)
+        const int budget = smem_per_sm / want_ctas - 1024;
+        int stages = (budget - smem_fixed<BITS, D>(cap)) / (G::STAGE + 16);
+        if (stages > 32)
+            stages = 32;
+        if (env_s)
+            stages = atoi(env_s);
+        if (stages < 4)
+            stages = 4;
+        const int smem = smem_bytes<BITS, D>(stages, cap);
+        if (smem > 227 * 1024 || !layout_ok<BITS, D>(stages, cap))
+            continue;
+        int ncl = max_active_clusters<BITS, D, DT>(C, smem);
+        if (ncl <= 0)
+            continue;
+        if (ncl > rows)
+            ncl = rows;
+        // balance: each cluster takes ceil(rows / ncl) rows; parallel slack penalised
+        const double rounds = (double)((rows + ncl - 1) / ncl);
+        const double eff = ((double)rows / ncl) / rounds * std::min(1.0, (double)(ncl * C) / (3.0 * sm_count));
+        if (eff > best_eff + 1e-9) {
+            best_eff = eff;
+            best.cluster = C;
+            best.clusters = ncl;
+            best.stages = stages;
+            best.smem = smem;
+            best.threads = kThreads;
+            best.cap = cap;
+        }
+    }
+    return best;
+}
+
+}  // namespace
+
+DecodeShape decode_shape(int bits, int D, int dtype, int rows, int max_blocks)
 {
     const bool bf = dtype == LOOPKV_DTYPE_BF16;
     if (bits == 4) {
         if (D == 128)
-            return bf ? launch_t<4, 128, __nv_bfloat16>(a, B, shp, s) : launch_t<4, 128, float>(a, B, shp, s);
-        return bf ? launch_t<4, 64, __nv_bfloat16>(a, B, shp, s) : launch_t<4, 64, float>(a, B, shp, s);
+            return bf ? shape_t<4, 128, __nv_bfloat16>(rows, max_blocks) : shape_t<4, 128, float>(rows, max_blocks);
+        return bf ? shape_t<4, 64, __nv_bfloat16>(rows, max_blocks) : shape_t<4, 64, float>(rows, max_blocks);
     }
     if (D == 128)
-        return bf ? launch_t<2, 128, __nv_bfloat16>(a, B, shp, s) : launch_t<2, 128, float>(a, B, shp, s);
-    return bf ? launch_t<2, 64, __nv_bfloat16>(a, B, shp, s) : launch_t<2, 64, float>(a, B, shp, s);
+        return bf ? shape_t<2, 128, __nv_bfloat16>(rows, max_blocks) : shape_t<2, 128, float>(rows, max_blocks);
+    return bf ? shape_t<2, 64, __nv_bfloat16>(rows, max_blocks) : shape_t<2, 64, float>(rows, max_blocks);
+}
+
+int launch_decode(const DecodeArgs &a, int bits, int D, int dtype, const DecodeShape &shp, cudaStream_t s)
+{
+    if (shp.cluster <= 0 || shp.clusters <= 0)
+        return LOOPKV_ERR_CUDA;
+    const bool bf = dtype == LOOPKV_DTYPE_BF16;
+    if (bits == 4) {
+        if (D == 128)
+            return bf ? launch_t<4, 128, __nv_bfloat16>(a, shp, s) : launch_t<4, 128, float>(a, shp, s);
+        return bf ? launch_t<4, 64, __nv_bfloat16>(a, shp, s) : launch_t<4, 64, float>(a, shp, s);
+    }
+    if (D == 128)
+        return bf ? launch_t<2, 128, __nv_bfloat16>(a, shp, s) : launch_t<2, 128, float>(a, shp, s);
+    return bf ? launch_t<2, 64, __nv_bfloat16>(a, shp, s) : launch_t<2, 64, float>(a, shp, s);
 }
 
 }  // namespace lkv

@@ -44,6 +44,7 @@ struct DecodeArgs {
     float *row_sum;             // optional [B][H]
     int64_t pool_blocks;
     int H;
+    int rows;                   // B * H (request, head) rows
     int max_blocks;
     int bitmap_words;
     int cap_groups;             // score capacity per CTA, in 32-token groups
@@ -53,16 +54,17 @@ struct DecodeArgs {
 };
 
 struct DecodeShape {
-    int cluster;   // CTAs per (request, head) row
-    int stages;    // pipeline depth
-    int smem;      // dynamic shared memory bytes
+    int cluster;   // CTAs per cluster; a cluster reads one (request, head) row at a time
+    int clusters;  // persistent clusters in the grid
+    int stages;    // pipeline depth (shared-memory ring slots per CTA)
+    int smem;      // dynamic shared memory bytes per CTA
     int threads;
+    int cap;       // score capacity per CTA and row, in 32-token groups
 };
 
 // Launchers (defined in the .cu files).  Return LOOPKV_OK or an error code.
-int launch_decode(const DecodeArgs &a, int bits, int D, int dtype, int B, const DecodeShape &shp,
-                  cudaStream_t s);
-DecodeShape decode_shape(int bits, int D, int rows, int max_blocks);
+int launch_decode(const DecodeArgs &a, int bits, int D, int dtype, const DecodeShape &shp, cudaStream_t s);
+DecodeShape decode_shape(int bits, int D, int dtype, int rows, int max_blocks);
 
 int launch_init_state(const DevState &st, cudaStream_t s);
 int launch_append(const DevState &st, int cell, int H, int D, int dtype, int max_batch, const void *k,

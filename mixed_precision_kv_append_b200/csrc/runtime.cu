@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <new>
 #include <vector>
 
@@ -27,6 +28,19 @@ struct loopkv_plan {
 
 struct loopkv_cache {
     loopkv_plan plan;
+    // decode launch shapes by (storage bits, batch), computed once (occupancy queries
+    // must not run while a stream is being captured)
+    std::map<std::pair<int, int>, lkv::DecodeShape> shapes;
+    const lkv::DecodeShape &shape(int bits, int B)
+    {
+        auto key = std::make_pair(bits, B);
+        auto it = shapes.find(key);
+        if (it == shapes.end())
+            it = shapes.emplace(key, lkv::decode_shape(bits, plan.cfg.head_dim, plan.cfg.in_dtype,
+                                                       B * plan.cfg.n_heads, plan.cfg.max_blocks_per_seq))
+                     .first;
+        return it->second;
+    }
     lkv::DevState st;
     uint8_t *modes_dev;
     int32_t *req_stage; // [max_batch] request ids of the last loopkv_append with req_ids
@@ -401,11 +415,12 @@ int loopkv_reset_request(loopkv_cache *cache, int req, void *stream)
                              static_cast<cudaStream_t>(stream));
 }
 
-int loopkv_decode_debug(const loopkv_plan *plan, int loop, int layer, const void *q, const loopkv_cache *cache,
+int loopkv_decode_debug(const loopkv_plan *plan, int loop, int layer, const void *q, const loopkv_cache *ccache,
                         float *out, int B, void *stream, uint32_t *s_bitmap, float *row_max, float *row_sum)
 {
-    if (!plan || !cache || !q || !out)
+    if (!plan || !ccache || !q || !out)
         return LOOPKV_ERR_INVALID_ARG;
+    loopkv_cache *cache = const_cast<loopkv_cache *>(ccache); // only the launch-shape memo changes
     int rc = check_cell(plan, loop, layer);
     if (rc)
         return rc;
@@ -434,14 +449,15 @@ int loopkv_decode_debug(const loopkv_plan *plan, int loop, int layer, const void
     a.row_sum = row_sum;
     a.pool_blocks = bits == 4 ? cache->st.n4 : cache->st.n2;
     a.H = H;
+    a.rows = B * H;
     a.max_blocks = MB;
     a.bitmap_words = MB / 2;
     a.qscale = (float)(1.4426950408889634 / std::sqrt((double)D));
     a.tau = plan->tau;
     a.tau_mode = plan->tau_mode;
-    lkv::DecodeShape shp = lkv::decode_shape(bits, D, B * H, MB);
-    a.cap_groups = (MB / 2 + shp.cluster - 1) / shp.cluster;
-    return lkv::launch_decode(a, bits, D, cp.cfg.in_dtype, B, shp, static_cast<cudaStream_t>(stream));
+    const lkv::DecodeShape &shp = cache->shape(bits, B);
+    a.cap_groups = shp.cap;
+    return lkv::launch_decode(a, bits, D, cp.cfg.in_dtype, shp, static_cast<cudaStream_t>(stream));
 }
 
 int loopkv_decode(const loopkv_plan *plan, int loop, int layer, const void *q, const loopkv_cache *cache, float *out,
@@ -512,15 +528,18 @@ int loopkv_decode_shape(const loopkv_plan *plan, int B, int *cluster_size, int *
 {
     if (!plan || B <= 0)
         return LOOPKV_ERR_INVALID_ARG;
-    // the widest shape over the cells (4-bit sources need the larger stage)
-    lkv::DecodeShape shp = lkv::decode_shape(4, plan->cfg.head_dim, B * plan->cfg.n_heads, plan->cfg.max_blocks_per_seq);
+    if (check_device())
+        return LOOPKV_ERR_NO_DEVICE; // the shape comes from an occupancy query of the device
+    // the shape of a 4-bit source cell (the larger pipeline stage)
+    lkv::DecodeShape shp = lkv::decode_shape(4, plan->cfg.head_dim, plan->cfg.in_dtype, B * plan->cfg.n_heads,
+                                             plan->cfg.max_blocks_per_seq);
     if (cluster_size)
         *cluster_size = shp.cluster;
     if (ctas)
-        *ctas = shp.cluster * B * plan->cfg.n_heads;
+        *ctas = shp.cluster * shp.clusters;
     if (smem_bytes)
         *smem_bytes = shp.smem;
-    return LOOPKV_OK;
+    return shp.cluster > 0 ? LOOPKV_OK : LOOPKV_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -133,10 +133,3 @@ def test_alloc_without_device_fails_loudly():
     with pytest.raises(L.LoopKVError) as e:
         L.loopkv_alloc(p.handle, buf, stream=0)
     assert e.value.code in (-12, -8)
-
-
-def test_decode_shape_reports_cluster_launch():
-    p = L.Plan(24, 4, 16, 128, 8, 514, [0] * 96, 0.0)
-    shp = p.decode_shape(8)
-    assert shp["cluster"] in (1, 2, 4, 8, 16) and shp["ctas"] == shp["cluster"] * 8 * 16
-    assert 0 < shp["smem"] <= 227 * 1024

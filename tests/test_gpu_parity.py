@@ -220,7 +220,7 @@ def test_full_size_sampled_rows(name, B, T, modes, tau, steps):
 
 
 def test_graph_replay_matches_eager():
-    modes = [L.CELL_4B, L.CELL_2B, L.CELL_SHARE, L.CELL_4B]
+    modes = [L.CELL_4B, L.CELL_SHARE, L.CELL_2B, L.CELL_4B]  # loop 0: [4b, share], loop 1: [2b, 4b]
     w = synth.Workload("graph", 2, 2, 4, 128, 3, [33, 64, 200], torch.bfloat16, modes, 0.01, append_steps=40,
                        seed=11)
     m = Model(w)
@@ -228,10 +228,13 @@ def test_graph_replay_matches_eager():
     qs = [[_q(w, 0, layer, lp) for lp in range(2)] for layer in range(2)]
     _, ks, vs = synth.step_tokens(w, 0, 0, device="cuda")
     outs = [[torch.empty_like(qs[0][0], dtype=torch.float32) for _ in range(2)] for _ in range(2)]
+    for layer in range(2):  # eager decodes fix each cell's launch shape before the capture
+        for lp in range(2):
+            m.cache.decode(lp, layer, qs[layer][lp])
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
-        m.cache.flush(stream=s)  # warm the launch attributes outside the capture
+        m.cache.flush(stream=s)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=s):
             m.cache.flush(stream=s)
@@ -327,3 +330,10 @@ def test_empty_row_is_reported():
     rc, bits = cache.status()
     assert rc == -11 and bits & L.DEV_EMPTY_ROW
     assert torch.all(out == 0)
+
+
+def test_decode_shape_reports_cluster_launch():
+    p = L.Plan(24, 4, 16, 128, 8, 514, [0] * 96, 0.0)
+    shp = p.decode_shape(8)
+    assert shp["cluster"] in (1, 2, 4, 8, 16) and shp["ctas"] % shp["cluster"] == 0
+    assert shp["ctas"] >= 148 and 0 < shp["smem"] <= 227 * 1024
