@@ -45,8 +45,8 @@
 namespace lkv {
 namespace {
 
-constexpr int kConsumerWarps = 4;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kWarps = 4; // every warp both issues the copies of its stages and computes on them
+constexpr int kThreads = kWarps * 32;
 constexpr int kMinCtasPerSm = 4;
 constexpr int kVScaleExp = 40; // V accumulators hold code * w * s * 2^(p - 40)
 
@@ -149,70 +149,65 @@ __device__ __forceinline__ int value_channel(int e, int n) { return 8 * (n & 1) 
 __device__ __forceinline__ int value_pos(int n) { return n < 6 ? 4 * n : (n == 6 ? 8 : 12); }
 
 struct Smem {
-    uint8_t *ring;     // [stages][STAGE]
-    uint64_t *full;    // [stages]
-    uint64_t *empty;   // [stages]
-    float *scores;     // [2][cap * 32 + 32] scores of a row (history, then tail), by row parity
-    float *stat;       // [3][kConsumerWarps][2] per-warp (max, sum exp(s - max)), by row index mod 3
+    uint8_t *ring;     // [kWarps][spw][STAGE] stage slots, a private slice per warp
+    uint64_t *full;    // [kWarps][spw] completion barriers of the slots
+    float *scores;     // [2][kWarps][capw * 32] scores of a warp's groups, by row parity
+    float *tscores;    // [2][32] tail scores, by row parity
+    float *aw;         // [kWarps][D] key factors
+    float *stat;       // [3][kWarps][2] per-warp (max, sum exp(s - max)), by row index mod 3
     float *part;       // [2][D + 1] CTA partial o and l of a row, by row parity
-    float *aw;         // [kConsumerWarps][D] key factors
-    float *wv;         // [kConsumerWarps][32] weights of the group a warp reads
-    float *red;        // [kConsumerWarps][D + 1]
-    int32_t *ids;      // [2][2 * cap] block ids of a row's groups (even, odd block), by row parity
+    float *wv;         // [kWarps][32] weights of the group a warp reads
+    float *red;        // [kWarps][D + 1]
+    int32_t *ids;      // [3][kWarps][2 * capw] block ids of a warp's groups, by row index mod 3
 };
 
 // Byte offsets of the shared-memory regions; every region starts on a 16-byte boundary
 // (the key factors and the stage data are read with 16-byte vector loads).
 struct SmemLayout {
-    int full, empty, scores, stat, part, aw, wv, red, ids, total;
+    int full, scores, tscores, aw, stat, part, wv, red, ids, total;
 };
 
 __host__ __device__ constexpr int align16(int x) { return (x + 15) & ~15; }
 
-template <int BITS, int D> __host__ __device__ constexpr SmemLayout smem_layout(int stages, int cap)
+template <int BITS, int D> __host__ __device__ constexpr SmemLayout smem_layout(int spw, int capw)
 {
     SmemLayout L{};
-    int o = stages * Geo<BITS, D>::STAGE; // ring, 128-byte aligned slots
+    int o = kWarps * spw * Geo<BITS, D>::STAGE; // ring, 128-byte aligned slots
     L.full = o;
-    o = align16(o + stages * 8);
-    L.empty = o;
-    o = align16(o + stages * 8);
+    o = align16(o + kWarps * spw * 8);
     L.scores = o;
-    o = align16(o + 2 * (cap * 32 + 32) * 4);
+    o = align16(o + 2 * kWarps * capw * 32 * 4);
+    L.tscores = o;
+    o = align16(o + 2 * 32 * 4);
     L.aw = o;
-    o = align16(o + kConsumerWarps * D * 4);
+    o = align16(o + kWarps * D * 4);
     L.stat = o;
-    o = align16(o + 3 * kConsumerWarps * 2 * 4);
+    o = align16(o + 3 * kWarps * 2 * 4);
     L.part = o;
     o = align16(o + 2 * (D + 1) * 4);
     L.wv = o;
-    o = align16(o + kConsumerWarps * 32 * 4);
+    o = align16(o + kWarps * 32 * 4);
     L.red = o;
-    o = align16(o + kConsumerWarps * (D + 1) * 4);
+    o = align16(o + kWarps * (D + 1) * 4);
     L.ids = o;
-    o = align16(o + 2 * 2 * cap * 4);
+    o = align16(o + 3 * kWarps * 2 * capw * 4);
     L.total = o;
     return L;
 }
 
-template <int BITS, int D> __host__ __device__ constexpr int smem_bytes(int stages, int cap)
+template <int BITS, int D> __host__ __device__ constexpr int smem_bytes(int spw, int capw)
 {
-    return smem_layout<BITS, D>(stages, cap).total;
+    return smem_layout<BITS, D>(spw, capw).total;
 }
 
-template <int BITS, int D> __host__ __device__ constexpr int smem_fixed(int cap)
+template <int BITS, int D> __device__ Smem carve(uint8_t *base, int spw, int capw)
 {
-    return smem_layout<BITS, D>(0, cap).total;
-}
-
-template <int BITS, int D> __device__ Smem carve(uint8_t *base, int stages, int cap)
-{
-    const SmemLayout L = smem_layout<BITS, D>(stages, cap);
+    const SmemLayout L = smem_layout<BITS, D>(spw, capw);
     Smem s;
     s.ring = base;
     s.full = reinterpret_cast<uint64_t *>(base + L.full);
-    s.empty = reinterpret_cast<uint64_t *>(base + L.empty);
     s.scores = reinterpret_cast<float *>(base + L.scores);
+    s.tscores = reinterpret_cast<float *>(base + L.tscores);
     s.aw = reinterpret_cast<float *>(base + L.aw);
     s.stat = reinterpret_cast<float *>(base + L.stat);
     s.part = reinterpret_cast<float *>(base + L.part);
@@ -222,12 +217,12 @@ template <int BITS, int D> __device__ Smem carve(uint8_t *base, int stages, int 
     return s;
 }
 
-// Host check of a layout: every region 16-byte aligned and inside the allocation.
-template <int BITS, int D> bool layout_ok(int stages, int cap)
+// Host check of a layout: every region 16-byte aligned, in order, inside the allocation.
+template <int BITS, int D> bool layout_ok(int spw, int capw)
 {
-    const SmemLayout L = smem_layout<BITS, D>(stages, cap);
-    const int offs[] = {L.full, L.empty, L.scores, L.aw, L.stat, L.part, L.wv, L.red, L.ids};
-    int prev = stages * Geo<BITS, D>::STAGE;
+    const SmemLayout L = smem_layout<BITS, D>(spw, capw);
+    const int offs[] = {L.full, L.scores, L.tscores, L.aw, L.stat, L.part, L.wv, L.red, L.ids};
+    int prev = kWarps * spw * Geo<BITS, D>::STAGE;
     for (int o : offs) {
         if (o % 16 || o < prev)
             return false;
@@ -239,12 +234,12 @@ template <int BITS, int D> bool layout_ok(int stages, int cap)
 // One (request, head) row as seen by one CTA of its cluster.
 struct RowCtx {
     int row, b, h;
-    int hist, tail;   // validated lengths
-    int nmy;          // 32-token groups of the history owned by this CTA
-    bool tail_cta;    // this CTA also reads the tail
+    int tail;       // validated tail length
+    int nmy;        // 32-token groups of the history owned by this CTA
+    bool tail_cta;  // this CTA also reads the tail
 };
 
-__device__ __forceinline__ RowCtx row_ctx(const DecodeArgs &a, int row, uint32_t crank, uint32_t C)
+__device__ __forceinline__ RowCtx row_ctx(const DecodeArgs &a, int row, uint32_t crank, uint32_t C, bool report)
 {
     RowCtx r;
     r.row = row;
@@ -266,13 +261,18 @@ __device__ __forceinline__ RowCtx row_ctx(const DecodeArgs &a, int row, uint32_t
         bad = true;
         nmy = a.cap_groups;
     }
-    if (bad && threadIdx.x == 0)
+    if (bad && report)
         atomicOr(a.status, LOOPKV_DEV_STATE);
-    r.hist = hist;
     r.tail = tail;
     r.nmy = nmy;
     r.tail_cta = (crank == C - 1) && tail > 0;
     return r;
+}
+
+// Groups of a row owned by warp w of the CTA: local groups w, w + kWarps, ...
+__device__ __forceinline__ int owned(const RowCtx &rc, int w)
+{
+    return rc.nmy > w ? (rc.nmy - w + kWarps - 1) / kWarps : 0;
 }
 
 // Row max m (log2 units) and, for the normalised rule, l = sum_t 2^(s_t - m), from the
@@ -281,13 +281,13 @@ __device__ __forceinline__ void cluster_row_stats(const float *stat, uint32_t C,
 {
     m = -INFINITY;
     for (uint32_t r = 0; r < C; ++r)
-        for (int w = 0; w < kConsumerWarps; ++w)
+        for (int w = 0; w < kWarps; ++w)
             m = fmaxf(m, ld_dsmem_f32(stat + 2 * w, r));
     l = 0.f;
     if (m == -INFINITY)
         return;
     for (uint32_t r = 0; r < C; ++r)
-        for (int w = 0; w < kConsumerWarps; ++w) {
+        for (int w = 0; w < kWarps; ++w) {
             const float mw = ld_dsmem_f32(stat + 2 * w, r);
             if (mw != -INFINITY)
                 l += ld_dsmem_f32(stat + 2 * w + 1, r) * exp2f(mw - m);
@@ -301,143 +301,174 @@ __device__ __forceinline__ float row_threshold(const DecodeArgs &a, float m, flo
     return a.tau_mode == LOOPKV_TAU_ABS_PROB ? m + log2f(a.tau * l) : m + log2f(a.tau);
 }
 
-// First stage index >= base in [base, base + n) owned by warp w (stage s -> warp s % NW).
-__device__ __forceinline__ int first_owned(int base, int w)
+// Segment sig of a warp's stage sequence K(0), K(1), V(0), K(2), V(1), ..., V(n-1):
+// returns whether it is a V segment and its row index.
+__device__ __forceinline__ void segment(int sig, int nrows, bool &is_v, int &ri)
 {
-    return ((w - base) % kConsumerWarps + kConsumerWarps) % kConsumerWarps;
+    if (sig == 0) {
+        is_v = false;
+        ri = 0;
+    } else if (sig == 2 * nrows - 1) {
+        is_v = true;
+        ri = nrows - 1;
+    } else {
+        const int i = (sig + 1) / 2;
+        is_v = !(sig & 1);
+        ri = (sig & 1) ? i : i - 1;
+    }
 }
 
 template <int BITS, int D, typename DT>
-__global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const DecodeArgs a, const int stages)
+__global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const DecodeArgs a, const int spw)
 {
     using G = Geo<BITS, D>;
     extern __shared__ __align__(128) uint8_t smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t crank = cluster_ctarank(), C = cluster_nctarank();
     const int cid = blockIdx.x / (int)C, ncl = gridDim.x / (int)C;
-    const int rows = a.rows;
-    const int nrows = cid < rows ? (rows - 1 - cid) / ncl + 1 : 0; // rows cid, cid + ncl, ...
-    Smem sm = carve<BITS, D>(smem_raw, stages, a.cap_groups);
-    const int SC = a.cap_groups * 32 + 32; // score buffer stride
+    const int nrows = cid < a.rows ? (a.rows - 1 - cid) / ncl + 1 : 0; // rows cid, cid + ncl, ...
+    const int capw = (a.cap_groups + kWarps - 1) / kWarps;
+    Smem sm = carve<BITS, D>(smem_raw, spw, capw);
     const bool all_hot = (BITS == 4) && !(a.tau > 0.f);
     const bool decide = (BITS == 4) && (a.tau > 0.f); // lo planes depend on the row max
 
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < stages; ++i) {
-            mbar_init(&sm.full[i], 1);
-            mbar_init(&sm.empty[i], 1);
-        }
-        fence_mbar_init();
-    }
-    __syncthreads();
+    if (lane == 0)
+        for (int i = 0; i < spw; ++i)
+            mbar_init(&sm.full[warp * spw + i], 1);
+    fence_mbar_init();
+    __syncwarp();
 
-    if (warp == kConsumerWarps) {
-        // ------------------------------------------------------------ producer
-        auto load_ids = [&](const RowCtx &rc, int par) {
-            const int32_t *bt = a.block_table + (int64_t)rc.b * a.max_blocks;
-            int32_t *ids = sm.ids + par * 2 * a.cap_groups;
-            for (int k = lane; k < 2 * rc.nmy; k += 32) {
-                int id = bt[2 * ((int)crank + (k >> 1) * (int)C) + (k & 1)];
-                if (id < 0 || id >= a.pool_blocks) {
-                    atomicOr(a.status, LOOPKV_DEV_STATE);
-                    id = 0;
-                }
-                ids[k] = id;
+    uint8_t *ring = sm.ring + warp * spw * G::STAGE;
+    uint64_t *full = sm.full + warp * spw;
+    auto scores_of = [&](int ri) { return sm.scores + ((ri & 1) * kWarps + warp) * capw * 32; };
+    auto ids_of = [&](int ri) { return sm.ids + ((ri % 3) * kWarps + warp) * 2 * capw; };
+
+    // ---------------------------------------------------------------- issuing
+    // A warp issues the bulk copies of its own stages, `spw` stages ahead of its compute.
+    RowCtx ictx[3];   // rows known to the issuer, by row index mod 3
+    float ithr[3];    // thresholds known to the issuer
+    int vfirst[3];    // warp-local stage number of the first V stage of a row
+    int vissued[3];   // V stages of a row issued so far (their meta + hi parts)
+    int iss_sig = 0, iss_k = 0, iss_n = 0;
+
+    auto setup_row = [&](int ri) {
+        RowCtx rc = row_ctx(a, cid + ri * ncl, crank, C, false);
+        ictx[ri % 3] = rc;
+        ithr[ri % 3] = NAN;
+        vissued[ri % 3] = 0;
+        const int n = owned(rc, warp);
+        const int32_t *bt = a.block_table + (int64_t)rc.b * a.max_blocks;
+        int32_t *ids = ids_of(ri);
+        for (int k = lane; k < 2 * n; k += 32) {
+            const int g = (int)crank + (warp + (k >> 1) * kWarps) * (int)C;
+            int id = bt[2 * g + (k & 1)];
+            if (id < 0 || id >= a.pool_blocks) {
+                atomicOr(a.status, LOOPKV_DEV_STATE);
+                id = 0;
+            }
+            ids[k] = id;
+        }
+        __syncwarp();
+    };
+    // lo planes (4-bit sources) of the hot tokens of V stage k of row ri, then arrive
+    auto issue_lo = [&](int ri, int k, int n, float thr2) {
+        const RowCtx &rc = ictx[ri % 3];
+        const int32_t *ids = ids_of(ri);
+        uint8_t *st = ring + (n % spw) * G::STAGE;
+        uint64_t *fb = &full[n % spw];
+        uint32_t mask = 0;
+        if (BITS == 4)
+            mask = all_hot ? 0xFFFFFFFFu : __ballot_sync(0xFFFFFFFFu, scores_of(ri)[k * 32 + lane] >= thr2);
+        const int g = (int)crank + (warp + k * kWarps) * (int)C;
+        if (a.s_bitmap && lane == 0)
+            a.s_bitmap[(int64_t)rc.row * a.bitmap_words + g] = mask;
+        const int64_t b0 = ids[2 * k], b1 = ids[2 * k + 1];
+        const bool full_lo = BITS == 4 && mask == 0xFFFFFFFFu;
+        if (lane == 0) {
+            const uint32_t lo_bytes = full_lo ? 2 * G::LOB : (uint32_t)__popc(mask) * G::ROWV;
+            mbar_arrive_expect_tx(fb, lo_bytes);
+            if (full_lo) {
+                bulk_g2s(st + 2 * G::VB, a.lo + (b0 * a.H + rc.h) * G::LOB, G::LOB, fb);
+                bulk_g2s(st + 2 * G::VB + G::LOB, a.lo + (b1 * a.H + rc.h) * G::LOB, G::LOB, fb);
+            }
+        }
+        __syncwarp();
+        if (BITS == 4 && !full_lo && ((mask >> lane) & 1u)) {
+            const int blk = lane >> 4, r = lane & 15;
+            const int64_t bb = blk ? b1 : b0;
+            bulk_g2s(st + 2 * G::VB + blk * G::LOB + r * G::ROWV, a.lo + (bb * a.H + rc.h) * G::LOB + r * G::ROWV,
+                     G::ROWV, fb);
+        }
+        __syncwarp();
+    };
+    auto issue_stage = [&](bool is_v, int ri, int k, int n) {
+        const RowCtx &rc = ictx[ri % 3];
+        const int32_t *ids = ids_of(ri);
+        uint8_t *st = ring + (n % spw) * G::STAGE;
+        uint64_t *fb = &full[n % spw];
+        const int64_t b0 = ids[2 * k], b1 = ids[2 * k + 1];
+        if (!is_v) {
+            if (lane == 0) {
+                mbar_arrive_expect_tx(fb, 2 * G::KB);
+                bulk_g2s(st, a.main + (b0 * a.H + rc.h) * G::HM, G::KB, fb);
+                bulk_g2s(st + G::KB, a.main + (b1 * a.H + rc.h) * G::HM, G::KB, fb);
             }
             __syncwarp();
-        };
-        auto wait_empty = [&](int s) {
-            if (s >= stages)
-                mbar_wait(&sm.empty[s % stages], ((s / stages) - 1) & 1, a.status);
-        };
-        auto issue_k = [&](const RowCtx &rc, int par, int base) {
-            const int32_t *ids = sm.ids + par * 2 * a.cap_groups;
-            for (int i = 0; i < rc.nmy; ++i) {
-                const int s = base + i;
-                wait_empty(s);
-                if (lane == 0) {
-                    uint8_t *st = sm.ring + (s % stages) * G::STAGE;
-                    uint64_t *fb = &sm.full[s % stages];
-                    mbar_arrive_expect_tx(fb, 2 * G::KB);
-                    bulk_g2s(st, a.main + ((int64_t)ids[2 * i] * a.H + rc.h) * G::HM, G::KB, fb);
-                    bulk_g2s(st + G::KB, a.main + ((int64_t)ids[2 * i + 1] * a.H + rc.h) * G::HM, G::KB, fb);
-                }
-                __syncwarp();
-            }
-        };
-        auto issue_v = [&](const RowCtx &rc, int par, int base, float thr2) {
-            const int32_t *ids = sm.ids + par * 2 * a.cap_groups;
-            const float *sc = sm.scores + par * SC;
-            for (int i = 0; i < rc.nmy; ++i) {
-                const int s = base + i;
-                const int g = (int)crank + i * (int)C;
-                uint32_t mask = 0;
-                if (BITS == 4)
-                    mask = all_hot ? 0xFFFFFFFFu : __ballot_sync(0xFFFFFFFFu, sc[i * 32 + lane] >= thr2);
-                if (a.s_bitmap && lane == 0)
-                    a.s_bitmap[(int64_t)rc.row * a.bitmap_words + g] = mask;
-                wait_empty(s);
-                uint8_t *st = sm.ring + (s % stages) * G::STAGE;
-                uint64_t *fb = &sm.full[s % stages];
-                const int64_t b0 = ids[2 * i], b1 = ids[2 * i + 1];
-                const bool full_lo = BITS == 4 && mask == 0xFFFFFFFFu;
-                if (lane == 0) {
-                    const uint32_t lo_bytes = full_lo ? 2 * G::LOB : (uint32_t)__popc(mask) * G::ROWV;
-                    mbar_arrive_expect_tx(fb, 2 * G::VB + lo_bytes);
-                    bulk_g2s(st, a.main + (b0 * a.H + rc.h) * G::HM + G::KB, G::VB, fb);
-                    bulk_g2s(st + G::VB, a.main + (b1 * a.H + rc.h) * G::HM + G::KB, G::VB, fb);
-                    if (full_lo) {
-                        bulk_g2s(st + 2 * G::VB, a.lo + (b0 * a.H + rc.h) * G::LOB, G::LOB, fb);
-                        bulk_g2s(st + 2 * G::VB + G::LOB, a.lo + (b1 * a.H + rc.h) * G::LOB, G::LOB, fb);
+            return;
+        }
+        if (vissued[ri % 3] == 0)
+            vfirst[ri % 3] = n;
+        vissued[ri % 3]++;
+        if (lane == 0) {
+            mbar_expect_tx(fb, 2 * G::VB);
+            bulk_g2s(st, a.main + (b0 * a.H + rc.h) * G::HM + G::KB, G::VB, fb);
+            bulk_g2s(st + G::VB, a.main + (b1 * a.H + rc.h) * G::HM + G::KB, G::VB, fb);
+        }
+        __syncwarp();
+        const float thr2 = ithr[ri % 3];
+        if (!decide || !isnan(thr2)) // the lo part needs the row threshold when tau > 0
+            issue_lo(ri, k, n, thr2);
+    };
+    int released = 0; // rows whose threshold the issuer has received
+    // Issue every stage numbered below `limit` that the sequence allows.  The issuer
+    // state of a row lives in slot (row mod 3), so row r is set up only after row r - 3
+    // has been released (all of its lo copies issued).
+    auto pump = [&](int limit) {
+        while (iss_n < limit && iss_sig < 2 * nrows) {
+            bool is_v;
+            int ri;
+            segment(iss_sig, nrows, is_v, ri);
+            if (iss_k >= owned(ictx[ri % 3], warp)) {
+                const int nsig = iss_sig + 1;
+                if (nsig < 2 * nrows) {
+                    bool nv;
+                    int nri;
+                    segment(nsig, nrows, nv, nri);
+                    if (!nv) {
+                        if (nri - 3 >= released)
+                            break;
+                        setup_row(nri);
                     }
                 }
-                __syncwarp();
-                if (BITS == 4 && !full_lo && ((mask >> lane) & 1u)) {
-                    const int blk = lane >> 4, r = lane & 15;
-                    const int64_t bb = blk ? b1 : b0;
-                    bulk_g2s(st + 2 * G::VB + blk * G::LOB + r * G::ROWV,
-                             a.lo + (bb * a.H + rc.h) * G::LOB + r * G::ROWV, G::ROWV, fb);
-                }
-                __syncwarp();
+                iss_sig = nsig;
+                iss_k = 0;
+                continue;
             }
-        };
+            issue_stage(is_v, ri, iss_k, iss_n);
+            ++iss_k;
+            ++iss_n;
+        }
+    };
+    // the threshold of row ri is known: finish the V stages issued without their lo part
+    auto release_row = [&](int ri, float thr2) {
+        ithr[ri % 3] = thr2;
+        if (decide)
+            for (int k = 0; k < vissued[ri % 3]; ++k)
+                issue_lo(ri, k, vfirst[ri % 3] + k, thr2);
+        released = ri + 1;
+    };
 
-        int pos = 0;
-        RowCtx prev{};
-        if (nrows > 0) {
-            prev = row_ctx(a, cid, crank, C);
-            load_ids(prev, 0);
-            issue_k(prev, 0, pos);
-            pos += prev.nmy;
-        }
-        cluster_arrive(); // row 0
-        for (int i = 1; i < nrows; ++i) {
-            const RowCtx cur = row_ctx(a, cid + i * ncl, crank, C);
-            load_ids(cur, i & 1);
-            issue_k(cur, i & 1, pos);
-            pos += cur.nmy;
-            cluster_wait(); // row i - 1
-            float m2, l2;
-            cluster_row_stats(sm.stat + ((i - 1) % 3) * kConsumerWarps * 2, C, m2, l2);
-            issue_v(prev, (i - 1) & 1, pos, row_threshold(a, m2, l2, decide));
-            pos += prev.nmy;
-            prev = cur;
-            cluster_arrive(); // row i
-        }
-        cluster_wait(); // last row
-        if (nrows > 0) {
-            float m2, l2;
-            cluster_row_stats(sm.stat + ((nrows - 1) % 3) * kConsumerWarps * 2, C, m2, l2);
-            issue_v(prev, (nrows - 1) & 1, pos, row_threshold(a, m2, l2, decide));
-        }
-        cluster_arrive(); // partials of the last row
-        cluster_wait();
-        cluster_arrive(); // remote reads done
-        cluster_wait();
-        return;
-    }
-
-    // ---------------------------------------------------------------- consumers
+    // ---------------------------------------------------------------- compute
     float *aw = sm.aw + warp * D;
     float *wv = sm.wv + warp * 32;
     int kslot[D / 32];
@@ -449,32 +480,39 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
         kpow[k] = __int_as_float((24 - pos + 127) << 23);
     }
     const float vscale = 6.490371073168535e32f; // 2^(149 - kVScaleExp) = 2^109
+    int prc_n = 0;
+    bool timed_out = false; // after one bounded wait gives up, later waits are skipped
+    auto wait_stage = [&](int n) {
+        if (!timed_out)
+            timed_out = !mbar_wait(&full[n % spw], (n / spw) & 1, a.status);
+    };
 
-    // K pass of one row: scores into the row's buffer, per-warp (max, sum) into stat.
-    auto consume_k = [&](const RowCtx &rc, int idx, int base) {
-        const int par = idx & 1;
-        float *sc = sm.scores + par * SC;
+    // K pass of the warp's groups of row ri; per-warp (max, sum) into stat.
+    auto consume_k = [&](int ri) {
+        const RowCtx rc = row_ctx(a, cid + ri * ncl, crank, C, warp == 0 && lane == 0);
+        float *sc = scores_of(ri);
         const DT *qrow = reinterpret_cast<const DT *>(a.q) + (int64_t)rc.row * D;
         float qreg[D / 32];
 #pragma unroll
         for (int k = 0; k < D / 32; ++k)
             qreg[k] = to_f32(qrow[lane + 32 * k]) * a.qscale;
         float mx = -INFINITY;
-        for (int i = first_owned(base, warp); i < rc.nmy; i += kConsumerWarps) {
-            const int s = base + i;
-            const int slot = s % stages;
-            mbar_wait(&sm.full[slot], (s / stages) & 1, a.status);
-            const uint8_t *st = sm.ring + slot * G::STAGE;
+        const int nown = owned(rc, warp);
+        for (int k = 0; k < nown; ++k) {
+            const int n = prc_n++;
+            pump(n + spw);
+            wait_stage(n);
+            const uint8_t *st = ring + (n % spw) * G::STAGE;
             const __half *ksc = reinterpret_cast<const __half *>(st + G::KCODES);        // even block: scales
             const __half *kzp = reinterpret_cast<const __half *>(st + G::KB + G::KCODES); // odd block: zeros
             float av[D / 32];
             float zs = 0.f, amax = 0.f;
 #pragma unroll
-            for (int k = 0; k < D / 32; ++k) {
-                const int c = lane + 32 * k;
-                av[k] = qreg[k] * __half2float(ksc[c]);
-                zs = fmaf(qreg[k], __half2float(kzp[c]), zs);
-                amax = fmaxf(amax, fabsf(av[k]));
+            for (int c4 = 0; c4 < D / 32; ++c4) {
+                const int c = lane + 32 * c4;
+                av[c4] = qreg[c4] * __half2float(ksc[c]);
+                zs = fmaf(qreg[c4], __half2float(kzp[c]), zs);
+                amax = fmaxf(amax, fabsf(av[c4]));
             }
             zs = warp_sum(zs);
             amax = warp_max(amax);
@@ -485,14 +523,14 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
             if (E >= -25 && E <= 100 && abits >= 0x00800000u) { // warp-uniform fast path
                 const float f = __int_as_float((102 - E + 127) << 23); // 2^(102 - E)
 #pragma unroll
-                for (int k = 0; k < D / 32; ++k)
-                    aw[kslot[k]] = (av[k] * f) * kpow[k];
+                for (int c4 = 0; c4 < D / 32; ++c4)
+                    aw[kslot[c4]] = (av[c4] * f) * kpow[c4];
             } else {
 #pragma unroll
-                for (int k = 0; k < D / 32; ++k) {
+                for (int c4 = 0; c4 < D / 32; ++c4) {
                     int slot_c, pos;
-                    key_slot<BITS>(lane + 32 * k, slot_c, pos);
-                    aw[slot_c] = mul_pow2(av[k], 126 - E - pos);
+                    key_slot<BITS>(lane + 32 * c4, slot_c, pos);
+                    aw[slot_c] = mul_pow2(av[c4], 126 - E - pos);
                 }
             }
             __syncwarp();
@@ -516,47 +554,46 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
             }
             const float accs = acc.x + acc.y;
             const float s2 = (E <= 100 ? accs * __int_as_float((E + 150) << 23) : mul_pow2(accs, E + 23)) + zs;
-            sc[i * 32 + lane] = s2;
+            sc[k * 32 + lane] = s2;
             mx = fmaxf(mx, s2);
             __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&sm.empty[slot]);
         }
-        if (rc.tail_cta && warp == kConsumerWarps - 1) { // tail keys, exact; lane = tail token
+        float *tsc = sm.tscores + (ri & 1) * 32;
+        if (rc.tail_cta && warp == kWarps - 1) { // tail keys, exact; lane = tail token
             const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)rc.b * 2 * a.H + rc.h) * 32 * D;
             float s2 = 0.f;
 #pragma unroll
-            for (int k = 0; k < D / 32; ++k)
+            for (int c4 = 0; c4 < D / 32; ++c4)
                 for (int c = 0; c < 32; ++c) {
-                    const float qc = __shfl_sync(0xFFFFFFFFu, qreg[k], c);
+                    const float qc = __shfl_sync(0xFFFFFFFFu, qreg[c4], c);
                     if (lane < rc.tail)
-                        s2 = fmaf(qc, to_f32(kt[(int64_t)lane * D + 32 * k + c]), s2);
+                        s2 = fmaf(qc, to_f32(kt[(int64_t)lane * D + 32 * c4 + c]), s2);
                 }
             if (lane < rc.tail) {
-                sc[a.cap_groups * 32 + lane] = s2;
+                tsc[lane] = s2;
                 mx = fmaxf(mx, s2);
             }
         }
         mx = warp_max(mx);
         float ls = 0.f;
         if (a.tau_mode == LOOPKV_TAU_ABS_PROB && mx != -INFINITY) {
-            for (int i = first_owned(base, warp); i < rc.nmy; i += kConsumerWarps)
-                ls += exp2f(sc[i * 32 + lane] - mx);
-            if (rc.tail_cta && warp == kConsumerWarps - 1 && lane < rc.tail)
-                ls += exp2f(sc[a.cap_groups * 32 + lane] - mx);
+            for (int k = 0; k < nown; ++k)
+                ls += exp2f(sc[k * 32 + lane] - mx);
+            if (rc.tail_cta && warp == kWarps - 1 && lane < rc.tail)
+                ls += exp2f(tsc[lane] - mx);
             ls = warp_sum(ls);
         }
         if (lane == 0) {
-            float *st = sm.stat + (idx % 3) * kConsumerWarps * 2;
-            st[2 * warp] = mx;
-            st[2 * warp + 1] = ls;
+            float *stw = sm.stat + (ri % 3) * kWarps * 2;
+            stw[2 * warp] = mx;
+            stw[2 * warp + 1] = ls;
         }
     };
 
-    // V pass of one row, then the CTA partial (o, l) into part[row parity].
-    auto consume_v = [&](const RowCtx &rc, int idx, int base, float m2, float thr2) {
-        const int par = idx & 1;
-        const float *sc = sm.scores + par * SC;
+    // V pass of the warp's groups of row ri, then the CTA partial (o, l) into part.
+    auto consume_v = [&](int ri, float m2, float thr2) {
+        const RowCtx rc = row_ctx(a, cid + ri * ncl, crank, C, false);
+        const float *sc = scores_of(ri);
         const int cg = lane % G::NCG, ts = lane / G::NCG;
         float2 acc[2][2][4];
 #pragma unroll
@@ -567,18 +604,19 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
                 for (int n = 0; n < 4; ++n)
                     acc[k][e][n] = make_float2(0.f, 0.f);
         float zacc = 0.f, lsum = 0.f;
-        for (int i = first_owned(base, warp); i < rc.nmy; i += kConsumerWarps) {
-            const int s = base + i;
-            const int slot = s % stages;
-            const float s2l = sc[i * 32 + lane];
+        const int nown = owned(rc, warp);
+        for (int k = 0; k < nown; ++k) {
+            const int n = prc_n++;
+            pump(n + spw);
+            const float s2l = sc[k * 32 + lane];
             const float wl = exp2f(s2l - m2);
             const uint32_t hotmask =
                 all_hot ? 0xFFFFFFFFu : (BITS == 4 ? __ballot_sync(0xFFFFFFFFu, s2l >= thr2) : 0u);
             lsum += wl;
             wv[lane] = wl;
             __syncwarp();
-            mbar_wait(&sm.full[slot], (s / stages) & 1, a.status);
-            const uint8_t *st = sm.ring + slot * G::STAGE;
+            wait_stage(n);
+            const uint8_t *st = ring + (n % spw) * G::STAGE;
 #pragma unroll
             for (int u = 0; u < 32 / G::TPI; ++u) {
                 const int t = u * G::TPI + ts;
@@ -605,8 +643,6 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
                 value_word(hw.y, lw.y, Wp, acc[1]);
             }
             __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&sm.empty[slot]);
         }
         // reduce over the token slots of the warp (lanes with the same cg)
 #pragma unroll
@@ -639,36 +675,38 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
         if (lane == 0)
             red[D] = lsum;
         __syncwarp();
-        if (rc.tail_cta && warp == kConsumerWarps - 1) { // tail values, exact
+        if (rc.tail_cta && warp == kWarps - 1) { // tail values, exact
+            const float *tsc = sm.tscores + (ri & 1) * 32;
             const DT *vt0 = reinterpret_cast<const DT *>(a.tail) + ((int64_t)(rc.b * 2 + 1) * a.H + rc.h) * 32 * D;
             float tl = 0.f;
             for (int t = 0; t < rc.tail; ++t) {
-                const float w = exp2f(sc[a.cap_groups * 32 + t] - m2);
+                const float w = exp2f(tsc[t] - m2);
                 tl += w;
                 const DT *vt = vt0 + (int64_t)t * D;
 #pragma unroll
-                for (int k = 0; k < D / 32; ++k)
-                    red[lane + 32 * k] = fmaf(w, to_f32(vt[lane + 32 * k]), red[lane + 32 * k]);
+                for (int c4 = 0; c4 < D / 32; ++c4)
+                    red[lane + 32 * c4] = fmaf(w, to_f32(vt[lane + 32 * c4]), red[lane + 32 * c4]);
             }
             __syncwarp();
             if (lane == 0)
                 red[D] += tl;
         }
-        named_sync(1, kConsumerWarps * 32);
-        float *part = sm.part + par * (D + 1);
-        for (int c = threadIdx.x; c <= D; c += kConsumerWarps * 32) {
+        named_sync(1, kThreads);
+        float *part = sm.part + (ri & 1) * (D + 1);
+        for (int c = threadIdx.x; c <= D; c += kThreads) {
             float sum = 0.f;
 #pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w)
+            for (int w = 0; w < kWarps; ++w)
                 sum += sm.red[w * (D + 1) + c];
             part[c] = sum;
         }
     };
 
-    // CTA `crank` writes channels [crank*D/C, (crank+1)*D/C) of a row, summing the
+    // CTA `crank` writes channels [crank*D/C, (crank+1)*D/C) of row ri, summing the
     // partials of every CTA of the cluster.
-    auto merge = [&](const RowCtx &rc, int idx, float m2) {
-        const float *part = sm.part + (idx & 1) * (D + 1);
+    auto merge = [&](int ri, float m2) {
+        const int row = cid + ri * ncl;
+        const float *part = sm.part + (ri & 1) * (D + 1);
         const int per = D / (int)C;
         if ((int)threadIdx.x < per) {
             const int c = (int)crank * per + (int)threadIdx.x;
@@ -682,55 +720,51 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
                 out = o / l;
             else if (c == 0)
                 atomicOr(a.status, LOOPKV_DEV_EMPTY_ROW);
-            a.out[(int64_t)rc.row * D + c] = out;
+            a.out[(int64_t)row * D + c] = out;
             if (c == 0) {
                 if (a.row_max)
-                    a.row_max[rc.row] = m2 * 0.6931471805599453f;
+                    a.row_max[row] = m2 * 0.6931471805599453f;
                 if (a.row_sum)
-                    a.row_sum[rc.row] = l;
+                    a.row_sum[row] = l;
             }
         }
     };
 
-    int pos = 0;
-    RowCtx prev{}, prev2{};
     float m_prev = 0.f, m_prev2 = 0.f;
     if (nrows > 0) {
-        prev = row_ctx(a, cid, crank, C);
-        consume_k(prev, 0, pos);
-        pos += prev.nmy;
+        setup_row(0);
+        pump(spw);
+        consume_k(0);
     }
     cluster_arrive(); // row 0
     for (int i = 1; i < nrows; ++i) {
-        named_sync(1, kConsumerWarps * 32); // every consumer warp is done with row i - 2
-        const RowCtx cur = row_ctx(a, cid + i * ncl, crank, C);
-        consume_k(cur, i, pos);
-        pos += cur.nmy;
+        consume_k(i);
         cluster_wait(); // row i - 1: maxima of row i - 1, partials of row i - 2
         if (i >= 2)
-            merge(prev2, i - 2, m_prev2);
+            merge(i - 2, m_prev2);
         float m2, l2;
-        cluster_row_stats(sm.stat + ((i - 1) % 3) * kConsumerWarps * 2, C, m2, l2);
-        consume_v(prev, i - 1, pos, m2, row_threshold(a, m2, l2, decide));
-        pos += prev.nmy;
-        prev2 = prev;
+        cluster_row_stats(sm.stat + ((i - 1) % 3) * kWarps * 2, C, m2, l2);
+        const float thr2 = row_threshold(a, m2, l2, decide);
+        release_row(i - 1, thr2);
+        consume_v(i - 1, m2, thr2);
         m_prev2 = m2;
-        prev = cur;
         cluster_arrive(); // row i
     }
     cluster_wait(); // last row
     if (nrows >= 2)
-        merge(prev2, nrows - 2, m_prev2);
+        merge(nrows - 2, m_prev2);
     if (nrows > 0) {
         float m2, l2;
-        cluster_row_stats(sm.stat + ((nrows - 1) % 3) * kConsumerWarps * 2, C, m2, l2);
-        consume_v(prev, nrows - 1, pos, m2, row_threshold(a, m2, l2, decide));
+        cluster_row_stats(sm.stat + ((nrows - 1) % 3) * kWarps * 2, C, m2, l2);
+        const float thr2 = row_threshold(a, m2, l2, decide);
+        release_row(nrows - 1, thr2);
+        consume_v(nrows - 1, m2, thr2);
         m_prev = m2;
     }
     cluster_arrive(); // partials of the last row
     cluster_wait();
     if (nrows > 0)
-        merge(prev, nrows - 1, m_prev);
+        merge(nrows - 1, m_prev);
     cluster_arrive(); // remote reads done
     cluster_wait();
 }
@@ -807,38 +841,39 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
     const char *env_c = getenv("LOOPKV_DECODE_CLUSTER");
     const char *env_s = getenv("LOOPKV_DECODE_STAGES");
     const char *env_o = getenv("LOOPKV_DECODE_CTAS_PER_SM");
-    const int want_ctas = env_o ? atoi(env_o) : 4;
+    const int want_ctas = env_o ? atoi(env_o) : kMinCtasPerSm;
     for (int C = 1; C <= 16; C *= 2) {
         if (env_c && atoi(env_c) != C)
             continue;
         if (D / C < 4)
             continue;
         const int cap = (max_groups + C - 1) / C;
-        // stages: fill the shared memory of `want_ctas` CTAs per SM (1 KB reserved per CTA)
+        const int capw = (cap + kWarps - 1) / kWarps;
+        // slots per warp: fill the shared memory of `want_ctas` CTAs per SM (1 KB reserved per CTA)
         const int budget = smem_per_sm / want_ctas - 1024;
-        int stages = (budget - smem_fixed<BITS, D>(cap)) / (G::STAGE + 16);
-        if (stages > 32)
-            stages = 32;
+        int spw = (budget - smem_bytes<BITS, D>(0, capw)) / (kWarps * (G::STAGE + 8));
+        if (spw > 8)
+            spw = 8;
         if (env_s)
-            stages = atoi(env_s);
-        if (stages < 4)
-            stages = 4;
-        const int smem = smem_bytes<BITS, D>(stages, cap);
-        if (smem > 227 * 1024 || !layout_ok<BITS, D>(stages, cap))
+            spw = atoi(env_s);
+        if (spw < 2)
+            spw = 2;
+        const int smem = smem_bytes<BITS, D>(spw, capw);
+        if (smem > 227 * 1024 || !layout_ok<BITS, D>(spw, capw))
             continue;
         int ncl = max_active_clusters<BITS, D, DT>(C, smem);
         if (ncl <= 0)
             continue;
         if (ncl > rows)
             ncl = rows;
-        // balance: each cluster takes ceil(rows / ncl) rows; parallel slack penalised
+        // balance: each cluster takes ceil(rows / ncl) rows; too few CTAs per SM penalised
         const double rounds = (double)((rows + ncl - 1) / ncl);
         const double eff = ((double)rows / ncl) / rounds * std::min(1.0, (double)(ncl * C) / (3.0 * sm_count));
         if (eff > best_eff + 1e-9) {
             best_eff = eff;
             best.cluster = C;
             best.clusters = ncl;
-            best.stages = stages;
+            best.stages = spw;
             best.smem = smem;
             best.threads = kThreads;
             best.cap = cap;
