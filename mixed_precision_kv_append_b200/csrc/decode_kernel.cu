@@ -156,15 +156,19 @@ struct Smem {
     float *aw;         // [kWarps][D] key factors
     float *stat;       // [3][kWarps][2] per-warp (max, sum exp(s - max)), by row index mod 3
     float *part;       // [2][D + 1] CTA partial o and l of a row, by row parity
-    float *wv;         // [kWarps][32] weights of the group a warp reads
+    float *wv;         // [kWarps][32][4] per token and 32-channel group: w * s * 2^109
     float *red;        // [kWarps][D + 1]
     int32_t *ids;      // [3][kWarps][2 * capw] block ids of a warp's groups, by row index mod 3
+    int32_t *irow;     // [3][kWarps][8] issuer state of a row, by row index mod 3
 };
+
+// Issuer state of one row (int fields of Smem::irow).
+enum { IR_ROW = 0, IR_H, IR_OWN, IR_VFIRST, IR_VISSUED, IR_THR, IR_N = 8 };
 
 // Byte offsets of the shared-memory regions; every region starts on a 16-byte boundary
 // (the key factors and the stage data are read with 16-byte vector loads).
 struct SmemLayout {
-    int full, scores, tscores, aw, stat, part, wv, red, ids, total;
+    int full, scores, tscores, aw, stat, part, wv, red, ids, irow, total;
 };
 
 __host__ __device__ constexpr int align16(int x) { return (x + 15) & ~15; }
@@ -186,11 +190,13 @@ template <int BITS, int D> __host__ __device__ constexpr SmemLayout smem_layout(
     L.part = o;
     o = align16(o + 2 * (D + 1) * 4);
     L.wv = o;
-    o = align16(o + kWarps * 32 * 4);
+    o = align16(o + kWarps * 32 * 4 * 4);
     L.red = o;
     o = align16(o + kWarps * (D + 1) * 4);
     L.ids = o;
     o = align16(o + 3 * kWarps * 2 * capw * 4);
+    L.irow = o;
+    o = align16(o + 3 * kWarps * IR_N * 4);
     L.total = o;
     return L;
 }
@@ -214,6 +220,7 @@ template <int BITS, int D> __device__ Smem carve(uint8_t *base, int spw, int cap
     s.wv = reinterpret_cast<float *>(base + L.wv);
     s.red = reinterpret_cast<float *>(base + L.red);
     s.ids = reinterpret_cast<int32_t *>(base + L.ids);
+    s.irow = reinterpret_cast<int32_t *>(base + L.irow);
     return s;
 }
 
@@ -221,14 +228,14 @@ template <int BITS, int D> __device__ Smem carve(uint8_t *base, int spw, int cap
 template <int BITS, int D> bool layout_ok(int spw, int capw)
 {
     const SmemLayout L = smem_layout<BITS, D>(spw, capw);
-    const int offs[] = {L.full, L.scores, L.tscores, L.aw, L.stat, L.part, L.wv, L.red, L.ids};
+    const int offs[] = {L.full, L.scores, L.tscores, L.aw, L.stat, L.part, L.wv, L.red, L.ids, L.irow};
     int prev = kWarps * spw * Geo<BITS, D>::STAGE;
     for (int o : offs) {
         if (o % 16 || o < prev)
             return false;
         prev = o;
     }
-    return (Geo<BITS, D>::STAGE % 128) == 0 && L.total >= prev;
+    return (Geo<BITS, D>::STAGE % 128) == 0 && L.total >= prev && (spw & (spw - 1)) == 0;
 }
 
 // One (request, head) row as seen by one CTA of its cluster.
@@ -244,7 +251,7 @@ __device__ __forceinline__ RowCtx row_ctx(const DecodeArgs &a, int row, uint32_t
     RowCtx r;
     r.row = row;
     r.b = row / a.H;
-    r.h = row % a.H;
+    r.h = row - r.b * a.H;
     int hist = a.hist_len[r.b], tail = a.tail_len[r.b];
     bool bad = false;
     if (hist < 0 || hist > a.max_blocks * 16 || (hist & 31)) {
@@ -270,10 +277,7 @@ __device__ __forceinline__ RowCtx row_ctx(const DecodeArgs &a, int row, uint32_t
 }
 
 // Groups of a row owned by warp w of the CTA: local groups w, w + kWarps, ...
-__device__ __forceinline__ int owned(const RowCtx &rc, int w)
-{
-    return rc.nmy > w ? (rc.nmy - w + kWarps - 1) / kWarps : 0;
-}
+__device__ __forceinline__ int owned(int nmy, int w) { return nmy > w ? (nmy - w + kWarps - 1) / kWarps : 0; }
 
 // Row max m (log2 units) and, for the normalised rule, l = sum_t 2^(s_t - m), from the
 // per-warp pairs of every CTA of the cluster (fixed order: every caller gets the same).
@@ -312,18 +316,19 @@ __device__ __forceinline__ void segment(int sig, int nrows, bool &is_v, int &ri)
         is_v = true;
         ri = nrows - 1;
     } else {
-        const int i = (sig + 1) / 2;
+        const int i = (sig + 1) >> 1;
         is_v = !(sig & 1);
         ri = (sig & 1) ? i : i - 1;
     }
 }
 
 template <int BITS, int D, typename DT>
-__global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const DecodeArgs a, const int spw)
+__global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const DecodeArgs a, const int spw_log2)
 {
     using G = Geo<BITS, D>;
     extern __shared__ __align__(128) uint8_t smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int spw = 1 << spw_log2, smask = spw - 1;
     const uint32_t crank = cluster_ctarank(), C = cluster_nctarank();
     const int cid = blockIdx.x / (int)C, ncl = gridDim.x / (int)C;
     const int nrows = cid < a.rows ? (a.rows - 1 - cid) / ncl + 1 : 0; // rows cid, cid + ncl, ...
@@ -342,21 +347,19 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
     uint64_t *full = sm.full + warp * spw;
     auto scores_of = [&](int ri) { return sm.scores + ((ri & 1) * kWarps + warp) * capw * 32; };
     auto ids_of = [&](int ri) { return sm.ids + ((ri % 3) * kWarps + warp) * 2 * capw; };
+    auto irow_of = [&](int ri) { return sm.irow + ((ri % 3) * kWarps + warp) * IR_N; };
 
     // ---------------------------------------------------------------- issuing
     // A warp issues the bulk copies of its own stages, `spw` stages ahead of its compute.
-    RowCtx ictx[3];   // rows known to the issuer, by row index mod 3
-    float ithr[3];    // thresholds known to the issuer
-    int vfirst[3];    // warp-local stage number of the first V stage of a row
-    int vissued[3];   // V stages of a row issued so far (their meta + hi parts)
     int iss_sig = 0, iss_k = 0, iss_n = 0;
+    int seg_len = 0, seg_ri = 0;   // current segment: own stages and row index
+    bool seg_v = false;
+    int released = 0;              // rows whose threshold the issuer has received
 
     auto setup_row = [&](int ri) {
-        RowCtx rc = row_ctx(a, cid + ri * ncl, crank, C, false);
-        ictx[ri % 3] = rc;
-        ithr[ri % 3] = NAN;
-        vissued[ri % 3] = 0;
-        const int n = owned(rc, warp);
+        const RowCtx rc = row_ctx(a, cid + ri * ncl, crank, C, false);
+        const int n = owned(rc.nmy, warp);
+        int32_t *st = irow_of(ri);
         const int32_t *bt = a.block_table + (int64_t)rc.b * a.max_blocks;
         int32_t *ids = ids_of(ri);
         for (int k = lane; k < 2 * n; k += 32) {
@@ -368,115 +371,136 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
             }
             ids[k] = id;
         }
+        if (lane == 0) {
+            st[IR_ROW] = rc.row;
+            st[IR_H] = rc.h;
+            st[IR_OWN] = n;
+            st[IR_VFIRST] = 0;
+            st[IR_VISSUED] = 0;
+            st[IR_THR] = __float_as_int(NAN);
+        }
         __syncwarp();
+    };
+    auto load_segment = [&]() {
+        segment(iss_sig, nrows, seg_v, seg_ri);
+        seg_len = irow_of(seg_ri)[IR_OWN];
     };
     // lo planes (4-bit sources) of the hot tokens of V stage k of row ri, then arrive
     auto issue_lo = [&](int ri, int k, int n, float thr2) {
-        const RowCtx &rc = ictx[ri % 3];
+        const int32_t *st_row = irow_of(ri);
+        const int h = st_row[IR_H];
         const int32_t *ids = ids_of(ri);
-        uint8_t *st = ring + (n % spw) * G::STAGE;
-        uint64_t *fb = &full[n % spw];
+        uint8_t *st = ring + (n & smask) * G::STAGE;
+        uint64_t *fb = &full[n & smask];
         uint32_t mask = 0;
         if (BITS == 4)
             mask = all_hot ? 0xFFFFFFFFu : __ballot_sync(0xFFFFFFFFu, scores_of(ri)[k * 32 + lane] >= thr2);
-        const int g = (int)crank + (warp + k * kWarps) * (int)C;
-        if (a.s_bitmap && lane == 0)
-            a.s_bitmap[(int64_t)rc.row * a.bitmap_words + g] = mask;
+        if (a.s_bitmap && lane == 0) {
+            const int g = (int)crank + (warp + k * kWarps) * (int)C;
+            a.s_bitmap[(int64_t)st_row[IR_ROW] * a.bitmap_words + g] = mask;
+        }
         const int64_t b0 = ids[2 * k], b1 = ids[2 * k + 1];
         const bool full_lo = BITS == 4 && mask == 0xFFFFFFFFu;
         if (lane == 0) {
             const uint32_t lo_bytes = full_lo ? 2 * G::LOB : (uint32_t)__popc(mask) * G::ROWV;
             mbar_arrive_expect_tx(fb, lo_bytes);
             if (full_lo) {
-                bulk_g2s(st + 2 * G::VB, a.lo + (b0 * a.H + rc.h) * G::LOB, G::LOB, fb);
-                bulk_g2s(st + 2 * G::VB + G::LOB, a.lo + (b1 * a.H + rc.h) * G::LOB, G::LOB, fb);
+                bulk_g2s(st + 2 * G::VB, a.lo + (b0 * a.H + h) * G::LOB, G::LOB, fb);
+                bulk_g2s(st + 2 * G::VB + G::LOB, a.lo + (b1 * a.H + h) * G::LOB, G::LOB, fb);
             }
         }
         __syncwarp();
         if (BITS == 4 && !full_lo && ((mask >> lane) & 1u)) {
             const int blk = lane >> 4, r = lane & 15;
             const int64_t bb = blk ? b1 : b0;
-            bulk_g2s(st + 2 * G::VB + blk * G::LOB + r * G::ROWV, a.lo + (bb * a.H + rc.h) * G::LOB + r * G::ROWV,
+            bulk_g2s(st + 2 * G::VB + blk * G::LOB + r * G::ROWV, a.lo + (bb * a.H + h) * G::LOB + r * G::ROWV,
                      G::ROWV, fb);
         }
         __syncwarp();
     };
-    auto issue_stage = [&](bool is_v, int ri, int k, int n) {
-        const RowCtx &rc = ictx[ri % 3];
+    auto issue_stage = [&](int n) {
+        const int k = iss_k, ri = seg_ri;
+        int32_t *st_row = irow_of(ri);
+        const int h = st_row[IR_H];
         const int32_t *ids = ids_of(ri);
-        uint8_t *st = ring + (n % spw) * G::STAGE;
-        uint64_t *fb = &full[n % spw];
+        uint8_t *st = ring + (n & smask) * G::STAGE;
+        uint64_t *fb = &full[n & smask];
         const int64_t b0 = ids[2 * k], b1 = ids[2 * k + 1];
-        if (!is_v) {
+        if (!seg_v) {
             if (lane == 0) {
                 mbar_arrive_expect_tx(fb, 2 * G::KB);
-                bulk_g2s(st, a.main + (b0 * a.H + rc.h) * G::HM, G::KB, fb);
-                bulk_g2s(st + G::KB, a.main + (b1 * a.H + rc.h) * G::HM, G::KB, fb);
+                bulk_g2s(st, a.main + (b0 * a.H + h) * G::HM, G::KB, fb);
+                bulk_g2s(st + G::KB, a.main + (b1 * a.H + h) * G::HM, G::KB, fb);
             }
             __syncwarp();
             return;
         }
-        if (vissued[ri % 3] == 0)
-            vfirst[ri % 3] = n;
-        vissued[ri % 3]++;
         if (lane == 0) {
+            if (k == 0)
+                st_row[IR_VFIRST] = n;
+            st_row[IR_VISSUED] = k + 1;
             mbar_expect_tx(fb, 2 * G::VB);
-            bulk_g2s(st, a.main + (b0 * a.H + rc.h) * G::HM + G::KB, G::VB, fb);
-            bulk_g2s(st + G::VB, a.main + (b1 * a.H + rc.h) * G::HM + G::KB, G::VB, fb);
+            bulk_g2s(st, a.main + (b0 * a.H + h) * G::HM + G::KB, G::VB, fb);
+            bulk_g2s(st + G::VB, a.main + (b1 * a.H + h) * G::HM + G::KB, G::VB, fb);
         }
         __syncwarp();
-        const float thr2 = ithr[ri % 3];
+        const float thr2 = __int_as_float(st_row[IR_THR]);
         if (!decide || !isnan(thr2)) // the lo part needs the row threshold when tau > 0
             issue_lo(ri, k, n, thr2);
     };
-    int released = 0; // rows whose threshold the issuer has received
     // Issue every stage numbered below `limit` that the sequence allows.  The issuer
     // state of a row lives in slot (row mod 3), so row r is set up only after row r - 3
     // has been released (all of its lo copies issued).
     auto pump = [&](int limit) {
         while (iss_n < limit && iss_sig < 2 * nrows) {
-            bool is_v;
-            int ri;
-            segment(iss_sig, nrows, is_v, ri);
-            if (iss_k >= owned(ictx[ri % 3], warp)) {
-                const int nsig = iss_sig + 1;
-                if (nsig < 2 * nrows) {
-                    bool nv;
-                    int nri;
-                    segment(nsig, nrows, nv, nri);
-                    if (!nv) {
-                        if (nri - 3 >= released)
-                            break;
-                        setup_row(nri);
-                    }
-                }
-                iss_sig = nsig;
-                iss_k = 0;
+            if (iss_k < seg_len) {
+                issue_stage(iss_n);
+                ++iss_k;
+                ++iss_n;
                 continue;
             }
-            issue_stage(is_v, ri, iss_k, iss_n);
-            ++iss_k;
-            ++iss_n;
+            const int nsig = iss_sig + 1;
+            if (nsig < 2 * nrows) {
+                bool nv;
+                int nri;
+                segment(nsig, nrows, nv, nri);
+                if (!nv) {
+                    if (nri - 3 >= released)
+                        break;
+                    setup_row(nri);
+                }
+            }
+            iss_sig = nsig;
+            iss_k = 0;
+            if (iss_sig < 2 * nrows)
+                load_segment();
         }
     };
     // the threshold of row ri is known: finish the V stages issued without their lo part
     auto release_row = [&](int ri, float thr2) {
-        ithr[ri % 3] = thr2;
+        int32_t *st_row = irow_of(ri);
+        const int vfirst = st_row[IR_VFIRST], vissued = st_row[IR_VISSUED];
+        __syncwarp();
+        if (lane == 0)
+            st_row[IR_THR] = __float_as_int(thr2);
+        __syncwarp();
         if (decide)
-            for (int k = 0; k < vissued[ri % 3]; ++k)
-                issue_lo(ri, k, vfirst[ri % 3] + k, thr2);
+            for (int k = 0; k < vissued; ++k)
+                issue_lo(ri, k, vfirst + k, thr2);
         released = ri + 1;
     };
 
     // ---------------------------------------------------------------- compute
     float *aw = sm.aw + warp * D;
-    float *wv = sm.wv + warp * 32;
+    float4 *wv4 = reinterpret_cast<float4 *>(sm.wv) + warp * 32;
+    const float *wvf = sm.wv + warp * 128;
+    // a lane owns the channel pairs (2*lane + 64j, 2*lane + 1 + 64j), j < D/64
     int kslot[D / 32];
     float kpow[D / 32];
 #pragma unroll
     for (int k = 0; k < D / 32; ++k) {
         int pos;
-        key_slot<BITS>(lane + 32 * k, kslot[k], pos);
+        key_slot<BITS>(2 * lane + 64 * (k >> 1) + (k & 1), kslot[k], pos);
         kpow[k] = __int_as_float((24 - pos + 127) << 23);
     }
     const float vscale = 6.490371073168535e32f; // 2^(149 - kVScaleExp) = 2^109
@@ -484,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
     bool timed_out = false; // after one bounded wait gives up, later waits are skipped
     auto wait_stage = [&](int n) {
         if (!timed_out)
-            timed_out = !mbar_wait(&full[n % spw], (n / spw) & 1, a.status);
+            timed_out = !mbar_wait(&full[n & smask], (n >> spw_log2) & 1, a.status);
     };
 
     // K pass of the warp's groups of row ri; per-warp (max, sum) into stat.
@@ -495,24 +519,28 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
         float qreg[D / 32];
 #pragma unroll
         for (int k = 0; k < D / 32; ++k)
-            qreg[k] = to_f32(qrow[lane + 32 * k]) * a.qscale;
+            qreg[k] = to_f32(qrow[2 * lane + 64 * (k >> 1) + (k & 1)]) * a.qscale;
         float mx = -INFINITY;
-        const int nown = owned(rc, warp);
+        const int nown = owned(rc.nmy, warp);
         for (int k = 0; k < nown; ++k) {
             const int n = prc_n++;
-            pump(n + spw);
+            if (iss_n < n + spw)
+                pump(n + spw);
             wait_stage(n);
-            const uint8_t *st = ring + (n % spw) * G::STAGE;
-            const __half *ksc = reinterpret_cast<const __half *>(st + G::KCODES);        // even block: scales
-            const __half *kzp = reinterpret_cast<const __half *>(st + G::KB + G::KCODES); // odd block: zeros
+            const uint8_t *st = ring + (n & smask) * G::STAGE;
+            const __half2 *ksc = reinterpret_cast<const __half2 *>(st + G::KCODES);        // even: scales
+            const __half2 *kzp = reinterpret_cast<const __half2 *>(st + G::KB + G::KCODES); // odd: zeros
             float av[D / 32];
             float zs = 0.f, amax = 0.f;
 #pragma unroll
-            for (int c4 = 0; c4 < D / 32; ++c4) {
-                const int c = lane + 32 * c4;
-                av[c4] = qreg[c4] * __half2float(ksc[c]);
-                zs = fmaf(qreg[c4], __half2float(kzp[c]), zs);
-                amax = fmaxf(amax, fabsf(av[c4]));
+            for (int j = 0; j < D / 64; ++j) {
+                const float2 sv = __half22float2(ksc[lane + 32 * j]);
+                const float2 zv = __half22float2(kzp[lane + 32 * j]);
+                av[2 * j] = qreg[2 * j] * sv.x;
+                av[2 * j + 1] = qreg[2 * j + 1] * sv.y;
+                zs = fmaf(qreg[2 * j], zv.x, zs);
+                zs = fmaf(qreg[2 * j + 1], zv.y, zs);
+                amax = fmaxf(amax, fmaxf(fabsf(av[2 * j]), fabsf(av[2 * j + 1])));
             }
             zs = warp_sum(zs);
             amax = warp_max(amax);
@@ -529,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
 #pragma unroll
                 for (int c4 = 0; c4 < D / 32; ++c4) {
                     int slot_c, pos;
-                    key_slot<BITS>(lane + 32 * c4, slot_c, pos);
+                    key_slot<BITS>(2 * lane + 64 * (c4 >> 1) + (c4 & 1), slot_c, pos);
                     aw[slot_c] = mul_pow2(av[c4], 126 - E - pos);
                 }
             }
@@ -564,10 +592,11 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
             float s2 = 0.f;
 #pragma unroll
             for (int c4 = 0; c4 < D / 32; ++c4)
-                for (int c = 0; c < 32; ++c) {
-                    const float qc = __shfl_sync(0xFFFFFFFFu, qreg[c4], c);
+                for (int l = 0; l < 32; ++l) {
+                    const float qc = __shfl_sync(0xFFFFFFFFu, qreg[c4], l);
+                    const int c = 2 * l + 64 * (c4 >> 1) + (c4 & 1);
                     if (lane < rc.tail)
-                        s2 = fmaf(qc, to_f32(kt[(int64_t)lane * D + 32 * c4 + c]), s2);
+                        s2 = fmaf(qc, to_f32(kt[(int64_t)lane * D + c]), s2);
                 }
             if (lane < rc.tail) {
                 tsc[lane] = s2;
@@ -603,42 +632,54 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
 #pragma unroll
                 for (int n = 0; n < 4; ++n)
                     acc[k][e][n] = make_float2(0.f, 0.f);
-        float zacc = 0.f, lsum = 0.f;
-        const int nown = owned(rc, warp);
+        float zl[G::NCG];
+#pragma unroll
+        for (int j = 0; j < G::NCG; ++j)
+            zl[j] = 0.f;
+        float lsum = 0.f;
+        const int nown = owned(rc.nmy, warp);
         for (int k = 0; k < nown; ++k) {
             const int n = prc_n++;
-            pump(n + spw);
+            if (iss_n < n + spw)
+                pump(n + spw);
             const float s2l = sc[k * 32 + lane];
             const float wl = exp2f(s2l - m2);
-            const uint32_t hotmask =
-                all_hot ? 0xFFFFFFFFu : (BITS == 4 ? __ballot_sync(0xFFFFFFFFu, s2l >= thr2) : 0u);
+            const bool hotl = all_hot || (BITS == 4 && s2l >= thr2);
+            const uint32_t hotmask = __ballot_sync(0xFFFFFFFFu, hotl);
             lsum += wl;
-            wv[lane] = wl;
-            __syncwarp();
             wait_stage(n);
-            const uint8_t *st = ring + (n % spw) * G::STAGE;
+            const uint8_t *st = ring + (n & smask) * G::STAGE;
+            {   // token `lane`: fold its value scales and zeros into the weight and a running sum
+                const uint8_t *mrow = st + (lane >> 4) * G::VB + (lane & 15) * G::NCG * 4;
+                float wsc[4];
+#pragma unroll
+                for (int j = 0; j < G::NCG; ++j) {
+                    const float2 m = __half22float2(reinterpret_cast<const __half2 *>(mrow)[j]); // (scale, zero)
+                    if (BITS == 4) {
+                        zl[j] = fmaf(wl, hotl ? m.y : fmaf(1.5f, m.x, m.y), zl[j]);
+                        wsc[j] = wl * m.x * vscale;
+                    } else {
+                        zl[j] = fmaf(wl, m.y, zl[j]);
+                        wsc[j] = wl * m.x * (0.25f * vscale);
+                    }
+                }
+                if (G::NCG == 4)
+                    wv4[lane] = make_float4(wsc[0], wsc[1], wsc[2], wsc[3]);
+                else
+                    reinterpret_cast<float2 *>(wv4)[lane] = make_float2(wsc[0], wsc[1]);
+            }
+            __syncwarp();
 #pragma unroll
             for (int u = 0; u < 32 / G::TPI; ++u) {
                 const int t = u * G::TPI + ts;
-                const float w = wv[t];
+                const float Wp = wvf[t * G::NCG + cg];
                 const bool hot = (hotmask >> t) & 1u;
                 const int blk = t >> 4, r = t & 15;
-                const uint8_t *vb = st + blk * G::VB;
-                const __half2 meta = *reinterpret_cast<const __half2 *>(vb + r * G::NCG * 4 + cg * 4);
-                const float vs = __low2float(meta), vz = __high2float(meta);
-                const uint2 hw = *reinterpret_cast<const uint2 *>(vb + G::VMETA + r * G::ROWV + cg * 8);
+                const uint2 hw =
+                    *reinterpret_cast<const uint2 *>(st + blk * G::VB + G::VMETA + r * G::ROWV + cg * 8);
                 uint2 lw = make_uint2(0u, 0u);
-                float W;
-                if (BITS == 4) {
-                    if (hot)
-                        lw = *reinterpret_cast<const uint2 *>(st + 2 * G::VB + blk * G::LOB + r * G::ROWV + cg * 8);
-                    W = w * vs;
-                    zacc = fmaf(w, hot ? vz : fmaf(1.5f, vs, vz), zacc);
-                } else {
-                    W = w * vs * 0.25f;
-                    zacc = fmaf(w, vz, zacc);
-                }
-                const float Wp = W * vscale;
+                if (BITS == 4 && hot)
+                    lw = *reinterpret_cast<const uint2 *>(st + 2 * G::VB + blk * G::LOB + r * G::ROWV + cg * 8);
                 value_word(hw.x, lw.x, Wp, acc[0]);
                 value_word(hw.y, lw.y, Wp, acc[1]);
             }
@@ -656,7 +697,13 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
                         acc[k][e][n].x += __shfl_xor_sync(0xFFFFFFFFu, acc[k][e][n].x, off);
                         acc[k][e][n].y += __shfl_xor_sync(0xFFFFFFFFu, acc[k][e][n].y, off);
                     }
-            zacc += __shfl_xor_sync(0xFFFFFFFFu, zacc, off);
+        }
+        float zacc = 0.f;
+#pragma unroll
+        for (int j = 0; j < G::NCG; ++j) {
+            const float z = warp_sum(zl[j]);
+            if (cg == j)
+                zacc = z;
         }
         lsum = warp_sum(lsum);
         float *red = sm.red + warp * (D + 1);
@@ -733,6 +780,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
     float m_prev = 0.f, m_prev2 = 0.f;
     if (nrows > 0) {
         setup_row(0);
+        load_segment();
         pump(spw);
         consume_k(0);
     }
@@ -792,7 +840,7 @@ int launch_t(const DecodeArgs &a, const DecodeShape &shp, cudaStream_t s)
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, a, shp.stages);
+    e = cudaLaunchKernelEx(&cfg, kern, a, shp.stages_log2);
     return e == cudaSuccess ? LOOPKV_OK : LOOPKV_ERR_CUDA;
 }
 
@@ -849,15 +897,13 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
             continue;
         const int cap = (max_groups + C - 1) / C;
         const int capw = (cap + kWarps - 1) / kWarps;
-        // slots per warp: fill the shared memory of `want_ctas` CTAs per SM (1 KB reserved per CTA)
+        // slots per warp (a power of two): fill the shared memory of `want_ctas` CTAs per SM
         const int budget = smem_per_sm / want_ctas - 1024;
-        int spw = (budget - smem_bytes<BITS, D>(0, capw)) / (kWarps * (G::STAGE + 8));
-        if (spw > 8)
-            spw = 8;
+        int spw = 8;
+        while (spw > 2 && smem_bytes<BITS, D>(spw, capw) > budget)
+            spw >>= 1;
         if (env_s)
             spw = atoi(env_s);
-        if (spw < 2)
-            spw = 2;
         const int smem = smem_bytes<BITS, D>(spw, capw);
         if (smem > 227 * 1024 || !layout_ok<BITS, D>(spw, capw))
             continue;
@@ -874,6 +920,7 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
             best.cluster = C;
             best.clusters = ncl;
             best.stages = spw;
+            best.stages_log2 = __builtin_ctz(spw);
             best.smem = smem;
             best.threads = kThreads;
             best.cap = cap;

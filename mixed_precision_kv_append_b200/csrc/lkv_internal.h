@@ -56,7 +56,8 @@ struct DecodeArgs {
 struct DecodeShape {
     int cluster;   // CTAs per cluster; a cluster reads one (request, head) row at a time
     int clusters;  // persistent clusters in the grid
-    int stages;    // pipeline depth (shared-memory ring slots per CTA)
+    int stages;    // ring slots per warp (a power of two)
+    int stages_log2;
     int smem;      // dynamic shared memory bytes per CTA
     int threads;
     int cap;       // score capacity per CTA and row, in 32-token groups
