@@ -34,6 +34,24 @@ from mixed_precision_kv_append_b200 import synth  # noqa: E402
 METRIC = "fused loop-aware decode attention: KV GB/s (% of HBM peak) and decode steps/s"
 
 
+def _profiled_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary of this workload, if the
+    decode kernel sources are unchanged since the capture (else None)."""
+    import hashlib
+    import re
+
+    path = os.path.join(ROOT, "profiles", f"decode_kernel_{workload}.md")
+    csrc = os.path.join(ROOT, "mixed_precision_kv_append_b200", "csrc")
+    try:
+        text = open(path).read()
+        traffic = int(re.search(r"traffic_bytes_per_launch: (\d+)", text).group(1))
+        want = re.search(r"kernel_source_sha256: ([0-9a-f]+)", text).group(1)
+        src = b"".join(open(os.path.join(csrc, f), "rb").read() for f in ("decode_kernel.cu", "lkv_device.cuh"))
+    except Exception:
+        return None
+    return traffic if hashlib.sha256(src).hexdigest() == want else None
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -92,6 +110,16 @@ class ClockSampler:
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
                 "reasons": sorted(reasons), "samples": len(self.samples)}
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise maximum over all ranks of per-rank timings (identity without a process group).
+    Every rank must call it at the same point; the tensor lives on `device` (CUDA for NCCL, CPU for gloo)."""
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return list(values)
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
 
 
 # ----------------------------------------------------------------------------- workload
@@ -232,10 +260,7 @@ def run_ours(args, rank, world, device):
         dist.barrier()
     t_e2e = _time_graph(runner, args.steps, True, host_q, host_out)
     runner.cache.check("timed steps")
-    if world > 1:
-        tt = torch.tensor([t, t_e2e], device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t, t_e2e = tt.tolist()
+    t, t_e2e = max_over_ranks([t, t_e2e], device)
     peak, peak_kind = _peaks()
     ms = t / args.steps * 1e3
     gbs = algo_bytes * world * args.steps / t / 1e9
@@ -272,7 +297,8 @@ def run_ours(args, rank, world, device):
                 "d2h_bytes_per_step": int(runner.out.numel() * 4),
                 "ms_per_step": round(t_e2e / args.steps * 1e3, 4)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4),
+                     "traffic": _profiled_traffic(w.name) if not args.layers else None,
                      "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"},
         "gpu_launches": runner.launches_per_step * args.steps * 2,
         "clocks": clk.summary(),

@@ -28,11 +28,16 @@
 // both the per-warp maxima (with their partial exponential sums, for the normalised
 // rule) of row r and the partial outputs of row r-1.
 //
-// Code extraction: a field masked out of a packed word, read as an fp32 bit pattern
-// x < 2^24, has the value x * 2^-149 exactly (subnormal or smallest-exponent normal
-// numbers).  Multiplying it by a factor pre-scaled with 2^(149 - p) (p = the field's
-// bit position) gives code * factor with one AND and one FMA per code and no int->
-// float conversion; fp32 FMA on sm_100a keeps subnormal inputs (no flush to zero).
+// Keys: the dot product of a 32-token group is computed exactly in integers.  The
+// group's per-channel factor q_c * s_c (key scale folded into the query once per group,
+// as the paper's reader does) is rounded to a 22-bit fixed-point integer and split into
+// three signed 8-bit digits; the 4-bit (or 2-bit) codes are unpacked four at a time into
+// bytes with one AND, and dp4a accumulates code * digit in int32 with no rounding.
+// Values: a field masked out of a packed word, read as an fp32 bit pattern x < 2^24, has
+// the value x * 2^-149 exactly (subnormal or smallest-exponent normal numbers);
+// multiplied by a weight pre-scaled with 2^(149 - p) (p = the field's bit position) it
+// gives code * weight with one AND and half a packed FMA per code; fp32 FMA on sm_100a
+// keeps subnormal inputs (no flush to zero).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -47,7 +52,7 @@ namespace {
 
 constexpr int kWarps = 4; // every warp both issues the copies of its stages and computes on them
 constexpr int kThreads = kWarps * 32;
-constexpr int kMinCtasPerSm = 4;
+constexpr int kMinCtasPerSm = 4; // default register bound: 4 CTAs of 128 threads per SM (<= 128 registers)
 constexpr int kVScaleExp = 40; // V accumulators hold code * w * s * 2^(p - 40)
 
 template <int BITS, int D> struct Geo {
@@ -69,23 +74,6 @@ template <int BITS, int D> struct Geo {
     static constexpr int TPI = 32 / NCG;      // tokens per V iteration of a warp
 };
 
-// Slot of channel c in the per-word factor table, and the bit position its field is
-// read from (fields above bit 23 are read from the word shifted right by 16).
-template <int BITS> __device__ __forceinline__ void key_slot(int c, int &slot, int &pos)
-{
-    if (BITS == 4) {
-        int w = c >> 3, r = c & 7;
-        int j = r < 4 ? 2 * r : 2 * (r - 4) + 1; // nibble index in the word
-        slot = 8 * w + j;
-        pos = j < 6 ? 4 * j : (j == 6 ? 8 : 12);
-    } else {
-        int w = c >> 4, r = c & 15;
-        int b = r & 3, i = r >> 2; // field at bit 8b + 2i
-        slot = 16 * w + 4 * b + i;
-        pos = b < 3 ? 8 * b + 2 * i : 8 + 2 * i;
-    }
-}
-
 __device__ __forceinline__ float fbits(uint32_t x) { return __uint_as_float(x); }
 
 __device__ __forceinline__ void ffma2(float2 &acc, float a, float b, float2 f)
@@ -93,34 +81,36 @@ __device__ __forceinline__ void ffma2(float2 &acc, float a, float b, float2 f)
     acc = __ffma2_rn(make_float2(a, b), f, acc);
 }
 
-// acc += sum over the 8 nibbles of w of nibble * A[slot]
-__device__ __forceinline__ void key_word4(uint32_t w, const float *A, float2 &acc)
+// acc += sum of the four unsigned bytes of `u` times the four signed bytes of `d`
+__device__ __forceinline__ void dp4a_us(int &acc, uint32_t u, int d)
 {
-    const float4 a0 = reinterpret_cast<const float4 *>(A)[0];
-    const float4 a1 = reinterpret_cast<const float4 *>(A)[1];
-    const uint32_t h = w >> 16;
-    ffma2(acc, fbits(w & 0xFu), fbits(w & 0xF0u), make_float2(a0.x, a0.y));
-    ffma2(acc, fbits(w & 0xF00u), fbits(w & 0xF000u), make_float2(a0.z, a0.w));
-    ffma2(acc, fbits(w & 0xF0000u), fbits(w & 0xF00000u), make_float2(a1.x, a1.y));
-    ffma2(acc, fbits(h & 0xF00u), fbits(h & 0xF000u), make_float2(a1.z, a1.w));
+    asm("dp4a.u32.s32 %0, %1, %2, %0;" : "+r"(acc) : "r"(u), "r"(d));
 }
 
-// acc += sum over the 16 two-bit fields of w of field * A[slot]
-__device__ __forceinline__ void key_word2(uint32_t w, const float *A, float2 &acc)
+// Quad q of a key row = channels 4q..4q+3 as four bytes.  4-bit word w holds quads 2w
+// (low nibbles) and 2w+1 (high nibbles); 2-bit word w holds quads 4w+i at bit 2i.
+template <int BITS>
+__device__ __forceinline__ void key_word(uint32_t w, const int4 *dig, int (&acc)[2][3])
 {
-    const float4 a0 = reinterpret_cast<const float4 *>(A)[0];
-    const float4 a1 = reinterpret_cast<const float4 *>(A)[1];
-    const float4 a2 = reinterpret_cast<const float4 *>(A)[2];
-    const float4 a3 = reinterpret_cast<const float4 *>(A)[3];
-    const uint32_t h = w >> 16;
-    ffma2(acc, fbits(w & 0x3u), fbits(w & 0xCu), make_float2(a0.x, a0.y));
-    ffma2(acc, fbits(w & 0x30u), fbits(w & 0xC0u), make_float2(a0.z, a0.w));
-    ffma2(acc, fbits(w & 0x300u), fbits(w & 0xC00u), make_float2(a1.x, a1.y));
-    ffma2(acc, fbits(w & 0x3000u), fbits(w & 0xC000u), make_float2(a1.z, a1.w));
-    ffma2(acc, fbits(w & 0x30000u), fbits(w & 0xC0000u), make_float2(a2.x, a2.y));
-    ffma2(acc, fbits(w & 0x300000u), fbits(w & 0xC00000u), make_float2(a2.z, a2.w));
-    ffma2(acc, fbits(h & 0x300u), fbits(h & 0xC00u), make_float2(a3.x, a3.y));
-    ffma2(acc, fbits(h & 0x3000u), fbits(h & 0xC000u), make_float2(a3.z, a3.w));
+    if (BITS == 4) {
+        const uint32_t u0 = w & 0x0F0F0F0Fu, u1 = (w >> 4) & 0x0F0F0F0Fu;
+        const int4 d0 = dig[0], d1 = dig[1];
+        dp4a_us(acc[0][0], u0, d0.x);
+        dp4a_us(acc[0][1], u0, d0.y);
+        dp4a_us(acc[0][2], u0, d0.z);
+        dp4a_us(acc[1][0], u1, d1.x);
+        dp4a_us(acc[1][1], u1, d1.y);
+        dp4a_us(acc[1][2], u1, d1.z);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t u = (w >> (2 * i)) & 0x03030303u;
+            const int4 d = dig[i];
+            dp4a_us(acc[i & 1][0], u, d.x);
+            dp4a_us(acc[i & 1][1], u, d.y);
+            dp4a_us(acc[i & 1][2], u, d.z);
+        }
+    }
 }
 
 // Value word pair (hi, lo) of 16 channels -> 4-bit codes 4h+l in two nibble words.
@@ -153,11 +143,11 @@ struct Smem {
     uint64_t *full;    // [kWarps][spw] completion barriers of the slots
     float *scores;     // [2][kWarps][capw * 32] scores of a warp's groups, by row parity
     float *tscores;    // [2][32] tail scores, by row parity
-    float *aw;         // [kWarps][D] key factors
+    uint8_t *scr;      // [kWarps][SCR] per-warp scratch, used in turn as: key-factor digits
+                       // [D/4][4] during a K stage, value weights [32][D/32] during a V
+                       // stage, the warp's partial o and l [D + 1] at the end of a V pass
     float *stat;       // [3][kWarps][2] per-warp (max, sum exp(s - max)), by row index mod 3
     float *part;       // [2][D + 1] CTA partial o and l of a row, by row parity
-    float *wv;         // [kWarps][32][4] per token and 32-channel group: w * s * 2^109
-    float *red;        // [kWarps][D + 1]
     int32_t *ids;      // [3][kWarps][2 * capw] block ids of a warp's groups, by row index mod 3
     int32_t *irow;     // [3][kWarps][8] issuer state of a row, by row index mod 3
 };
@@ -168,31 +158,37 @@ enum { IR_ROW = 0, IR_H, IR_OWN, IR_VFIRST, IR_VISSUED, IR_THR, IR_N = 8 };
 // Byte offsets of the shared-memory regions; every region starts on a 16-byte boundary
 // (the key factors and the stage data are read with 16-byte vector loads).
 struct SmemLayout {
-    int full, scores, tscores, aw, stat, part, wv, red, ids, irow, total;
+    int full, scores, tscores, scr, stat, part, ids, irow, total;
 };
 
 __host__ __device__ constexpr int align16(int x) { return (x + 15) & ~15; }
 
-template <int BITS, int D> __host__ __device__ constexpr SmemLayout smem_layout(int spw, int capw)
+// Bytes of a warp's scratch: the largest of its three uses.
+template <int D> __host__ __device__ constexpr int scratch_bytes()
+{
+    return align16((D * 4 > (D + 1) * 4 ? D * 4 : (D + 1) * 4) > 32 * (D / 32) * 4
+                       ? (D * 4 > (D + 1) * 4 ? D * 4 : (D + 1) * 4)
+                       : 32 * (D / 32) * 4);
+}
+
+// nbuf: score buffers (2 when a cluster reads more than one row, so that the next row's
+// keys can be scored while the current row's values are read).
+template <int BITS, int D> __host__ __device__ constexpr SmemLayout smem_layout(int spw, int capw, int nbuf)
 {
     SmemLayout L{};
     int o = kWarps * spw * Geo<BITS, D>::STAGE; // ring, 128-byte aligned slots
     L.full = o;
     o = align16(o + kWarps * spw * 8);
     L.scores = o;
-    o = align16(o + 2 * kWarps * capw * 32 * 4);
+    o = align16(o + nbuf * kWarps * capw * 32 * 4);
     L.tscores = o;
     o = align16(o + 2 * 32 * 4);
-    L.aw = o;
-    o = align16(o + kWarps * D * 4);
+    L.scr = o;
+    o = align16(o + kWarps * scratch_bytes<D>());
     L.stat = o;
     o = align16(o + 3 * kWarps * 2 * 4);
     L.part = o;
     o = align16(o + 2 * (D + 1) * 4);
-    L.wv = o;
-    o = align16(o + kWarps * 32 * 4 * 4);
-    L.red = o;
-    o = align16(o + kWarps * (D + 1) * 4);
     L.ids = o;
     o = align16(o + 3 * kWarps * 2 * capw * 4);
     L.irow = o;
@@ -201,41 +197,40 @@ template <int BITS, int D> __host__ __device__ constexpr SmemLayout smem_layout(
     return L;
 }
 
-template <int BITS, int D> __host__ __device__ constexpr int smem_bytes(int spw, int capw)
+template <int BITS, int D> __host__ __device__ constexpr int smem_bytes(int spw, int capw, int nbuf)
 {
-    return smem_layout<BITS, D>(spw, capw).total;
+    return smem_layout<BITS, D>(spw, capw, nbuf).total;
 }
 
-template <int BITS, int D> __device__ Smem carve(uint8_t *base, int spw, int capw)
+template <int BITS, int D> __device__ Smem carve(uint8_t *base, int spw, int capw, int nbuf)
 {
-    const SmemLayout L = smem_layout<BITS, D>(spw, capw);
+    const SmemLayout L = smem_layout<BITS, D>(spw, capw, nbuf);
     Smem s;
     s.ring = base;
     s.full = reinterpret_cast<uint64_t *>(base + L.full);
     s.scores = reinterpret_cast<float *>(base + L.scores);
     s.tscores = reinterpret_cast<float *>(base + L.tscores);
-    s.aw = reinterpret_cast<float *>(base + L.aw);
+    s.scr = base + L.scr;
     s.stat = reinterpret_cast<float *>(base + L.stat);
     s.part = reinterpret_cast<float *>(base + L.part);
-    s.wv = reinterpret_cast<float *>(base + L.wv);
-    s.red = reinterpret_cast<float *>(base + L.red);
     s.ids = reinterpret_cast<int32_t *>(base + L.ids);
     s.irow = reinterpret_cast<int32_t *>(base + L.irow);
     return s;
 }
 
 // Host check of a layout: every region 16-byte aligned, in order, inside the allocation.
-template <int BITS, int D> bool layout_ok(int spw, int capw)
+template <int BITS, int D> bool layout_ok(int spw, int capw, int nbuf)
 {
-    const SmemLayout L = smem_layout<BITS, D>(spw, capw);
-    const int offs[] = {L.full, L.scores, L.tscores, L.aw, L.stat, L.part, L.wv, L.red, L.ids, L.irow};
+    const SmemLayout L = smem_layout<BITS, D>(spw, capw, nbuf);
+    const int offs[] = {L.full, L.scores, L.tscores, L.scr, L.stat, L.part, L.ids, L.irow};
     int prev = kWarps * spw * Geo<BITS, D>::STAGE;
     for (int o : offs) {
         if (o % 16 || o < prev)
             return false;
         prev = o;
     }
-    return (Geo<BITS, D>::STAGE % 128) == 0 && L.total >= prev && (spw & (spw - 1)) == 0;
+    return (Geo<BITS, D>::STAGE % 128) == 0 && L.total >= prev && (spw & (spw - 1)) == 0 &&
+           scratch_bytes<D>() >= D * 4 && scratch_bytes<D>() >= (D + 1) * 4 && scratch_bytes<D>() >= 32 * (D / 32) * 4;
 }
 
 // One (request, head) row as seen by one CTA of its cluster.
@@ -322,8 +317,9 @@ __device__ __forceinline__ void segment(int sig, int nrows, bool &is_v, int &ri)
     }
 }
 
-template <int BITS, int D, typename DT>
-__global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const DecodeArgs a, const int spw_log2)
+// MINCTA: CTAs per SM the registers are budgeted for (4: <= 128 registers, 5: <= 96).
+template <int BITS, int D, typename DT, int MINCTA>
+__global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeArgs a, const int spw_log2, const int nbuf)
 {
     using G = Geo<BITS, D>;
     extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -333,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
     const int cid = blockIdx.x / (int)C, ncl = gridDim.x / (int)C;
     const int nrows = cid < a.rows ? (a.rows - 1 - cid) / ncl + 1 : 0; // rows cid, cid + ncl, ...
     const int capw = (a.cap_groups + kWarps - 1) / kWarps;
-    Smem sm = carve<BITS, D>(smem_raw, spw, capw);
+    Smem sm = carve<BITS, D>(smem_raw, spw, capw, nbuf);
     const bool all_hot = (BITS == 4) && !(a.tau > 0.f);
     const bool decide = (BITS == 4) && (a.tau > 0.f); // lo planes depend on the row max
 
@@ -345,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
 
     uint8_t *ring = sm.ring + warp * spw * G::STAGE;
     uint64_t *full = sm.full + warp * spw;
-    auto scores_of = [&](int ri) { return sm.scores + ((ri & 1) * kWarps + warp) * capw * 32; };
+    auto scores_of = [&](int ri) { return sm.scores + (((nbuf == 2) ? (ri & 1) : 0) * kWarps + warp) * capw * 32; };
     auto ids_of = [&](int ri) { return sm.ids + ((ri % 3) * kWarps + warp) * 2 * capw; };
     auto irow_of = [&](int ri) { return sm.irow + ((ri % 3) * kWarps + warp) * IR_N; };
 
@@ -491,18 +487,13 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
     };
 
     // ---------------------------------------------------------------- compute
-    float *aw = sm.aw + warp * D;
-    float4 *wv4 = reinterpret_cast<float4 *>(sm.wv) + warp * 32;
-    const float *wvf = sm.wv + warp * 128;
+    constexpr int SCR = scratch_bytes<D>();
+    uint8_t *scr = sm.scr + warp * SCR;
+    uint8_t *awb = scr;                                    // K stage: digit table, 16 bytes per quad
+    const int4 *aw4 = reinterpret_cast<const int4 *>(scr);
+    float4 *wv4 = reinterpret_cast<float4 *>(scr);         // V stage: weights per token and group
+    const float *wvf = reinterpret_cast<const float *>(scr);
     // a lane owns the channel pairs (2*lane + 64j, 2*lane + 1 + 64j), j < D/64
-    int kslot[D / 32];
-    float kpow[D / 32];
-#pragma unroll
-    for (int k = 0; k < D / 32; ++k) {
-        int pos;
-        key_slot<BITS>(2 * lane + 64 * (k >> 1) + (k & 1), kslot[k], pos);
-        kpow[k] = __int_as_float((24 - pos + 127) << 23);
-    }
     const float vscale = 6.490371073168535e32f; // 2^(149 - kVScaleExp) = 2^109
     int prc_n = 0;
     bool timed_out = false; // after one bounded wait gives up, later waits are skipped
@@ -544,44 +535,43 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
             }
             zs = warp_sum(zs);
             amax = warp_max(amax);
-            // Factor of channel c: a_c * 2^(149 - pos - K), K = E + 23, E = exponent of amax,
-            // so |factor| < 2^127 and every product code * factor is exact up to one rounding.
+            // Fixed point: I_c = round(a_c * 2^F) with F = 21 - E (E = exponent of max |a|),
+            // so |I_c| <= 2^22; balanced base-256 digits d0 + 256 d1 + 65536 d2, |d2| <= 65.
             const uint32_t abits = __float_as_uint(amax);
-            const int E = abits >= 0x00800000u ? (int)(abits >> 23) - 127 : 0;
-            if (E >= -25 && E <= 100 && abits >= 0x00800000u) { // warp-uniform fast path
-                const float f = __int_as_float((102 - E + 127) << 23); // 2^(102 - E)
+            const int E = abits >= 0x00800000u ? (int)(abits >> 23) - 127 : -126;
+            const int F = 21 - E;
+            const bool fast = F >= -126 && F <= 127 && E - 21 >= -126;
+            const float fs = fast ? __int_as_float((F + 127) << 23) : 0.f;
 #pragma unroll
-                for (int c4 = 0; c4 < D / 32; ++c4)
-                    aw[kslot[c4]] = (av[c4] * f) * kpow[c4];
-            } else {
-#pragma unroll
-                for (int c4 = 0; c4 < D / 32; ++c4) {
-                    int slot_c, pos;
-                    key_slot<BITS>(2 * lane + 64 * (c4 >> 1) + (c4 & 1), slot_c, pos);
-                    aw[slot_c] = mul_pow2(av[c4], 126 - E - pos);
-                }
+            for (int c4 = 0; c4 < D / 32; ++c4) {
+                const int c = 2 * lane + 64 * (c4 >> 1) + (c4 & 1);
+                const float x = fast ? av[c4] * fs : mul_pow2(av[c4], F);
+                const int I = __float2int_rn(x);
+                const int d0 = (I << 24) >> 24;
+                const int I1 = (I - d0) >> 8;
+                const int d1 = (I1 << 24) >> 24;
+                const int d2 = (I1 - d1) >> 8;
+                uint8_t *q = awb + (c >> 2) * 16 + (c & 3);
+                q[0] = (uint8_t)d0;
+                q[4] = (uint8_t)d1;
+                q[8] = (uint8_t)d2;
             }
             __syncwarp();
             const uint32_t *kr =
                 reinterpret_cast<const uint32_t *>(st + (lane >> 4) * G::KB + (lane & 15) * G::ROWK);
-            float2 acc = make_float2(0.f, 0.f);
+            int acc[2][3] = {{0, 0, 0}, {0, 0, 0}};
+            constexpr int QPW = BITS == 4 ? 2 : 4; // quads per code word
 #pragma unroll
             for (int w4 = 0; w4 < G::WORDSK / 4; ++w4) {
                 const uint4 cw = reinterpret_cast<const uint4 *>(kr)[w4];
-                if (BITS == 4) {
-                    key_word4(cw.x, aw + 8 * (4 * w4 + 0), acc);
-                    key_word4(cw.y, aw + 8 * (4 * w4 + 1), acc);
-                    key_word4(cw.z, aw + 8 * (4 * w4 + 2), acc);
-                    key_word4(cw.w, aw + 8 * (4 * w4 + 3), acc);
-                } else {
-                    key_word2(cw.x, aw + 16 * (4 * w4 + 0), acc);
-                    key_word2(cw.y, aw + 16 * (4 * w4 + 1), acc);
-                    key_word2(cw.z, aw + 16 * (4 * w4 + 2), acc);
-                    key_word2(cw.w, aw + 16 * (4 * w4 + 3), acc);
-                }
+                key_word<BITS>(cw.x, aw4 + QPW * (4 * w4 + 0), acc);
+                key_word<BITS>(cw.y, aw4 + QPW * (4 * w4 + 1), acc);
+                key_word<BITS>(cw.z, aw4 + QPW * (4 * w4 + 2), acc);
+                key_word<BITS>(cw.w, aw4 + QPW * (4 * w4 + 3), acc);
             }
-            const float accs = acc.x + acc.y;
-            const float s2 = (E <= 100 ? accs * __int_as_float((E + 150) << 23) : mul_pow2(accs, E + 23)) + zs;
+            const float dot = fmaf((float)(acc[0][2] + acc[1][2]), 65536.f,
+                                   fmaf((float)(acc[0][1] + acc[1][1]), 256.f, (float)(acc[0][0] + acc[1][0])));
+            const float s2 = (fast ? dot * __int_as_float((127 - F) << 23) : mul_pow2(dot, -F)) + zs;
             sc[k * 32 + lane] = s2;
             mx = fmaxf(mx, s2);
             __syncwarp();
@@ -706,7 +696,8 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
                 zacc = z;
         }
         lsum = warp_sum(lsum);
-        float *red = sm.red + warp * (D + 1);
+        __syncwarp();
+        float *red = reinterpret_cast<float *>(scr); // end of the V pass: the warp's partial o, l
         if (lane < G::NCG) {
 #pragma unroll
             for (int k = 0; k < 2; ++k)
@@ -744,9 +735,10 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
             float sum = 0.f;
 #pragma unroll
             for (int w = 0; w < kWarps; ++w)
-                sum += sm.red[w * (D + 1) + c];
+                sum += reinterpret_cast<const float *>(sm.scr + w * SCR)[c];
             part[c] = sum;
         }
+        named_sync(1, kThreads); // every warp's scratch is free again
     };
 
     // CTA `crank` writes channels [crank*D/C, (crank+1)*D/C) of row ri, summing the
@@ -820,7 +812,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasPerSm) decode_kernel(const D
 template <int BITS, int D, typename DT>
 int launch_t(const DecodeArgs &a, const DecodeShape &shp, cudaStream_t s)
 {
-    auto kern = decode_kernel<BITS, D, DT>;
+    auto kern = shp.min_ctas == 5 ? decode_kernel<BITS, D, DT, 5> : decode_kernel<BITS, D, DT, 4>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, shp.smem);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
@@ -840,14 +832,14 @@ int launch_t(const DecodeArgs &a, const DecodeShape &shp, cudaStream_t s)
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, a, shp.stages_log2);
+    e = cudaLaunchKernelEx(&cfg, kern, a, shp.stages_log2, shp.score_bufs);
     return e == cudaSuccess ? LOOPKV_OK : LOOPKV_ERR_CUDA;
 }
 
 // Clusters of size C that can be resident at once for this kernel and shared memory.
-template <int BITS, int D, typename DT> int max_active_clusters(int C, int smem)
+template <int BITS, int D, typename DT> int max_active_clusters(int C, int smem, int min_ctas)
 {
-    auto kern = decode_kernel<BITS, D, DT>;
+    auto kern = min_ctas == 5 ? decode_kernel<BITS, D, DT, 5> : decode_kernel<BITS, D, DT, 4>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return 0;
     cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
@@ -889,7 +881,9 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
     const char *env_c = getenv("LOOPKV_DECODE_CLUSTER");
     const char *env_s = getenv("LOOPKV_DECODE_STAGES");
     const char *env_o = getenv("LOOPKV_DECODE_CTAS_PER_SM");
-    const int want_ctas = env_o ? atoi(env_o) : kMinCtasPerSm;
+    for (int want_ctas = 4; want_ctas <= 5; ++want_ctas) {
+    if (env_o && atoi(env_o) != want_ctas)
+        continue;
     for (int C = 1; C <= 16; C *= 2) {
         if (env_c && atoi(env_c) != C)
             continue;
@@ -897,34 +891,47 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
             continue;
         const int cap = (max_groups + C - 1) / C;
         const int capw = (cap + kWarps - 1) / kWarps;
-        // slots per warp (a power of two): fill the shared memory of `want_ctas` CTAs per SM
         const int budget = smem_per_sm / want_ctas - 1024;
-        int spw = 8;
-        while (spw > 2 && smem_bytes<BITS, D>(spw, capw) > budget)
-            spw >>= 1;
-        if (env_s)
-            spw = atoi(env_s);
-        const int smem = smem_bytes<BITS, D>(spw, capw);
-        if (smem > 227 * 1024 || !layout_ok<BITS, D>(spw, capw))
-            continue;
-        int ncl = max_active_clusters<BITS, D, DT>(C, smem);
-        if (ncl <= 0)
-            continue;
-        if (ncl > rows)
-            ncl = rows;
-        // balance: each cluster takes ceil(rows / ncl) rows; too few CTAs per SM penalised
-        const double rounds = (double)((rows + ncl - 1) / ncl);
-        const double eff = ((double)rows / ncl) / rounds * std::min(1.0, (double)(ncl * C) / (3.0 * sm_count));
-        if (eff > best_eff + 1e-9) {
-            best_eff = eff;
-            best.cluster = C;
-            best.clusters = ncl;
-            best.stages = spw;
-            best.stages_log2 = __builtin_ctz(spw);
-            best.smem = smem;
-            best.threads = kThreads;
-            best.cap = cap;
+        for (int nbuf = 1; nbuf <= 2; ++nbuf) {
+            // slots per warp (a power of two): fill the shared memory of `want_ctas` CTAs per SM
+            int spw = 8;
+            while (spw > 2 && smem_bytes<BITS, D>(spw, capw, nbuf) > budget)
+                spw >>= 1;
+            if (env_s)
+                spw = atoi(env_s);
+            const int smem = smem_bytes<BITS, D>(spw, capw, nbuf);
+            if (smem > 227 * 1024 || !layout_ok<BITS, D>(spw, capw, nbuf))
+                continue;
+            int ncl = max_active_clusters<BITS, D, DT>(C, smem, want_ctas);
+            if (ncl <= 0)
+                continue;
+            if (ncl > rows)
+                ncl = rows;
+            if (nbuf == 1 && ncl < rows)
+                continue; // a cluster would read several rows: it needs two score buffers
+            // balance: each cluster takes ceil(rows / ncl) rows; too few CTAs per SM penalised;
+            // more resident CTAs (warps to hide latency) and deeper rings (bytes in flight)
+            // preferred
+            const double rounds = (double)((rows + ncl - 1) / ncl);
+            const double eff = ((double)rows / ncl) / rounds *
+                               std::min(1.0, (double)(ncl * C) / (3.0 * sm_count)) *
+                               (1.0 + 0.3 * std::min(1.0, (double)(ncl * C) / (want_ctas * sm_count))) *
+                               (1.0 + 0.01 * spw);
+            if (eff > best_eff + 1e-9) {
+                best_eff = eff;
+                best.cluster = C;
+                best.clusters = ncl;
+                best.stages = spw;
+                best.stages_log2 = __builtin_ctz(spw);
+                best.score_bufs = nbuf;
+                best.smem = smem;
+                best.threads = kThreads;
+                best.cap = cap;
+                best.min_ctas = want_ctas;
+            }
+            break;
         }
+    }
     }
     return best;
 }

@@ -58,6 +58,8 @@ struct DecodeShape {
     int clusters;  // persistent clusters in the grid
     int stages;    // ring slots per warp (a power of two)
     int stages_log2;
+    int score_bufs; // 1, or 2 when a cluster reads several rows
+    int min_ctas;   // register budget of the kernel build: CTAs per SM (4 or 5)
     int smem;      // dynamic shared memory bytes per CTA
     int threads;
     int cap;       // score capacity per CTA and row, in 32-token groups

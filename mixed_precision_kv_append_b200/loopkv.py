@@ -14,7 +14,8 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libloopkv.so")
+# LOOPKV_LIB selects another build of the same library (for comparing builds)
+LIB_PATH = os.environ.get("LOOPKV_LIB") or os.path.join(_PKG, "libloopkv.so")
 
 LOOPKV_OK = 0
 ERRORS = {
