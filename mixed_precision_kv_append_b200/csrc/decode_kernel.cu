@@ -4,35 +4,37 @@
 // of persistent thread-block clusters of C CTAs; cluster c serves the (request, head)
 // rows c, c + NC, c + 2NC, ... one after another.  Inside a row, CTA k of the cluster
 // owns the 32-token groups k, k+C, k+2C, ... of the history, and CTA C-1 also the
-// unquantized tail.  For each row a CTA:
-//   1. K pass: streams the key codes and per-channel key scale/zero of its groups
-//      into shared memory with bulk asynchronous copies (a producer warp, an
-//      mbarrier ring), and computes every score from the full 4-bit (or 2-bit) keys
-//      with the key scale folded into q once per group (Appendix "History reader").
-//      Scores stay in shared memory.
-//   2. Exact row maximum: the CTAs exchange their maxima through distributed shared
-//      memory across a cluster barrier, so every CTA knows the exact m -- the
+// unquantized tail.  Warp w of a CTA owns the CTA's groups w, w+4, ...  For each row a
+// warp:
+//   1. K pass: streams the key codes and the per-channel key scale/zero of its groups
+//      into shared memory with bulk asynchronous copies that it issues itself (one
+//      elected lane, a private mbarrier ring), and computes every score from the full
+//      4-bit (or 2-bit) keys with the key scale folded into q once per group (Appendix
+//      "History reader").  Scores stay in shared memory.
+//   2. Exact row maximum: the CTAs exchange their per-warp maxima through distributed
+//      shared memory across a cluster barrier, so every CTA knows the exact m -- the
 //      "ideal" rule of §3.3 (a token is cold if its weight is below tau times the
-//      largest in its row), not a streaming seed.  With the normalised-weight rule
-//      a second exchange gives sum_t exp(s_t - m).
-//   3. V pass: streams V scale/zero and the hi plane of every token; the producer
-//      fetches a token's lo plane only if its weight passes the threshold (§3.3
-//      "Read-time V precision").  Hot tokens decode to z + s(4h+l), cold ones to the
-//      middle of their bucket z + s(4h+1.5), 2-bit cells to z + s*code; the per-token
-//      scale and zero are folded into the weight and a running sum.
-//   4. Merge: since all CTAs used the same m, their partial sums add directly; the
-//      CTAs reduce them through distributed shared memory and write out = o / l.
-// Rows are software-pipelined: while the cluster barrier that publishes row r's
-// maxima completes, the CTA already streams and scores the keys of row r+1, so the
-// memory pipe never drains at a row boundary.  One cluster barrier per row carries
-// both the per-warp maxima (with their partial exponential sums, for the normalised
-// rule) of row r and the partial outputs of row r-1.
+//      largest in its row), not a streaming seed.  With the normalised-weight rule the
+//      same exchange carries the partial sums of exp(s_t - m_w).
+//   3. V pass: streams V scale/zero and the hi plane of every token; the lo plane of a
+//      token is fetched only if its weight passes the threshold (§3.3 "Read-time V
+//      precision").  Hot tokens decode to z + s(4h+l), cold ones to the middle of their
+//      bucket z + s(4h+1.5), 2-bit cells to z + s*code; the per-token scale and zero
+//      are folded into the weight and a running sum.
+//   4. Merge: since all CTAs used the same m, their partial sums add directly; the CTAs
+//      reduce them through distributed shared memory and write out = o / l.
+// Rows are software-pipelined: while the cluster barrier that publishes row r's maxima
+// completes, the warp already streams and scores the keys of row r+1, so the memory pipe
+// never drains at a row boundary.  One cluster barrier per row carries both the
+// per-warp maxima of row r and the partial outputs of row r-1.
 //
 // Keys: the dot product of a 32-token group is computed exactly in integers.  The
-// group's per-channel factor q_c * s_c (key scale folded into the query once per group,
-// as the paper's reader does) is rounded to a 22-bit fixed-point integer and split into
-// three signed 8-bit digits; the 4-bit (or 2-bit) codes are unpacked four at a time into
-// bytes with one AND, and dp4a accumulates code * digit in int32 with no rounding.
+// group's per-channel factor a_c = q_c * s_c is rounded to a 22-bit fixed-point integer
+// I_c with one FMA against 1.5 * 2^23 (the float's low 23 bits are then I_c + 2^22), and
+// the three bytes of that field become three 8-bit digits (the top one re-centred to a
+// signed byte) with byte permutes.  The 4-bit (or 2-bit) codes are unpacked four at a
+// time into bytes with one AND, and dp4a accumulates code * digit in int32 with no
+// rounding.
 // Values: a field masked out of a packed word, read as an fp32 bit pattern x < 2^24, has
 // the value x * 2^-149 exactly (subnormal or smallest-exponent normal numbers);
 // multiplied by a weight pre-scaled with 2^(149 - p) (p = the field's bit position) it
@@ -52,7 +54,6 @@ namespace {
 
 constexpr int kWarps = 4; // every warp both issues the copies of its stages and computes on them
 constexpr int kThreads = kWarps * 32;
-constexpr int kMinCtasPerSm = 4; // default register bound: 4 CTAs of 128 threads per SM (<= 128 registers)
 constexpr int kVScaleExp = 40; // V accumulators hold code * w * s * 2^(p - 40)
 
 template <int BITS, int D> struct Geo {
@@ -72,6 +73,7 @@ template <int BITS, int D> struct Geo {
     static constexpr int ROWV = D / 4;        // value plane bytes per token
     static constexpr int NCG = D / 32;        // 32-channel value groups per token
     static constexpr int TPI = 32 / NCG;      // tokens per V iteration of a warp
+    static constexpr int NQ = D / 4;          // channel quads
 };
 
 __device__ __forceinline__ float fbits(uint32_t x) { return __uint_as_float(x); }
@@ -81,34 +83,90 @@ __device__ __forceinline__ void ffma2(float2 &acc, float a, float b, float2 f)
     acc = __ffma2_rn(make_float2(a, b), f, acc);
 }
 
+// acc += sum of the four unsigned bytes of `u` times the four unsigned bytes of `d`
+__device__ __forceinline__ void dp4a_uu(uint32_t &acc, uint32_t u, uint32_t d)
+{
+    asm("dp4a.u32.u32 %0, %1, %2, %0;" : "+r"(acc) : "r"(u), "r"(d));
+}
+
 // acc += sum of the four unsigned bytes of `u` times the four signed bytes of `d`
-__device__ __forceinline__ void dp4a_us(int &acc, uint32_t u, int d)
+__device__ __forceinline__ void dp4a_us(int &acc, uint32_t u, uint32_t d)
 {
     asm("dp4a.u32.s32 %0, %1, %2, %0;" : "+r"(acc) : "r"(u), "r"(d));
 }
 
-// Quad q of a key row = channels 4q..4q+3 as four bytes.  4-bit word w holds quads 2w
-// (low nibbles) and 2w+1 (high nibbles); 2-bit word w holds quads 4w+i at bit 2i.
+// max over the warp of |v|
+__device__ __forceinline__ float warp_max_abs(float v)
+{
+    float r;
+    asm volatile("redux.sync.max.abs.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+    return r;
+}
+
+
+// Accumulate one key word: quads `rec[0..]` hold the digits of the word's channels.
+// 4-bit word: low nibbles = quad 2w, high nibbles = quad 2w+1; 2-bit word: quad 4w+i at
+// bit 2i of every byte.
+struct KeyAcc {
+    uint32_t a0[2], a1[2];
+    int a2[2];
+};
+
 template <int BITS>
-__device__ __forceinline__ void key_word(uint32_t w, const int4 *dig, int (&acc)[2][3])
+__device__ __forceinline__ void key_word(uint32_t w, const uint4 *rec, KeyAcc &acc)
 {
     if (BITS == 4) {
         const uint32_t u0 = w & 0x0F0F0F0Fu, u1 = (w >> 4) & 0x0F0F0F0Fu;
-        const int4 d0 = dig[0], d1 = dig[1];
-        dp4a_us(acc[0][0], u0, d0.x);
-        dp4a_us(acc[0][1], u0, d0.y);
-        dp4a_us(acc[0][2], u0, d0.z);
-        dp4a_us(acc[1][0], u1, d1.x);
-        dp4a_us(acc[1][1], u1, d1.y);
-        dp4a_us(acc[1][2], u1, d1.z);
+        const uint4 r0 = rec[0], r1 = rec[1];
+        dp4a_uu(acc.a0[0], u0, r0.x);
+        dp4a_uu(acc.a1[0], u0, r0.y);
+        dp4a_us(acc.a2[0], u0, r0.z);
+        dp4a_uu(acc.a0[1], u1, r1.x);
+        dp4a_uu(acc.a1[1], u1, r1.y);
+        dp4a_us(acc.a2[1], u1, r1.z);
     } else {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const uint32_t u = (w >> (2 * i)) & 0x03030303u;
-            const int4 d = dig[i];
-            dp4a_us(acc[i & 1][0], u, d.x);
-            dp4a_us(acc[i & 1][1], u, d.y);
-            dp4a_us(acc[i & 1][2], u, d.z);
+            const uint4 r = rec[i];
+            dp4a_uu(acc.a0[i & 1], u, r.x);
+            dp4a_uu(acc.a1[i & 1], u, r.y);
+            dp4a_us(acc.a2[i & 1], u, r.z);
+        }
+    }
+}
+
+// One code word of two tokens against the same digit records.
+template <int BITS>
+__device__ __forceinline__ void key_word2(uint32_t wa, uint32_t wb, const uint4 *rec, KeyAcc &a, KeyAcc &b)
+{
+    if (BITS == 4) {
+        const uint32_t ua0 = wa & 0x0F0F0F0Fu, ua1 = (wa >> 4) & 0x0F0F0F0Fu;
+        const uint32_t ub0 = wb & 0x0F0F0F0Fu, ub1 = (wb >> 4) & 0x0F0F0F0Fu;
+        const uint4 r0 = rec[0], r1 = rec[1];
+        dp4a_uu(a.a0[0], ua0, r0.x);
+        dp4a_uu(b.a0[0], ub0, r0.x);
+        dp4a_uu(a.a1[0], ua0, r0.y);
+        dp4a_uu(b.a1[0], ub0, r0.y);
+        dp4a_us(a.a2[0], ua0, r0.z);
+        dp4a_us(b.a2[0], ub0, r0.z);
+        dp4a_uu(a.a0[1], ua1, r1.x);
+        dp4a_uu(b.a0[1], ub1, r1.x);
+        dp4a_uu(a.a1[1], ua1, r1.y);
+        dp4a_uu(b.a1[1], ub1, r1.y);
+        dp4a_us(a.a2[1], ua1, r1.z);
+        dp4a_us(b.a2[1], ub1, r1.z);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t ua = (wa >> (2 * i)) & 0x03030303u, ub = (wb >> (2 * i)) & 0x03030303u;
+            const uint4 r = rec[i];
+            dp4a_uu(a.a0[i & 1], ua, r.x);
+            dp4a_uu(b.a0[i & 1], ub, r.x);
+            dp4a_uu(a.a1[i & 1], ua, r.y);
+            dp4a_uu(b.a1[i & 1], ub, r.y);
+            dp4a_us(a.a2[i & 1], ua, r.z);
+            dp4a_us(b.a2[i & 1], ub, r.z);
         }
     }
 }
@@ -133,30 +191,36 @@ __device__ __forceinline__ void value_word(uint32_t hi, uint32_t lo, float W, fl
     ffma2(acc[1][3], fbits(Oh & 0xF00u), fbits(Oh & 0xF000u), w2);
 }
 
-// Channel offset (within 16) and bit position of accumulator (e, n): e = 0 for E,
-// 1 for O; n = nibble index 0..7.
-__device__ __forceinline__ int value_channel(int e, int n) { return 8 * (n & 1) + (n >> 1) + 4 * e; }
-__device__ __forceinline__ int value_pos(int n) { return n < 6 ? 4 * n : (n == 6 ? 8 : 12); }
+// Accumulator element i = 16k + 8e + n (k: 16-channel half, e: E or O word, n: nibble)
+// -> channel offset within the 32-channel group and bit position of its field.
+__host__ __device__ constexpr int value_channel(int i)
+{
+    return 16 * (i >> 4) + 8 * (i & 1) + ((i & 7) >> 1) + 4 * ((i >> 3) & 1);
+}
+__host__ __device__ constexpr int value_pos(int i)
+{
+    return (i & 7) < 6 ? 4 * (i & 7) : ((i & 7) == 6 ? 8 : 12);
+}
 
 struct Smem {
     uint8_t *ring;     // [kWarps][spw][STAGE] stage slots, a private slice per warp
     uint64_t *full;    // [kWarps][spw] completion barriers of the slots
-    float *scores;     // [2][kWarps][capw * 32] scores of a warp's groups, by row parity
+    float *scores;     // [nbuf][kWarps][capw * 32] scores of a warp's groups, by row parity
     float *tscores;    // [2][32] tail scores, by row parity
-    uint8_t *scr;      // [kWarps][SCR] per-warp scratch, used in turn as: key-factor digits
-                       // [D/4][4] during a K stage, value weights [32][D/32] during a V
+    uint8_t *scr;      // [kWarps][SCR] per-warp scratch, used in turn as: key digit records
+                       // [D/4][16 B] during a K stage, value weights [32][D/32] during a V
                        // stage, the warp's partial o and l [D + 1] at the end of a V pass
     float *stat;       // [3][kWarps][2] per-warp (max, sum exp(s - max)), by row index mod 3
     float *part;       // [2][D + 1] CTA partial o and l of a row, by row parity
     int32_t *ids;      // [3][kWarps][2 * capw] block ids of a warp's groups, by row index mod 3
-    int32_t *irow;     // [3][kWarps][8] issuer state of a row, by row index mod 3
+    int32_t *irow;     // [3][kWarps][IR_N] row parameters and issuer state, by row index mod 3
 };
 
-// Issuer state of one row (int fields of Smem::irow).
-enum { IR_ROW = 0, IR_H, IR_OWN, IR_VFIRST, IR_VISSUED, IR_THR, IR_N = 8 };
+// Fields of a row slot (Smem::irow).
+enum { IR_ROW = 0, IR_B, IR_H, IR_N, IR_TAIL, IR_VFIRST, IR_VISSUED, IR_THR, IR_N_FIELDS = 12 };
 
 // Byte offsets of the shared-memory regions; every region starts on a 16-byte boundary
-// (the key factors and the stage data are read with 16-byte vector loads).
+// (digit records, weights and stage data are read with 16-byte vector loads).
 struct SmemLayout {
     int full, scores, tscores, scr, stat, part, ids, irow, total;
 };
@@ -166,9 +230,7 @@ __host__ __device__ constexpr int align16(int x) { return (x + 15) & ~15; }
 // Bytes of a warp's scratch: the largest of its three uses.
 template <int D> __host__ __device__ constexpr int scratch_bytes()
 {
-    return align16((D * 4 > (D + 1) * 4 ? D * 4 : (D + 1) * 4) > 32 * (D / 32) * 4
-                       ? (D * 4 > (D + 1) * 4 ? D * 4 : (D + 1) * 4)
-                       : 32 * (D / 32) * 4);
+    return align16((D / 4) * 16 > (D + 1) * 4 ? (D / 4) * 16 : (D + 1) * 4);
 }
 
 // nbuf: score buffers (2 when a cluster reads more than one row, so that the next row's
@@ -192,7 +254,7 @@ template <int BITS, int D> __host__ __device__ constexpr SmemLayout smem_layout(
     L.ids = o;
     o = align16(o + 3 * kWarps * 2 * capw * 4);
     L.irow = o;
-    o = align16(o + 3 * kWarps * IR_N * 4);
+    o = align16(o + 3 * kWarps * IR_N_FIELDS * 4);
     L.total = o;
     return L;
 }
@@ -218,7 +280,8 @@ template <int BITS, int D> __device__ Smem carve(uint8_t *base, int spw, int cap
     return s;
 }
 
-// Host check of a layout: every region 16-byte aligned, in order, inside the allocation.
+// Host check of a layout: every region 16-byte aligned, in order, inside the allocation;
+// the per-warp id lists 8-byte aligned (read as pairs).
 template <int BITS, int D> bool layout_ok(int spw, int capw, int nbuf)
 {
     const SmemLayout L = smem_layout<BITS, D>(spw, capw, nbuf);
@@ -230,75 +293,12 @@ template <int BITS, int D> bool layout_ok(int spw, int capw, int nbuf)
         prev = o;
     }
     return (Geo<BITS, D>::STAGE % 128) == 0 && L.total >= prev && (spw & (spw - 1)) == 0 &&
-           scratch_bytes<D>() >= D * 4 && scratch_bytes<D>() >= (D + 1) * 4 && scratch_bytes<D>() >= 32 * (D / 32) * 4;
-}
-
-// One (request, head) row as seen by one CTA of its cluster.
-struct RowCtx {
-    int row, b, h;
-    int tail;       // validated tail length
-    int nmy;        // 32-token groups of the history owned by this CTA
-    bool tail_cta;  // this CTA also reads the tail
-};
-
-__device__ __forceinline__ RowCtx row_ctx(const DecodeArgs &a, int row, uint32_t crank, uint32_t C, bool report)
-{
-    RowCtx r;
-    r.row = row;
-    r.b = row / a.H;
-    r.h = row - r.b * a.H;
-    int hist = a.hist_len[r.b], tail = a.tail_len[r.b];
-    bool bad = false;
-    if (hist < 0 || hist > a.max_blocks * 16 || (hist & 31)) {
-        bad = true;
-        hist = 0;
-    }
-    if (tail < 0 || tail > 32) {
-        bad = true;
-        tail = 0;
-    }
-    const int ngroups = hist >> 5;
-    int nmy = ngroups > (int)crank ? (ngroups - (int)crank + (int)C - 1) / (int)C : 0;
-    if (nmy > a.cap_groups) {
-        bad = true;
-        nmy = a.cap_groups;
-    }
-    if (bad && report)
-        atomicOr(a.status, LOOPKV_DEV_STATE);
-    r.tail = tail;
-    r.nmy = nmy;
-    r.tail_cta = (crank == C - 1) && tail > 0;
-    return r;
+           scratch_bytes<D>() >= (D / 4) * 16 && scratch_bytes<D>() >= (D + 1) * 4 &&
+           scratch_bytes<D>() >= 32 * (D / 32) * 4 && (2 * capw * 4) % 8 == 0;
 }
 
 // Groups of a row owned by warp w of the CTA: local groups w, w + kWarps, ...
 __device__ __forceinline__ int owned(int nmy, int w) { return nmy > w ? (nmy - w + kWarps - 1) / kWarps : 0; }
-
-// Row max m (log2 units) and, for the normalised rule, l = sum_t 2^(s_t - m), from the
-// per-warp pairs of every CTA of the cluster (fixed order: every caller gets the same).
-__device__ __forceinline__ void cluster_row_stats(const float *stat, uint32_t C, float &m, float &l)
-{
-    m = -INFINITY;
-    for (uint32_t r = 0; r < C; ++r)
-        for (int w = 0; w < kWarps; ++w)
-            m = fmaxf(m, ld_dsmem_f32(stat + 2 * w, r));
-    l = 0.f;
-    if (m == -INFINITY)
-        return;
-    for (uint32_t r = 0; r < C; ++r)
-        for (int w = 0; w < kWarps; ++w) {
-            const float mw = ld_dsmem_f32(stat + 2 * w, r);
-            if (mw != -INFINITY)
-                l += ld_dsmem_f32(stat + 2 * w + 1, r) * exp2f(mw - m);
-        }
-}
-
-__device__ __forceinline__ float row_threshold(const DecodeArgs &a, float m, float l, bool decide)
-{
-    if (!decide)
-        return -INFINITY;
-    return a.tau_mode == LOOPKV_TAU_ABS_PROB ? m + log2f(a.tau * l) : m + log2f(a.tau);
-}
 
 // Segment sig of a warp's stage sequence K(0), K(1), V(0), K(2), V(1), ..., V(n-1):
 // returns whether it is a V segment and its row index.
@@ -317,6 +317,33 @@ __device__ __forceinline__ void segment(int sig, int nrows, bool &is_v, int &ri)
     }
 }
 
+// Row max m (log2 units) and, for the normalised rule, l = sum_t 2^(s_t - m), from the
+// per-warp pairs of every CTA of the cluster.  Lane j < C * kWarps fetches pair j; the
+// warp reductions give every lane the same m and l.
+__device__ __forceinline__ void cluster_row_stats(const float *stat, uint32_t C, int lane, float &m, float &l)
+{
+    float mw = -INFINITY, lw = 0.f;
+    for (int j = lane; j < (int)C * kWarps; j += 32) {
+        const float mj = ld_dsmem_f32(stat + 2 * (j % kWarps), (uint32_t)(j / kWarps));
+        const float lj = ld_dsmem_f32(stat + 2 * (j % kWarps) + 1, (uint32_t)(j / kWarps));
+        if (mj == -INFINITY)
+            continue;
+        if (mw == -INFINITY) {
+            mw = mj;
+            lw = lj;
+        } else {
+            const float mn = fmaxf(mw, mj);
+            lw = lw * exp2f(mw - mn) + lj * exp2f(mj - mn);
+            mw = mn;
+        }
+    }
+    m = warp_max(mw);
+    l = 0.f;
+    if (m == -INFINITY)
+        return;
+    l = __shfl_sync(0xFFFFFFFFu, warp_sum(mw == -INFINITY ? 0.f : lw * exp2f(mw - m)), 0); // one value for all lanes
+}
+
 // MINCTA: CTAs per SM the registers are budgeted for (4: <= 128 registers, 5: <= 96).
 template <int BITS, int D, typename DT, int MINCTA>
 __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeArgs a, const int spw_log2, const int nbuf)
@@ -332,6 +359,8 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     Smem sm = carve<BITS, D>(smem_raw, spw, capw, nbuf);
     const bool all_hot = (BITS == 4) && !(a.tau > 0.f);
     const bool decide = (BITS == 4) && (a.tau > 0.f); // lo planes depend on the row max
+    // byte distance between consecutive block ids in the pools (one block = H heads)
+    const uint32_t bstride = (uint32_t)a.H * G::HM, lstride = (uint32_t)a.H * G::LOB;
 
     if (lane == 0)
         for (int i = 0; i < spw; ++i)
@@ -343,20 +372,42 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     uint64_t *full = sm.full + warp * spw;
     auto scores_of = [&](int ri) { return sm.scores + (((nbuf == 2) ? (ri & 1) : 0) * kWarps + warp) * capw * 32; };
     auto ids_of = [&](int ri) { return sm.ids + ((ri % 3) * kWarps + warp) * 2 * capw; };
-    auto irow_of = [&](int ri) { return sm.irow + ((ri % 3) * kWarps + warp) * IR_N; };
+    auto irow_of = [&](int ri) { return sm.irow + ((ri % 3) * kWarps + warp) * IR_N_FIELDS; };
 
     // ---------------------------------------------------------------- issuing
     // A warp issues the bulk copies of its own stages, `spw` stages ahead of its compute.
-    int iss_sig = 0, iss_k = 0, iss_n = 0;
+    int iss_sig = -1, iss_k = 0, iss_n = 0; // the sequence starts before its first segment
     int seg_len = 0, seg_ri = 0;   // current segment: own stages and row index
     bool seg_v = false;
-    int released = 0;              // rows whose threshold the issuer has received
+    const uint8_t *seg_src = nullptr; // main pool + head offset (+ K part) of the segment's row
+    const uint8_t *seg_lo = nullptr;  // lo pool + head offset of the segment's row
+    const int2 *seg_ids = nullptr;
+    int setup_upto = -1;           // rows 0..setup_upto have their parameters and ids in place
 
+    // Row parameters, validation and the warp's block ids of row ri.
     auto setup_row = [&](int ri) {
-        const RowCtx rc = row_ctx(a, cid + ri * ncl, crank, C, false);
-        const int n = owned(rc.nmy, warp);
-        int32_t *st = irow_of(ri);
-        const int32_t *bt = a.block_table + (int64_t)rc.b * a.max_blocks;
+        const int row = cid + ri * ncl;
+        const int b = row / a.H, h = row - b * a.H;
+        int hist = a.hist_len[b], tail = a.tail_len[b];
+        bool bad = false;
+        if (hist < 0 || hist > a.max_blocks * 16 || (hist & 31)) {
+            bad = true;
+            hist = 0;
+        }
+        if (tail < 0 || tail > 32) {
+            bad = true;
+            tail = 0;
+        }
+        const int ngroups = hist >> 5;
+        int nmy = ngroups > (int)crank ? (ngroups - (int)crank + (int)C - 1) / (int)C : 0;
+        if (nmy > a.cap_groups) {
+            bad = true;
+            nmy = a.cap_groups;
+        }
+        if (bad && warp == 0 && lane == 0)
+            atomicOr(a.status, LOOPKV_DEV_STATE);
+        const int n = owned(nmy, warp);
+        const int32_t *bt = a.block_table + (int64_t)b * a.max_blocks;
         int32_t *ids = ids_of(ri);
         for (int k = lane; k < 2 * n; k += 32) {
             const int g = (int)crank + (warp + (k >> 1) * kWarps) * (int)C;
@@ -367,10 +418,13 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             }
             ids[k] = id;
         }
+        int32_t *st = irow_of(ri);
         if (lane == 0) {
-            st[IR_ROW] = rc.row;
-            st[IR_H] = rc.h;
-            st[IR_OWN] = n;
+            st[IR_ROW] = row;
+            st[IR_B] = b;
+            st[IR_H] = h;
+            st[IR_N] = n;
+            st[IR_TAIL] = (crank == C - 1) ? tail : 0;
             st[IR_VFIRST] = 0;
             st[IR_VISSUED] = 0;
             st[IR_THR] = __float_as_int(NAN);
@@ -379,121 +433,126 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     };
     auto load_segment = [&]() {
         segment(iss_sig, nrows, seg_v, seg_ri);
-        seg_len = irow_of(seg_ri)[IR_OWN];
+        const int32_t *st = irow_of(seg_ri);
+        seg_len = st[IR_N];
+        seg_src = a.main + (size_t)st[IR_H] * G::HM + (seg_v ? G::KB : 0);
+        seg_lo = a.lo + (size_t)st[IR_H] * G::LOB;
+        seg_ids = reinterpret_cast<const int2 *>(ids_of(seg_ri));
     };
-    // lo planes (4-bit sources) of the hot tokens of V stage k of row ri, then arrive
-    auto issue_lo = [&](int ri, int k, int n, float thr2) {
+    // lo planes (4-bit sources, tau > 0) of the hot tokens of V stage k of row ri, then
+    // the arrival that completes the stage's barrier phase
+    auto issue_lo = [&](int ri, int k, int n, int2 id, float thr2) {
         const int32_t *st_row = irow_of(ri);
-        const int h = st_row[IR_H];
-        const int32_t *ids = ids_of(ri);
-        uint8_t *st = ring + (n & smask) * G::STAGE;
+        uint8_t *st = ring + (n & smask) * G::STAGE + 2 * G::VB;
         uint64_t *fb = &full[n & smask];
-        uint32_t mask = 0;
-        if (BITS == 4)
-            mask = all_hot ? 0xFFFFFFFFu : __ballot_sync(0xFFFFFFFFu, scores_of(ri)[k * 32 + lane] >= thr2);
-        if (a.s_bitmap && lane == 0) {
-            const int g = (int)crank + (warp + k * kWarps) * (int)C;
-            a.s_bitmap[(int64_t)st_row[IR_ROW] * a.bitmap_words + g] = mask;
-        }
-        const int64_t b0 = ids[2 * k], b1 = ids[2 * k + 1];
-        const bool full_lo = BITS == 4 && mask == 0xFFFFFFFFu;
-        if (lane == 0) {
-            const uint32_t lo_bytes = full_lo ? 2 * G::LOB : (uint32_t)__popc(mask) * G::ROWV;
-            mbar_arrive_expect_tx(fb, lo_bytes);
-            if (full_lo) {
-                bulk_g2s(st + 2 * G::VB, a.lo + (b0 * a.H + h) * G::LOB, G::LOB, fb);
-                bulk_g2s(st + 2 * G::VB + G::LOB, a.lo + (b1 * a.H + h) * G::LOB, G::LOB, fb);
+        const uint32_t mask = __ballot_sync(0xFFFFFFFFu, scores_of(ri)[k * 32 + lane] >= thr2);
+        const uint8_t *lob = a.lo + (size_t)st_row[IR_H] * G::LOB;
+        if (mask == 0xFFFFFFFFu) {
+            if (lane == 0) {
+                mbar_arrive_expect_tx(fb, 2 * G::LOB);
+                bulk_g2s(st, lob + (uint64_t)(uint32_t)id.x * lstride, G::LOB, fb);
+                bulk_g2s(st + G::LOB, lob + (uint64_t)(uint32_t)id.y * lstride, G::LOB, fb);
             }
+            return;
         }
+        if (lane == 0)
+            mbar_arrive_expect_tx(fb, (uint32_t)__popc(mask) * G::ROWV);
         __syncwarp();
-        if (BITS == 4 && !full_lo && ((mask >> lane) & 1u)) {
+        if ((mask >> lane) & 1u) {
             const int blk = lane >> 4, r = lane & 15;
-            const int64_t bb = blk ? b1 : b0;
-            bulk_g2s(st + 2 * G::VB + blk * G::LOB + r * G::ROWV, a.lo + (bb * a.H + h) * G::LOB + r * G::ROWV,
-                     G::ROWV, fb);
+            const uint32_t bid = (uint32_t)(blk ? id.y : id.x);
+            bulk_g2s(st + blk * G::LOB + r * G::ROWV, lob + (uint64_t)bid * lstride + r * G::ROWV, G::ROWV, fb);
         }
         __syncwarp();
     };
     auto issue_stage = [&](int n) {
-        const int k = iss_k, ri = seg_ri;
-        int32_t *st_row = irow_of(ri);
-        const int h = st_row[IR_H];
-        const int32_t *ids = ids_of(ri);
+        const int k = iss_k;
+        const int2 id = seg_ids[k];
         uint8_t *st = ring + (n & smask) * G::STAGE;
         uint64_t *fb = &full[n & smask];
-        const int64_t b0 = ids[2 * k], b1 = ids[2 * k + 1];
+        const uint8_t *s0 = seg_src + (uint64_t)(uint32_t)id.x * bstride;
+        const uint8_t *s1 = seg_src + (uint64_t)(uint32_t)id.y * bstride;
         if (!seg_v) {
             if (lane == 0) {
                 mbar_arrive_expect_tx(fb, 2 * G::KB);
-                bulk_g2s(st, a.main + (b0 * a.H + h) * G::HM, G::KB, fb);
-                bulk_g2s(st + G::KB, a.main + (b1 * a.H + h) * G::HM, G::KB, fb);
+                bulk_g2s(st, s0, G::KB, fb);
+                bulk_g2s(st + G::KB, s1, G::KB, fb);
             }
-            __syncwarp();
             return;
         }
+        if (!decide) { // the whole V stage now: hi parts, and lo planes of every token (4-bit)
+            if (lane == 0) {
+                mbar_arrive_expect_tx(fb, 2 * G::VB + 2 * G::LOB);
+                bulk_g2s(st, s0, G::VB, fb);
+                bulk_g2s(st + G::VB, s1, G::VB, fb);
+                if (BITS == 4) {
+                    bulk_g2s(st + 2 * G::VB, seg_lo + (uint64_t)(uint32_t)id.x * lstride, G::LOB, fb);
+                    bulk_g2s(st + 2 * G::VB + G::LOB, seg_lo + (uint64_t)(uint32_t)id.y * lstride, G::LOB, fb);
+                }
+            }
+            return;
+        }
+        int32_t *st_row = irow_of(seg_ri);
         if (lane == 0) {
             if (k == 0)
                 st_row[IR_VFIRST] = n;
             st_row[IR_VISSUED] = k + 1;
             mbar_expect_tx(fb, 2 * G::VB);
-            bulk_g2s(st, a.main + (b0 * a.H + h) * G::HM + G::KB, G::VB, fb);
-            bulk_g2s(st + G::VB, a.main + (b1 * a.H + h) * G::HM + G::KB, G::VB, fb);
+            bulk_g2s(st, s0, G::VB, fb);
+            bulk_g2s(st + G::VB, s1, G::VB, fb);
         }
         __syncwarp();
         const float thr2 = __int_as_float(st_row[IR_THR]);
-        if (!decide || !isnan(thr2)) // the lo part needs the row threshold when tau > 0
-            issue_lo(ri, k, n, thr2);
+        if (!isnan(thr2)) // the lo part needs the row threshold
+            issue_lo(seg_ri, k, n, id, thr2);
     };
-    // Issue every stage numbered below `limit` that the sequence allows.  The issuer
-    // state of a row lives in slot (row mod 3), so row r is set up only after row r - 3
-    // has been released (all of its lo copies issued).
+    // Issue every stage numbered below `limit` that the sequence allows.  The K segment
+    // of a row waits until the row is set up (the compute side sets up row r + 1 when it
+    // starts scoring row r, see consume_k).
     auto pump = [&](int limit) {
-        while (iss_n < limit && iss_sig < 2 * nrows) {
+        for (;;) {
             if (iss_k < seg_len) {
+                if (iss_n >= limit)
+                    break;
                 issue_stage(iss_n);
                 ++iss_k;
                 ++iss_n;
                 continue;
             }
             const int nsig = iss_sig + 1;
-            if (nsig < 2 * nrows) {
-                bool nv;
-                int nri;
-                segment(nsig, nrows, nv, nri);
-                if (!nv) {
-                    if (nri - 3 >= released)
-                        break;
-                    setup_row(nri);
-                }
-            }
+            if (nsig >= 2 * nrows)
+                break;
+            bool nv;
+            int nri;
+            segment(nsig, nrows, nv, nri);
+            if (!nv && nri > setup_upto)
+                break;
             iss_sig = nsig;
             iss_k = 0;
-            if (iss_sig < 2 * nrows)
-                load_segment();
+            load_segment();
         }
     };
     // the threshold of row ri is known: finish the V stages issued without their lo part
     auto release_row = [&](int ri, float thr2) {
-        int32_t *st_row = irow_of(ri);
-        const int vfirst = st_row[IR_VFIRST], vissued = st_row[IR_VISSUED];
-        __syncwarp();
-        if (lane == 0)
-            st_row[IR_THR] = __float_as_int(thr2);
-        __syncwarp();
-        if (decide)
+        if (decide) {
+            int32_t *st_row = irow_of(ri);
+            const int vfirst = st_row[IR_VFIRST], vissued = st_row[IR_VISSUED];
+            __syncwarp();
+            if (lane == 0)
+                st_row[IR_THR] = __float_as_int(thr2);
+            __syncwarp();
+            const int2 *ids = reinterpret_cast<const int2 *>(ids_of(ri));
             for (int k = 0; k < vissued; ++k)
-                issue_lo(ri, k, vfirst + k, thr2);
-        released = ri + 1;
+                issue_lo(ri, k, vfirst + k, ids[k], thr2);
+        }
     };
 
     // ---------------------------------------------------------------- compute
     constexpr int SCR = scratch_bytes<D>();
     uint8_t *scr = sm.scr + warp * SCR;
-    uint8_t *awb = scr;                                    // K stage: digit table, 16 bytes per quad
-    const int4 *aw4 = reinterpret_cast<const int4 *>(scr);
-    float4 *wv4 = reinterpret_cast<float4 *>(scr);         // V stage: weights per token and group
+    const uint4 *rec = reinterpret_cast<const uint4 *>(scr); // K stage: digit records, one per quad
+    float4 *wv4 = reinterpret_cast<float4 *>(scr);           // V stage: weights per token and group
     const float *wvf = reinterpret_cast<const float *>(scr);
-    // a lane owns the channel pairs (2*lane + 64j, 2*lane + 1 + 64j), j < D/64
     const float vscale = 6.490371073168535e32f; // 2^(149 - kVScaleExp) = 2^109
     int prc_n = 0;
     bool timed_out = false; // after one bounded wait gives up, later waits are skipped
@@ -504,91 +563,135 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
 
     // K pass of the warp's groups of row ri; per-warp (max, sum) into stat.
     auto consume_k = [&](int ri) {
-        const RowCtx rc = row_ctx(a, cid + ri * ncl, crank, C, warp == 0 && lane == 0);
+        // Set up row ri + 1 (and row 0 first).  Its slot (ri + 1) mod 3 last held row
+        // ri - 2, whose values were read and whose lo copies were all issued in the
+        // previous iteration, so nothing reads that slot any more.
+        for (int r = ri == 0 ? 0 : ri + 1; r <= ri + 1 && r < nrows; ++r) {
+            setup_row(r);
+            setup_upto = r;
+        }
+        const int32_t *srow = irow_of(ri);
+        const int row = srow[IR_ROW], nown = srow[IR_N], tail = srow[IR_TAIL];
         float *sc = scores_of(ri);
-        const DT *qrow = reinterpret_cast<const DT *>(a.q) + (int64_t)rc.row * D;
-        float qreg[D / 32];
+        // lane owns the channel quad 4*lane .. 4*lane+3 (lanes >= D/4 own none)
+        const bool ownq = lane < G::NQ;
+        float qreg[4];
+        {
+            const DT *qrow = reinterpret_cast<const DT *>(a.q) + (int64_t)row * D + 4 * lane;
 #pragma unroll
-        for (int k = 0; k < D / 32; ++k)
-            qreg[k] = to_f32(qrow[2 * lane + 64 * (k >> 1) + (k & 1)]) * a.qscale;
+            for (int i = 0; i < 4; ++i)
+                qreg[i] = ownq ? to_f32(qrow[i]) * a.qscale : 0.f;
+        }
         float mx = -INFINITY;
-        const int nown = owned(rc.nmy, warp);
         for (int k = 0; k < nown; ++k) {
             const int n = prc_n++;
             if (iss_n < n + spw)
                 pump(n + spw);
             wait_stage(n);
             const uint8_t *st = ring + (n & smask) * G::STAGE;
-            const __half2 *ksc = reinterpret_cast<const __half2 *>(st + G::KCODES);        // even: scales
-            const __half2 *kzp = reinterpret_cast<const __half2 *>(st + G::KB + G::KCODES); // odd: zeros
-            float av[D / 32];
-            float zs = 0.f, amax = 0.f;
+            // the lane's code words (two tokens, one channel half), loaded before the digit
+            // build so that their latency overlaps it
+            const int hf = lane >> 4;
+            constexpr int HW = G::WORDSK / 2; // code words per channel half
+            const uint8_t *krA = st + (lane & 15) * G::ROWK + hf * (G::ROWK / 2);
+            const uint8_t *krB = krA + G::KB;
+            uint32_t cwA[HW], cwB[HW];
 #pragma unroll
-            for (int j = 0; j < D / 64; ++j) {
-                const float2 sv = __half22float2(ksc[lane + 32 * j]);
-                const float2 zv = __half22float2(kzp[lane + 32 * j]);
-                av[2 * j] = qreg[2 * j] * sv.x;
-                av[2 * j + 1] = qreg[2 * j + 1] * sv.y;
-                zs = fmaf(qreg[2 * j], zv.x, zs);
-                zs = fmaf(qreg[2 * j + 1], zv.y, zs);
-                amax = fmaxf(amax, fmaxf(fabsf(av[2 * j]), fabsf(av[2 * j + 1])));
+            for (int w = 0; w < HW; w += (HW % 4 == 0 ? 4 : 2)) {
+                if (HW % 4 == 0) {
+                    const uint4 ca = *reinterpret_cast<const uint4 *>(krA + 4 * w);
+                    const uint4 cb = *reinterpret_cast<const uint4 *>(krB + 4 * w);
+                    cwA[w] = ca.x, cwA[w + 1] = ca.y, cwA[w + 2] = ca.z, cwA[w + 3] = ca.w;
+                    cwB[w] = cb.x, cwB[w + 1] = cb.y, cwB[w + 2] = cb.z, cwB[w + 3] = cb.w;
+                } else {
+                    const uint2 ca = *reinterpret_cast<const uint2 *>(krA + 4 * w);
+                    const uint2 cb = *reinterpret_cast<const uint2 *>(krB + 4 * w);
+                    cwA[w] = ca.x, cwA[w + 1] = ca.y;
+                    cwB[w] = cb.x, cwB[w + 1] = cb.y;
+                }
             }
+            // factors a_c = q_c s_c of the lane's quad and the zero term sum_c q_c z_c
+            float av[4], zs = 0.f;
+            {
+                uint2 sr = make_uint2(0u, 0u), zr = make_uint2(0u, 0u);
+                if (ownq) {
+                    sr = *reinterpret_cast<const uint2 *>(st + G::KCODES + 8 * lane);          // scales (even block)
+                    zr = *reinterpret_cast<const uint2 *>(st + G::KB + G::KCODES + 8 * lane); // zeros (odd block)
+                }
+                const float2 s01 = __half22float2(*reinterpret_cast<const __half2 *>(&sr.x));
+                const float2 s23 = __half22float2(*reinterpret_cast<const __half2 *>(&sr.y));
+                const float2 z01 = __half22float2(*reinterpret_cast<const __half2 *>(&zr.x));
+                const float2 z23 = __half22float2(*reinterpret_cast<const __half2 *>(&zr.y));
+                av[0] = qreg[0] * s01.x;
+                av[1] = qreg[1] * s01.y;
+                av[2] = qreg[2] * s23.x;
+                av[3] = qreg[3] * s23.y;
+                zs = fmaf(qreg[0], z01.x, fmaf(qreg[1], z01.y, fmaf(qreg[2], z23.x, qreg[3] * z23.y)));
+            }
+            const float amax = warp_max_abs(fmaxf(fmaxf(fabsf(av[0]), fabsf(av[1])), fmaxf(fabsf(av[2]), fabsf(av[3]))));
             zs = warp_sum(zs);
-            amax = warp_max(amax);
-            // Fixed point: I_c = round(a_c * 2^F) with F = 21 - E (E = exponent of max |a|),
-            // so |I_c| <= 2^22; balanced base-256 digits d0 + 256 d1 + 65536 d2, |d2| <= 65.
-            const uint32_t abits = __float_as_uint(amax);
-            const int E = abits >= 0x00800000u ? (int)(abits >> 23) - 127 : -126;
-            const int F = 21 - E;
-            const bool fast = F >= -126 && F <= 127 && E - 21 >= -126;
-            const float fs = fast ? __int_as_float((F + 127) << 23) : 0.f;
-#pragma unroll
-            for (int c4 = 0; c4 < D / 32; ++c4) {
-                const int c = 2 * lane + 64 * (c4 >> 1) + (c4 & 1);
-                const float x = fast ? av[c4] * fs : mul_pow2(av[c4], F);
-                const int I = __float2int_rn(x);
-                const int d0 = (I << 24) >> 24;
-                const int I1 = (I - d0) >> 8;
-                const int d1 = (I1 << 24) >> 24;
-                const int d2 = (I1 - d1) >> 8;
-                uint8_t *q = awb + (c >> 2) * 16 + (c & 3);
-                q[0] = (uint8_t)d0;
-                q[4] = (uint8_t)d1;
-                q[8] = (uint8_t)d2;
+            // I_c = round(a_c 2^F), F = 21 - E (E = exponent of max |a|), so |I_c| < 2^22
+            // (one less when the rounding of the largest could reach 2^22); F is capped so
+            // that 2^F and 2^-F stay normal.
+            const uint32_t ab = __float_as_uint(amax);
+            int F = 21 - ((int)(ab >> 23) - 127) - ((ab & 0x7FFFFFu) >= 0x7FFFFEu ? 1 : 0);
+            F = F > 126 ? 126 : F;
+            const float fs = __int_as_float((F + 127) << 23), fsi = __int_as_float((127 - F) << 23);
+            if (ownq) {
+                // low 23 bits of y = I + 2^22: bytes b0, b1 and b2 < 128
+                const uint32_t y0 = __float_as_uint(fmaf(av[0], fs, 12582912.f));
+                const uint32_t y1 = __float_as_uint(fmaf(av[1], fs, 12582912.f));
+                const uint32_t y2 = __float_as_uint(fmaf(av[2], fs, 12582912.f));
+                const uint32_t y3 = __float_as_uint(fmaf(av[3], fs, 12582912.f));
+                const uint32_t t01 = __byte_perm(y0, y1, 0x5140), t23 = __byte_perm(y2, y3, 0x5140);
+                const uint32_t u01 = __byte_perm(y0, y1, 0x0062), u23 = __byte_perm(y2, y3, 0x0062);
+                const uint32_t d0 = __byte_perm(t01, t23, 0x5410), d1 = __byte_perm(t01, t23, 0x7632);
+                // top digit b2 - 64 as a signed byte: flip bit 6, copy the new bit 6 into bit 7
+                const uint32_t x2 = __byte_perm(u01, u23, 0x5410) ^ 0x40404040u;
+                const uint32_t d2 = x2 | ((x2 & 0x40404040u) << 1);
+                reinterpret_cast<uint4 *>(scr)[lane] = make_uint4(d0, d1, d2, 0u);
             }
             __syncwarp();
-            const uint32_t *kr =
-                reinterpret_cast<const uint32_t *>(st + (lane >> 4) * G::KB + (lane & 15) * G::ROWK);
-            int acc[2][3] = {{0, 0, 0}, {0, 0, 0}};
+            // Lane L sums channel half hf = L / 16 of tokens tA = L % 16 (block 0) and
+            // tB = tA + 16 (block 1); both share every digit-record load.  The halves are
+            // then exchanged so that lane L ends with the whole dot product of token L.
             constexpr int QPW = BITS == 4 ? 2 : 4; // quads per code word
+            const uint4 *rh = rec + hf * (G::NQ / 2);
+            KeyAcc accA = {{0u, 0u}, {0u, 0u}, {0, 0}}, accB = {{0u, 0u}, {0u, 0u}, {0, 0}};
 #pragma unroll
-            for (int w4 = 0; w4 < G::WORDSK / 4; ++w4) {
-                const uint4 cw = reinterpret_cast<const uint4 *>(kr)[w4];
-                key_word<BITS>(cw.x, aw4 + QPW * (4 * w4 + 0), acc);
-                key_word<BITS>(cw.y, aw4 + QPW * (4 * w4 + 1), acc);
-                key_word<BITS>(cw.z, aw4 + QPW * (4 * w4 + 2), acc);
-                key_word<BITS>(cw.w, aw4 + QPW * (4 * w4 + 3), acc);
-            }
-            const float dot = fmaf((float)(acc[0][2] + acc[1][2]), 65536.f,
-                                   fmaf((float)(acc[0][1] + acc[1][1]), 256.f, (float)(acc[0][0] + acc[1][0])));
-            const float s2 = (fast ? dot * __int_as_float((127 - F) << 23) : mul_pow2(dot, -F)) + zs;
+            for (int w = 0; w < HW; ++w)
+                key_word2<BITS>(cwA[w], cwB[w], rh + QPW * w, accA, accB);
+            // per token and half: A01 = sum of d0 terms + 256 * sum of d1 terms (< 2^30),
+            // A2 = sum of d2 terms; both exact in 32-bit integers
+            const uint32_t a01A = accA.a0[0] + accA.a0[1] + ((accA.a1[0] + accA.a1[1]) << 8);
+            const uint32_t a01B = accB.a0[0] + accB.a0[1] + ((accB.a1[0] + accB.a1[1]) << 8);
+            const int a2A = accA.a2[0] + accA.a2[1], a2B = accB.a2[0] + accB.a2[1];
+            // lane L keeps token L: half 0 keeps A and sends B, half 1 keeps B and sends A
+            const uint32_t a01 = (hf ? a01B : a01A) + __shfl_xor_sync(0xFFFFFFFFu, hf ? a01A : a01B, 16);
+            const int a2 = (hf ? a2B : a2A) + __shfl_xor_sync(0xFFFFFFFFu, hf ? a2A : a2B, 16);
+            // sum_c code_c I_c = A01 + 65536 A2 (A01 < 2^31); one rounding when they are added
+            const float dot = fmaf((float)a2, 65536.f, (float)a01);
+            const float s2 = fmaf(dot, fsi, zs);
             sc[k * 32 + lane] = s2;
             mx = fmaxf(mx, s2);
             __syncwarp();
         }
         float *tsc = sm.tscores + (ri & 1) * 32;
-        if (rc.tail_cta && warp == kWarps - 1) { // tail keys, exact; lane = tail token
-            const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)rc.b * 2 * a.H + rc.h) * 32 * D;
+        if (tail > 0 && warp == kWarps - 1) { // tail keys, exact; lane = tail token
+            const int b = srow[IR_B], h = srow[IR_H];
+            const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)b * 2 * a.H + h) * 32 * D;
             float s2 = 0.f;
+            for (int q4 = 0; q4 < G::NQ; ++q4) {
+                float kv[4] = {0.f, 0.f, 0.f, 0.f};
+                if (lane < tail)
 #pragma unroll
-            for (int c4 = 0; c4 < D / 32; ++c4)
-                for (int l = 0; l < 32; ++l) {
-                    const float qc = __shfl_sync(0xFFFFFFFFu, qreg[c4], l);
-                    const int c = 2 * l + 64 * (c4 >> 1) + (c4 & 1);
-                    if (lane < rc.tail)
-                        s2 = fmaf(qc, to_f32(kt[(int64_t)lane * D + c]), s2);
-                }
-            if (lane < rc.tail) {
+                    for (int i = 0; i < 4; ++i)
+                        kv[i] = to_f32(kt[(int64_t)lane * D + 4 * q4 + i]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    s2 = fmaf(__shfl_sync(0xFFFFFFFFu, qreg[i], q4), kv[i], s2);
+            }
+            if (lane < tail) {
                 tsc[lane] = s2;
                 mx = fmaxf(mx, s2);
             }
@@ -598,7 +701,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         if (a.tau_mode == LOOPKV_TAU_ABS_PROB && mx != -INFINITY) {
             for (int k = 0; k < nown; ++k)
                 ls += exp2f(sc[k * 32 + lane] - mx);
-            if (rc.tail_cta && warp == kWarps - 1 && lane < rc.tail)
+            if (tail > 0 && warp == kWarps - 1 && lane < tail)
                 ls += exp2f(tsc[lane] - mx);
             ls = warp_sum(ls);
         }
@@ -611,7 +714,8 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
 
     // V pass of the warp's groups of row ri, then the CTA partial (o, l) into part.
     auto consume_v = [&](int ri, float m2, float thr2) {
-        const RowCtx rc = row_ctx(a, cid + ri * ncl, crank, C, false);
+        const int32_t *srow = irow_of(ri);
+        const int nown = srow[IR_N], tail = srow[IR_TAIL];
         const float *sc = scores_of(ri);
         const int cg = lane % G::NCG, ts = lane / G::NCG;
         float2 acc[2][2][4];
@@ -627,7 +731,6 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         for (int j = 0; j < G::NCG; ++j)
             zl[j] = 0.f;
         float lsum = 0.f;
-        const int nown = owned(rc.nmy, warp);
         for (int k = 0; k < nown; ++k) {
             const int n = prc_n++;
             if (iss_n < n + spw)
@@ -636,22 +739,49 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             const float wl = exp2f(s2l - m2);
             const bool hotl = all_hot || (BITS == 4 && s2l >= thr2);
             const uint32_t hotmask = __ballot_sync(0xFFFFFFFFu, hotl);
+            if (a.s_bitmap && lane == 0) {
+                const int g = (int)crank + (warp + k * kWarps) * (int)C;
+                a.s_bitmap[(int64_t)srow[IR_ROW] * a.bitmap_words + g] = hotmask;
+            }
             lsum += wl;
             wait_stage(n);
             const uint8_t *st = ring + (n & smask) * G::STAGE;
+            // the lane's plane words of its 32 / TPI tokens, loaded before the weight build so
+            // that their latency overlaps it (lo words only where they were copied)
+            uint2 hwv[32 / G::TPI], lwv[32 / G::TPI];
+#pragma unroll
+            for (int u = 0; u < 32 / G::TPI; ++u) {
+                const int t = u * G::TPI + ts;
+                const int blk = t >> 4, r = t & 15;
+                hwv[u] = *reinterpret_cast<const uint2 *>(st + blk * G::VB + G::VMETA + r * G::ROWV + cg * 8);
+                lwv[u] = make_uint2(0u, 0u);
+                if (BITS == 4 && (all_hot || ((hotmask >> t) & 1u)))
+                    lwv[u] = *reinterpret_cast<const uint2 *>(st + 2 * G::VB + blk * G::LOB + r * G::ROWV + cg * 8);
+            }
             {   // token `lane`: fold its value scales and zeros into the weight and a running sum
                 const uint8_t *mrow = st + (lane >> 4) * G::VB + (lane & 15) * G::NCG * 4;
                 float wsc[4];
+                uint32_t mw[4];
+                if (G::NCG == 4) {
+                    const uint4 m4 = *reinterpret_cast<const uint4 *>(mrow);
+                    mw[0] = m4.x;
+                    mw[1] = m4.y;
+                    mw[2] = m4.z;
+                    mw[3] = m4.w;
+                } else {
+                    const uint2 m2w = *reinterpret_cast<const uint2 *>(mrow);
+                    mw[0] = m2w.x;
+                    mw[1] = m2w.y;
+                }
+                const float wls = wl * (BITS == 4 ? vscale : 0.25f * vscale);
 #pragma unroll
                 for (int j = 0; j < G::NCG; ++j) {
-                    const float2 m = __half22float2(reinterpret_cast<const __half2 *>(mrow)[j]); // (scale, zero)
-                    if (BITS == 4) {
+                    const float2 m = __half22float2(*reinterpret_cast<const __half2 *>(&mw[j])); // (scale, zero)
+                    if (BITS == 4)
                         zl[j] = fmaf(wl, hotl ? m.y : fmaf(1.5f, m.x, m.y), zl[j]);
-                        wsc[j] = wl * m.x * vscale;
-                    } else {
+                    else
                         zl[j] = fmaf(wl, m.y, zl[j]);
-                        wsc[j] = wl * m.x * (0.25f * vscale);
-                    }
+                    wsc[j] = wls * m.x;
                 }
                 if (G::NCG == 4)
                     wv4[lane] = make_float4(wsc[0], wsc[1], wsc[2], wsc[3]);
@@ -661,63 +791,70 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             __syncwarp();
 #pragma unroll
             for (int u = 0; u < 32 / G::TPI; ++u) {
-                const int t = u * G::TPI + ts;
-                const float Wp = wvf[t * G::NCG + cg];
-                const bool hot = (hotmask >> t) & 1u;
-                const int blk = t >> 4, r = t & 15;
-                const uint2 hw =
-                    *reinterpret_cast<const uint2 *>(st + blk * G::VB + G::VMETA + r * G::ROWV + cg * 8);
-                uint2 lw = make_uint2(0u, 0u);
-                if (BITS == 4 && hot)
-                    lw = *reinterpret_cast<const uint2 *>(st + 2 * G::VB + blk * G::LOB + r * G::ROWV + cg * 8);
-                value_word(hw.x, lw.x, Wp, acc[0]);
-                value_word(hw.y, lw.y, Wp, acc[1]);
+                const float Wp = wvf[(u * G::TPI + ts) * G::NCG + cg];
+                value_word(hwv[u].x, lwv[u].x, Wp, acc[0]);
+                value_word(hwv[u].y, lwv[u].y, Wp, acc[1]);
             }
             __syncwarp();
         }
-        // reduce over the token slots of the warp (lanes with the same cg)
+        // Reduce over the token slots of the warp (lanes with the same cg), scattering the
+        // 32 accumulators of a channel group over its 32 / NCG lanes: after the steps lane
+        // (ts, cg) holds elements NCG*ts + j, j < NCG.
+        float v[32];
 #pragma unroll
-        for (int off = G::NCG; off < 32; off <<= 1) {
+        for (int k = 0; k < 2; ++k)
 #pragma unroll
-            for (int k = 0; k < 2; ++k)
+            for (int e = 0; e < 2; ++e)
 #pragma unroll
-                for (int e = 0; e < 2; ++e)
+                for (int n = 0; n < 4; ++n) {
+                    v[16 * k + 8 * e + 2 * n] = acc[k][e][n].x;
+                    v[16 * k + 8 * e + 2 * n + 1] = acc[k][e][n].y;
+                }
 #pragma unroll
-                    for (int n = 0; n < 4; ++n) {
-                        acc[k][e][n].x += __shfl_xor_sync(0xFFFFFFFFu, acc[k][e][n].x, off);
-                        acc[k][e][n].y += __shfl_xor_sync(0xFFFFFFFFu, acc[k][e][n].y, off);
-                    }
+        for (int s = 0; (16 >> s) >= G::NCG; ++s) {
+            const int off = 16 >> s, half = 16 >> s;
+            const bool up = (lane & off) != 0;
+#pragma unroll
+            for (int j = 0; j < half; ++j) {
+                const float send = up ? v[j] : v[j + half];
+                const float keep = up ? v[j + half] : v[j];
+                v[j] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, off);
+            }
         }
-        float zacc = 0.f;
+        // zero terms: lane ends with the sum over the warp of zl[cg]
 #pragma unroll
-        for (int j = 0; j < G::NCG; ++j) {
-            const float z = warp_sum(zl[j]);
-            if (cg == j)
-                zacc = z;
+        for (int s = 0; (1 << s) < G::NCG; ++s) {
+            const int off = 1 << s, len = G::NCG >> (s + 1);
+            const bool up = (lane & off) != 0;
+#pragma unroll
+            for (int m = 0; m < len; ++m) {
+                const float send = up ? zl[2 * m] : zl[2 * m + 1];
+                const float keep = up ? zl[2 * m + 1] : zl[2 * m];
+                zl[m] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, off);
+            }
         }
+        float zacc = zl[0];
+#pragma unroll
+        for (int off = G::NCG; off < 32; off <<= 1)
+            zacc += __shfl_xor_sync(0xFFFFFFFFu, zacc, off);
         lsum = warp_sum(lsum);
         __syncwarp();
         float *red = reinterpret_cast<float *>(scr); // end of the V pass: the warp's partial o, l
-        if (lane < G::NCG) {
 #pragma unroll
-            for (int k = 0; k < 2; ++k)
-#pragma unroll
-                for (int e = 0; e < 2; ++e)
-#pragma unroll
-                    for (int n = 0; n < 8; ++n) {
-                        const float v = (n & 1) ? acc[k][e][n >> 1].y : acc[k][e][n >> 1].x;
-                        const int ch = 32 * cg + 16 * k + value_channel(e, n);
-                        red[ch] = mul_pow2(v, kVScaleExp - value_pos(n)) + zacc;
-                    }
+        for (int j = 0; j < G::NCG; ++j) {
+            const int i = G::NCG * ts + j;
+            const float f = __int_as_float((127 + kVScaleExp - value_pos(i)) << 23);
+            red[32 * cg + value_channel(i)] = fmaf(v[j], f, zacc);
         }
         if (lane == 0)
             red[D] = lsum;
         __syncwarp();
-        if (rc.tail_cta && warp == kWarps - 1) { // tail values, exact
+        if (tail > 0 && warp == kWarps - 1) { // tail values, exact
+            const int b = srow[IR_B], h = srow[IR_H];
             const float *tsc = sm.tscores + (ri & 1) * 32;
-            const DT *vt0 = reinterpret_cast<const DT *>(a.tail) + ((int64_t)(rc.b * 2 + 1) * a.H + rc.h) * 32 * D;
+            const DT *vt0 = reinterpret_cast<const DT *>(a.tail) + ((int64_t)(b * 2 + 1) * a.H + h) * 32 * D;
             float tl = 0.f;
-            for (int t = 0; t < rc.tail; ++t) {
+            for (int t = 0; t < tail; ++t) {
                 const float w = exp2f(tsc[t] - m2);
                 tl += w;
                 const DT *vt = vt0 + (int64_t)t * D;
@@ -741,14 +878,14 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         named_sync(1, kThreads); // every warp's scratch is free again
     };
 
-    // CTA `crank` writes channels [crank*D/C, (crank+1)*D/C) of row ri, summing the
-    // partials of every CTA of the cluster.
+    // CTA `crank` writes channels [crank*per, min(D, (crank+1)*per)) of row ri, per =
+    // ceil(D / C), summing the partials of every CTA of the cluster.
     auto merge = [&](int ri, float m2) {
         const int row = cid + ri * ncl;
         const float *part = sm.part + (ri & 1) * (D + 1);
-        const int per = D / (int)C;
-        if ((int)threadIdx.x < per) {
-            const int c = (int)crank * per + (int)threadIdx.x;
+        const int per = (D + (int)C - 1) / (int)C;
+        const int c = (int)crank * per + (int)threadIdx.x;
+        if ((int)threadIdx.x < per && c < D) {
             float o = 0.f, l = 0.f;
             for (uint32_t r = 0; r < C; ++r) {
                 o += ld_dsmem_f32(part + c, r);
@@ -769,40 +906,33 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         }
     };
 
-    float m_prev = 0.f, m_prev2 = 0.f;
-    if (nrows > 0) {
-        setup_row(0);
-        load_segment();
-        pump(spw);
-        consume_k(0);
+    auto row_threshold = [&](float m, float l) {
+        if (!decide)
+            return -INFINITY;
+        return a.tau_mode == LOOPKV_TAU_ABS_PROB ? m + log2f(a.tau * l) : m + log2f(a.tau);
+    };
+
+    // Iteration i scores row i and reads the values of row i - 1; each phase has a single
+    // call site (keeps the kernel's code small).  Barrier i publishes the maxima of row i
+    // and the partials of row i - 1.
+    float m_prev = 0.f;
+    for (int i = 0; i <= nrows; ++i) {
+        if (i < nrows)
+            consume_k(i);
+        if (i > 0) {
+            cluster_wait(); // barrier i - 1: maxima of row i - 1, partials of row i - 2
+            if (i >= 2)
+                merge(i - 2, m_prev);
+            float m2, l2;
+            cluster_row_stats(sm.stat + ((i - 1) % 3) * kWarps * 2, C, lane, m2, l2);
+            const float thr2 = row_threshold(m2, l2);
+            release_row(i - 1, thr2);
+            consume_v(i - 1, m2, thr2);
+            m_prev = m2;
+        }
+        cluster_arrive(); // barrier i
     }
-    cluster_arrive(); // row 0
-    for (int i = 1; i < nrows; ++i) {
-        consume_k(i);
-        cluster_wait(); // row i - 1: maxima of row i - 1, partials of row i - 2
-        if (i >= 2)
-            merge(i - 2, m_prev2);
-        float m2, l2;
-        cluster_row_stats(sm.stat + ((i - 1) % 3) * kWarps * 2, C, m2, l2);
-        const float thr2 = row_threshold(a, m2, l2, decide);
-        release_row(i - 1, thr2);
-        consume_v(i - 1, m2, thr2);
-        m_prev2 = m2;
-        cluster_arrive(); // row i
-    }
-    cluster_wait(); // last row
-    if (nrows >= 2)
-        merge(nrows - 2, m_prev2);
-    if (nrows > 0) {
-        float m2, l2;
-        cluster_row_stats(sm.stat + ((nrows - 1) % 3) * kWarps * 2, C, m2, l2);
-        const float thr2 = row_threshold(a, m2, l2, decide);
-        release_row(nrows - 1, thr2);
-        consume_v(nrows - 1, m2, thr2);
-        m_prev = m2;
-    }
-    cluster_arrive(); // partials of the last row
-    cluster_wait();
+    cluster_wait(); // partials of the last row
     if (nrows > 0)
         merge(nrows - 1, m_prev);
     cluster_arrive(); // remote reads done
@@ -884,10 +1014,8 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
     for (int want_ctas = 4; want_ctas <= 5; ++want_ctas) {
     if (env_o && atoi(env_o) != want_ctas)
         continue;
-    for (int C = 1; C <= 16; C *= 2) {
+    for (int C = 1; C <= 16; C = C < 8 ? C + 1 : 2 * C) { // 1..8, 16
         if (env_c && atoi(env_c) != C)
-            continue;
-        if (D / C < 4)
             continue;
         const int cap = (max_groups + C - 1) / C;
         const int capw = (cap + kWarps - 1) / kWarps;

@@ -37,9 +37,11 @@ __device__ __forceinline__ void fence_mbar_init()
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
+// Relaxed: the arriving thread publishes no data of its own through the barrier (the
+// bytes are written by the bulk copies that complete on it), so no release fence.
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t tx)
 {
-    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+    asm volatile("mbarrier.arrive.expect_tx.relaxed.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
                  "r"(tx)
                  : "memory");
 }
