@@ -55,6 +55,7 @@ namespace {
 constexpr int kWarps = 4; // every warp both issues the copies of its stages and computes on them
 constexpr int kThreads = kWarps * 32;
 constexpr int kVScaleExp = 40; // V accumulators hold code * w * s * 2^(p - 40)
+constexpr int kGPS = 2;        // 32-token groups per pipeline stage (one barrier, one slot)
 
 template <int BITS, int D> struct Geo {
     static constexpr int KCODES = BITS == 4 ? 16 * D / 2 : 16 * D / 4;
@@ -67,7 +68,8 @@ template <int BITS, int D> struct Geo {
     static constexpr int VB = VMETA + VPLANE;                   // V meta + hi part
     static constexpr int KSTAGE = 2 * KB;
     static constexpr int VSTAGE = 2 * VB + 2 * LOB;
-    static constexpr int STAGE = ((KSTAGE > VSTAGE ? KSTAGE : VSTAGE) + 127) / 128 * 128;
+    static constexpr int GSLOT = ((KSTAGE > VSTAGE ? KSTAGE : VSTAGE) + 127) / 128 * 128; // one group
+    static constexpr int STAGE = kGPS * GSLOT;
     static constexpr int ROWK = KCODES / 16;  // key bytes per token
     static constexpr int WORDSK = ROWK / 4;
     static constexpr int ROWV = D / 4;        // value plane bytes per token
@@ -203,7 +205,7 @@ __host__ __device__ constexpr int value_pos(int i)
 }
 
 struct Smem {
-    uint8_t *ring;     // [kWarps][spw][STAGE] stage slots, a private slice per warp
+    uint8_t *ring;     // [kWarps][spw][STAGE] stage slots (kGPS groups each), a private slice per warp
     uint64_t *full;    // [kWarps][spw] completion barriers of the slots
     float *scores;     // [nbuf][kWarps][capw * 32] scores of a warp's groups, by row parity
     float *tscores;    // [2][32] tail scores, by row parity
@@ -292,7 +294,7 @@ template <int BITS, int D> bool layout_ok(int spw, int capw, int nbuf)
             return false;
         prev = o;
     }
-    return (Geo<BITS, D>::STAGE % 128) == 0 && L.total >= prev && (spw & (spw - 1)) == 0 &&
+    return (Geo<BITS, D>::GSLOT % 128) == 0 && L.total >= prev && (spw & (spw - 1)) == 0 &&
            scratch_bytes<D>() >= (D / 4) * 16 && scratch_bytes<D>() >= (D + 1) * 4 &&
            scratch_bytes<D>() >= 32 * (D / 32) * 4 && (2 * capw * 4) % 8 == 0;
 }
@@ -378,6 +380,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     // A warp issues the bulk copies of its own stages, `spw` stages ahead of its compute.
     int iss_sig = -1, iss_k = 0, iss_n = 0; // the sequence starts before its first segment
     int seg_len = 0, seg_ri = 0;   // current segment: own stages and row index
+    int seg_n = 0;                 // groups of the segment's row owned by this warp
     bool seg_v = false;
     const uint8_t *seg_src = nullptr; // main pool + head offset (+ K part) of the segment's row
     const uint8_t *seg_lo = nullptr;  // lo pool + head offset of the segment's row
@@ -434,77 +437,102 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     auto load_segment = [&]() {
         segment(iss_sig, nrows, seg_v, seg_ri);
         const int32_t *st = irow_of(seg_ri);
-        seg_len = st[IR_N];
+        seg_n = st[IR_N];
+        seg_len = (seg_n + kGPS - 1) / kGPS;
         seg_src = a.main + (size_t)st[IR_H] * G::HM + (seg_v ? G::KB : 0);
         seg_lo = a.lo + (size_t)st[IR_H] * G::LOB;
         seg_ids = reinterpret_cast<const int2 *>(ids_of(seg_ri));
     };
-    // lo planes (4-bit sources, tau > 0) of the hot tokens of V stage k of row ri, then
-    // the arrival that completes the stage's barrier phase
-    auto issue_lo = [&](int ri, int k, int n, int2 id, float thr2) {
+    // lo planes (4-bit sources, tau > 0) of the hot tokens of V stage k2 of row ri, then
+    // the one arrival that completes the stage's barrier phase
+    auto issue_lo = [&](int ri, int k2, int n, float thr2) {
         const int32_t *st_row = irow_of(ri);
-        uint8_t *st = ring + (n & smask) * G::STAGE + 2 * G::VB;
+        const int ng = min(kGPS, st_row[IR_N] - kGPS * k2);
+        uint8_t *stg = ring + (n & smask) * G::STAGE + 2 * G::VB;
         uint64_t *fb = &full[n & smask];
-        const uint32_t mask = __ballot_sync(0xFFFFFFFFu, scores_of(ri)[k * 32 + lane] >= thr2);
         const uint8_t *lob = a.lo + (size_t)st_row[IR_H] * G::LOB;
-        if (mask == 0xFFFFFFFFu) {
-            if (lane == 0) {
-                mbar_arrive_expect_tx(fb, 2 * G::LOB);
-                bulk_g2s(st, lob + (uint64_t)(uint32_t)id.x * lstride, G::LOB, fb);
-                bulk_g2s(st + G::LOB, lob + (uint64_t)(uint32_t)id.y * lstride, G::LOB, fb);
-            }
-            return;
+        const int2 *ids = reinterpret_cast<const int2 *>(ids_of(ri)) + kGPS * k2;
+        const float *sc = scores_of(ri) + kGPS * k2 * 32;
+        uint32_t mask[kGPS];
+        uint32_t bytes = 0;
+#pragma unroll
+        for (int j = 0; j < kGPS; ++j) {
+            mask[j] = j < ng ? __ballot_sync(0xFFFFFFFFu, sc[j * 32 + lane] >= thr2) : 0u;
+            bytes += mask[j] == 0xFFFFFFFFu ? 2 * G::LOB : (uint32_t)__popc(mask[j]) * G::ROWV;
         }
         if (lane == 0)
-            mbar_arrive_expect_tx(fb, (uint32_t)__popc(mask) * G::ROWV);
+            mbar_arrive_expect_tx(fb, bytes);
         __syncwarp();
-        if ((mask >> lane) & 1u) {
-            const int blk = lane >> 4, r = lane & 15;
-            const uint32_t bid = (uint32_t)(blk ? id.y : id.x);
-            bulk_g2s(st + blk * G::LOB + r * G::ROWV, lob + (uint64_t)bid * lstride + r * G::ROWV, G::ROWV, fb);
+#pragma unroll
+        for (int j = 0; j < kGPS; ++j) {
+            if (j >= ng)
+                break;
+            const int2 id = ids[j];
+            uint8_t *st = stg + j * G::GSLOT;
+            if (mask[j] == 0xFFFFFFFFu) {
+                if (lane == 0) {
+                    bulk_g2s(st, lob + (uint64_t)(uint32_t)id.x * lstride, G::LOB, fb);
+                    bulk_g2s(st + G::LOB, lob + (uint64_t)(uint32_t)id.y * lstride, G::LOB, fb);
+                }
+            } else if ((mask[j] >> lane) & 1u) {
+                const int blk = lane >> 4, r = lane & 15;
+                const uint32_t bid = (uint32_t)(blk ? id.y : id.x);
+                bulk_g2s(st + blk * G::LOB + r * G::ROWV, lob + (uint64_t)bid * lstride + r * G::ROWV, G::ROWV, fb);
+            }
         }
         __syncwarp();
     };
+    // Stage k2 of the current segment: groups kGPS*k2 .. kGPS*k2 + ng - 1 of the row, group
+    // j into sub-slot j.
     auto issue_stage = [&](int n) {
-        const int k = iss_k;
-        const int2 id = seg_ids[k];
-        uint8_t *st = ring + (n & smask) * G::STAGE;
+        const int k2 = iss_k;
+        const int ng = min(kGPS, seg_n - kGPS * k2);
+        uint8_t *stg = ring + (n & smask) * G::STAGE;
         uint64_t *fb = &full[n & smask];
-        const uint8_t *s0 = seg_src + (uint64_t)(uint32_t)id.x * bstride;
-        const uint8_t *s1 = seg_src + (uint64_t)(uint32_t)id.y * bstride;
+        const int2 *ids = seg_ids + kGPS * k2;
         if (!seg_v) {
             if (lane == 0) {
-                mbar_arrive_expect_tx(fb, 2 * G::KB);
-                bulk_g2s(st, s0, G::KB, fb);
-                bulk_g2s(st + G::KB, s1, G::KB, fb);
+                mbar_arrive_expect_tx(fb, (uint32_t)ng * 2 * G::KB);
+                for (int j = 0; j < ng; ++j) {
+                    const int2 id = ids[j];
+                    bulk_g2s(stg + j * G::GSLOT, seg_src + (uint64_t)(uint32_t)id.x * bstride, G::KB, fb);
+                    bulk_g2s(stg + j * G::GSLOT + G::KB, seg_src + (uint64_t)(uint32_t)id.y * bstride, G::KB, fb);
+                }
             }
             return;
         }
         if (!decide) { // the whole V stage now: hi parts, and lo planes of every token (4-bit)
             if (lane == 0) {
-                mbar_arrive_expect_tx(fb, 2 * G::VB + 2 * G::LOB);
-                bulk_g2s(st, s0, G::VB, fb);
-                bulk_g2s(st + G::VB, s1, G::VB, fb);
-                if (BITS == 4) {
-                    bulk_g2s(st + 2 * G::VB, seg_lo + (uint64_t)(uint32_t)id.x * lstride, G::LOB, fb);
-                    bulk_g2s(st + 2 * G::VB + G::LOB, seg_lo + (uint64_t)(uint32_t)id.y * lstride, G::LOB, fb);
+                mbar_arrive_expect_tx(fb, (uint32_t)ng * (2 * G::VB + 2 * G::LOB));
+                for (int j = 0; j < ng; ++j) {
+                    const int2 id = ids[j];
+                    uint8_t *st = stg + j * G::GSLOT;
+                    bulk_g2s(st, seg_src + (uint64_t)(uint32_t)id.x * bstride, G::VB, fb);
+                    bulk_g2s(st + G::VB, seg_src + (uint64_t)(uint32_t)id.y * bstride, G::VB, fb);
+                    if (BITS == 4) {
+                        bulk_g2s(st + 2 * G::VB, seg_lo + (uint64_t)(uint32_t)id.x * lstride, G::LOB, fb);
+                        bulk_g2s(st + 2 * G::VB + G::LOB, seg_lo + (uint64_t)(uint32_t)id.y * lstride, G::LOB, fb);
+                    }
                 }
             }
             return;
         }
         int32_t *st_row = irow_of(seg_ri);
         if (lane == 0) {
-            if (k == 0)
+            if (k2 == 0)
                 st_row[IR_VFIRST] = n;
-            st_row[IR_VISSUED] = k + 1;
-            mbar_expect_tx(fb, 2 * G::VB);
-            bulk_g2s(st, s0, G::VB, fb);
-            bulk_g2s(st + G::VB, s1, G::VB, fb);
+            st_row[IR_VISSUED] = k2 + 1;
+            mbar_expect_tx(fb, (uint32_t)ng * 2 * G::VB);
+            for (int j = 0; j < ng; ++j) {
+                const int2 id = ids[j];
+                bulk_g2s(stg + j * G::GSLOT, seg_src + (uint64_t)(uint32_t)id.x * bstride, G::VB, fb);
+                bulk_g2s(stg + j * G::GSLOT + G::VB, seg_src + (uint64_t)(uint32_t)id.y * bstride, G::VB, fb);
+            }
         }
         __syncwarp();
         const float thr2 = __int_as_float(st_row[IR_THR]);
         if (!isnan(thr2)) // the lo part needs the row threshold
-            issue_lo(seg_ri, k, n, id, thr2);
+            issue_lo(seg_ri, k2, n, thr2);
     };
     // Issue every stage numbered below `limit` that the sequence allows.  The K segment
     // of a row waits until the row is set up (the compute side sets up row r + 1 when it
@@ -541,9 +569,8 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             if (lane == 0)
                 st_row[IR_THR] = __float_as_int(thr2);
             __syncwarp();
-            const int2 *ids = reinterpret_cast<const int2 *>(ids_of(ri));
-            for (int k = 0; k < vissued; ++k)
-                issue_lo(ri, k, vfirst + k, ids[k], thr2);
+            for (int k2 = 0; k2 < vissued; ++k2)
+                issue_lo(ri, k2, vfirst + k2, thr2);
         }
     };
 
@@ -583,12 +610,16 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
                 qreg[i] = ownq ? to_f32(qrow[i]) * a.qscale : 0.f;
         }
         float mx = -INFINITY;
+        const uint8_t *stg = ring;
         for (int k = 0; k < nown; ++k) {
-            const int n = prc_n++;
-            if (iss_n < n + spw)
-                pump(n + spw);
-            wait_stage(n);
-            const uint8_t *st = ring + (n & smask) * G::STAGE;
+            if (k % kGPS == 0) { // first group of a stage
+                const int n = prc_n++;
+                if (iss_n < n + spw)
+                    pump(n + spw);
+                wait_stage(n);
+                stg = ring + (n & smask) * G::STAGE;
+            }
+            const uint8_t *st = stg + (k % kGPS) * G::GSLOT;
             // the lane's code words (two tokens, one channel half), loaded before the digit
             // build so that their latency overlaps it
             const int hf = lane >> 4;
@@ -731,10 +762,15 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         for (int j = 0; j < G::NCG; ++j)
             zl[j] = 0.f;
         float lsum = 0.f;
+        const uint8_t *stg = ring;
         for (int k = 0; k < nown; ++k) {
-            const int n = prc_n++;
-            if (iss_n < n + spw)
-                pump(n + spw);
+            const bool first = k % kGPS == 0; // first group of a stage
+            int n = 0;
+            if (first) {
+                n = prc_n++;
+                if (iss_n < n + spw)
+                    pump(n + spw);
+            }
             const float s2l = sc[k * 32 + lane];
             const float wl = exp2f(s2l - m2);
             const bool hotl = all_hot || (BITS == 4 && s2l >= thr2);
@@ -744,8 +780,11 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
                 a.s_bitmap[(int64_t)srow[IR_ROW] * a.bitmap_words + g] = hotmask;
             }
             lsum += wl;
-            wait_stage(n);
-            const uint8_t *st = ring + (n & smask) * G::STAGE;
+            if (first) {
+                wait_stage(n);
+                stg = ring + (n & smask) * G::STAGE;
+            }
+            const uint8_t *st = stg + (k % kGPS) * G::GSLOT;
             // the lane's plane words of its 32 / TPI tokens, loaded before the weight build so
             // that their latency overlaps it (lo words only where they were copied)
             uint2 hwv[32 / G::TPI], lwv[32 / G::TPI];
@@ -994,11 +1033,18 @@ template <int BITS, int D, typename DT> int max_active_clusters(int C, int smem,
     return n;
 }
 
+// Launch shape.  Model: a cluster of C CTAs serves ceil(rows / clusters) rows one after
+// another; a CTA's share of one row costs (groups / C + kRowFixed) group-times, and an SM
+// running n CTAs gives each 1 / max(n, kSaturate) of its throughput.  Time is then
+// rounds * (G / C + kRowFixed) * max(n, kSaturate) with n the CTAs on the busiest SM.
+// Among equal times the deeper ring (more bytes in flight) wins.
+constexpr double kRowFixed = 6.0;  // per-CTA cost of a row outside its groups (setup, merge, bubble)
+constexpr double kSaturate = 3.5;  // CTAs per SM that keep its issue slots busy
+
 template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_blocks)
 {
-    using G = Geo<BITS, D>;
     DecodeShape best = {};
-    double best_eff = -1.0;
+    double best_t = 1e300;
     const int max_groups = max_blocks / 2;
     int sm_count = 148;
     {
@@ -1012,54 +1058,50 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
     const char *env_s = getenv("LOOPKV_DECODE_STAGES");
     const char *env_o = getenv("LOOPKV_DECODE_CTAS_PER_SM");
     for (int want_ctas = 4; want_ctas <= 5; ++want_ctas) {
-    if (env_o && atoi(env_o) != want_ctas)
-        continue;
-    for (int C = 1; C <= 16; C = C < 8 ? C + 1 : 2 * C) { // 1..8, 16
-        if (env_c && atoi(env_c) != C)
+        if (env_o && atoi(env_o) != want_ctas)
             continue;
-        const int cap = (max_groups + C - 1) / C;
-        const int capw = (cap + kWarps - 1) / kWarps;
-        const int budget = smem_per_sm / want_ctas - 1024;
-        for (int nbuf = 1; nbuf <= 2; ++nbuf) {
-            // slots per warp (a power of two): fill the shared memory of `want_ctas` CTAs per SM
-            int spw = 8;
-            while (spw > 2 && smem_bytes<BITS, D>(spw, capw, nbuf) > budget)
-                spw >>= 1;
-            if (env_s)
-                spw = atoi(env_s);
-            const int smem = smem_bytes<BITS, D>(spw, capw, nbuf);
-            if (smem > 227 * 1024 || !layout_ok<BITS, D>(spw, capw, nbuf))
+        for (int C = 1; C <= 16; C = C < 8 ? C + 1 : 2 * C) { // 1..8, 16
+            if (env_c && atoi(env_c) != C)
                 continue;
-            int ncl = max_active_clusters<BITS, D, DT>(C, smem, want_ctas);
-            if (ncl <= 0)
-                continue;
-            if (ncl > rows)
-                ncl = rows;
-            if (nbuf == 1 && ncl < rows)
-                continue; // a cluster would read several rows: it needs two score buffers
-            // balance: each cluster takes ceil(rows / ncl) rows; too few CTAs per SM penalised;
-            // more resident CTAs (warps to hide latency) and deeper rings (bytes in flight)
-            // preferred
-            const double rounds = (double)((rows + ncl - 1) / ncl);
-            const double eff = ((double)rows / ncl) / rounds *
-                               std::min(1.0, (double)(ncl * C) / (3.0 * sm_count)) *
-                               (1.0 + 0.3 * std::min(1.0, (double)(ncl * C) / (want_ctas * sm_count))) *
-                               (1.0 + 0.01 * spw);
-            if (eff > best_eff + 1e-9) {
-                best_eff = eff;
-                best.cluster = C;
-                best.clusters = ncl;
-                best.stages = spw;
-                best.stages_log2 = __builtin_ctz(spw);
-                best.score_bufs = nbuf;
-                best.smem = smem;
-                best.threads = kThreads;
-                best.cap = cap;
-                best.min_ctas = want_ctas;
+            const int cap = (max_groups + C - 1) / C;
+            const int capw = (cap + kWarps - 1) / kWarps;
+            const int budget = smem_per_sm / want_ctas - 1024;
+            for (int nbuf = 1; nbuf <= 2; ++nbuf) {
+                // slots per warp (a power of two): fill the shared memory of `want_ctas` CTAs per SM
+                int spw = 8;
+                while (spw > 2 && smem_bytes<BITS, D>(spw, capw, nbuf) > budget)
+                    spw >>= 1;
+                if (env_s)
+                    spw = atoi(env_s);
+                const int smem = smem_bytes<BITS, D>(spw, capw, nbuf);
+                if (smem > 227 * 1024 || !layout_ok<BITS, D>(spw, capw, nbuf))
+                    continue;
+                int ncl = max_active_clusters<BITS, D, DT>(C, smem, want_ctas);
+                if (ncl <= 0)
+                    continue;
+                if (ncl > rows)
+                    ncl = rows;
+                if (nbuf == 1 && ncl < rows)
+                    continue; // a cluster would read several rows: it needs two score buffers
+                const int rounds = (rows + ncl - 1) / ncl;
+                const int per_sm = (ncl * C + sm_count - 1) / sm_count;
+                const double t = rounds * ((double)max_groups / C + kRowFixed) * std::max((double)per_sm, kSaturate) *
+                                 (1.0 - 0.01 * spw);
+                if (t < best_t * (1.0 - 1e-9)) {
+                    best_t = t;
+                    best.cluster = C;
+                    best.clusters = ncl;
+                    best.stages = spw;
+                    best.stages_log2 = __builtin_ctz(spw);
+                    best.score_bufs = nbuf;
+                    best.smem = smem;
+                    best.threads = kThreads;
+                    best.cap = cap;
+                    best.min_ctas = want_ctas;
+                }
+                break;
             }
-            break;
         }
-    }
     }
     return best;
 }
