@@ -35,11 +35,11 @@
 // signed byte) with byte permutes.  The 4-bit (or 2-bit) codes are unpacked four at a
 // time into bytes with one AND, and dp4a accumulates code * digit in int32 with no
 // rounding.
-// Values: a field masked out of a packed word, read as an fp32 bit pattern x < 2^24, has
-// the value x * 2^-149 exactly (subnormal or smallest-exponent normal numbers);
-// multiplied by a weight pre-scaled with 2^(149 - p) (p = the field's bit position) it
-// gives code * weight with one AND and half a packed FMA per code; fp32 FMA on sm_100a
-// keeps subnormal inputs (no flush to zero).
+// Values: a value-plane word holds 4 tokens x 4 channels (token in the byte).  The hi and
+// lo words merge into 4-bit codes (lo bits of cold tokens masked off), one AND unpacks the
+// codes of one channel for 4 tokens, and dp4a against 8-bit digits of the tokens' 21-bit
+// fixed-point weights w * scale sums code * weight over tokens exactly in int32; each
+// 32-token group's sum is rounded to fp32 once.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -54,7 +54,6 @@ namespace {
 
 constexpr int kWarps = 4; // every warp both issues the copies of its stages and computes on them
 constexpr int kThreads = kWarps * 32;
-constexpr int kVScaleExp = 40; // V accumulators hold code * w * s * 2^(p - 40)
 constexpr int kGPS = 2;        // 32-token groups per pipeline stage (one barrier, one slot)
 
 template <int BITS, int D> struct Geo {
@@ -78,13 +77,6 @@ template <int BITS, int D> struct Geo {
     static constexpr int NQ = D / 4;          // channel quads
 };
 
-__device__ __forceinline__ float fbits(uint32_t x) { return __uint_as_float(x); }
-
-__device__ __forceinline__ void ffma2(float2 &acc, float a, float b, float2 f)
-{
-    acc = __ffma2_rn(make_float2(a, b), f, acc);
-}
-
 // acc += sum of the four unsigned bytes of `u` times the four unsigned bytes of `d`
 __device__ __forceinline__ void dp4a_uu(uint32_t &acc, uint32_t u, uint32_t d)
 {
@@ -95,6 +87,31 @@ __device__ __forceinline__ void dp4a_uu(uint32_t &acc, uint32_t u, uint32_t d)
 __device__ __forceinline__ void dp4a_us(int &acc, uint32_t u, uint32_t d)
 {
     asm("dp4a.u32.s32 %0, %1, %2, %0;" : "+r"(acc) : "r"(u), "r"(d));
+}
+
+// 2^x by the hardware approximation (relative error about 2^-22; tiny results flush to 0)
+__device__ __forceinline__ float ex2(float x)
+{
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// Byte b of the result = 0xFF if bit 8b+7 of x is set, else 0 (prmt's sign-replicating
+// selector values 8..11).
+__device__ __forceinline__ uint32_t byte_signs(uint32_t x)
+{
+    uint32_t r;
+    asm("prmt.b32 %0, %1, 0, 0xBA98;" : "=r"(r) : "r"(x));
+    return r;
+}
+
+// max over the warp of v
+__device__ __forceinline__ float warp_max_f(float v)
+{
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+    return r;
 }
 
 // max over the warp of |v|
@@ -173,45 +190,16 @@ __device__ __forceinline__ void key_word2(uint32_t wa, uint32_t wb, const uint4 
     }
 }
 
-// Value word pair (hi, lo) of 16 channels -> 4-bit codes 4h+l in two nibble words.
-// Field of channel 4i+b sits at bit 8b+2i in both planes.  E holds the channels with
-// even i (nibble at 8b+4m is channel 8m+b), O those with odd i (channel 8m+4+b).
-// With lo = 0 the nibbles are 4h: the cold / 2-bit decode in the same scale domain.
-__device__ __forceinline__ void value_word(uint32_t hi, uint32_t lo, float W, float2 (&acc)[2][4])
-{
-    const uint32_t E = ((hi << 2) & 0xCCCCCCCCu) | (lo & 0x33333333u);
-    const uint32_t O = (hi & 0xCCCCCCCCu) | ((lo >> 2) & 0x33333333u);
-    const uint32_t Eh = E >> 16, Oh = O >> 16;
-    const float2 w2 = make_float2(W, W);
-    ffma2(acc[0][0], fbits(E & 0xFu), fbits(E & 0xF0u), w2);
-    ffma2(acc[0][1], fbits(E & 0xF00u), fbits(E & 0xF000u), w2);
-    ffma2(acc[0][2], fbits(E & 0xF0000u), fbits(E & 0xF00000u), w2);
-    ffma2(acc[0][3], fbits(Eh & 0xF00u), fbits(Eh & 0xF000u), w2);
-    ffma2(acc[1][0], fbits(O & 0xFu), fbits(O & 0xF0u), w2);
-    ffma2(acc[1][1], fbits(O & 0xF00u), fbits(O & 0xF000u), w2);
-    ffma2(acc[1][2], fbits(O & 0xF0000u), fbits(O & 0xF00000u), w2);
-    ffma2(acc[1][3], fbits(Oh & 0xF00u), fbits(Oh & 0xF000u), w2);
-}
-
-// Accumulator element i = 16k + 8e + n (k: 16-channel half, e: E or O word, n: nibble)
-// -> channel offset within the 32-channel group and bit position of its field.
-__host__ __device__ constexpr int value_channel(int i)
-{
-    return 16 * (i >> 4) + 8 * (i & 1) + ((i & 7) >> 1) + 4 * ((i >> 3) & 1);
-}
-__host__ __device__ constexpr int value_pos(int i)
-{
-    return (i & 7) < 6 ? 4 * (i & 7) : ((i & 7) == 6 ? 8 : 12);
-}
-
 struct Smem {
     uint8_t *ring;     // [kWarps][spw][STAGE] stage slots (kGPS groups each), a private slice per warp
     uint64_t *full;    // [kWarps][spw] completion barriers of the slots
     float *scores;     // [nbuf][kWarps][capw * 32] scores of a warp's groups, by row parity
     float *tscores;    // [2][32] tail scores, by row parity
     uint8_t *scr;      // [kWarps][SCR] per-warp scratch, used in turn as: key digit records
-                       // [D/4][16 B] during a K stage, value weights [32][D/32] during a V
-                       // stage, the warp's partial o and l [D + 1] at the end of a V pass
+                       // [D/4][16 B] during a K stage, the fixed-point weight transpose
+                       // [D/32][40 words] (overwritten in place by the value digit records)
+                       // and 2^-F during a V stage, the warp's partial o and l [D + 1] at
+                       // the end of a V pass
     float *stat;       // [3][kWarps][2] per-warp (max, sum exp(s - max)), by row index mod 3
     float *part;       // [2][D + 1] CTA partial o and l of a row, by row parity
     int32_t *ids;      // [3][kWarps][2 * capw] block ids of a warp's groups, by row index mod 3
@@ -232,7 +220,7 @@ __host__ __device__ constexpr int align16(int x) { return (x + 15) & ~15; }
 // Bytes of a warp's scratch: the largest of its three uses.
 template <int D> __host__ __device__ constexpr int scratch_bytes()
 {
-    return align16((D / 4) * 16 > (D + 1) * 4 ? (D / 4) * 16 : (D + 1) * 4);
+    return align16(std::max((D / 4) * 16, std::max((D + 1) * 4, (D / 32) * 40 * 4 + 4)));
 }
 
 // nbuf: score buffers (2 when a cluster reads more than one row, so that the next row's
@@ -296,7 +284,7 @@ template <int BITS, int D> bool layout_ok(int spw, int capw, int nbuf)
     }
     return (Geo<BITS, D>::GSLOT % 128) == 0 && L.total >= prev && (spw & (spw - 1)) == 0 &&
            scratch_bytes<D>() >= (D / 4) * 16 && scratch_bytes<D>() >= (D + 1) * 4 &&
-           scratch_bytes<D>() >= 32 * (D / 32) * 4 && (2 * capw * 4) % 8 == 0;
+           scratch_bytes<D>() >= (D / 32) * 40 * 4 + 4 && (2 * capw * 4) % 8 == 0;
 }
 
 // Groups of a row owned by warp w of the CTA: local groups w, w + kWarps, ...
@@ -444,7 +432,9 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         seg_ids = reinterpret_cast<const int2 *>(ids_of(seg_ri));
     };
     // lo planes (4-bit sources, tau > 0) of the hot tokens of V stage k2 of row ri, then
-    // the one arrival that completes the stage's barrier phase
+    // the one arrival that completes the stage's barrier phase.  The lo plane holds 4
+    // tokens per word, so a 4-token quad with a hot token is copied whole (D bytes); a
+    // group whose 32 tokens are all hot copies both blocks' planes.
     auto issue_lo = [&](int ri, int k2, int n, float thr2) {
         const int32_t *st_row = irow_of(ri);
         const int ng = min(kGPS, st_row[IR_N] - kGPS * k2);
@@ -457,8 +447,13 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         uint32_t bytes = 0;
 #pragma unroll
         for (int j = 0; j < kGPS; ++j) {
-            mask[j] = j < ng ? __ballot_sync(0xFFFFFFFFu, sc[j * 32 + lane] >= thr2) : 0u;
-            bytes += mask[j] == 0xFFFFFFFFu ? 2 * G::LOB : (uint32_t)__popc(mask[j]) * G::ROWV;
+            const uint32_t tm = j < ng ? __ballot_sync(0xFFFFFFFFu, sc[j * 32 + lane] >= thr2) : 0u;
+            uint32_t qm = 0; // bit q: token quad q has a hot token
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                qm |= ((tm >> (4 * q)) & 0xFu) ? 1u << q : 0u;
+            mask[j] = tm == 0xFFFFFFFFu ? 0xFFFFFFFFu : qm;
+            bytes += tm == 0xFFFFFFFFu ? 2 * G::LOB : (uint32_t)__popc(qm) * D;
         }
         if (lane == 0)
             mbar_arrive_expect_tx(fb, bytes);
@@ -474,10 +469,10 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
                     bulk_g2s(st, lob + (uint64_t)(uint32_t)id.x * lstride, G::LOB, fb);
                     bulk_g2s(st + G::LOB, lob + (uint64_t)(uint32_t)id.y * lstride, G::LOB, fb);
                 }
-            } else if ((mask[j] >> lane) & 1u) {
-                const int blk = lane >> 4, r = lane & 15;
+            } else if (lane < 8 && ((mask[j] >> lane) & 1u)) { // lane = token quad
+                const int blk = lane >> 2, tau = lane & 3;
                 const uint32_t bid = (uint32_t)(blk ? id.y : id.x);
-                bulk_g2s(st + blk * G::LOB + r * G::ROWV, lob + (uint64_t)bid * lstride + r * G::ROWV, G::ROWV, fb);
+                bulk_g2s(st + blk * G::LOB + tau * D, lob + (uint64_t)bid * lstride + tau * D, D, fb);
             }
         }
         __syncwarp();
@@ -578,9 +573,6 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     constexpr int SCR = scratch_bytes<D>();
     uint8_t *scr = sm.scr + warp * SCR;
     const uint4 *rec = reinterpret_cast<const uint4 *>(scr); // K stage: digit records, one per quad
-    float4 *wv4 = reinterpret_cast<float4 *>(scr);           // V stage: weights per token and group
-    const float *wvf = reinterpret_cast<const float *>(scr);
-    const float vscale = 6.490371073168535e32f; // 2^(149 - kVScaleExp) = 2^109
     int prc_n = 0;
     bool timed_out = false; // after one bounded wait gives up, later waits are skipped
     auto wait_stage = [&](int n) {
@@ -744,23 +736,38 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     };
 
     // V pass of the warp's groups of row ri, then the CTA partial (o, l) into part.
+    //
+    // Per group, lane t takes token t: weight w = 2^(s - m), the zero terms, W_g = w * scale_g
+    // (a quarter of it for 2-bit codes, which sit in the hi position) and, with F from the
+    // exact maximum of W over the group, the 21-bit fixed-point I_g = round(W_g 2^F) as the
+    // low bits of W_g 2^F + 2^23.  Through a padded shared transpose, lane (t8, g) then packs
+    // the three byte digits of I_g of the 4 tokens of token quad t8 into a record
+    // {d0, d1, d2, hot-byte mask}.  Consumer lane vk owns channel quad vk and, for every token
+    // quad, merges its hi and lo plane words into 4-bit codes (lo bits kept for hot tokens
+    // only), unpacks the four channels' codes of the four tokens with one AND each and
+    // accumulates code * digit over tokens with dp4a, exact in int32; the group's sum goes
+    // to fp32 with one rounding.
     auto consume_v = [&](int ri, float m2, float thr2) {
         const int32_t *srow = irow_of(ri);
         const int nown = srow[IR_N], tail = srow[IR_TAIL];
         const float *sc = scores_of(ri);
-        const int cg = lane % G::NCG, ts = lane / G::NCG;
-        float2 acc[2][2][4];
+        constexpr int NCG = G::NCG;
+        constexpr int YS = 40; // word stride of a group's row in the transpose (conflict-free both ways)
+        const int pt8 = lane / NCG, pg = lane % NCG;  // record lane: token quad, channel group
+        const bool pv = pt8 < 8;
+        constexpr int BPL = G::NQ == 32 ? 2 : 1;      // blocks of a group per consumer lane
+        const int vk = lane % G::NQ, vg = vk >> 3;     // consumer lane: channel quad and its group
+        const int vb0 = G::NQ == 32 ? 0 : lane / G::NQ;
+        // [NCG][YS] fixed-point words of the tokens; record (g, t8) is then written in place
+        // over words 4 t8 .. 4 t8 + 3 of row g, the only words its lane reads
+        uint32_t *ybuf = reinterpret_cast<uint32_t *>(scr);
+        float *fsit = reinterpret_cast<float *>(ybuf + NCG * YS);
+        const float wscale = BITS == 4 ? 1.f : 0.25f;
+        float facc[4] = {0.f, 0.f, 0.f, 0.f};
+        float zl[NCG];
 #pragma unroll
-        for (int k = 0; k < 2; ++k)
-#pragma unroll
-            for (int e = 0; e < 2; ++e)
-#pragma unroll
-                for (int n = 0; n < 4; ++n)
-                    acc[k][e][n] = make_float2(0.f, 0.f);
-        float zl[G::NCG];
-#pragma unroll
-        for (int j = 0; j < G::NCG; ++j)
-            zl[j] = 0.f;
+        for (int g = 0; g < NCG; ++g)
+            zl[g] = 0.f;
         float lsum = 0.f;
         const uint8_t *stg = ring;
         for (int k = 0; k < nown; ++k) {
@@ -772,98 +779,93 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
                     pump(n + spw);
             }
             const float s2l = sc[k * 32 + lane];
-            const float wl = exp2f(s2l - m2);
+            const float wl = ex2(s2l - m2);
             const bool hotl = all_hot || (BITS == 4 && s2l >= thr2);
-            const uint32_t hotmask = __ballot_sync(0xFFFFFFFFu, hotl);
-            if (a.s_bitmap && lane == 0) {
-                const int g = (int)crank + (warp + k * kWarps) * (int)C;
-                a.s_bitmap[(int64_t)srow[IR_ROW] * a.bitmap_words + g] = hotmask;
-            }
+            const uint32_t hm = __ballot_sync(0xFFFFFFFFu, hotl);
+            if (a.s_bitmap && lane == 0) // refine set of the debug entry point, one bit per token
+                a.s_bitmap[(int64_t)srow[IR_ROW] * a.bitmap_words + (int)crank + (warp + k * kWarps) * (int)C] = hm;
             lsum += wl;
             if (first) {
                 wait_stage(n);
                 stg = ring + (n & smask) * G::STAGE;
             }
             const uint8_t *st = stg + (k % kGPS) * G::GSLOT;
-            // the lane's plane words of its 32 / TPI tokens, loaded before the weight build so
-            // that their latency overlaps it (lo words only where they were copied)
-            uint2 hwv[32 / G::TPI], lwv[32 / G::TPI];
+            // ---- token lane: zero terms, fixed-point weights
+            {
+                const uint8_t *vm = st + (lane >> 4) * G::VB + (lane & 15) * 4; // (scale, zero) of group g at + 64 g
+                float W[NCG], wmax = 0.f;
 #pragma unroll
-            for (int u = 0; u < 32 / G::TPI; ++u) {
-                const int t = u * G::TPI + ts;
-                const int blk = t >> 4, r = t & 15;
-                hwv[u] = *reinterpret_cast<const uint2 *>(st + blk * G::VB + G::VMETA + r * G::ROWV + cg * 8);
-                lwv[u] = make_uint2(0u, 0u);
-                if (BITS == 4 && (all_hot || ((hotmask >> t) & 1u)))
-                    lwv[u] = *reinterpret_cast<const uint2 *>(st + 2 * G::VB + blk * G::LOB + r * G::ROWV + cg * 8);
-            }
-            {   // token `lane`: fold its value scales and zeros into the weight and a running sum
-                const uint8_t *mrow = st + (lane >> 4) * G::VB + (lane & 15) * G::NCG * 4;
-                float wsc[4];
-                uint32_t mw[4];
-                if (G::NCG == 4) {
-                    const uint4 m4 = *reinterpret_cast<const uint4 *>(mrow);
-                    mw[0] = m4.x;
-                    mw[1] = m4.y;
-                    mw[2] = m4.z;
-                    mw[3] = m4.w;
-                } else {
-                    const uint2 m2w = *reinterpret_cast<const uint2 *>(mrow);
-                    mw[0] = m2w.x;
-                    mw[1] = m2w.y;
+                for (int g = 0; g < NCG; ++g) {
+                    const float2 m = __half22float2(*reinterpret_cast<const __half2 *>(vm + 64 * g));
+                    zl[g] = fmaf(wl, (BITS == 4 && !hotl) ? fmaf(1.5f, m.x, m.y) : m.y, zl[g]);
+                    W[g] = wl * wscale * m.x;
+                    wmax = fmaxf(wmax, W[g]);
                 }
-                const float wls = wl * (BITS == 4 ? vscale : 0.25f * vscale);
+                wmax = warp_max_f(wmax);
+                // I < 2^21 + 1 with F = 20 - E (E = exponent of the maximum), capped so that
+                // 2^F and 2^-F stay normal
+                int F = 20 - ((int)(__float_as_uint(wmax) >> 23) - 127);
+                F = F > 126 ? 126 : F;
+                const float fs = __int_as_float((F + 127) << 23);
 #pragma unroll
-                for (int j = 0; j < G::NCG; ++j) {
-                    const float2 m = __half22float2(*reinterpret_cast<const __half2 *>(&mw[j])); // (scale, zero)
-                    if (BITS == 4)
-                        zl[j] = fmaf(wl, hotl ? m.y : fmaf(1.5f, m.x, m.y), zl[j]);
-                    else
-                        zl[j] = fmaf(wl, m.y, zl[j]);
-                    wsc[j] = wls * m.x;
-                }
-                if (G::NCG == 4)
-                    wv4[lane] = make_float4(wsc[0], wsc[1], wsc[2], wsc[3]);
-                else
-                    reinterpret_cast<float2 *>(wv4)[lane] = make_float2(wsc[0], wsc[1]);
+                for (int g = 0; g < NCG; ++g)
+                    ybuf[g * YS + lane] = __float_as_uint(fmaf(W[g], fs, 8388608.f));
+                if (lane == 0)
+                    *fsit = __int_as_float((127 - F) << 23);
             }
             __syncwarp();
-#pragma unroll
-            for (int u = 0; u < 32 / G::TPI; ++u) {
-                const float Wp = wvf[(u * G::TPI + ts) * G::NCG + cg];
-                value_word(hwv[u].x, lwv[u].x, Wp, acc[0]);
-                value_word(hwv[u].y, lwv[u].y, Wp, acc[1]);
+            // ---- record lane (t8, g): byte digits of the 4 tokens of quad t8, hot-byte mask
+            if (pv) {
+                const uint4 y = *reinterpret_cast<const uint4 *>(ybuf + pg * YS + 4 * pt8);
+                const uint32_t t01 = __byte_perm(y.x, y.y, 0x5140), t23 = __byte_perm(y.z, y.w, 0x5140);
+                const uint32_t u01 = __byte_perm(y.x, y.y, 0x0062), u23 = __byte_perm(y.z, y.w, 0x0062);
+                // bit b of the quad's 4 hot bits to bit 8b+7, then each byte takes its top bit
+                const uint32_t hb = byte_signs(((hm >> (4 * pt8)) & 0xFu) * 0x10204080u);
+                reinterpret_cast<uint4 *>(ybuf + pg * YS)[pt8] = make_uint4(__byte_perm(t01, t23, 0x5410), __byte_perm(t01, t23, 0x7632),
+                                                __byte_perm(u01, u23, 0x5410), hb);
             }
             __syncwarp();
-        }
-        // Reduce over the token slots of the warp (lanes with the same cg), scattering the
-        // 32 accumulators of a channel group over its 32 / NCG lanes: after the steps lane
-        // (ts, cg) holds elements NCG*ts + j, j < NCG.
-        float v[32];
+            // ---- accumulate: channel quad vk, dp4a over the tokens of each token quad
+            uint32_t a0[4] = {0u, 0u, 0u, 0u}, a1[4] = {0u, 0u, 0u, 0u}, a2[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-        for (int k = 0; k < 2; ++k)
+            for (int bb = 0; bb < BPL; ++bb) {
+                const int blk = vb0 + bb;
+                const uint4 h4 = *reinterpret_cast<const uint4 *>(st + blk * G::VB + G::VMETA + 16 * vk);
+                const uint32_t hwv[4] = {h4.x, h4.y, h4.z, h4.w};
 #pragma unroll
-            for (int e = 0; e < 2; ++e)
+                for (int tau = 0; tau < 4; ++tau) {
+                    const uint4 rc = reinterpret_cast<const uint4 *>(ybuf + vg * YS)[4 * blk + tau];
+                    uint32_t lw = 0u;
+                    if (BITS == 4 && (all_hot || rc.w != 0u)) { // lo words exist for quads with a hot token
+                        lw = *reinterpret_cast<const uint32_t *>(st + 2 * G::VB + blk * G::LOB + tau * D + 4 * vk);
+                        if (!all_hot)
+                            lw &= rc.w;
+                    }
+                    const uint32_t hw = hwv[tau];
+                    const uint32_t E = ((hw << 2) & 0xCCCCCCCCu) | (lw & 0x33333333u);
+                    const uint32_t O = (hw & 0xCCCCCCCCu) | ((lw >> 2) & 0x33333333u);
+                    const uint32_t c4[4] = {E & 0x0F0F0F0Fu, O & 0x0F0F0F0Fu, (E >> 4) & 0x0F0F0F0Fu,
+                                            (O >> 4) & 0x0F0F0F0Fu};
 #pragma unroll
-                for (int n = 0; n < 4; ++n) {
-                    v[16 * k + 8 * e + 2 * n] = acc[k][e][n].x;
-                    v[16 * k + 8 * e + 2 * n + 1] = acc[k][e][n].y;
+                    for (int i = 0; i < 4; ++i) {
+                        dp4a_uu(a0[i], c4[i], rc.x);
+                        dp4a_uu(a1[i], c4[i], rc.y);
+                        dp4a_uu(a2[i], c4[i], rc.z);
+                    }
                 }
-#pragma unroll
-        for (int s = 0; (16 >> s) >= G::NCG; ++s) {
-            const int off = 16 >> s, half = 16 >> s;
-            const bool up = (lane & off) != 0;
-#pragma unroll
-            for (int j = 0; j < half; ++j) {
-                const float send = up ? v[j] : v[j + half];
-                const float keep = up ? v[j + half] : v[j];
-                v[j] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, off);
             }
-        }
-        // zero terms: lane ends with the sum over the warp of zl[cg]
+            // sum_t code * I < 2^31: exact in 32 bits; one rounding to fp32
+            const float fsi = *fsit;
 #pragma unroll
-        for (int s = 0; (1 << s) < G::NCG; ++s) {
-            const int off = 1 << s, len = G::NCG >> (s + 1);
+            for (int i = 0; i < 4; ++i)
+                facc[i] = fmaf((float)(a0[i] + (a1[i] << 8) + (a2[i] << 16)), fsi, facc[i]);
+            __syncwarp();
+        }
+        // zero terms: lane ends with the warp's sum of zl[lane % NCG] (reduce-scatter over
+        // the group bits, then a sum over the other lanes); lane vk takes its group's from lane vg
+#pragma unroll
+        for (int s2 = 0; (1 << s2) < NCG; ++s2) {
+            const int off = 1 << s2, len = NCG >> (s2 + 1);
             const bool up = (lane & off) != 0;
 #pragma unroll
             for (int m = 0; m < len; ++m) {
@@ -872,19 +874,21 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
                 zl[m] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, off);
             }
         }
-        float zacc = zl[0];
+        float zsum = zl[0];
 #pragma unroll
-        for (int off = G::NCG; off < 32; off <<= 1)
-            zacc += __shfl_xor_sync(0xFFFFFFFFu, zacc, off);
+        for (int off = NCG; off < 32; off <<= 1)
+            zsum += __shfl_xor_sync(0xFFFFFFFFu, zsum, off);
+        const float zacc = __shfl_sync(0xFFFFFFFFu, zsum, vg);
         lsum = warp_sum(lsum);
+        if (BPL == 1) // D = 64: the two halves of the warp read the two blocks
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                facc[i] += __shfl_xor_sync(0xFFFFFFFFu, facc[i], 16);
         __syncwarp();
         float *red = reinterpret_cast<float *>(scr); // end of the V pass: the warp's partial o, l
-#pragma unroll
-        for (int j = 0; j < G::NCG; ++j) {
-            const int i = G::NCG * ts + j;
-            const float f = __int_as_float((127 + kVScaleExp - value_pos(i)) << 23);
-            red[32 * cg + value_channel(i)] = fmaf(v[j], f, zacc);
-        }
+        if (lane < G::NQ)
+            *reinterpret_cast<float4 *>(red + 4 * vk) =
+                make_float4(facc[0] + zacc, facc[1] + zacc, facc[2] + zacc, facc[3] + zacc);
         if (lane == 0)
             red[D] = lsum;
         __syncwarp();

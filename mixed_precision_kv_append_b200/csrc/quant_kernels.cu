@@ -142,7 +142,9 @@ __device__ void quant_group_head(const DT *ksrc, const DT *vsrc, int64_t tok_str
         uint8_t *m = (t < 16) ? main0 : main1;
         reinterpret_cast<uint32_t *>(m + (t & 15) * ROWK)[w] = word;
     }
-    // Values: one thread per (token, 32-channel group).
+    __syncthreads(); // the key rows are packed: the scratch now takes the value codes
+    // Values: one thread per (token, 32-channel group); the (scale, zero) pair goes to
+    // [group][token] of the block's V meta, the codes to the scratch.
     constexpr int NCG = D / 32;
     for (int u = tid; u < 32 * NCG; u += kQThreads) {
         int t = u / NCG, j = u % NCG;
@@ -155,21 +157,32 @@ __device__ void quant_group_head(const DT *ksrc, const DT *vsrc, int64_t tok_str
         uint8_t code[32];
         err |= quant32<L>(x, zb, sb, code);
         uint8_t *m = (t < 16) ? main0 : main1;
-        int r = t & 15;
-        uint16_t *meta = reinterpret_cast<uint16_t *>(m + KCODES + G::KMETA + r * NCG * 4 + j * 4);
+        uint16_t *meta = reinterpret_cast<uint16_t *>(m + KCODES + G::KMETA + (j * 16 + (t & 15)) * 4);
         meta[0] = sb;
         meta[1] = zb;
-        uint32_t *plane = reinterpret_cast<uint32_t *>(m + KCODES + G::KMETA + G::VMETA + r * (D / 4));
-        if (BITS == 4) {
-            uint32_t *lop = reinterpret_cast<uint32_t *>(((t < 16) ? lo0 : lo1) + r * (D / 4));
-            plane[2 * j] = pack2_16(code, 2, 3);
-            plane[2 * j + 1] = pack2_16(code + 16, 2, 3);
-            lop[2 * j] = pack2_16(code, 0, 3);
-            lop[2 * j + 1] = pack2_16(code + 16, 0, 3);
-        } else {
-            plane[2 * j] = pack2_16(code, 0, 3);
-            plane[2 * j + 1] = pack2_16(code + 16, 0, 3);
-        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            kc_smem[t * D + 32 * j + i] = code[i];
+    }
+    __syncthreads();
+    // Planes: one thread per (block, channel quad kappa, token quad tau) word; byte b of a
+    // word is token 4tau+b, its bits 2i..2i+1 channel 4kappa+i.  hi words (the 2-bit codes
+    // of a 2-bit cell) at index 4kappa+tau, lo words at tau*(D/4)+kappa.
+    for (int n = tid; n < 2 * D; n += kQThreads) {
+        const int blk = n / D, kappa = (n % D) >> 2, tau = n & 3;
+        uint32_t hw = 0, lw = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t code = kc_smem[(16 * blk + 4 * tau + b) * D + 4 * kappa + i];
+                hw |= (BITS == 4 ? code >> 2 : code) << (8 * b + 2 * i);
+                lw |= (code & 3u) << (8 * b + 2 * i);
+            }
+        uint8_t *m = blk ? main1 : main0;
+        reinterpret_cast<uint32_t *>(m + KCODES + G::KMETA + G::VMETA)[4 * kappa + tau] = hw;
+        if (BITS == 4)
+            reinterpret_cast<uint32_t *>(blk ? lo1 : lo0)[tau * (D / 4) + kappa] = lw;
     }
     if (err)
         atomicOr(status, err);

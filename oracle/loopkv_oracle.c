@@ -309,11 +309,37 @@ int orc_head_main_bytes(int bits, int D)
 }
 int orc_head_lo_bytes(int bits, int D) { return bits == 4 ? 16 * D / 4 : 0; }
 
+static void put_u32(uint8_t *p, uint32_t v)
+{
+    p[0] = (uint8_t)(v & 0xff);
+    p[1] = (uint8_t)((v >> 8) & 0xff);
+    p[2] = (uint8_t)((v >> 16) & 0xff);
+    p[3] = (uint8_t)(v >> 24);
+}
+
+/*
+ * One word of a value plane: 4 tokens x 4 channels of 2-bit values plane[16][D].
+ * Byte b holds token 4*tau + b; in it, bits 2i..2i+1 hold channel 4*kappa + i.
+ * (The pages fix two 2-bit planes, not their bit order; this is the reading.)
+ */
+static uint32_t plane_word(const uint8_t *plane, int D, int kappa, int tau)
+{
+    uint32_t w = 0;
+    for (int b = 0; b < 4; ++b)
+        for (int i = 0; i < 4; ++i)
+            w |= (uint32_t)(plane[(size_t)(4 * tau + b) * D + 4 * kappa + i] & 3) << (8 * b + 2 * i);
+    return w;
+}
+
 /*
  * Pack one head of one block.  kcodes[16][D], kmeta[D] (scales if the block is
  * even in its group, zeros if odd), vcodes[16][D] (4-bit or 2-bit codes),
  * vscale/vzero[16][D/32].  main_out gets orc_head_main_bytes, lo_out (4-bit
  * only) orc_head_lo_bytes.
+ *   K rows: token-major, orc_pack_row4 / orc_pack_row2 per token.
+ *   V meta: (scale, zero) fp16 pairs ordered [channel group j][token t].
+ *   V planes: words of plane_word; the hi plane (or the 2-bit codes) ordered
+ *   [channel quad kappa][token quad tau], the lo plane [tau][kappa].
  */
 void orc_pack_head_block(int bits, int D, const uint8_t *kcodes, const uint16_t *kmeta,
                          const uint8_t *vcodes, const uint16_t *vscale, const uint16_t *vzero,
@@ -321,7 +347,6 @@ void orc_pack_head_block(int bits, int D, const uint8_t *kcodes, const uint16_t 
 {
     int G = D / ORC_GROUP;
     uint8_t *p = main_out;
-    uint8_t tmp[512];
     for (int t = 0; t < 16; ++t) {
         if (bits == 4) {
             orc_pack_row4(kcodes + (size_t)t * D, D, p);
@@ -333,25 +358,26 @@ void orc_pack_head_block(int bits, int D, const uint8_t *kcodes, const uint16_t 
     }
     for (int c = 0; c < D; ++c, p += 2)
         put_u16(p, kmeta[c]);
-    for (int t = 0; t < 16; ++t)
-        for (int j = 0; j < G; ++j) {
+    for (int j = 0; j < G; ++j)
+        for (int t = 0; t < 16; ++t) {
             put_u16(p, vscale[t * G + j]);
             put_u16(p + 2, vzero[t * G + j]);
             p += 4;
         }
-    for (int t = 0; t < 16; ++t) {
-        if (bits == 4) {
-            for (int c = 0; c < D; ++c)
-                tmp[c] = (uint8_t)(vcodes[(size_t)t * D + c] >> 2); /* hi plane */
-            orc_pack_row2(tmp, D, p);
-            for (int c = 0; c < D; ++c)
-                tmp[c] = (uint8_t)(vcodes[(size_t)t * D + c] & 3); /* lo plane */
-            orc_pack_row2(tmp, D, lo_out + (size_t)t * (D / 4));
-        } else {
-            orc_pack_row2(vcodes + (size_t)t * D, D, p);
-        }
-        p += D / 4;
+    uint8_t *hi = (uint8_t *)malloc((size_t)16 * D), *lo = (uint8_t *)malloc((size_t)16 * D);
+    for (int i = 0; i < 16 * D; ++i) {
+        hi[i] = bits == 4 ? (uint8_t)(vcodes[i] >> 2) : vcodes[i];
+        lo[i] = (uint8_t)(vcodes[i] & 3);
     }
+    for (int kappa = 0; kappa < D / 4; ++kappa)
+        for (int tau = 0; tau < 4; ++tau)
+            put_u32(p + 4 * (kappa * 4 + tau), plane_word(hi, D, kappa, tau));
+    if (bits == 4)
+        for (int tau = 0; tau < 4; ++tau)
+            for (int kappa = 0; kappa < D / 4; ++kappa)
+                put_u32(lo_out + 4 * (tau * (D / 4) + kappa), plane_word(lo, D, kappa, tau));
+    free(hi);
+    free(lo);
 }
 
 /* ------------------------------------------------------------------------- */

@@ -14,14 +14,26 @@ from oracle import oracle as O
 GOLD = os.path.join(os.path.dirname(__file__), "golden", "pack_examples.txt")
 
 
-def _examples():
+def _lines(kind):
     for line in open(GOLD):
         line = line.strip()
-        if not line or line.startswith("#"):
-            continue
-        kind, rest = line.split(None, 1)
-        codes, out = rest.split("->")
-        yield kind, [int(c) for c in codes.split(",")], bytes.fromhex(out.replace(" ", ""))
+        if line and not line.startswith("#") and line.split(None, 1)[0] == kind:
+            yield line.split(None, 1)[1]
+
+
+def _examples():
+    for kind in ("row4", "row2"):
+        for rest in _lines(kind):
+            codes, out = rest.split("->")
+            yield kind, [int(c) for c in codes.split(",")], bytes.fromhex(out.replace(" ", ""))
+
+
+def _plane_examples():
+    for rest in _lines("vplane"):
+        lhs, rhs = rest.split("->")
+        D, t, c, code = (int(x) for x in lhs.split())
+        hb, hv, lb, lv = rhs.split()
+        yield D, t, c, code, int(hb), int(hv, 16), int(lb), int(lv, 16)
 
 
 @pytest.mark.parametrize("ex", list(_examples()), ids=lambda e: e[0])
@@ -29,6 +41,33 @@ def test_hand_derived_rows(ex):
     kind, codes, expect = ex
     got = O.pack_row4(codes) if kind == "row4" else O.pack_row2(codes)
     assert bytes(got) == expect
+
+
+@pytest.mark.parametrize("ex", list(_plane_examples()), ids=lambda e: f"D{e[0]}_t{e[1]}_c{e[2]}")
+def test_hand_derived_value_planes(ex):
+    """One 4-bit value code in an otherwise zero block lands on the hand-derived bytes of the
+    hi and lo planes, and nowhere else."""
+    D, t, c, code, hbyte, hval, lbyte, lval = ex
+    vc = np.zeros((16, D), np.uint8)
+    vc[t, c] = code
+    z16 = np.zeros(16 * (D // 32), np.uint16)
+    main, lo = O.pack_head_block(4, D, np.zeros((16, D), np.uint8), np.zeros(D, np.uint16), vc, z16, z16)
+    hi = main[-16 * D // 4:]
+    assert np.flatnonzero(hi).tolist() == [hbyte] and hi[hbyte] == hval
+    assert np.flatnonzero(lo).tolist() == [lbyte] and lo[lbyte] == lval
+
+
+def _unpack_plane(words_bytes, D, kappa_major):
+    """Decode a packed plane back to [16][D] 2-bit values by walking every field."""
+    w = np.frombuffer(bytes(words_bytes), dtype="<u4")
+    out = np.zeros((16, D), np.uint8)
+    for kappa in range(D // 4):
+        for tau in range(4):
+            word = int(w[4 * kappa + tau] if kappa_major else w[tau * (D // 4) + kappa])
+            for b in range(4):
+                for i in range(4):
+                    out[4 * tau + b, 4 * kappa + i] = (word >> (8 * b + 2 * i)) & 3
+    return out
 
 
 @pytest.mark.parametrize("bits,width", [(4, 4), (2, 2)])
@@ -74,10 +113,10 @@ def test_head_block_roundtrip_fields():
         assert bytes(m[:D // 2]) == bytes(O.pack_row4(h.kc[16 * b]))
         meta = m[kc_bytes:kc_bytes + 2 * D].view(np.uint16)
         assert np.array_equal(meta, h.kz[0] if b else h.ks[0])
-        vmeta = m[kc_bytes + 2 * D: kc_bytes + 2 * D + 16 * (D // 32) * 4].view(np.uint16).reshape(16, D // 32, 2)
-        assert np.array_equal(vmeta[..., 0], h.vs[16 * b:16 * b + 16])
-        assert np.array_equal(vmeta[..., 1], h.vz[16 * b:16 * b + 16])
-        hi = m[-16 * D // 4:].reshape(16, D // 4)
-        for t in range(16):
-            assert bytes(hi[t]) == bytes(O.pack_row2(h.vc[16 * b + t] >> 2))
-            assert bytes(los[b].reshape(16, D // 4)[t]) == bytes(O.pack_row2(h.vc[16 * b + t] & 3))
+        # V meta pairs ordered [channel group][token]
+        vmeta = m[kc_bytes + 2 * D: kc_bytes + 2 * D + 16 * (D // 32) * 4].view(np.uint16).reshape(D // 32, 16, 2)
+        assert np.array_equal(vmeta[..., 0].T, h.vs[16 * b:16 * b + 16])
+        assert np.array_equal(vmeta[..., 1].T, h.vz[16 * b:16 * b + 16])
+        # every field of both planes decodes back to its (token, channel) code
+        assert np.array_equal(_unpack_plane(m[-16 * D // 4:], D, True), h.vc[16 * b:16 * b + 16] >> 2)
+        assert np.array_equal(_unpack_plane(los[b], D, False), h.vc[16 * b:16 * b + 16] & 3)
