@@ -204,6 +204,7 @@ struct Smem {
     float *part;       // [2][D + 1] CTA partial o and l of a row, by row parity
     int32_t *ids;      // [3][kWarps][2 * capw] block ids of a warp's groups, by row index mod 3
     int32_t *irow;     // [3][kWarps][IR_N] row parameters and issuer state, by row index mod 3
+    int32_t *order;    // [kMaxOrder] requests by decreasing history length, then index
 };
 
 // Fields of a row slot (Smem::irow).
@@ -212,8 +213,10 @@ enum { IR_ROW = 0, IR_B, IR_H, IR_N, IR_TAIL, IR_VFIRST, IR_VISSUED, IR_THR, IR_
 // Byte offsets of the shared-memory regions; every region starts on a 16-byte boundary
 // (digit records, weights and stage data are read with 16-byte vector loads).
 struct SmemLayout {
-    int full, scores, tscores, scr, stat, part, ids, irow, total;
+    int full, scores, tscores, scr, stat, part, ids, irow, order, total;
 };
+
+constexpr int kMaxOrder = 64; // batches up to this size are ordered longest request first
 
 __host__ __device__ constexpr int align16(int x) { return (x + 15) & ~15; }
 
@@ -245,6 +248,8 @@ template <int BITS, int D> __host__ __device__ constexpr SmemLayout smem_layout(
     o = align16(o + 3 * kWarps * 2 * capw * 4);
     L.irow = o;
     o = align16(o + 3 * kWarps * IR_N_FIELDS * 4);
+    L.order = o;
+    o = align16(o + 2 * kMaxOrder * 4);
     L.total = o;
     return L;
 }
@@ -267,6 +272,7 @@ template <int BITS, int D> __device__ Smem carve(uint8_t *base, int spw, int cap
     s.part = reinterpret_cast<float *>(base + L.part);
     s.ids = reinterpret_cast<int32_t *>(base + L.ids);
     s.irow = reinterpret_cast<int32_t *>(base + L.irow);
+    s.order = reinterpret_cast<int32_t *>(base + L.order);
     return s;
 }
 
@@ -275,7 +281,7 @@ template <int BITS, int D> __device__ Smem carve(uint8_t *base, int spw, int cap
 template <int BITS, int D> bool layout_ok(int spw, int capw, int nbuf)
 {
     const SmemLayout L = smem_layout<BITS, D>(spw, capw, nbuf);
-    const int offs[] = {L.full, L.scores, L.tscores, L.scr, L.stat, L.part, L.ids, L.irow};
+    const int offs[] = {L.full, L.scores, L.tscores, L.scr, L.stat, L.part, L.ids, L.irow, L.order};
     int prev = kWarps * spw * Geo<BITS, D>::STAGE;
     for (int o : offs) {
         if (o % 16 || o < prev)
@@ -344,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     const int spw = 1 << spw_log2, smask = spw - 1;
     const uint32_t crank = cluster_ctarank(), C = cluster_nctarank();
     const int cid = blockIdx.x / (int)C, ncl = gridDim.x / (int)C;
-    const int nrows = cid < a.rows ? (a.rows - 1 - cid) / ncl + 1 : 0; // rows cid, cid + ncl, ...
+
     const int capw = (a.cap_groups + kWarps - 1) / kWarps;
     Smem sm = carve<BITS, D>(smem_raw, spw, capw, nbuf);
     const bool all_hot = (BITS == 4) && !(a.tau > 0.f);
@@ -352,11 +358,49 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     // byte distance between consecutive block ids in the pools (one block = H heads)
     const uint32_t bstride = (uint32_t)a.H * G::HM, lstride = (uint32_t)a.H * G::LOB;
 
+    // Programmatic dependent launch: the next kernel of the stream may start its CTAs once
+    // every CTA of this grid has run this (so it never takes resources this grid still
+    // needs); they wait in griddepcontrol.wait for this grid to finish before reading q.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (lane == 0)
         for (int i = 0; i < spw; ++i)
             mbar_init(&sm.full[warp * spw + i], 1);
     fence_mbar_init();
-    __syncwarp();
+    // Row schedule.  Requests of equal history length: cluster c takes rows c, c + ncl, ...
+    // Otherwise (batches up to kMaxOrder) a pass-by-pass deal of the rows ordered longest
+    // request first: pass j gives positions j*ncl .. j*ncl + ncl - 1 to clusters 0..ncl-1
+    // (even j) or ncl-1..0 (odd j), position p being head p % H of the (p / H)-th longest
+    // request, so that a cluster drawing a long row early draws a short one next.
+    const int nreq = a.rows / a.H;
+    bool ordered = false;
+    if (nreq <= kMaxOrder) { // rank the requests by history length (every CTA derives the same order)
+        int32_t *lens = sm.order + kMaxOrder;
+        for (int b = threadIdx.x; b < nreq; b += kThreads)
+            lens[b] = a.hist_len[b];
+        __syncthreads();
+        for (int b = threadIdx.x; b < nreq; b += kThreads) {
+            const int lb = lens[b];
+            int rank = 0;
+            for (int b2 = 0; b2 < nreq; ++b2) {
+                const int l2 = lens[b2];
+                rank += (l2 > lb) || (l2 == lb && b2 < b);
+            }
+            sm.order[rank] = b;
+        }
+        for (int b = 1; b < nreq; ++b)
+            ordered |= lens[b] != lens[0];
+    }
+    __syncthreads();
+    const int full_passes = a.rows / ncl, rem = a.rows % ncl;
+    const int nrows = !ordered ? (cid < a.rows ? (a.rows - 1 - cid) / ncl + 1 : 0)
+                               : full_passes + ((full_passes & 1) ? (cid >= ncl - rem) : (cid < rem));
+    auto row_of = [&](int ri) {
+        if (!ordered)
+            return cid + ri * ncl;
+        const int p = ri * ncl + ((ri & 1) ? ncl - 1 - cid : cid);
+        const int q = p / a.H;
+        return sm.order[q] * a.H + (p - q * a.H);
+    };
 
     uint8_t *ring = sm.ring + warp * spw * G::STAGE;
     uint64_t *full = sm.full + warp * spw;
@@ -377,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
 
     // Row parameters, validation and the warp's block ids of row ri.
     auto setup_row = [&](int ri) {
-        const int row = cid + ri * ncl;
+        const int row = row_of(ri);
         const int b = row / a.H, h = row - b * a.H;
         int hist = a.hist_len[b], tail = a.tail_len[b];
         bool bad = false;
@@ -592,6 +636,14 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         const int32_t *srow = irow_of(ri);
         const int row = srow[IR_ROW], nown = srow[IR_N], tail = srow[IR_TAIL];
         float *sc = scores_of(ri);
+        if (ri == 0) {
+            // Prefetch the first stages (pools, block tables and lengths come from earlier
+            // flush / append / ingest launches, which let dependents start only when they
+            // complete), then wait for the previous grid of the stream: q, and the outputs
+            // this grid writes, may be shared with it.
+            pump(prc_n + spw);
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+        }
         // lane owns the channel quad 4*lane .. 4*lane+3 (lanes >= D/4 own none)
         const bool ownq = lane < G::NQ;
         float qreg[4];
@@ -738,7 +790,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     // V pass of the warp's groups of row ri, then the CTA partial (o, l) into part.
     //
     // Per group, lane t takes token t: weight w = 2^(s - m), the zero terms, W_g = w * scale_g
-    // (a quarter of it for 2-bit codes, which sit in the hi position) and, with F from the
+    // and, with F from the
     // exact maximum of W over the group, the 21-bit fixed-point I_g = round(W_g 2^F) as the
     // low bits of W_g 2^F + 2^23.  Through a padded shared transpose, lane (t8, g) then packs
     // the three byte digits of I_g of the 4 tokens of token quad t8 into a record
@@ -762,7 +814,6 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         // over words 4 t8 .. 4 t8 + 3 of row g, the only words its lane reads
         uint32_t *ybuf = reinterpret_cast<uint32_t *>(scr);
         float *fsit = reinterpret_cast<float *>(ybuf + NCG * YS);
-        const float wscale = BITS == 4 ? 1.f : 0.25f;
         float facc[4] = {0.f, 0.f, 0.f, 0.f};
         float zl[NCG];
 #pragma unroll
@@ -798,7 +849,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
                 for (int g = 0; g < NCG; ++g) {
                     const float2 m = __half22float2(*reinterpret_cast<const __half2 *>(vm + 64 * g));
                     zl[g] = fmaf(wl, (BITS == 4 && !hotl) ? fmaf(1.5f, m.x, m.y) : m.y, zl[g]);
-                    W[g] = wl * wscale * m.x;
+                    W[g] = wl * m.x;
                     wmax = fmaxf(wmax, W[g]);
                 }
                 wmax = warp_max_f(wmax);
@@ -827,30 +878,55 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             __syncwarp();
             // ---- accumulate: channel quad vk, dp4a over the tokens of each token quad
             uint32_t a0[4] = {0u, 0u, 0u, 0u}, a1[4] = {0u, 0u, 0u, 0u}, a2[4] = {0u, 0u, 0u, 0u};
+            // codes of channel 4vk+i of the quad's 4 tokens, one per byte, into the sums
+            auto acc_quad = [&](const uint32_t (&c4)[4], const uint4 &rc) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    dp4a_uu(a0[i], c4[i], rc.x);
+                    dp4a_uu(a1[i], c4[i], rc.y);
+                    dp4a_uu(a2[i], c4[i], rc.z);
+                }
+            };
+            // 4-bit codes 4h + l from a hi and a lo word: nibble 0 of each byte is channel 0
+            // (E) or 1 (O), nibble 1 channel 2 (E) or 3 (O)
+            auto merged = [](uint32_t hw, uint32_t lw, uint32_t (&c4)[4]) {
+                const uint32_t E = ((hw << 2) & 0xCCCCCCCCu) | (lw & 0x33333333u);
+                const uint32_t O = (hw & 0xCCCCCCCCu) | ((lw >> 2) & 0x33333333u);
+                c4[0] = E & 0x0F0F0F0Fu;
+                c4[1] = O & 0x0F0F0F0Fu;
+                c4[2] = (E >> 4) & 0x0F0F0F0Fu;
+                c4[3] = (O >> 4) & 0x0F0F0F0Fu;
+            };
 #pragma unroll
             for (int bb = 0; bb < BPL; ++bb) {
                 const int blk = vb0 + bb;
                 const uint4 h4 = *reinterpret_cast<const uint4 *>(st + blk * G::VB + G::VMETA + 16 * vk);
                 const uint32_t hwv[4] = {h4.x, h4.y, h4.z, h4.w};
+                const uint8_t *lop = st + 2 * G::VB + blk * G::LOB + 4 * vk;
+                const uint4 *rq = reinterpret_cast<const uint4 *>(ybuf + vg * YS) + 4 * blk;
+                if (BITS == 2) { // own 2-bit codes: channel i of every byte at bit 2i
 #pragma unroll
-                for (int tau = 0; tau < 4; ++tau) {
-                    const uint4 rc = reinterpret_cast<const uint4 *>(ybuf + vg * YS)[4 * blk + tau];
-                    uint32_t lw = 0u;
-                    if (BITS == 4 && (all_hot || rc.w != 0u)) { // lo words exist for quads with a hot token
-                        lw = *reinterpret_cast<const uint32_t *>(st + 2 * G::VB + blk * G::LOB + tau * D + 4 * vk);
-                        if (!all_hot)
-                            lw &= rc.w;
+                    for (int tau = 0; tau < 4; ++tau) {
+                        const uint32_t hw = hwv[tau];
+                        const uint32_t c4[4] = {hw & 0x03030303u, (hw >> 2) & 0x03030303u, (hw >> 4) & 0x03030303u,
+                                                (hw >> 6) & 0x03030303u};
+                        acc_quad(c4, rq[tau]);
                     }
-                    const uint32_t hw = hwv[tau];
-                    const uint32_t E = ((hw << 2) & 0xCCCCCCCCu) | (lw & 0x33333333u);
-                    const uint32_t O = (hw & 0xCCCCCCCCu) | ((lw >> 2) & 0x33333333u);
-                    const uint32_t c4[4] = {E & 0x0F0F0F0Fu, O & 0x0F0F0F0Fu, (E >> 4) & 0x0F0F0F0Fu,
-                                            (O >> 4) & 0x0F0F0F0Fu};
+                } else if (all_hot) { // every lo word was copied
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        dp4a_uu(a0[i], c4[i], rc.x);
-                        dp4a_uu(a1[i], c4[i], rc.y);
-                        dp4a_uu(a2[i], c4[i], rc.z);
+                    for (int tau = 0; tau < 4; ++tau) {
+                        uint32_t c4[4];
+                        merged(hwv[tau], *reinterpret_cast<const uint32_t *>(lop + tau * D), c4);
+                        acc_quad(c4, rq[tau]);
+                    }
+                } else { // lo words exist for quads with a hot token; keep the hot tokens' bits
+#pragma unroll
+                    for (int tau = 0; tau < 4; ++tau) {
+                        const uint4 rc = rq[tau];
+                        const uint32_t lw = rc.w ? *reinterpret_cast<const uint32_t *>(lop + tau * D) & rc.w : 0u;
+                        uint32_t c4[4];
+                        merged(hwv[tau], lw, c4);
+                        acc_quad(c4, rc);
                     }
                 }
             }
@@ -924,7 +1000,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     // CTA `crank` writes channels [crank*per, min(D, (crank+1)*per)) of row ri, per =
     // ceil(D / C), summing the partials of every CTA of the cluster.
     auto merge = [&](int ri, float m2) {
-        const int row = cid + ri * ncl;
+        const int row = row_of(ri);
         const float *part = sm.part + (ri & 1) * (D + 1);
         const int per = (D + (int)C - 1) / (int)C;
         const int c = (int)crank * per + (int)threadIdx.x;
@@ -998,13 +1074,15 @@ int launch_t(const DecodeArgs &a, const DecodeShape &shp, cudaStream_t s)
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = shp.smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = shp.cluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization; // see griddepcontrol in the kernel
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = shp.pdl ? 2 : 1;
     e = cudaLaunchKernelEx(&cfg, kern, a, shp.stages_log2, shp.score_bufs);
     return e == cudaSuccess ? LOOPKV_OK : LOOPKV_ERR_CUDA;
 }
@@ -1044,6 +1122,17 @@ template <int BITS, int D, typename DT> int max_active_clusters(int C, int smem,
 // Among equal times the deeper ring (more bytes in flight) wins.
 constexpr double kRowFixed = 6.0;  // per-CTA cost of a row outside its groups (setup, merge, bubble)
 constexpr double kSaturate = 3.5;  // CTAs per SM that keep its issue slots busy
+
+// Overlap with the previous launch of the stream (programmatic dependent launch): measured
+// faster with clusters of up to 4 CTAs and slower with larger ones; LOOPKV_DECODE_PDL=0/1
+// overrides.
+inline int pdl_default(int C)
+{
+    const char *env = getenv("LOOPKV_DECODE_PDL");
+    if (env)
+        return atoi(env) != 0;
+    return C <= 4;
+}
 
 template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_blocks)
 {
@@ -1102,6 +1191,7 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
                     best.threads = kThreads;
                     best.cap = cap;
                     best.min_ctas = want_ctas;
+                    best.pdl = pdl_default(C);
                 }
                 break;
             }

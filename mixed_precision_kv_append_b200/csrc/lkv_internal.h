@@ -63,6 +63,7 @@ struct DecodeShape {
     int smem;      // dynamic shared memory bytes per CTA
     int threads;
     int cap;       // score capacity per CTA and row, in 32-token groups
+    int pdl;       // launch with programmatic stream serialization (overlap the previous launch)
 };
 
 // Launchers (defined in the .cu files).  Return LOOPKV_OK or an error code.
