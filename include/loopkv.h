@@ -53,6 +53,7 @@ extern "C" {
 #define LOOPKV_ERR_STATE (-10)         /* ingest into a non-empty (cell, request), bad block id */
 #define LOOPKV_ERR_EMPTY_ROW (-11)     /* decode of a row with no token at all */
 #define LOOPKV_ERR_NO_DEVICE (-12)     /* no CUDA device of compute capability 10.x */
+#define LOOPKV_ERR_INFEASIBLE (-13)    /* plan search: no plan meets the budgets */
 
 /* Device status word bits (loopkv_status); each maps to one code above. */
 #define LOOPKV_DEV_NONFINITE 0x01u
@@ -142,6 +143,36 @@ void loopkv_plan_free(loopkv_plan *plan);
  * Host-only; touches no device.
  */
 int loopkv_plan_bytes(const loopkv_plan *plan, const float *hot_fraction, loopkv_byte_report *out);
+
+/*
+ * Offline plan search (LoopKV paper §3.1 "Allocation"): choose one storage option per
+ * cell of loops 0 .. n_loops-2 -- LOOPKV_CELL_4B, LOOPKV_CELL_2B, or LOOPKV_CELL_SHARE
+ * (reads the final loop's cell of the same layer, §3.2) -- that minimizes the bytes read
+ * per token subject to
+ *     sum over all cells of damage[cell][option] <= damage_budget, and
+ *     stored bytes per token <= storage_budget (no storage budget if <= 0).
+ * Cells of the final loop keep 4-bit codes.  Bytes per token and head: 4-bit stores and
+ * reads 1.25 D (every lo plane counted), 2-bit 0.75 D, share stores 0 and reads 1.25 D.
+ * Damages add up over cells (the paper's profile: summed single-cell damages predict a
+ * plan's KL).  Among the plans with the fewest reads the result has the least damage, then
+ * the least storage; remaining ties are broken deterministically.  Exact (dynamic program
+ * over cells).  Host-only; touches no device.
+ *   damage:    host [n_loops * n_layers][3] (loop-major cells, option index =
+ *              loopkv_cell_mode), finite and >= 0; of final-loop cells only the 4B entry
+ *              is read.
+ *   modes_out: host [n_loops * n_layers], the plan's modes for loopkv_plan_create.
+ *   report:    may be NULL; read / stored bytes per token and total damage of the plan.
+ * Returns LOOPKV_OK, LOOPKV_ERR_INVALID_ARG, or LOOPKV_ERR_INFEASIBLE (modes_out then
+ * untouched).
+ */
+typedef struct {
+    double read_bytes_per_token;   /* every lo plane read */
+    double stored_bytes_per_token;
+    double damage;                 /* sum over all cells, final loop included */
+} loopkv_plan_search_report;
+
+int loopkv_plan_search(const loopkv_config *cfg, const double *damage, double damage_budget,
+                       double storage_budget, uint8_t *modes_out, loopkv_plan_search_report *report);
 
 /* Device bytes a cache needs so that every non-share cell can hold max_batch x
  * max_blocks_per_seq blocks.  Host-only. */

@@ -190,6 +190,8 @@ const char *loopkv_strerror(int code)
         return "decode row with no token";
     case LOOPKV_ERR_NO_DEVICE:
         return "no CUDA device of compute capability 10.x";
+    case LOOPKV_ERR_INFEASIBLE:
+        return "no plan meets the damage and storage budgets";
     default:
         return "unknown error";
     }

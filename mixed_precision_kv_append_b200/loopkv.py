@@ -21,6 +21,7 @@ LOOPKV_OK = 0
 ERRORS = {
     -1: "INVALID_ARG", -2: "SHAPE", -3: "PLAN", -4: "POOL_EXHAUSTED", -5: "NONFINITE", -6: "RANGE",
     -7: "TIMEOUT", -8: "CUDA", -9: "TAIL_FULL", -10: "STATE", -11: "EMPTY_ROW", -12: "NO_DEVICE",
+    -13: "INFEASIBLE",
 }
 CELL_4B, CELL_2B, CELL_SHARE = 0, 1, 2
 TAU_REL_MAX, TAU_ABS_PROB = 0, 1
@@ -32,7 +33,7 @@ EXPORTS = [
     "loopkv_plan_create", "loopkv_plan_free", "loopkv_plan_bytes", "loopkv_required_bytes", "loopkv_alloc",
     "loopkv_free", "loopkv_ingest", "loopkv_append", "loopkv_flush", "loopkv_reset_request", "loopkv_decode",
     "loopkv_decode_debug", "loopkv_status", "loopkv_cell_view_get", "loopkv_decode_shape", "loopkv_strerror",
-    "loopkv_version",
+    "loopkv_version", "loopkv_plan_search",
 ]
 
 
@@ -53,6 +54,11 @@ class ByteReport(ctypes.Structure):
     _fields_ = [("stored_bytes_per_token", ctypes.c_double), ("read_bytes_per_token", ctypes.c_double),
                 ("read_bytes_all_hot", ctypes.c_double), ("read_bytes_all_cold", ctypes.c_double),
                 ("bf16_bytes_per_token", ctypes.c_double)]
+
+
+class PlanSearchReport(ctypes.Structure):
+    _fields_ = [("read_bytes_per_token", ctypes.c_double), ("stored_bytes_per_token", ctypes.c_double),
+                ("damage", ctypes.c_double)]
 
 
 class CellView(ctypes.Structure):
@@ -95,6 +101,9 @@ def lib() -> ctypes.CDLL:
         L.loopkv_strerror.argtypes = [i]
         L.loopkv_strerror.restype = ctypes.c_char_p
         L.loopkv_version.argtypes = []
+        L.loopkv_plan_search.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(ctypes.c_double), ctypes.c_double,
+                                         ctypes.c_double, ctypes.POINTER(ctypes.c_uint8),
+                                         ctypes.POINTER(PlanSearchReport)]
         for name in EXPORTS:
             if name not in ("loopkv_plan_free", "loopkv_free", "loopkv_strerror"):
                 getattr(L, name).restype = ctypes.c_int
@@ -130,6 +139,22 @@ def _dtype_code(dt: torch.dtype) -> int:
 
 
 # ------------------------------------------------------------ C-named functions
+
+def loopkv_plan_search(cfg: Config, damage, damage_budget: float, storage_budget: float = 0.0):
+    """Exact plan search (host-only).  damage: [n_loops * n_layers][3] per cell and option.
+    Returns (modes list, report dict)."""
+    n = cfg.n_loops * cfg.n_layers
+    flat = [float(x) for row in damage for x in row]
+    if len(flat) != 3 * n:
+        raise ValueError("damage must hold 3 values per cell")
+    d = (ctypes.c_double * len(flat))(*flat)
+    modes = (ctypes.c_uint8 * n)()
+    rep = PlanSearchReport()
+    _check(lib().loopkv_plan_search(ctypes.byref(cfg), d, float(damage_budget), float(storage_budget), modes,
+                                    ctypes.byref(rep)), "loopkv_plan_search")
+    return list(modes), {"read_bytes_per_token": rep.read_bytes_per_token,
+                         "stored_bytes_per_token": rep.stored_bytes_per_token, "damage": rep.damage}
+
 
 def loopkv_plan_create(cfg: Config, modes, tau: float, tau_mode: int = TAU_REL_MAX) -> ctypes.c_void_p:
     arr = (ctypes.c_uint8 * len(modes))(*[int(m) for m in modes])
