@@ -74,7 +74,8 @@ def seeded_plan(n_layers, n_loops, loops, p2, psh, seed) -> list:
 
 
 def workload(name: str, seed: int = 0) -> Workload:
-    """The five workloads of the benchmark configuration list, by name."""
+    """The benchmark workloads by name: the five of the configuration list and the Ouro-2.6B
+    fixed-length sweep."""
     if name == "tiny":
         return Workload("tiny", 1, 2, 2, 64, 1, [256], torch.float32, [CELL_4B, CELL_2B], 0.02, seed=seed)
     if name == "kivi4_8k":
@@ -91,10 +92,19 @@ def workload(name: str, seed: int = 0) -> Workload:
         lengths = torch.randint(4096, 32768 + 1, (8,), generator=g).tolist()
         modes = seeded_plan(48, 4, [0, 1, 2], 0.35, 0.25, seed)
         return Workload("ragged_2p6b", 48, 4, 16, 128, 8, lengths, torch.bfloat16, modes, 0.01, seed=seed)
+    if name.startswith("ouro2p6b_"):
+        # Ouro-2.6B fixed-length sweep (the paper's 8K / 16K / 32K throughput tables): 48 layers
+        # x 4 loops, the ragged workload's plan, batch halving as the context doubles so that
+        # the stored KV stays about 87 GB on one GPU
+        T = {"ouro2p6b_8k": 8192, "ouro2p6b_16k": 16384, "ouro2p6b_32k": 32768}[name]
+        B = 32 * 8192 // T
+        modes = seeded_plan(48, 4, [0, 1, 2], 0.35, 0.25, seed)
+        return Workload(name, 48, 4, 16, 128, B, [T] * B, torch.bfloat16, modes, 0.01, seed=seed)
     raise KeyError(name)
 
 
-WORKLOADS = ["tiny", "kivi4_8k", "mixed_8k", "long_16k", "ragged_2p6b"]
+WORKLOADS = ["tiny", "kivi4_8k", "mixed_8k", "long_16k", "ragged_2p6b", "ouro2p6b_8k", "ouro2p6b_16k",
+             "ouro2p6b_32k"]
 
 
 def _gen(seed: int, device) -> torch.Generator:

@@ -200,6 +200,7 @@ def test_share_cell_with_final_loop_query_is_bit_identical():
     ("mixed_8k", 32, [8192] * 32, [0, 1, 2, 0], 0.01, 0),
     ("long_16k", 32, [16384] * 32, [0, 2, 1, 0], 0.005, 2),
     ("ragged_2p6b", 8, None, [1, 2, 0, 0], 0.01, 0),
+    ("ouro2p6b_32k", 8, [32768] * 8, [2, 1, 0, 0], 0.01, 0),
 ])
 def test_full_size_sampled_rows(name, B, T, modes, tau, steps):
     """Benchmark shapes (one layer of four loops): the launch configuration the benchmark times,
