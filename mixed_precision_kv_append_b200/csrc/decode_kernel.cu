@@ -71,9 +71,7 @@ template <int BITS, int D> struct Geo {
     static constexpr int STAGE = kGPS * GSLOT;
     static constexpr int ROWK = KCODES / 16;  // key bytes per token
     static constexpr int WORDSK = ROWK / 4;
-    static constexpr int ROWV = D / 4;        // value plane bytes per token
     static constexpr int NCG = D / 32;        // 32-channel value groups per token
-    static constexpr int TPI = 32 / NCG;      // tokens per V iteration of a warp
     static constexpr int NQ = D / 4;          // channel quads
 };
 
@@ -219,11 +217,12 @@ struct SmemLayout {
 constexpr int kMaxOrder = 64; // batches up to this size are ordered longest request first
 
 __host__ __device__ constexpr int align16(int x) { return (x + 15) & ~15; }
+__host__ __device__ constexpr int imax(int a, int b) { return a > b ? a : b; }
 
 // Bytes of a warp's scratch: the largest of its three uses.
 template <int D> __host__ __device__ constexpr int scratch_bytes()
 {
-    return align16(std::max((D / 4) * 16, std::max((D + 1) * 4, (D / 32) * 40 * 4 + 4)));
+    return align16(imax((D / 4) * 16, imax((D + 1) * 4, (D / 32) * 40 * 4 + 4)));
 }
 
 // nbuf: score buffers (2 when a cluster reads more than one row, so that the next row's
@@ -1058,10 +1057,576 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     cluster_wait();
 }
 
-template <int BITS, int D, typename DT>
-int launch_t(const DecodeArgs &a, const DecodeShape &shp, cudaStream_t s)
+// ---------------------------------------------------------------------------------------
+// Single-pass reader for rows whose refine set does not depend on the row maximum: 4-bit
+// sources read with tau <= 0 (every lo plane is read) and 2-bit sources (no lo plane, S
+// empty).  For these, softmax with a running maximum per warp (rescaling the warp's sums
+// whenever it grows) gives the result of the exact-maximum reader up to rounding, so a
+// group's keys and values are read from one stage and its scores stay in registers: no
+// score buffer, no exchange of maxima inside a row, one merge of (m, l, o) per row over
+// the warps and CTAs of the cluster.  The smaller shared footprint lets 5 CTAs share an SM.
+//
+// A stage holds one 32-token group: the whole head region of both of its blocks (key
+// codes and meta, value meta, hi plane) and, for 4-bit sources, both lo regions.
+template <int BITS, int D> struct Geo1 {
+    using G = Geo<BITS, D>;
+    static constexpr int STAGE = (2 * G::HM + 2 * G::LOB + 127) / 128 * 128;
+    static constexpr int LOFF = 2 * G::HM; // lo regions of the stage
+};
+
+struct SmemLayout1 {
+    int full, scr, wm, part, ids, irow, order, total;
+};
+
+// Row slots (ids, irow) by row parity: while a warp reads row r its issuer may start row
+// r + 1.  CTA partials (o[D], l, m) by row index mod 3 (see the barrier note in the kernel).
+template <int BITS, int D> __host__ __device__ constexpr SmemLayout1 smem_layout1(int spw, int capw)
 {
-    auto kern = shp.min_ctas == 5 ? decode_kernel<BITS, D, DT, 5> : decode_kernel<BITS, D, DT, 4>;
+    SmemLayout1 L{};
+    int o = kWarps * spw * Geo1<BITS, D>::STAGE;
+    L.full = o;
+    o = align16(o + kWarps * spw * 8);
+    L.scr = o;
+    o = align16(o + kWarps * scratch_bytes<D>());
+    L.wm = o;
+    o = align16(o + kWarps * 4);
+    L.part = o;
+    o = align16(o + 3 * (D + 2) * 4);
+    L.ids = o;
+    o = align16(o + 2 * kWarps * 2 * capw * 4);
+    L.irow = o;
+    o = align16(o + 2 * kWarps * IR_N_FIELDS * 4);
+    L.order = o;
+    o = align16(o + kMaxOrder * 4);
+    L.total = o;
+    return L;
+}
+
+template <int BITS, int D> bool layout1_ok(int spw, int capw)
+{
+    const SmemLayout1 L = smem_layout1<BITS, D>(spw, capw);
+    const int offs[] = {L.full, L.scr, L.wm, L.part, L.ids, L.irow, L.order};
+    int prev = kWarps * spw * Geo1<BITS, D>::STAGE;
+    for (int o : offs) {
+        if (o % 16 || o < prev)
+            return false;
+        prev = o;
+    }
+    // the request lengths are ranked in the warps' scratch at kernel start
+    return L.total >= prev && (spw & (spw - 1)) == 0 && kWarps * scratch_bytes<D>() >= kMaxOrder * 4 &&
+           (Geo1<BITS, D>::STAGE % 128) == 0 && (Geo<BITS, D>::HM % 16) == 0 && (Geo<BITS, D>::LOB % 16) == 0;
+}
+
+template <int BITS, int D, typename DT, int MINCTA>
+__global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const DecodeArgs a, const int spw_log2)
+{
+    using G = Geo<BITS, D>;
+    using G1 = Geo1<BITS, D>;
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int spw = 1 << spw_log2, smask = spw - 1;
+    const uint32_t crank = cluster_ctarank(), C = cluster_nctarank();
+    const int cid = blockIdx.x / (int)C, ncl = gridDim.x / (int)C;
+    const int capw = (a.cap_groups + kWarps - 1) / kWarps;
+    const SmemLayout1 LY = smem_layout1<BITS, D>(spw, capw);
+    constexpr int SCR = scratch_bytes<D>();
+    uint64_t *fullb = reinterpret_cast<uint64_t *>(smem_raw + LY.full);
+    uint8_t *scr_all = smem_raw + LY.scr;
+    float *wm = reinterpret_cast<float *>(smem_raw + LY.wm);
+    float *parts = reinterpret_cast<float *>(smem_raw + LY.part);
+    int32_t *ids_all = reinterpret_cast<int32_t *>(smem_raw + LY.ids);
+    int32_t *irow_all = reinterpret_cast<int32_t *>(smem_raw + LY.irow);
+    int32_t *order = reinterpret_cast<int32_t *>(smem_raw + LY.order);
+    const uint32_t bstride = (uint32_t)a.H * G::HM, lstride = (uint32_t)a.H * G::LOB;
+
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); // as in decode_kernel
+    if (lane == 0)
+        for (int i = 0; i < spw; ++i)
+            mbar_init(&fullb[warp * spw + i], 1);
+    fence_mbar_init();
+    // row schedule of decode_kernel; the lengths are ranked in the scratch
+    const int nreq = a.rows / a.H;
+    bool ordered = false;
+    if (nreq <= kMaxOrder) {
+        int32_t *lens = reinterpret_cast<int32_t *>(scr_all);
+        for (int b = threadIdx.x; b < nreq; b += kThreads)
+            lens[b] = a.hist_len[b];
+        __syncthreads();
+        for (int b = threadIdx.x; b < nreq; b += kThreads) {
+            const int lb = lens[b];
+            int rank = 0;
+            for (int b2 = 0; b2 < nreq; ++b2) {
+                const int l2 = lens[b2];
+                rank += (l2 > lb) || (l2 == lb && b2 < b);
+            }
+            order[rank] = b;
+        }
+        for (int b = 1; b < nreq; ++b)
+            ordered |= lens[b] != lens[0];
+    }
+    __syncthreads(); // the scratch is free again
+    const int full_passes = a.rows / ncl, rem = a.rows % ncl;
+    const int nrows = !ordered ? (cid < a.rows ? (a.rows - 1 - cid) / ncl + 1 : 0)
+                               : full_passes + ((full_passes & 1) ? (cid >= ncl - rem) : (cid < rem));
+    auto row_of = [&](int ri) {
+        if (!ordered)
+            return cid + ri * ncl;
+        const int p = ri * ncl + ((ri & 1) ? ncl - 1 - cid : cid);
+        const int q = p / a.H;
+        return order[q] * a.H + (p - q * a.H);
+    };
+
+    uint8_t *ring = smem_raw + warp * spw * G1::STAGE;
+    uint64_t *full = fullb + warp * spw;
+    uint8_t *scr = scr_all + warp * SCR;
+    auto ids_of = [&](int ri) { return ids_all + ((ri & 1) * kWarps + warp) * 2 * capw; };
+    auto irow_of = [&](int ri) { return irow_all + ((ri & 1) * kWarps + warp) * IR_N_FIELDS; };
+
+    // ---------------------------------------------------------------- issuing
+    int iss_n = 0, iss_row = -1, iss_k = 0, seg_n = 0, setup_upto = -1;
+    const uint8_t *seg_src = nullptr, *seg_lo = nullptr;
+    const int2 *seg_ids = nullptr;
+    // row parameters, validation and the warp's block ids of row ri (as in decode_kernel)
+    auto setup_row = [&](int ri) {
+        const int row = row_of(ri);
+        const int b = row / a.H, h = row - b * a.H;
+        int hist = a.hist_len[b], tail = a.tail_len[b];
+        bool bad = false;
+        if (hist < 0 || hist > a.max_blocks * 16 || (hist & 31)) {
+            bad = true;
+            hist = 0;
+        }
+        if (tail < 0 || tail > 32) {
+            bad = true;
+            tail = 0;
+        }
+        const int ngroups = hist >> 5;
+        int nmy = ngroups > (int)crank ? (ngroups - (int)crank + (int)C - 1) / (int)C : 0;
+        if (nmy > a.cap_groups) {
+            bad = true;
+            nmy = a.cap_groups;
+        }
+        if (bad && warp == 0 && lane == 0)
+            atomicOr(a.status, LOOPKV_DEV_STATE);
+        const int n = owned(nmy, warp);
+        const int32_t *bt = a.block_table + (int64_t)b * a.max_blocks;
+        int32_t *ids = ids_of(ri);
+        for (int k = lane; k < 2 * n; k += 32) {
+            const int g = (int)crank + (warp + (k >> 1) * kWarps) * (int)C;
+            int id = bt[2 * g + (k & 1)];
+            if (id < 0 || id >= a.pool_blocks) {
+                atomicOr(a.status, LOOPKV_DEV_STATE);
+                id = 0;
+            }
+            ids[k] = id;
+        }
+        int32_t *st = irow_of(ri);
+        if (lane == 0) {
+            st[IR_ROW] = row;
+            st[IR_B] = b;
+            st[IR_H] = h;
+            st[IR_N] = n;
+            st[IR_TAIL] = (crank == C - 1) ? tail : 0;
+        }
+        __syncwarp();
+    };
+    // stage n = the next group of the issuing row: both head regions (+ both lo regions)
+    auto issue_stage = [&](int n) {
+        const int2 id = seg_ids[iss_k];
+        uint8_t *st = ring + (n & smask) * G1::STAGE;
+        uint64_t *fb = &full[n & smask];
+        if (lane == 0) {
+            mbar_arrive_expect_tx(fb, 2 * G::HM + 2 * G::LOB);
+            bulk_g2s(st, seg_src + (uint64_t)(uint32_t)id.x * bstride, G::HM, fb);
+            bulk_g2s(st + G::HM, seg_src + (uint64_t)(uint32_t)id.y * bstride, G::HM, fb);
+            if (BITS == 4) {
+                bulk_g2s(st + G1::LOFF, seg_lo + (uint64_t)(uint32_t)id.x * lstride, G::LOB, fb);
+                bulk_g2s(st + G1::LOFF + G::LOB, seg_lo + (uint64_t)(uint32_t)id.y * lstride, G::LOB, fb);
+            }
+        }
+    };
+    // issue every stage numbered below `limit`; a row's stages follow once it is set up
+    auto pump = [&](int limit) {
+        for (;;) {
+            if (iss_k < seg_n) {
+                if (iss_n >= limit)
+                    break;
+                issue_stage(iss_n);
+                ++iss_k;
+                ++iss_n;
+                continue;
+            }
+            if (iss_row + 1 >= nrows || iss_row + 1 > setup_upto)
+                break;
+            ++iss_row;
+            iss_k = 0;
+            const int32_t *st = irow_of(iss_row);
+            seg_n = st[IR_N];
+            seg_src = a.main + (size_t)st[IR_H] * G::HM;
+            seg_lo = a.lo + (size_t)st[IR_H] * G::LOB;
+            seg_ids = reinterpret_cast<const int2 *>(ids_of(iss_row));
+        }
+    };
+
+    // ---------------------------------------------------------------- compute
+    const uint4 *rec = reinterpret_cast<const uint4 *>(scr);
+    int prc_n = 0;
+    bool timed_out = false;
+    auto wait_stage = [&](int n) {
+        if (!timed_out)
+            timed_out = !mbar_wait(&full[n & smask], (n >> spw_log2) & 1, a.status);
+    };
+    const bool ownq = lane < G::NQ;
+    constexpr int NCG = G::NCG;
+    constexpr int YS = 40;
+    const int pt8 = lane / NCG, pg = lane % NCG;
+    const bool pv = pt8 < 8;
+    constexpr int BPL = G::NQ == 32 ? 2 : 1;
+    const int vk = lane % G::NQ, vg = vk >> 3;
+    const int vb0 = G::NQ == 32 ? 0 : lane / G::NQ;
+    uint32_t *ybuf = reinterpret_cast<uint32_t *>(scr);
+    float *fsit = reinterpret_cast<float *>(ybuf + NCG * YS);
+
+    // Row ri of this CTA: the warps' groups, the tail (last CTA), the CTA partial
+    // (o, l in units of 2^-m, and m) into parts[ri % 3].
+    auto row_pass = [&](int ri) {
+        // set up row ri + 1 (row 0 first); its slot last held row ri - 1, whose stages were
+        // all issued and read
+        for (int r = ri == 0 ? 0 : ri + 1; r <= ri + 1 && r < nrows; ++r) {
+            setup_row(r);
+            setup_upto = r;
+        }
+        const int32_t *srow = irow_of(ri);
+        const int row = srow[IR_ROW], nown = srow[IR_N], tail = srow[IR_TAIL];
+        if (ri == 0) { // prefetch, then wait for the previous grid of the stream (see decode_kernel)
+            pump(prc_n + spw);
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+        }
+        float qreg[4];
+        {
+            const DT *qrow = reinterpret_cast<const DT *>(a.q) + (int64_t)row * D + 4 * lane;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                qreg[i] = ownq ? to_f32(qrow[i]) * a.qscale : 0.f;
+        }
+        float m_run = -INFINITY, lsum = 0.f;
+        float facc[4] = {0.f, 0.f, 0.f, 0.f};
+        float zl[NCG];
+#pragma unroll
+        for (int g = 0; g < NCG; ++g)
+            zl[g] = 0.f;
+        for (int k = 0; k < nown; ++k) {
+            const int n = prc_n++;
+            if (iss_n < n + spw)
+                pump(n + spw);
+            wait_stage(n);
+            const uint8_t *st = ring + (n & smask) * G1::STAGE;
+            // ---- keys: the exact integer dot products of decode_kernel's key pass
+            const int hf = lane >> 4;
+            constexpr int HW = G::WORDSK / 2;
+            const uint8_t *krA = st + (lane & 15) * G::ROWK + hf * (G::ROWK / 2);
+            const uint8_t *krB = krA + G::HM;
+            uint32_t cwA[HW], cwB[HW];
+#pragma unroll
+            for (int w = 0; w < HW; w += (HW % 4 == 0 ? 4 : 2)) {
+                if (HW % 4 == 0) {
+                    const uint4 ca = *reinterpret_cast<const uint4 *>(krA + 4 * w);
+                    const uint4 cb = *reinterpret_cast<const uint4 *>(krB + 4 * w);
+                    cwA[w] = ca.x, cwA[w + 1] = ca.y, cwA[w + 2] = ca.z, cwA[w + 3] = ca.w;
+                    cwB[w] = cb.x, cwB[w + 1] = cb.y, cwB[w + 2] = cb.z, cwB[w + 3] = cb.w;
+                } else {
+                    const uint2 ca = *reinterpret_cast<const uint2 *>(krA + 4 * w);
+                    const uint2 cb = *reinterpret_cast<const uint2 *>(krB + 4 * w);
+                    cwA[w] = ca.x, cwA[w + 1] = ca.y;
+                    cwB[w] = cb.x, cwB[w + 1] = cb.y;
+                }
+            }
+            float av[4], zs = 0.f;
+            {
+                uint2 sr = make_uint2(0u, 0u), zr = make_uint2(0u, 0u);
+                if (ownq) {
+                    sr = *reinterpret_cast<const uint2 *>(st + G::KCODES + 8 * lane);          // scales (even block)
+                    zr = *reinterpret_cast<const uint2 *>(st + G::HM + G::KCODES + 8 * lane); // zeros (odd block)
+                }
+                const float2 s01 = __half22float2(*reinterpret_cast<const __half2 *>(&sr.x));
+                const float2 s23 = __half22float2(*reinterpret_cast<const __half2 *>(&sr.y));
+                const float2 z01 = __half22float2(*reinterpret_cast<const __half2 *>(&zr.x));
+                const float2 z23 = __half22float2(*reinterpret_cast<const __half2 *>(&zr.y));
+                av[0] = qreg[0] * s01.x;
+                av[1] = qreg[1] * s01.y;
+                av[2] = qreg[2] * s23.x;
+                av[3] = qreg[3] * s23.y;
+                zs = fmaf(qreg[0], z01.x, fmaf(qreg[1], z01.y, fmaf(qreg[2], z23.x, qreg[3] * z23.y)));
+            }
+            const float amax = warp_max_abs(fmaxf(fmaxf(fabsf(av[0]), fabsf(av[1])), fmaxf(fabsf(av[2]), fabsf(av[3]))));
+            zs = warp_sum(zs);
+            const uint32_t ab = __float_as_uint(amax);
+            int F = 21 - ((int)(ab >> 23) - 127) - ((ab & 0x7FFFFFu) >= 0x7FFFFEu ? 1 : 0);
+            F = F > 126 ? 126 : F;
+            const float fs = __int_as_float((F + 127) << 23), fsk = __int_as_float((127 - F) << 23);
+            if (ownq) {
+                const uint32_t y0 = __float_as_uint(fmaf(av[0], fs, 12582912.f));
+                const uint32_t y1 = __float_as_uint(fmaf(av[1], fs, 12582912.f));
+                const uint32_t y2 = __float_as_uint(fmaf(av[2], fs, 12582912.f));
+                const uint32_t y3 = __float_as_uint(fmaf(av[3], fs, 12582912.f));
+                const uint32_t t01 = __byte_perm(y0, y1, 0x5140), t23 = __byte_perm(y2, y3, 0x5140);
+                const uint32_t u01 = __byte_perm(y0, y1, 0x0062), u23 = __byte_perm(y2, y3, 0x0062);
+                const uint32_t d0 = __byte_perm(t01, t23, 0x5410), d1 = __byte_perm(t01, t23, 0x7632);
+                const uint32_t x2 = __byte_perm(u01, u23, 0x5410) ^ 0x40404040u;
+                const uint32_t d2 = x2 | ((x2 & 0x40404040u) << 1);
+                reinterpret_cast<uint4 *>(scr)[lane] = make_uint4(d0, d1, d2, 0u);
+            }
+            __syncwarp();
+            constexpr int QPW = BITS == 4 ? 2 : 4;
+            const uint4 *rh = rec + hf * (G::NQ / 2);
+            KeyAcc accA = {{0u, 0u}, {0u, 0u}, {0, 0}}, accB = {{0u, 0u}, {0u, 0u}, {0, 0}};
+#pragma unroll
+            for (int w = 0; w < HW; ++w)
+                key_word2<BITS>(cwA[w], cwB[w], rh + QPW * w, accA, accB);
+            const uint32_t a01A = accA.a0[0] + accA.a0[1] + ((accA.a1[0] + accA.a1[1]) << 8);
+            const uint32_t a01B = accB.a0[0] + accB.a0[1] + ((accB.a1[0] + accB.a1[1]) << 8);
+            const int a2A = accA.a2[0] + accA.a2[1], a2B = accB.a2[0] + accB.a2[1];
+            const uint32_t a01 = (hf ? a01B : a01A) + __shfl_xor_sync(0xFFFFFFFFu, hf ? a01A : a01B, 16);
+            const int a2 = (hf ? a2B : a2A) + __shfl_xor_sync(0xFFFFFFFFu, hf ? a2A : a2B, 16);
+            const float s2l = fmaf(fmaf((float)a2, 65536.f, (float)a01), fsk, zs); // score of token `lane`
+            // ---- running maximum (warp-uniform): rescale the warp's sums when it grows
+            const float mg = warp_max_f(s2l);
+            if (mg > m_run) {
+                const float f = ex2(m_run - mg); // 0 at the first group
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    facc[i] *= f;
+#pragma unroll
+                for (int g = 0; g < NCG; ++g)
+                    zl[g] *= f;
+                lsum *= f;
+                m_run = mg;
+            }
+            const float wl = ex2(s2l - m_run);
+            lsum += wl;
+            if (a.s_bitmap && lane == 0) // refine set: every token (4-bit, tau <= 0) or none (2-bit)
+                a.s_bitmap[(int64_t)row * a.bitmap_words + (int)crank + (warp + k * kWarps) * (int)C] =
+                    BITS == 4 ? 0xFFFFFFFFu : 0u;
+            __syncwarp(); // the key digit records are read: the scratch takes the value weights
+            // ---- values: decode_kernel's value pass with every token hot
+            {
+                const uint8_t *vm = st + (lane >> 4) * G::HM + G::KB + (lane & 15) * 4; // (scale, zero) of group g at + 64 g
+                float W[NCG], wmax = 0.f;
+#pragma unroll
+                for (int g = 0; g < NCG; ++g) {
+                    const float2 m = __half22float2(*reinterpret_cast<const __half2 *>(vm + 64 * g));
+                    zl[g] = fmaf(wl, m.y, zl[g]);
+                    W[g] = wl * m.x;
+                    wmax = fmaxf(wmax, W[g]);
+                }
+                wmax = warp_max_f(wmax);
+                int Fv = 20 - ((int)(__float_as_uint(wmax) >> 23) - 127);
+                Fv = Fv > 126 ? 126 : Fv;
+                const float fv = __int_as_float((Fv + 127) << 23);
+#pragma unroll
+                for (int g = 0; g < NCG; ++g)
+                    ybuf[g * YS + lane] = __float_as_uint(fmaf(W[g], fv, 8388608.f));
+                if (lane == 0)
+                    *fsit = __int_as_float((127 - Fv) << 23);
+            }
+            __syncwarp();
+            if (pv) {
+                const uint4 y = *reinterpret_cast<const uint4 *>(ybuf + pg * YS + 4 * pt8);
+                const uint32_t t01 = __byte_perm(y.x, y.y, 0x5140), t23 = __byte_perm(y.z, y.w, 0x5140);
+                const uint32_t u01 = __byte_perm(y.x, y.y, 0x0062), u23 = __byte_perm(y.z, y.w, 0x0062);
+                reinterpret_cast<uint4 *>(ybuf + pg * YS)[pt8] =
+                    make_uint4(__byte_perm(t01, t23, 0x5410), __byte_perm(t01, t23, 0x7632),
+                               __byte_perm(u01, u23, 0x5410), 0u);
+            }
+            __syncwarp();
+            uint32_t a0[4] = {0u, 0u, 0u, 0u}, a1[4] = {0u, 0u, 0u, 0u}, a2v[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int bb = 0; bb < BPL; ++bb) {
+                const int blk = vb0 + bb;
+                const uint4 h4 = *reinterpret_cast<const uint4 *>(st + blk * G::HM + G::KB + G::VMETA + 16 * vk);
+                const uint32_t hwv[4] = {h4.x, h4.y, h4.z, h4.w};
+                const uint8_t *lop = st + G1::LOFF + blk * G::LOB + 4 * vk;
+                const uint4 *rq = reinterpret_cast<const uint4 *>(ybuf + vg * YS) + 4 * blk;
+#pragma unroll
+                for (int tau = 0; tau < 4; ++tau) {
+                    const uint4 rc = rq[tau];
+                    const uint32_t hw = hwv[tau];
+                    uint32_t c4[4];
+                    if (BITS == 2) { // own 2-bit codes: channel i of every byte at bit 2i
+                        c4[0] = hw & 0x03030303u;
+                        c4[1] = (hw >> 2) & 0x03030303u;
+                        c4[2] = (hw >> 4) & 0x03030303u;
+                        c4[3] = (hw >> 6) & 0x03030303u;
+                    } else { // 4h + l
+                        const uint32_t lw = *reinterpret_cast<const uint32_t *>(lop + tau * D);
+                        const uint32_t E = ((hw << 2) & 0xCCCCCCCCu) | (lw & 0x33333333u);
+                        const uint32_t O = (hw & 0xCCCCCCCCu) | ((lw >> 2) & 0x33333333u);
+                        c4[0] = E & 0x0F0F0F0Fu;
+                        c4[1] = O & 0x0F0F0F0Fu;
+                        c4[2] = (E >> 4) & 0x0F0F0F0Fu;
+                        c4[3] = (O >> 4) & 0x0F0F0F0Fu;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        dp4a_uu(a0[i], c4[i], rc.x);
+                        dp4a_uu(a1[i], c4[i], rc.y);
+                        dp4a_uu(a2v[i], c4[i], rc.z);
+                    }
+                }
+            }
+            const float fsi = *fsit;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                facc[i] = fmaf((float)(a0[i] + (a1[i] << 8) + (a2v[i] << 16)), fsi, facc[i]);
+            __syncwarp();
+        }
+        // the warp's zero terms (reduce-scatter as in decode_kernel), sums and partial o, l
+#pragma unroll
+        for (int s2 = 0; (1 << s2) < NCG; ++s2) {
+            const int off = 1 << s2, len = NCG >> (s2 + 1);
+            const bool up = (lane & off) != 0;
+#pragma unroll
+            for (int m = 0; m < len; ++m) {
+                const float send = up ? zl[2 * m] : zl[2 * m + 1];
+                const float keep = up ? zl[2 * m + 1] : zl[2 * m];
+                zl[m] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, off);
+            }
+        }
+        float zsum = zl[0];
+#pragma unroll
+        for (int off = NCG; off < 32; off <<= 1)
+            zsum += __shfl_xor_sync(0xFFFFFFFFu, zsum, off);
+        const float zacc = __shfl_sync(0xFFFFFFFFu, zsum, vg);
+        lsum = warp_sum(lsum);
+        if (BPL == 1)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                facc[i] += __shfl_xor_sync(0xFFFFFFFFu, facc[i], 16);
+        __syncwarp();
+        float *red = reinterpret_cast<float *>(scr);
+        if (lane < G::NQ)
+            *reinterpret_cast<float4 *>(red + 4 * vk) =
+                make_float4(facc[0] + zacc, facc[1] + zacc, facc[2] + zacc, facc[3] + zacc);
+        if (lane == 0)
+            red[D] = lsum;
+        __syncwarp();
+        if (tail > 0 && warp == kWarps - 1) { // tail tokens, exact; lane = tail token
+            const int b = srow[IR_B], h = srow[IR_H];
+            const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)b * 2 * a.H + h) * 32 * D;
+            float s2 = 0.f;
+            for (int q4 = 0; q4 < G::NQ; ++q4) {
+                float kv[4] = {0.f, 0.f, 0.f, 0.f};
+                if (lane < tail)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        kv[i] = to_f32(kt[(int64_t)lane * D + 4 * q4 + i]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    s2 = fmaf(__shfl_sync(0xFFFFFFFFu, qreg[i], q4), kv[i], s2);
+            }
+            const float mt = warp_max_f(lane < tail ? s2 : -INFINITY);
+            if (mt > m_run) { // rescale the warp's partial in the scratch
+                const float f = ex2(m_run - mt);
+                for (int c = lane; c <= D; c += 32)
+                    red[c] *= f;
+                m_run = mt;
+            }
+            __syncwarp();
+            const DT *vt0 = reinterpret_cast<const DT *>(a.tail) + ((int64_t)(b * 2 + 1) * a.H + h) * 32 * D;
+            float tl = 0.f;
+            for (int t = 0; t < tail; ++t) {
+                const float w = ex2(__shfl_sync(0xFFFFFFFFu, s2, t) - m_run);
+                tl += w;
+                const DT *vt = vt0 + (int64_t)t * D;
+#pragma unroll
+                for (int c4 = 0; c4 < D / 32; ++c4)
+                    red[lane + 32 * c4] = fmaf(w, to_f32(vt[lane + 32 * c4]), red[lane + 32 * c4]);
+            }
+            __syncwarp();
+            if (lane == 0)
+                red[D] += tl;
+        }
+        if (lane == 0)
+            wm[warp] = m_run;
+        named_sync(1, kThreads);
+        // CTA partial relative to the CTA's maximum mc
+        float mc = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w)
+            mc = fmaxf(mc, wm[w]);
+        float fw[kWarps];
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w)
+            fw[w] = wm[w] == -INFINITY ? 0.f : ex2(wm[w] - mc);
+        float *part = parts + (ri % 3) * (D + 2);
+        for (int c = threadIdx.x; c <= D; c += kThreads) {
+            float sum = 0.f;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w)
+                sum += fw[w] * reinterpret_cast<const float *>(scr_all + w * SCR)[c];
+            part[c] = sum;
+        }
+        if (threadIdx.x == 0)
+            part[D + 1] = mc;
+        named_sync(1, kThreads); // every warp's scratch and wm are free again
+    };
+
+    // CTA `crank` writes channels [crank*per, min(D, (crank+1)*per)) of row ri, per =
+    // ceil(D / C), from the partials of every CTA rescaled to the row maximum M.
+    auto merge = [&](int ri) {
+        const int row = row_of(ri);
+        const float *part = parts + (ri % 3) * (D + 2);
+        const int per = (D + (int)C - 1) / (int)C;
+        const int c = (int)crank * per + (int)threadIdx.x;
+        if ((int)threadIdx.x < per && c < D) {
+            float M = -INFINITY;
+            for (uint32_t r = 0; r < C; ++r)
+                M = fmaxf(M, ld_dsmem_f32(part + D + 1, r));
+            float o = 0.f, l = 0.f;
+            if (M != -INFINITY)
+                for (uint32_t r = 0; r < C; ++r) {
+                    const float mr = ld_dsmem_f32(part + D + 1, r);
+                    const float f = mr == -INFINITY ? 0.f : ex2(mr - M);
+                    o = fmaf(f, ld_dsmem_f32(part + c, r), o);
+                    l = fmaf(f, ld_dsmem_f32(part + D, r), l);
+                }
+            float out = 0.f;
+            if (l > 0.f)
+                out = o / l;
+            else if (c == 0)
+                atomicOr(a.status, LOOPKV_DEV_EMPTY_ROW);
+            a.out[(int64_t)row * D + c] = out;
+            if (c == 0) {
+                if (a.row_max)
+                    a.row_max[row] = M * 0.6931471805599453f;
+                if (a.row_sum)
+                    a.row_sum[row] = l;
+            }
+        }
+    };
+
+    // One cluster barrier per row: barrier i publishes the partials of row i, merged after
+    // the next row's pass.  parts[i % 3] is written again at row i + 3, after this CTA
+    // passed barrier i + 1, which every CTA reaches only after its merge of row i.
+    for (int i = 0; i <= nrows; ++i) {
+        if (i < nrows)
+            row_pass(i);
+        if (i > 0) {
+            cluster_wait(); // barrier i - 1
+            merge(i - 1);
+        }
+        if (i < nrows)
+            cluster_arrive(); // barrier i
+    }
+    cluster_arrive(); // the remote reads of the last merge are done
+    cluster_wait();
+}
+
+// Launch `kern` with the shape's grid, cluster and shared memory (and programmatic
+// stream serialization when the shape asks for it).
+template <typename K, typename... Args>
+int launch_shape(K kern, const DecodeShape &shp, cudaStream_t s, Args... args)
+{
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, shp.smem);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
@@ -1079,18 +1644,26 @@ int launch_t(const DecodeArgs &a, const DecodeShape &shp, cudaStream_t s)
     attr[0].val.clusterDim.x = shp.cluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization; // see griddepcontrol in the kernel
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization; // see griddepcontrol in the kernels
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = shp.pdl ? 2 : 1;
-    e = cudaLaunchKernelEx(&cfg, kern, a, shp.stages_log2, shp.score_bufs);
+    e = cudaLaunchKernelEx(&cfg, kern, args...);
     return e == cudaSuccess ? LOOPKV_OK : LOOPKV_ERR_CUDA;
 }
 
-// Clusters of size C that can be resident at once for this kernel and shared memory.
-template <int BITS, int D, typename DT> int max_active_clusters(int C, int smem, int min_ctas)
+template <int BITS, int D, typename DT>
+int launch_t(const DecodeArgs &a, const DecodeShape &shp, cudaStream_t s)
 {
-    auto kern = min_ctas == 5 ? decode_kernel<BITS, D, DT, 5> : decode_kernel<BITS, D, DT, 4>;
+    if (shp.onepass)
+        return launch_shape(decode_kernel_1p<BITS, D, DT, 4>, shp, s, a, shp.stages_log2);
+    auto kern = shp.min_ctas == 5 ? decode_kernel<BITS, D, DT, 5> : decode_kernel<BITS, D, DT, 4>;
+    return launch_shape(kern, shp, s, a, shp.stages_log2, shp.score_bufs);
+}
+
+// Clusters of size C that can be resident at once for this kernel and shared memory.
+template <typename K> int max_active_clusters(K kern, int C, int smem)
+{
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return 0;
     cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
@@ -1134,7 +1707,15 @@ inline int pdl_default(int C)
     return C <= 4;
 }
 
-template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_blocks)
+// Shared memory of a kernel with `spw` ring slots per warp.
+template <int BITS, int D> int kernel_smem(bool onepass, int spw, int capw, int nbuf)
+{
+    if (onepass)
+        return layout1_ok<BITS, D>(spw, capw) ? smem_layout1<BITS, D>(spw, capw).total : -1;
+    return layout_ok<BITS, D>(spw, capw, nbuf) ? smem_bytes<BITS, D>(spw, capw, nbuf) : -1;
+}
+
+template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_blocks, bool onepass)
 {
     DecodeShape best = {};
     double best_t = 1e300;
@@ -1150,7 +1731,8 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
     const char *env_c = getenv("LOOPKV_DECODE_CLUSTER");
     const char *env_s = getenv("LOOPKV_DECODE_STAGES");
     const char *env_o = getenv("LOOPKV_DECODE_CTAS_PER_SM");
-    for (int want_ctas = 4; want_ctas <= 5; ++want_ctas) {
+    // the single-pass kernel is built for 4 CTAs per SM; the two-phase one for 4 or 5
+    for (int want_ctas = 4; want_ctas <= (onepass ? 4 : 5); ++want_ctas) {
         if (env_o && atoi(env_o) != want_ctas)
             continue;
         for (int C = 1; C <= 16; C = C < 8 ? C + 1 : 2 * C) { // 1..8, 16
@@ -1162,19 +1744,21 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
             for (int nbuf = 1; nbuf <= 2; ++nbuf) {
                 // slots per warp (a power of two): fill the shared memory of `want_ctas` CTAs per SM
                 int spw = 8;
-                while (spw > 2 && smem_bytes<BITS, D>(spw, capw, nbuf) > budget)
+                while (spw > 2 && kernel_smem<BITS, D>(onepass, spw, capw, nbuf) > budget)
                     spw >>= 1;
                 if (env_s)
                     spw = atoi(env_s);
-                const int smem = smem_bytes<BITS, D>(spw, capw, nbuf);
-                if (smem > 227 * 1024 || !layout_ok<BITS, D>(spw, capw, nbuf))
+                const int smem = kernel_smem<BITS, D>(onepass, spw, capw, nbuf);
+                if (smem <= 0 || smem > 227 * 1024)
                     continue;
-                int ncl = max_active_clusters<BITS, D, DT>(C, smem, want_ctas);
+                int ncl = onepass ? max_active_clusters(decode_kernel_1p<BITS, D, DT, 4>, C, smem)
+                          : want_ctas == 5 ? max_active_clusters(decode_kernel<BITS, D, DT, 5>, C, smem)
+                                           : max_active_clusters(decode_kernel<BITS, D, DT, 4>, C, smem);
                 if (ncl <= 0)
                     continue;
                 if (ncl > rows)
                     ncl = rows;
-                if (nbuf == 1 && ncl < rows)
+                if (!onepass && nbuf == 1 && ncl < rows)
                     continue; // a cluster would read several rows: it needs two score buffers
                 const int rounds = (rows + ncl - 1) / ncl;
                 const int per_sm = (ncl * C + sm_count - 1) / sm_count;
@@ -1186,12 +1770,13 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
                     best.clusters = ncl;
                     best.stages = spw;
                     best.stages_log2 = __builtin_ctz(spw);
-                    best.score_bufs = nbuf;
+                    best.score_bufs = onepass ? 0 : nbuf;
                     best.smem = smem;
                     best.threads = kThreads;
                     best.cap = cap;
                     best.min_ctas = want_ctas;
                     best.pdl = pdl_default(C);
+                    best.onepass = onepass;
                 }
                 break;
             }
@@ -1202,17 +1787,18 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
 
 }  // namespace
 
-DecodeShape decode_shape(int bits, int D, int dtype, int rows, int max_blocks)
+DecodeShape decode_shape(int bits, int D, int dtype, int rows, int max_blocks, bool onepass)
 {
     const bool bf = dtype == LOOPKV_DTYPE_BF16;
+    const int mb = max_blocks;
     if (bits == 4) {
         if (D == 128)
-            return bf ? shape_t<4, 128, __nv_bfloat16>(rows, max_blocks) : shape_t<4, 128, float>(rows, max_blocks);
-        return bf ? shape_t<4, 64, __nv_bfloat16>(rows, max_blocks) : shape_t<4, 64, float>(rows, max_blocks);
+            return bf ? shape_t<4, 128, __nv_bfloat16>(rows, mb, onepass) : shape_t<4, 128, float>(rows, mb, onepass);
+        return bf ? shape_t<4, 64, __nv_bfloat16>(rows, mb, onepass) : shape_t<4, 64, float>(rows, mb, onepass);
     }
     if (D == 128)
-        return bf ? shape_t<2, 128, __nv_bfloat16>(rows, max_blocks) : shape_t<2, 128, float>(rows, max_blocks);
-    return bf ? shape_t<2, 64, __nv_bfloat16>(rows, max_blocks) : shape_t<2, 64, float>(rows, max_blocks);
+        return bf ? shape_t<2, 128, __nv_bfloat16>(rows, mb, onepass) : shape_t<2, 128, float>(rows, mb, onepass);
+    return bf ? shape_t<2, 64, __nv_bfloat16>(rows, mb, onepass) : shape_t<2, 64, float>(rows, mb, onepass);
 }
 
 int launch_decode(const DecodeArgs &a, int bits, int D, int dtype, const DecodeShape &shp, cudaStream_t s)

@@ -64,11 +64,14 @@ struct DecodeShape {
     int threads;
     int cap;       // score capacity per CTA and row, in 32-token groups
     int pdl;       // launch with programmatic stream serialization (overlap the previous launch)
+    int onepass;   // single-pass kernel (refine set independent of the row maximum)
 };
 
 // Launchers (defined in the .cu files).  Return LOOPKV_OK or an error code.
 int launch_decode(const DecodeArgs &a, int bits, int D, int dtype, const DecodeShape &shp, cudaStream_t s);
-DecodeShape decode_shape(int bits, int D, int dtype, int rows, int max_blocks);
+// onepass: the rows' refine set does not depend on the row maximum (2-bit source, or a
+// 4-bit source read with tau <= 0), so the single-pass kernel may read them.
+DecodeShape decode_shape(int bits, int D, int dtype, int rows, int max_blocks, bool onepass);
 
 int launch_init_state(const DevState &st, cudaStream_t s);
 int launch_append(const DevState &st, int cell, int H, int D, int dtype, int max_batch, const void *k,

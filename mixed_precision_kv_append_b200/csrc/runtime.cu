@@ -8,6 +8,7 @@
 #include <cstring>
 #include <map>
 #include <new>
+#include <tuple>
 #include <vector>
 
 #include "lkv_internal.h"
@@ -28,16 +29,16 @@ struct loopkv_plan {
 
 struct loopkv_cache {
     loopkv_plan plan;
-    // decode launch shapes by (storage bits, batch), computed once (occupancy queries
-    // must not run while a stream is being captured)
-    std::map<std::pair<int, int>, lkv::DecodeShape> shapes;
-    const lkv::DecodeShape &shape(int bits, int B)
+    // decode launch shapes by (storage bits, batch, single-pass), computed once (occupancy
+    // queries must not run while a stream is being captured)
+    std::map<std::tuple<int, int, bool>, lkv::DecodeShape> shapes;
+    const lkv::DecodeShape &shape(int bits, int B, bool onepass)
     {
-        auto key = std::make_pair(bits, B);
+        auto key = std::make_tuple(bits, B, onepass);
         auto it = shapes.find(key);
         if (it == shapes.end())
             it = shapes.emplace(key, lkv::decode_shape(bits, plan.cfg.head_dim, plan.cfg.in_dtype,
-                                                       B * plan.cfg.n_heads, plan.cfg.max_blocks_per_seq))
+                                                       B * plan.cfg.n_heads, plan.cfg.max_blocks_per_seq, onepass))
                      .first;
         return it->second;
     }
@@ -57,6 +58,19 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 int dtype_size(int dt) { return dt == LOOPKV_DTYPE_BF16 ? 2 : 4; }
 
 int head_main_bytes(int bits, int D) { return bits == 4 ? LKV_HEAD_MAIN_4B(D) : LKV_HEAD_MAIN_2B(D); }
+
+// Whether a read's refine set is fixed before any score is known: a 2-bit source has no lo
+// plane (S empty), a 4-bit source read with tau <= 0 refines every token.  Such reads go to
+// the single-pass kernel (running maximum); LOOPKV_DECODE_ONEPASS=0 keeps them on the
+// two-phase one.
+bool single_pass(int bits, float tau)
+{
+    static const bool allowed = [] {
+        const char *env = getenv("LOOPKV_DECODE_ONEPASS");
+        return !env || atoi(env) != 0;
+    }();
+    return allowed && (bits == 2 || !(tau > 0.f));
+}
 
 int check_config(const loopkv_config *c)
 {
@@ -457,7 +471,7 @@ int loopkv_decode_debug(const loopkv_plan *plan, int loop, int layer, const void
     a.qscale = (float)(1.4426950408889634 / std::sqrt((double)D));
     a.tau = plan->tau;
     a.tau_mode = plan->tau_mode;
-    const lkv::DecodeShape &shp = cache->shape(bits, B);
+    const lkv::DecodeShape &shp = cache->shape(bits, B, single_pass(bits, plan->tau));
     a.cap_groups = shp.cap;
     return lkv::launch_decode(a, bits, D, cp.cfg.in_dtype, shp, static_cast<cudaStream_t>(stream));
 }
@@ -532,9 +546,9 @@ int loopkv_decode_shape(const loopkv_plan *plan, int B, int *cluster_size, int *
         return LOOPKV_ERR_INVALID_ARG;
     if (check_device())
         return LOOPKV_ERR_NO_DEVICE; // the shape comes from an occupancy query of the device
-    // the shape of a 4-bit source cell (the larger pipeline stage)
+    // the shape of a 4-bit source cell (the larger pipeline stage) under the plan's tau
     lkv::DecodeShape shp = lkv::decode_shape(4, plan->cfg.head_dim, plan->cfg.in_dtype, B * plan->cfg.n_heads,
-                                             plan->cfg.max_blocks_per_seq);
+                                             plan->cfg.max_blocks_per_seq, single_pass(4, plan->tau));
     if (cluster_size)
         *cluster_size = shp.cluster;
     if (ctas)
