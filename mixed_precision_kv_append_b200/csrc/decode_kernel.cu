@@ -1075,11 +1075,15 @@ template <int BITS, int D> struct Geo1 {
 };
 
 struct SmemLayout1 {
-    int full, scr, wm, part, ids, irow, order, total;
+    int full, scr, part, ids, irow, order, total;
 };
 
-// Row slots (ids, irow) by row parity: while a warp reads row r its issuer may start row
-// r + 1.  CTA partials (o[D], l, m) by row index mod 3 (see the barrier note in the kernel).
+// One row slot (block ids, row fields) per warp: the next row is set up once the current
+// row's stages are all issued.  A warp's maximum sits in its scratch after its partial
+// (word D + 1).  CTA partials (o[D], l, m) by row parity (see the barrier note in the
+// kernel).
+constexpr int kFields1 = 8;
+
 template <int BITS, int D> __host__ __device__ constexpr SmemLayout1 smem_layout1(int spw, int capw)
 {
     SmemLayout1 L{};
@@ -1088,14 +1092,12 @@ template <int BITS, int D> __host__ __device__ constexpr SmemLayout1 smem_layout
     o = align16(o + kWarps * spw * 8);
     L.scr = o;
     o = align16(o + kWarps * scratch_bytes<D>());
-    L.wm = o;
-    o = align16(o + kWarps * 4);
     L.part = o;
-    o = align16(o + 3 * (D + 2) * 4);
+    o = align16(o + 2 * (D + 2) * 4);
     L.ids = o;
-    o = align16(o + 2 * kWarps * 2 * capw * 4);
+    o = align16(o + kWarps * 2 * capw * 4);
     L.irow = o;
-    o = align16(o + 2 * kWarps * IR_N_FIELDS * 4);
+    o = align16(o + kWarps * kFields1 * 4);
     L.order = o;
     o = align16(o + kMaxOrder * 4);
     L.total = o;
@@ -1105,16 +1107,295 @@ template <int BITS, int D> __host__ __device__ constexpr SmemLayout1 smem_layout
 template <int BITS, int D> bool layout1_ok(int spw, int capw)
 {
     const SmemLayout1 L = smem_layout1<BITS, D>(spw, capw);
-    const int offs[] = {L.full, L.scr, L.wm, L.part, L.ids, L.irow, L.order};
+    const int offs[] = {L.full, L.scr, L.part, L.ids, L.irow, L.order};
     int prev = kWarps * spw * Geo1<BITS, D>::STAGE;
     for (int o : offs) {
         if (o % 16 || o < prev)
             return false;
         prev = o;
     }
-    // the request lengths are ranked in the warps' scratch at kernel start
+    // the request lengths are ranked in the warps' scratch at kernel start; a warp's
+    // partial and maximum take D + 2 words of its scratch; id pairs are read as int2
     return L.total >= prev && (spw & (spw - 1)) == 0 && kWarps * scratch_bytes<D>() >= kMaxOrder * 4 &&
-           (Geo1<BITS, D>::STAGE % 128) == 0 && (Geo<BITS, D>::HM % 16) == 0 && (Geo<BITS, D>::LOB % 16) == 0;
+           scratch_bytes<D>() >= (D + 2) * 4 && (2 * capw * 4) % 8 == 0 && (Geo1<BITS, D>::STAGE % 128) == 0 &&
+           (Geo<BITS, D>::HM % 16) == 0 && (Geo<BITS, D>::LOB % 16) == 0;
+}
+
+// Running state of one warp over its groups of a row (single-pass reader): maximum m
+// (log2 units), l = sum of 2^(s - m), the lane's channel-quad sums o of 2^(s - m) * s_v *
+// code, and the lane-token's zero terms z per 32-channel group (also relative to 2^m).
+template <int D> struct Run1 {
+    float m, l;
+    float o[4];
+    float z[D / 32];
+};
+
+template <int D> __device__ __forceinline__ void run1_init(Run1<D> &r)
+{
+    r.m = -INFINITY;
+    r.l = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        r.o[i] = 0.f;
+#pragma unroll
+    for (int g = 0; g < D / 32; ++g)
+        r.z[g] = 0.f;
+}
+
+// One 32-token group: head regions of its two blocks at st and st + HM, their lo regions
+// at lo (4-bit).  Exact integer key dot products (the key pass of decode_kernel), the
+// running-maximum update, then the value pass of decode_kernel with every token refined
+// (4-bit source) or plain 2-bit codes.  scr: the warp's scratch.
+template <int BITS, int D>
+__device__ __forceinline__ void run1_group(const uint8_t *st, const uint8_t *lo, uint8_t *scr, const float (&qreg)[4],
+                                           const int lane, Run1<D> &r)
+{
+    using G = Geo<BITS, D>;
+    const uint4 *rec = reinterpret_cast<const uint4 *>(scr);
+    const bool ownq = lane < G::NQ;
+    constexpr int NCG = G::NCG;
+    constexpr int YS = 40;
+    const int pt8 = lane / NCG, pg = lane % NCG;
+    const bool pv = pt8 < 8;
+    constexpr int BPL = G::NQ == 32 ? 2 : 1;
+    const int vk = lane % G::NQ, vg = vk >> 3;
+    const int vb0 = G::NQ == 32 ? 0 : lane / G::NQ;
+    uint32_t *ybuf = reinterpret_cast<uint32_t *>(scr);
+    float *fsit = reinterpret_cast<float *>(ybuf + NCG * YS);
+    // ---- keys: the exact integer dot products of decode_kernel's key pass
+    const int hf = lane >> 4;
+    constexpr int HW = G::WORDSK / 2;
+    const uint8_t *krA = st + (lane & 15) * G::ROWK + hf * (G::ROWK / 2);
+    const uint8_t *krB = krA + G::HM;
+    uint32_t cwA[HW], cwB[HW];
+#pragma unroll
+    for (int w = 0; w < HW; w += (HW % 4 == 0 ? 4 : 2)) {
+        if (HW % 4 == 0) {
+            const uint4 ca = *reinterpret_cast<const uint4 *>(krA + 4 * w);
+            const uint4 cb = *reinterpret_cast<const uint4 *>(krB + 4 * w);
+            cwA[w] = ca.x, cwA[w + 1] = ca.y, cwA[w + 2] = ca.z, cwA[w + 3] = ca.w;
+            cwB[w] = cb.x, cwB[w + 1] = cb.y, cwB[w + 2] = cb.z, cwB[w + 3] = cb.w;
+        } else {
+            const uint2 ca = *reinterpret_cast<const uint2 *>(krA + 4 * w);
+            const uint2 cb = *reinterpret_cast<const uint2 *>(krB + 4 * w);
+            cwA[w] = ca.x, cwA[w + 1] = ca.y;
+            cwB[w] = cb.x, cwB[w + 1] = cb.y;
+        }
+    }
+    float av[4], zs = 0.f;
+    {
+        uint2 sr = make_uint2(0u, 0u), zr = make_uint2(0u, 0u);
+        if (ownq) {
+            sr = *reinterpret_cast<const uint2 *>(st + G::KCODES + 8 * lane);          // scales (even block)
+            zr = *reinterpret_cast<const uint2 *>(st + G::HM + G::KCODES + 8 * lane); // zeros (odd block)
+        }
+        const float2 s01 = __half22float2(*reinterpret_cast<const __half2 *>(&sr.x));
+        const float2 s23 = __half22float2(*reinterpret_cast<const __half2 *>(&sr.y));
+        const float2 z01 = __half22float2(*reinterpret_cast<const __half2 *>(&zr.x));
+        const float2 z23 = __half22float2(*reinterpret_cast<const __half2 *>(&zr.y));
+        av[0] = qreg[0] * s01.x;
+        av[1] = qreg[1] * s01.y;
+        av[2] = qreg[2] * s23.x;
+        av[3] = qreg[3] * s23.y;
+        zs = fmaf(qreg[0], z01.x, fmaf(qreg[1], z01.y, fmaf(qreg[2], z23.x, qreg[3] * z23.y)));
+    }
+    const float amax = warp_max_abs(fmaxf(fmaxf(fabsf(av[0]), fabsf(av[1])), fmaxf(fabsf(av[2]), fabsf(av[3]))));
+    zs = warp_sum(zs);
+    const uint32_t ab = __float_as_uint(amax);
+    int F = 21 - ((int)(ab >> 23) - 127) - ((ab & 0x7FFFFFu) >= 0x7FFFFEu ? 1 : 0);
+    F = F > 126 ? 126 : F;
+    const float fs = __int_as_float((F + 127) << 23), fsk = __int_as_float((127 - F) << 23);
+    if (ownq) {
+        const uint32_t y0 = __float_as_uint(fmaf(av[0], fs, 12582912.f));
+        const uint32_t y1 = __float_as_uint(fmaf(av[1], fs, 12582912.f));
+        const uint32_t y2 = __float_as_uint(fmaf(av[2], fs, 12582912.f));
+        const uint32_t y3 = __float_as_uint(fmaf(av[3], fs, 12582912.f));
+        const uint32_t t01 = __byte_perm(y0, y1, 0x5140), t23 = __byte_perm(y2, y3, 0x5140);
+        const uint32_t u01 = __byte_perm(y0, y1, 0x0062), u23 = __byte_perm(y2, y3, 0x0062);
+        const uint32_t d0 = __byte_perm(t01, t23, 0x5410), d1 = __byte_perm(t01, t23, 0x7632);
+        const uint32_t x2 = __byte_perm(u01, u23, 0x5410) ^ 0x40404040u;
+        const uint32_t d2 = x2 | ((x2 & 0x40404040u) << 1);
+        reinterpret_cast<uint4 *>(scr)[lane] = make_uint4(d0, d1, d2, 0u);
+    }
+    __syncwarp();
+    constexpr int QPW = BITS == 4 ? 2 : 4;
+    const uint4 *rh = rec + hf * (G::NQ / 2);
+    KeyAcc accA = {{0u, 0u}, {0u, 0u}, {0, 0}}, accB = {{0u, 0u}, {0u, 0u}, {0, 0}};
+#pragma unroll
+    for (int w = 0; w < HW; ++w)
+        key_word2<BITS>(cwA[w], cwB[w], rh + QPW * w, accA, accB);
+    const uint32_t a01A = accA.a0[0] + accA.a0[1] + ((accA.a1[0] + accA.a1[1]) << 8);
+    const uint32_t a01B = accB.a0[0] + accB.a0[1] + ((accB.a1[0] + accB.a1[1]) << 8);
+    const int a2A = accA.a2[0] + accA.a2[1], a2B = accB.a2[0] + accB.a2[1];
+    const uint32_t a01 = (hf ? a01B : a01A) + __shfl_xor_sync(0xFFFFFFFFu, hf ? a01A : a01B, 16);
+    const int a2 = (hf ? a2B : a2A) + __shfl_xor_sync(0xFFFFFFFFu, hf ? a2A : a2B, 16);
+    const float s2l = fmaf(fmaf((float)a2, 65536.f, (float)a01), fsk, zs); // score of token `lane`
+    // ---- running maximum (warp-uniform): rescale the warp's sums when it grows
+    const float mg = warp_max_f(s2l);
+    if (mg > r.m) {
+        const float f = ex2(r.m - mg); // 0 at the first group
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            r.o[i] *= f;
+#pragma unroll
+        for (int g = 0; g < NCG; ++g)
+            r.z[g] *= f;
+        r.l *= f;
+        r.m = mg;
+    }
+    const float wl = ex2(s2l - r.m);
+    r.l += wl;
+    __syncwarp(); // the key digit records are read: the scratch takes the value weights
+    // ---- values: decode_kernel's value pass with every token hot
+    {
+        const uint8_t *vm = st + (lane >> 4) * G::HM + G::KB + (lane & 15) * 4; // (scale, zero) of group g at + 64 g
+        float W[NCG], wmax = 0.f;
+#pragma unroll
+        for (int g = 0; g < NCG; ++g) {
+            const float2 m = __half22float2(*reinterpret_cast<const __half2 *>(vm + 64 * g));
+            r.z[g] = fmaf(wl, m.y, r.z[g]);
+            W[g] = wl * m.x;
+            wmax = fmaxf(wmax, W[g]);
+        }
+        wmax = warp_max_f(wmax);
+        int Fv = 20 - ((int)(__float_as_uint(wmax) >> 23) - 127);
+        Fv = Fv > 126 ? 126 : Fv;
+        const float fv = __int_as_float((Fv + 127) << 23);
+#pragma unroll
+        for (int g = 0; g < NCG; ++g)
+            ybuf[g * YS + lane] = __float_as_uint(fmaf(W[g], fv, 8388608.f));
+        if (lane == 0)
+            *fsit = __int_as_float((127 - Fv) << 23);
+    }
+    __syncwarp();
+    if (pv) {
+        const uint4 y = *reinterpret_cast<const uint4 *>(ybuf + pg * YS + 4 * pt8);
+        const uint32_t t01 = __byte_perm(y.x, y.y, 0x5140), t23 = __byte_perm(y.z, y.w, 0x5140);
+        const uint32_t u01 = __byte_perm(y.x, y.y, 0x0062), u23 = __byte_perm(y.z, y.w, 0x0062);
+        reinterpret_cast<uint4 *>(ybuf + pg * YS)[pt8] =
+            make_uint4(__byte_perm(t01, t23, 0x5410), __byte_perm(t01, t23, 0x7632),
+                       __byte_perm(u01, u23, 0x5410), 0u);
+    }
+    __syncwarp();
+    uint32_t a0[4] = {0u, 0u, 0u, 0u}, a1[4] = {0u, 0u, 0u, 0u}, a2v[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int bb = 0; bb < BPL; ++bb) {
+        const int blk = vb0 + bb;
+        const uint4 h4 = *reinterpret_cast<const uint4 *>(st + blk * G::HM + G::KB + G::VMETA + 16 * vk);
+        const uint32_t hwv[4] = {h4.x, h4.y, h4.z, h4.w};
+        const uint8_t *lop = lo + blk * G::LOB + 4 * vk;
+        const uint4 *rq = reinterpret_cast<const uint4 *>(ybuf + vg * YS) + 4 * blk;
+#pragma unroll
+        for (int tau = 0; tau < 4; ++tau) {
+            const uint4 rc = rq[tau];
+            const uint32_t hw = hwv[tau];
+            uint32_t c4[4];
+            if (BITS == 2) { // own 2-bit codes: channel i of every byte at bit 2i
+                c4[0] = hw & 0x03030303u;
+                c4[1] = (hw >> 2) & 0x03030303u;
+                c4[2] = (hw >> 4) & 0x03030303u;
+                c4[3] = (hw >> 6) & 0x03030303u;
+            } else { // 4h + l
+                const uint32_t lw = *reinterpret_cast<const uint32_t *>(lop + tau * D);
+                const uint32_t E = ((hw << 2) & 0xCCCCCCCCu) | (lw & 0x33333333u);
+                const uint32_t O = (hw & 0xCCCCCCCCu) | ((lw >> 2) & 0x33333333u);
+                c4[0] = E & 0x0F0F0F0Fu;
+                c4[1] = O & 0x0F0F0F0Fu;
+                c4[2] = (E >> 4) & 0x0F0F0F0Fu;
+                c4[3] = (O >> 4) & 0x0F0F0F0Fu;
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                dp4a_uu(a0[i], c4[i], rc.x);
+                dp4a_uu(a1[i], c4[i], rc.y);
+                dp4a_uu(a2v[i], c4[i], rc.z);
+            }
+        }
+    }
+    const float fsi = *fsit;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        r.o[i] = fmaf((float)(a0[i] + (a1[i] << 8) + (a2v[i] << 16)), fsi, r.o[i]);
+    __syncwarp();
+}
+
+// End of a row for one warp: its partial o (zero terms added) into red[0 .. D-1] and l into
+// red[D], relative to 2^r.m.
+template <int BITS, int D> __device__ __forceinline__ void run1_finish(Run1<D> &r, float *red, const int lane)
+{
+    using G = Geo<BITS, D>;
+    constexpr int NCG = G::NCG;
+    constexpr int BPL = G::NQ == 32 ? 2 : 1;
+    const int vk = lane % G::NQ, vg = vk >> 3;
+    // the warp's zero terms (reduce-scatter as in decode_kernel), sums and partial o, l
+#pragma unroll
+    for (int s2 = 0; (1 << s2) < NCG; ++s2) {
+        const int off = 1 << s2, len = NCG >> (s2 + 1);
+        const bool up = (lane & off) != 0;
+#pragma unroll
+        for (int m = 0; m < len; ++m) {
+            const float send = up ? r.z[2 * m] : r.z[2 * m + 1];
+            const float keep = up ? r.z[2 * m + 1] : r.z[2 * m];
+            r.z[m] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, off);
+        }
+    }
+    float zsum = r.z[0];
+#pragma unroll
+    for (int off = NCG; off < 32; off <<= 1)
+        zsum += __shfl_xor_sync(0xFFFFFFFFu, zsum, off);
+    const float zacc = __shfl_sync(0xFFFFFFFFu, zsum, vg);
+    r.l = warp_sum(r.l);
+    if (BPL == 1)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            r.o[i] += __shfl_xor_sync(0xFFFFFFFFu, r.o[i], 16);
+    __syncwarp();
+    if (lane < G::NQ)
+        *reinterpret_cast<float4 *>(red + 4 * vk) =
+            make_float4(r.o[0] + zacc, r.o[1] + zacc, r.o[2] + zacc, r.o[3] + zacc);
+    if (lane == 0)
+        red[D] = r.l;
+    __syncwarp();
+}
+
+// Tail tokens t < tail (exact; lane = tail token) folded into the warp's partial red:
+// keys kt [32][D] and values vt0 [32][D]; rescales red when a tail score raises r.m.
+template <int D, typename DT>
+__device__ __forceinline__ void run1_tail(Run1<D> &r, float *red, const int lane, const float (&qreg)[4], const DT *kt,
+                                          const DT *vt0, const int tail)
+{
+    constexpr int NQ = D / 4;
+    float s2 = 0.f;
+    for (int q4 = 0; q4 < NQ; ++q4) {
+        float kv[4] = {0.f, 0.f, 0.f, 0.f};
+        if (lane < tail)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                kv[i] = to_f32(kt[(int64_t)lane * D + 4 * q4 + i]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            s2 = fmaf(__shfl_sync(0xFFFFFFFFu, qreg[i], q4), kv[i], s2);
+    }
+    const float mt = warp_max_f(lane < tail ? s2 : -INFINITY);
+    if (mt > r.m) { // rescale the warp's partial in the scratch
+        const float f = ex2(r.m - mt);
+        for (int c = lane; c <= D; c += 32)
+            red[c] *= f;
+        r.m = mt;
+    }
+    __syncwarp();
+    float tl = 0.f;
+    for (int t = 0; t < tail; ++t) {
+        const float w = ex2(__shfl_sync(0xFFFFFFFFu, s2, t) - r.m);
+        tl += w;
+        const DT *vt = vt0 + (int64_t)t * D;
+#pragma unroll
+        for (int c4 = 0; c4 < D / 32; ++c4)
+            red[lane + 32 * c4] = fmaf(w, to_f32(vt[lane + 32 * c4]), red[lane + 32 * c4]);
+    }
+    __syncwarp();
+    if (lane == 0)
+        red[D] += tl;
 }
 
 template <int BITS, int D, typename DT, int MINCTA>
@@ -1132,10 +1413,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
     constexpr int SCR = scratch_bytes<D>();
     uint64_t *fullb = reinterpret_cast<uint64_t *>(smem_raw + LY.full);
     uint8_t *scr_all = smem_raw + LY.scr;
-    float *wm = reinterpret_cast<float *>(smem_raw + LY.wm);
     float *parts = reinterpret_cast<float *>(smem_raw + LY.part);
-    int32_t *ids_all = reinterpret_cast<int32_t *>(smem_raw + LY.ids);
-    int32_t *irow_all = reinterpret_cast<int32_t *>(smem_raw + LY.irow);
     int32_t *order = reinterpret_cast<int32_t *>(smem_raw + LY.order);
     const uint32_t bstride = (uint32_t)a.H * G::HM, lstride = (uint32_t)a.H * G::LOB;
 
@@ -1179,13 +1457,12 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
     uint8_t *ring = smem_raw + warp * spw * G1::STAGE;
     uint64_t *full = fullb + warp * spw;
     uint8_t *scr = scr_all + warp * SCR;
-    auto ids_of = [&](int ri) { return ids_all + ((ri & 1) * kWarps + warp) * 2 * capw; };
-    auto irow_of = [&](int ri) { return irow_all + ((ri & 1) * kWarps + warp) * IR_N_FIELDS; };
+    int32_t *ids = reinterpret_cast<int32_t *>(smem_raw + LY.ids) + warp * 2 * capw;
+    int32_t *irow = reinterpret_cast<int32_t *>(smem_raw + LY.irow) + warp * kFields1;
 
     // ---------------------------------------------------------------- issuing
     int iss_n = 0, iss_row = -1, iss_k = 0, seg_n = 0, setup_upto = -1;
     const uint8_t *seg_src = nullptr, *seg_lo = nullptr;
-    const int2 *seg_ids = nullptr;
     // row parameters, validation and the warp's block ids of row ri (as in decode_kernel)
     auto setup_row = [&](int ri) {
         const int row = row_of(ri);
@@ -1210,7 +1487,6 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
             atomicOr(a.status, LOOPKV_DEV_STATE);
         const int n = owned(nmy, warp);
         const int32_t *bt = a.block_table + (int64_t)b * a.max_blocks;
-        int32_t *ids = ids_of(ri);
         for (int k = lane; k < 2 * n; k += 32) {
             const int g = (int)crank + (warp + (k >> 1) * kWarps) * (int)C;
             int id = bt[2 * g + (k & 1)];
@@ -1220,19 +1496,19 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
             }
             ids[k] = id;
         }
-        int32_t *st = irow_of(ri);
         if (lane == 0) {
-            st[IR_ROW] = row;
-            st[IR_B] = b;
-            st[IR_H] = h;
-            st[IR_N] = n;
-            st[IR_TAIL] = (crank == C - 1) ? tail : 0;
+            irow[IR_ROW] = row;
+            irow[IR_B] = b;
+            irow[IR_H] = h;
+            irow[IR_N] = n;
+            irow[IR_TAIL] = (crank == C - 1) ? tail : 0;
         }
         __syncwarp();
+        setup_upto = ri;
     };
     // stage n = the next group of the issuing row: both head regions (+ both lo regions)
     auto issue_stage = [&](int n) {
-        const int2 id = seg_ids[iss_k];
+        const int2 id = reinterpret_cast<const int2 *>(ids)[iss_k];
         uint8_t *st = ring + (n & smask) * G1::STAGE;
         uint64_t *fb = &full[n & smask];
         if (lane == 0) {
@@ -1256,20 +1532,19 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
                 ++iss_n;
                 continue;
             }
-            if (iss_row + 1 >= nrows || iss_row + 1 > setup_upto)
+            // move to the row in the slot; rows set up and replaced before the issuer got
+            // to them had no group for this warp
+            if (iss_row >= setup_upto)
                 break;
-            ++iss_row;
+            iss_row = setup_upto;
             iss_k = 0;
-            const int32_t *st = irow_of(iss_row);
-            seg_n = st[IR_N];
-            seg_src = a.main + (size_t)st[IR_H] * G::HM;
-            seg_lo = a.lo + (size_t)st[IR_H] * G::LOB;
-            seg_ids = reinterpret_cast<const int2 *>(ids_of(iss_row));
+            seg_n = irow[IR_N];
+            seg_src = a.main + (size_t)irow[IR_H] * G::HM;
+            seg_lo = a.lo + (size_t)irow[IR_H] * G::LOB;
         }
     };
 
     // ---------------------------------------------------------------- compute
-    const uint4 *rec = reinterpret_cast<const uint4 *>(scr);
     int prc_n = 0;
     bool timed_out = false;
     auto wait_stage = [&](int n) {
@@ -1277,27 +1552,18 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
             timed_out = !mbar_wait(&full[n & smask], (n >> spw_log2) & 1, a.status);
     };
     const bool ownq = lane < G::NQ;
-    constexpr int NCG = G::NCG;
-    constexpr int YS = 40;
-    const int pt8 = lane / NCG, pg = lane % NCG;
-    const bool pv = pt8 < 8;
-    constexpr int BPL = G::NQ == 32 ? 2 : 1;
-    const int vk = lane % G::NQ, vg = vk >> 3;
-    const int vb0 = G::NQ == 32 ? 0 : lane / G::NQ;
-    uint32_t *ybuf = reinterpret_cast<uint32_t *>(scr);
-    float *fsit = reinterpret_cast<float *>(ybuf + NCG * YS);
 
-    // Row ri of this CTA: the warps' groups, the tail (last CTA), the CTA partial
-    // (o, l in units of 2^-m, and m) into parts[ri % 3].
+    // Row ri of this CTA: the warp's groups and, in the last CTA, the tail; leaves the
+    // warp's partial (o, l relative to 2^m) in its scratch, m at word D + 1.
     auto row_pass = [&](int ri) {
-        // set up row ri + 1 (row 0 first); its slot last held row ri - 1, whose stages were
-        // all issued and read
-        for (int r = ri == 0 ? 0 : ri + 1; r <= ri + 1 && r < nrows; ++r) {
-            setup_row(r);
-            setup_upto = r;
-        }
-        const int32_t *srow = irow_of(ri);
-        const int row = srow[IR_ROW], nown = srow[IR_N], tail = srow[IR_TAIL];
+        if (ri == 0)
+            setup_row(0);
+        const int row = irow[IR_ROW], nown = irow[IR_N], tail = irow[IR_TAIL], rb = irow[IR_B], rh = irow[IR_H];
+        // the slot takes row ri + 1 once row ri's stages are all issued (after the pump of
+        // group nown - spw, or at once when the warp has no group)
+        const int k_setup = nown > spw ? nown - spw : 0;
+        if (nown == 0 && ri + 1 < nrows)
+            setup_row(ri + 1);
         if (ri == 0) { // prefetch, then wait for the previous grid of the stream (see decode_kernel)
             pump(prc_n + spw);
             asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -1309,256 +1575,50 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
             for (int i = 0; i < 4; ++i)
                 qreg[i] = ownq ? to_f32(qrow[i]) * a.qscale : 0.f;
         }
-        float m_run = -INFINITY, lsum = 0.f;
-        float facc[4] = {0.f, 0.f, 0.f, 0.f};
-        float zl[NCG];
-#pragma unroll
-        for (int g = 0; g < NCG; ++g)
-            zl[g] = 0.f;
+        Run1<D> run;
+        run1_init(run);
         for (int k = 0; k < nown; ++k) {
             const int n = prc_n++;
             if (iss_n < n + spw)
                 pump(n + spw);
+            if (k == k_setup && ri + 1 < nrows) {
+                setup_row(ri + 1);
+                pump(n + spw);
+            }
             wait_stage(n);
             const uint8_t *st = ring + (n & smask) * G1::STAGE;
-            // ---- keys: the exact integer dot products of decode_kernel's key pass
-            const int hf = lane >> 4;
-            constexpr int HW = G::WORDSK / 2;
-            const uint8_t *krA = st + (lane & 15) * G::ROWK + hf * (G::ROWK / 2);
-            const uint8_t *krB = krA + G::HM;
-            uint32_t cwA[HW], cwB[HW];
-#pragma unroll
-            for (int w = 0; w < HW; w += (HW % 4 == 0 ? 4 : 2)) {
-                if (HW % 4 == 0) {
-                    const uint4 ca = *reinterpret_cast<const uint4 *>(krA + 4 * w);
-                    const uint4 cb = *reinterpret_cast<const uint4 *>(krB + 4 * w);
-                    cwA[w] = ca.x, cwA[w + 1] = ca.y, cwA[w + 2] = ca.z, cwA[w + 3] = ca.w;
-                    cwB[w] = cb.x, cwB[w + 1] = cb.y, cwB[w + 2] = cb.z, cwB[w + 3] = cb.w;
-                } else {
-                    const uint2 ca = *reinterpret_cast<const uint2 *>(krA + 4 * w);
-                    const uint2 cb = *reinterpret_cast<const uint2 *>(krB + 4 * w);
-                    cwA[w] = ca.x, cwA[w + 1] = ca.y;
-                    cwB[w] = cb.x, cwB[w + 1] = cb.y;
-                }
-            }
-            float av[4], zs = 0.f;
-            {
-                uint2 sr = make_uint2(0u, 0u), zr = make_uint2(0u, 0u);
-                if (ownq) {
-                    sr = *reinterpret_cast<const uint2 *>(st + G::KCODES + 8 * lane);          // scales (even block)
-                    zr = *reinterpret_cast<const uint2 *>(st + G::HM + G::KCODES + 8 * lane); // zeros (odd block)
-                }
-                const float2 s01 = __half22float2(*reinterpret_cast<const __half2 *>(&sr.x));
-                const float2 s23 = __half22float2(*reinterpret_cast<const __half2 *>(&sr.y));
-                const float2 z01 = __half22float2(*reinterpret_cast<const __half2 *>(&zr.x));
-                const float2 z23 = __half22float2(*reinterpret_cast<const __half2 *>(&zr.y));
-                av[0] = qreg[0] * s01.x;
-                av[1] = qreg[1] * s01.y;
-                av[2] = qreg[2] * s23.x;
-                av[3] = qreg[3] * s23.y;
-                zs = fmaf(qreg[0], z01.x, fmaf(qreg[1], z01.y, fmaf(qreg[2], z23.x, qreg[3] * z23.y)));
-            }
-            const float amax = warp_max_abs(fmaxf(fmaxf(fabsf(av[0]), fabsf(av[1])), fmaxf(fabsf(av[2]), fabsf(av[3]))));
-            zs = warp_sum(zs);
-            const uint32_t ab = __float_as_uint(amax);
-            int F = 21 - ((int)(ab >> 23) - 127) - ((ab & 0x7FFFFFu) >= 0x7FFFFEu ? 1 : 0);
-            F = F > 126 ? 126 : F;
-            const float fs = __int_as_float((F + 127) << 23), fsk = __int_as_float((127 - F) << 23);
-            if (ownq) {
-                const uint32_t y0 = __float_as_uint(fmaf(av[0], fs, 12582912.f));
-                const uint32_t y1 = __float_as_uint(fmaf(av[1], fs, 12582912.f));
-                const uint32_t y2 = __float_as_uint(fmaf(av[2], fs, 12582912.f));
-                const uint32_t y3 = __float_as_uint(fmaf(av[3], fs, 12582912.f));
-                const uint32_t t01 = __byte_perm(y0, y1, 0x5140), t23 = __byte_perm(y2, y3, 0x5140);
-                const uint32_t u01 = __byte_perm(y0, y1, 0x0062), u23 = __byte_perm(y2, y3, 0x0062);
-                const uint32_t d0 = __byte_perm(t01, t23, 0x5410), d1 = __byte_perm(t01, t23, 0x7632);
-                const uint32_t x2 = __byte_perm(u01, u23, 0x5410) ^ 0x40404040u;
-                const uint32_t d2 = x2 | ((x2 & 0x40404040u) << 1);
-                reinterpret_cast<uint4 *>(scr)[lane] = make_uint4(d0, d1, d2, 0u);
-            }
-            __syncwarp();
-            constexpr int QPW = BITS == 4 ? 2 : 4;
-            const uint4 *rh = rec + hf * (G::NQ / 2);
-            KeyAcc accA = {{0u, 0u}, {0u, 0u}, {0, 0}}, accB = {{0u, 0u}, {0u, 0u}, {0, 0}};
-#pragma unroll
-            for (int w = 0; w < HW; ++w)
-                key_word2<BITS>(cwA[w], cwB[w], rh + QPW * w, accA, accB);
-            const uint32_t a01A = accA.a0[0] + accA.a0[1] + ((accA.a1[0] + accA.a1[1]) << 8);
-            const uint32_t a01B = accB.a0[0] + accB.a0[1] + ((accB.a1[0] + accB.a1[1]) << 8);
-            const int a2A = accA.a2[0] + accA.a2[1], a2B = accB.a2[0] + accB.a2[1];
-            const uint32_t a01 = (hf ? a01B : a01A) + __shfl_xor_sync(0xFFFFFFFFu, hf ? a01A : a01B, 16);
-            const int a2 = (hf ? a2B : a2A) + __shfl_xor_sync(0xFFFFFFFFu, hf ? a2A : a2B, 16);
-            const float s2l = fmaf(fmaf((float)a2, 65536.f, (float)a01), fsk, zs); // score of token `lane`
-            // ---- running maximum (warp-uniform): rescale the warp's sums when it grows
-            const float mg = warp_max_f(s2l);
-            if (mg > m_run) {
-                const float f = ex2(m_run - mg); // 0 at the first group
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    facc[i] *= f;
-#pragma unroll
-                for (int g = 0; g < NCG; ++g)
-                    zl[g] *= f;
-                lsum *= f;
-                m_run = mg;
-            }
-            const float wl = ex2(s2l - m_run);
-            lsum += wl;
+            run1_group<BITS, D>(st, st + G1::LOFF, scr, qreg, lane, run);
             if (a.s_bitmap && lane == 0) // refine set: every token (4-bit, tau <= 0) or none (2-bit)
                 a.s_bitmap[(int64_t)row * a.bitmap_words + (int)crank + (warp + k * kWarps) * (int)C] =
                     BITS == 4 ? 0xFFFFFFFFu : 0u;
-            __syncwarp(); // the key digit records are read: the scratch takes the value weights
-            // ---- values: decode_kernel's value pass with every token hot
-            {
-                const uint8_t *vm = st + (lane >> 4) * G::HM + G::KB + (lane & 15) * 4; // (scale, zero) of group g at + 64 g
-                float W[NCG], wmax = 0.f;
-#pragma unroll
-                for (int g = 0; g < NCG; ++g) {
-                    const float2 m = __half22float2(*reinterpret_cast<const __half2 *>(vm + 64 * g));
-                    zl[g] = fmaf(wl, m.y, zl[g]);
-                    W[g] = wl * m.x;
-                    wmax = fmaxf(wmax, W[g]);
-                }
-                wmax = warp_max_f(wmax);
-                int Fv = 20 - ((int)(__float_as_uint(wmax) >> 23) - 127);
-                Fv = Fv > 126 ? 126 : Fv;
-                const float fv = __int_as_float((Fv + 127) << 23);
-#pragma unroll
-                for (int g = 0; g < NCG; ++g)
-                    ybuf[g * YS + lane] = __float_as_uint(fmaf(W[g], fv, 8388608.f));
-                if (lane == 0)
-                    *fsit = __int_as_float((127 - Fv) << 23);
-            }
-            __syncwarp();
-            if (pv) {
-                const uint4 y = *reinterpret_cast<const uint4 *>(ybuf + pg * YS + 4 * pt8);
-                const uint32_t t01 = __byte_perm(y.x, y.y, 0x5140), t23 = __byte_perm(y.z, y.w, 0x5140);
-                const uint32_t u01 = __byte_perm(y.x, y.y, 0x0062), u23 = __byte_perm(y.z, y.w, 0x0062);
-                reinterpret_cast<uint4 *>(ybuf + pg * YS)[pt8] =
-                    make_uint4(__byte_perm(t01, t23, 0x5410), __byte_perm(t01, t23, 0x7632),
-                               __byte_perm(u01, u23, 0x5410), 0u);
-            }
-            __syncwarp();
-            uint32_t a0[4] = {0u, 0u, 0u, 0u}, a1[4] = {0u, 0u, 0u, 0u}, a2v[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-            for (int bb = 0; bb < BPL; ++bb) {
-                const int blk = vb0 + bb;
-                const uint4 h4 = *reinterpret_cast<const uint4 *>(st + blk * G::HM + G::KB + G::VMETA + 16 * vk);
-                const uint32_t hwv[4] = {h4.x, h4.y, h4.z, h4.w};
-                const uint8_t *lop = st + G1::LOFF + blk * G::LOB + 4 * vk;
-                const uint4 *rq = reinterpret_cast<const uint4 *>(ybuf + vg * YS) + 4 * blk;
-#pragma unroll
-                for (int tau = 0; tau < 4; ++tau) {
-                    const uint4 rc = rq[tau];
-                    const uint32_t hw = hwv[tau];
-                    uint32_t c4[4];
-                    if (BITS == 2) { // own 2-bit codes: channel i of every byte at bit 2i
-                        c4[0] = hw & 0x03030303u;
-                        c4[1] = (hw >> 2) & 0x03030303u;
-                        c4[2] = (hw >> 4) & 0x03030303u;
-                        c4[3] = (hw >> 6) & 0x03030303u;
-                    } else { // 4h + l
-                        const uint32_t lw = *reinterpret_cast<const uint32_t *>(lop + tau * D);
-                        const uint32_t E = ((hw << 2) & 0xCCCCCCCCu) | (lw & 0x33333333u);
-                        const uint32_t O = (hw & 0xCCCCCCCCu) | ((lw >> 2) & 0x33333333u);
-                        c4[0] = E & 0x0F0F0F0Fu;
-                        c4[1] = O & 0x0F0F0F0Fu;
-                        c4[2] = (E >> 4) & 0x0F0F0F0Fu;
-                        c4[3] = (O >> 4) & 0x0F0F0F0Fu;
-                    }
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        dp4a_uu(a0[i], c4[i], rc.x);
-                        dp4a_uu(a1[i], c4[i], rc.y);
-                        dp4a_uu(a2v[i], c4[i], rc.z);
-                    }
-                }
-            }
-            const float fsi = *fsit;
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                facc[i] = fmaf((float)(a0[i] + (a1[i] << 8) + (a2v[i] << 16)), fsi, facc[i]);
-            __syncwarp();
         }
-        // the warp's zero terms (reduce-scatter as in decode_kernel), sums and partial o, l
-#pragma unroll
-        for (int s2 = 0; (1 << s2) < NCG; ++s2) {
-            const int off = 1 << s2, len = NCG >> (s2 + 1);
-            const bool up = (lane & off) != 0;
-#pragma unroll
-            for (int m = 0; m < len; ++m) {
-                const float send = up ? zl[2 * m] : zl[2 * m + 1];
-                const float keep = up ? zl[2 * m + 1] : zl[2 * m];
-                zl[m] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, off);
-            }
-        }
-        float zsum = zl[0];
-#pragma unroll
-        for (int off = NCG; off < 32; off <<= 1)
-            zsum += __shfl_xor_sync(0xFFFFFFFFu, zsum, off);
-        const float zacc = __shfl_sync(0xFFFFFFFFu, zsum, vg);
-        lsum = warp_sum(lsum);
-        if (BPL == 1)
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                facc[i] += __shfl_xor_sync(0xFFFFFFFFu, facc[i], 16);
-        __syncwarp();
         float *red = reinterpret_cast<float *>(scr);
-        if (lane < G::NQ)
-            *reinterpret_cast<float4 *>(red + 4 * vk) =
-                make_float4(facc[0] + zacc, facc[1] + zacc, facc[2] + zacc, facc[3] + zacc);
-        if (lane == 0)
-            red[D] = lsum;
-        __syncwarp();
-        if (tail > 0 && warp == kWarps - 1) { // tail tokens, exact; lane = tail token
-            const int b = srow[IR_B], h = srow[IR_H];
-            const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)b * 2 * a.H + h) * 32 * D;
-            float s2 = 0.f;
-            for (int q4 = 0; q4 < G::NQ; ++q4) {
-                float kv[4] = {0.f, 0.f, 0.f, 0.f};
-                if (lane < tail)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        kv[i] = to_f32(kt[(int64_t)lane * D + 4 * q4 + i]);
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    s2 = fmaf(__shfl_sync(0xFFFFFFFFu, qreg[i], q4), kv[i], s2);
-            }
-            const float mt = warp_max_f(lane < tail ? s2 : -INFINITY);
-            if (mt > m_run) { // rescale the warp's partial in the scratch
-                const float f = ex2(m_run - mt);
-                for (int c = lane; c <= D; c += 32)
-                    red[c] *= f;
-                m_run = mt;
-            }
-            __syncwarp();
-            const DT *vt0 = reinterpret_cast<const DT *>(a.tail) + ((int64_t)(b * 2 + 1) * a.H + h) * 32 * D;
-            float tl = 0.f;
-            for (int t = 0; t < tail; ++t) {
-                const float w = ex2(__shfl_sync(0xFFFFFFFFu, s2, t) - m_run);
-                tl += w;
-                const DT *vt = vt0 + (int64_t)t * D;
-#pragma unroll
-                for (int c4 = 0; c4 < D / 32; ++c4)
-                    red[lane + 32 * c4] = fmaf(w, to_f32(vt[lane + 32 * c4]), red[lane + 32 * c4]);
-            }
-            __syncwarp();
-            if (lane == 0)
-                red[D] += tl;
+        run1_finish<BITS, D>(run, red, lane);
+        if (tail > 0 && warp == kWarps - 1) {
+            const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)rb * 2 * a.H + rh) * 32 * D;
+            const DT *vt0 = reinterpret_cast<const DT *>(a.tail) + ((int64_t)(rb * 2 + 1) * a.H + rh) * 32 * D;
+            run1_tail<D, DT>(run, red, lane, qreg, kt, vt0, tail);
         }
         if (lane == 0)
-            wm[warp] = m_run;
+            red[D + 1] = run.m;
         named_sync(1, kThreads);
-        // CTA partial relative to the CTA's maximum mc
+    };
+
+    // The CTA's partial of row ri relative to the CTA's maximum mc, into parts[ri & 1].
+    auto cta_partial = [&](int ri) {
+        float wmx[kWarps];
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w)
+            wmx[w] = reinterpret_cast<const float *>(scr_all + w * SCR)[D + 1];
         float mc = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w)
-            mc = fmaxf(mc, wm[w]);
+            mc = fmaxf(mc, wmx[w]);
         float fw[kWarps];
 #pragma unroll
         for (int w = 0; w < kWarps; ++w)
-            fw[w] = wm[w] == -INFINITY ? 0.f : ex2(wm[w] - mc);
-        float *part = parts + (ri % 3) * (D + 2);
+            fw[w] = wmx[w] == -INFINITY ? 0.f : ex2(wmx[w] - mc);
+        float *part = parts + (ri & 1) * (D + 2);
         for (int c = threadIdx.x; c <= D; c += kThreads) {
             float sum = 0.f;
 #pragma unroll
@@ -1568,14 +1628,13 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
         }
         if (threadIdx.x == 0)
             part[D + 1] = mc;
-        named_sync(1, kThreads); // every warp's scratch and wm are free again
     };
 
     // CTA `crank` writes channels [crank*per, min(D, (crank+1)*per)) of row ri, per =
     // ceil(D / C), from the partials of every CTA rescaled to the row maximum M.
     auto merge = [&](int ri) {
         const int row = row_of(ri);
-        const float *part = parts + (ri % 3) * (D + 2);
+        const float *part = parts + (ri & 1) * (D + 2);
         const int per = (D + (int)C - 1) / (int)C;
         const int c = (int)crank * per + (int)threadIdx.x;
         if ((int)threadIdx.x < per && c < D) {
@@ -1605,9 +1664,10 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
         }
     };
 
-    // One cluster barrier per row: barrier i publishes the partials of row i, merged after
-    // the next row's pass.  parts[i % 3] is written again at row i + 3, after this CTA
-    // passed barrier i + 1, which every CTA reaches only after its merge of row i.
+    // One cluster barrier per row: barrier i publishes the CTA partials of row i, merged
+    // after the pass of row i + 1.  parts[i & 1] is written once this CTA has passed
+    // barrier i - 1, which every CTA reaches only after its merge of row i - 2, the last
+    // reader of that buffer.
     for (int i = 0; i <= nrows; ++i) {
         if (i < nrows)
             row_pass(i);
@@ -1615,8 +1675,11 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
             cluster_wait(); // barrier i - 1
             merge(i - 1);
         }
-        if (i < nrows)
-            cluster_arrive(); // barrier i
+        if (i < nrows) {
+            cta_partial(i);
+            named_sync(1, kThreads); // every warp's scratch is free again
+            cluster_arrive();       // barrier i
+        }
     }
     cluster_arrive(); // the remote reads of the last merge are done
     cluster_wait();
@@ -1656,7 +1719,8 @@ template <int BITS, int D, typename DT>
 int launch_t(const DecodeArgs &a, const DecodeShape &shp, cudaStream_t s)
 {
     if (shp.onepass)
-        return launch_shape(decode_kernel_1p<BITS, D, DT, 4>, shp, s, a, shp.stages_log2);
+        return launch_shape(shp.min_ctas == 5 ? decode_kernel_1p<BITS, D, DT, 5> : decode_kernel_1p<BITS, D, DT, 4>, shp,
+                            s, a, shp.stages_log2);
     auto kern = shp.min_ctas == 5 ? decode_kernel<BITS, D, DT, 5> : decode_kernel<BITS, D, DT, 4>;
     return launch_shape(kern, shp, s, a, shp.stages_log2, shp.score_bufs);
 }
@@ -1731,8 +1795,7 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
     const char *env_c = getenv("LOOPKV_DECODE_CLUSTER");
     const char *env_s = getenv("LOOPKV_DECODE_STAGES");
     const char *env_o = getenv("LOOPKV_DECODE_CTAS_PER_SM");
-    // the single-pass kernel is built for 4 CTAs per SM; the two-phase one for 4 or 5
-    for (int want_ctas = 4; want_ctas <= (onepass ? 4 : 5); ++want_ctas) {
+    for (int want_ctas = 4; want_ctas <= 5; ++want_ctas) { // builds for 4 and 5 CTAs per SM
         if (env_o && atoi(env_o) != want_ctas)
             continue;
         for (int C = 1; C <= 16; C = C < 8 ? C + 1 : 2 * C) { // 1..8, 16
@@ -1751,7 +1814,8 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
                 const int smem = kernel_smem<BITS, D>(onepass, spw, capw, nbuf);
                 if (smem <= 0 || smem > 227 * 1024)
                     continue;
-                int ncl = onepass ? max_active_clusters(decode_kernel_1p<BITS, D, DT, 4>, C, smem)
+                int ncl = onepass ? (want_ctas == 5 ? max_active_clusters(decode_kernel_1p<BITS, D, DT, 5>, C, smem)
+                                                    : max_active_clusters(decode_kernel_1p<BITS, D, DT, 4>, C, smem))
                           : want_ctas == 5 ? max_active_clusters(decode_kernel<BITS, D, DT, 5>, C, smem)
                                            : max_active_clusters(decode_kernel<BITS, D, DT, 4>, C, smem);
                 if (ncl <= 0)

@@ -183,6 +183,23 @@ def test_append_flush_sequence():
                 assert int(tail[req]) >= 1 and int(hist[req]) % 32 == 0 and int(hist[req]) + int(tail[req]) == n
 
 
+@pytest.mark.parametrize("lengths", [[4096, 1000, 33], [2048] * 3])
+def test_repeated_single_pass_decode_is_bit_identical(lengths):
+    # 2-bit cells and tau = 0 reads split long rows across CTAs and merge the pieces through
+    # per-row counters that the merging CTA resets: a second launch must repeat the first.
+    modes = [L.CELL_2B, L.CELL_4B]
+    w = synth.Workload("repeat", 1, 2, 4, 128, 3, lengths, torch.bfloat16, modes, 0.0, seed=11)
+    m = Model(w)
+    m.ingest()
+    for lp in range(2):
+        q = _q(w, 0, 0, lp)
+        first = m.cache.decode(lp, 0, q)
+        second = m.cache.decode(lp, 0, q)
+        m.cache.check("repeat")
+        assert torch.equal(first, second)
+        m.check_cell(lp, 0, q, where=f"repeat loop {lp}")
+
+
 def test_share_cell_with_final_loop_query_is_bit_identical():
     modes = [L.CELL_SHARE, L.CELL_4B]
     w = synth.Workload("share", 1, 2, 4, 128, 2, [512, 1024], torch.bfloat16, modes, 0.01, seed=9)
