@@ -37,9 +37,10 @@
 // rounding.
 // Values: a value-plane word holds 4 tokens x 4 channels (token in the byte).  The hi and
 // lo words merge into 4-bit codes (lo bits of cold tokens masked off), one AND unpacks the
-// codes of one channel for 4 tokens, and dp4a against 8-bit digits of the tokens' 21-bit
-// fixed-point weights w * scale sums code * weight over tokens exactly in int32; each
-// 32-token group's sum is rounded to fp32 once.
+// codes of one channel for 4 tokens, and dp4a against the two 8-bit digits of the tokens'
+// 15-bit fixed-point weights w * scale (relative step 2^-15 of the group's largest) sums
+// code * weight over tokens exactly in int32; each 32-token group's sum (< 2^24) converts
+// to fp32 exactly.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -790,14 +791,14 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     //
     // Per group, lane t takes token t: weight w = 2^(s - m), the zero terms, W_g = w * scale_g
     // and, with F from the
-    // exact maximum of W over the group, the 21-bit fixed-point I_g = round(W_g 2^F) as the
+    // exact maximum of W over the group, the 15-bit fixed-point I_g = round(W_g 2^F) as the
     // low bits of W_g 2^F + 2^23.  Through a padded shared transpose, lane (t8, g) then packs
-    // the three byte digits of I_g of the 4 tokens of token quad t8 into a record
-    // {d0, d1, d2, hot-byte mask}.  Consumer lane vk owns channel quad vk and, for every token
+    // the two byte digits of I_g of the 4 tokens of token quad t8 into a record
+    // {d0, d1, hot-byte mask}.  Consumer lane vk owns channel quad vk and, for every token
     // quad, merges its hi and lo plane words into 4-bit codes (lo bits kept for hot tokens
     // only), unpacks the four channels' codes of the four tokens with one AND each and
     // accumulates code * digit over tokens with dp4a, exact in int32; the group's sum goes
-    // to fp32 with one rounding.
+    // to fp32 exactly.
     auto consume_v = [&](int ri, float m2, float thr2) {
         const int32_t *srow = irow_of(ri);
         const int nown = srow[IR_N], tail = srow[IR_TAIL];
@@ -852,9 +853,9 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
                     wmax = fmaxf(wmax, W[g]);
                 }
                 wmax = warp_max_f(wmax);
-                // I < 2^21 + 1 with F = 20 - E (E = exponent of the maximum), capped so that
-                // 2^F and 2^-F stay normal
-                int F = 20 - ((int)(__float_as_uint(wmax) >> 23) - 127);
+                // I < 2^15 + 1 with F = 14 - E (E = exponent of the maximum), capped so that
+                // 2^F and 2^-F stay normal: two byte digits
+                int F = 14 - ((int)(__float_as_uint(wmax) >> 23) - 127);
                 F = F > 126 ? 126 : F;
                 const float fs = __int_as_float((F + 127) << 23);
 #pragma unroll
@@ -868,22 +869,20 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             if (pv) {
                 const uint4 y = *reinterpret_cast<const uint4 *>(ybuf + pg * YS + 4 * pt8);
                 const uint32_t t01 = __byte_perm(y.x, y.y, 0x5140), t23 = __byte_perm(y.z, y.w, 0x5140);
-                const uint32_t u01 = __byte_perm(y.x, y.y, 0x0062), u23 = __byte_perm(y.z, y.w, 0x0062);
                 // bit b of the quad's 4 hot bits to bit 8b+7, then each byte takes its top bit
                 const uint32_t hb = byte_signs(((hm >> (4 * pt8)) & 0xFu) * 0x10204080u);
-                reinterpret_cast<uint4 *>(ybuf + pg * YS)[pt8] = make_uint4(__byte_perm(t01, t23, 0x5410), __byte_perm(t01, t23, 0x7632),
-                                                __byte_perm(u01, u23, 0x5410), hb);
+                reinterpret_cast<uint4 *>(ybuf + pg * YS)[pt8] =
+                    make_uint4(__byte_perm(t01, t23, 0x5410), __byte_perm(t01, t23, 0x7632), hb, 0u);
             }
             __syncwarp();
             // ---- accumulate: channel quad vk, dp4a over the tokens of each token quad
-            uint32_t a0[4] = {0u, 0u, 0u, 0u}, a1[4] = {0u, 0u, 0u, 0u}, a2[4] = {0u, 0u, 0u, 0u};
+            uint32_t a0[4] = {0u, 0u, 0u, 0u}, a1[4] = {0u, 0u, 0u, 0u};
             // codes of channel 4vk+i of the quad's 4 tokens, one per byte, into the sums
             auto acc_quad = [&](const uint32_t (&c4)[4], const uint4 &rc) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     dp4a_uu(a0[i], c4[i], rc.x);
                     dp4a_uu(a1[i], c4[i], rc.y);
-                    dp4a_uu(a2[i], c4[i], rc.z);
                 }
             };
             // 4-bit codes 4h + l from a hi and a lo word: nibble 0 of each byte is channel 0
@@ -922,18 +921,18 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
 #pragma unroll
                     for (int tau = 0; tau < 4; ++tau) {
                         const uint4 rc = rq[tau];
-                        const uint32_t lw = rc.w ? *reinterpret_cast<const uint32_t *>(lop + tau * D) & rc.w : 0u;
+                        const uint32_t lw = rc.z ? *reinterpret_cast<const uint32_t *>(lop + tau * D) & rc.z : 0u;
                         uint32_t c4[4];
                         merged(hwv[tau], lw, c4);
                         acc_quad(c4, rc);
                     }
                 }
             }
-            // sum_t code * I < 2^31: exact in 32 bits; one rounding to fp32
+            // sum_t code * I <= 15 * 2^15 * 32 < 2^24: exact in 32 bits and in fp32
             const float fsi = *fsit;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                facc[i] = fmaf((float)(a0[i] + (a1[i] << 8) + (a2[i] << 16)), fsi, facc[i]);
+                facc[i] = fmaf((float)(a0[i] + (a1[i] << 8)), fsi, facc[i]);
             __syncwarp();
         }
         // zero terms: lane ends with the warp's sum of zl[lane % NCG] (reduce-scatter over
@@ -1258,7 +1257,9 @@ __device__ __forceinline__ void run1_group(const uint8_t *st, const uint8_t *lo,
             wmax = fmaxf(wmax, W[g]);
         }
         wmax = warp_max_f(wmax);
-        int Fv = 20 - ((int)(__float_as_uint(wmax) >> 23) - 127);
+        // I = round(W 2^F) < 2^15 + 1 with F = 14 - E: two byte digits (the 2^-15 relative
+        // step of a weight is far below the fp32 rounding of the sums it enters)
+        int Fv = 14 - ((int)(__float_as_uint(wmax) >> 23) - 127);
         Fv = Fv > 126 ? 126 : Fv;
         const float fv = __int_as_float((Fv + 127) << 23);
 #pragma unroll
@@ -1268,26 +1269,24 @@ __device__ __forceinline__ void run1_group(const uint8_t *st, const uint8_t *lo,
             *fsit = __int_as_float((127 - Fv) << 23);
     }
     __syncwarp();
-    if (pv) {
+    if (pv) { // record lane (t8, g): the two byte digits of the 4 tokens of quad t8
         const uint4 y = *reinterpret_cast<const uint4 *>(ybuf + pg * YS + 4 * pt8);
         const uint32_t t01 = __byte_perm(y.x, y.y, 0x5140), t23 = __byte_perm(y.z, y.w, 0x5140);
-        const uint32_t u01 = __byte_perm(y.x, y.y, 0x0062), u23 = __byte_perm(y.z, y.w, 0x0062);
-        reinterpret_cast<uint4 *>(ybuf + pg * YS)[pt8] =
-            make_uint4(__byte_perm(t01, t23, 0x5410), __byte_perm(t01, t23, 0x7632),
-                       __byte_perm(u01, u23, 0x5410), 0u);
+        *reinterpret_cast<uint2 *>(ybuf + pg * YS + 4 * pt8) =
+            make_uint2(__byte_perm(t01, t23, 0x5410), __byte_perm(t01, t23, 0x7632));
     }
     __syncwarp();
-    uint32_t a0[4] = {0u, 0u, 0u, 0u}, a1[4] = {0u, 0u, 0u, 0u}, a2v[4] = {0u, 0u, 0u, 0u};
+    uint32_t a0[4] = {0u, 0u, 0u, 0u}, a1[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
     for (int bb = 0; bb < BPL; ++bb) {
         const int blk = vb0 + bb;
         const uint4 h4 = *reinterpret_cast<const uint4 *>(st + blk * G::HM + G::KB + G::VMETA + 16 * vk);
         const uint32_t hwv[4] = {h4.x, h4.y, h4.z, h4.w};
         const uint8_t *lop = lo + blk * G::LOB + 4 * vk;
-        const uint4 *rq = reinterpret_cast<const uint4 *>(ybuf + vg * YS) + 4 * blk;
+        const uint32_t *rq = ybuf + vg * YS + 16 * blk; // record of token quad 4 blk + tau at + 4 tau
 #pragma unroll
         for (int tau = 0; tau < 4; ++tau) {
-            const uint4 rc = rq[tau];
+            const uint2 rc = *reinterpret_cast<const uint2 *>(rq + 4 * tau);
             const uint32_t hw = hwv[tau];
             uint32_t c4[4];
             if (BITS == 2) { // own 2-bit codes: channel i of every byte at bit 2i
@@ -1308,14 +1307,13 @@ __device__ __forceinline__ void run1_group(const uint8_t *st, const uint8_t *lo,
             for (int i = 0; i < 4; ++i) {
                 dp4a_uu(a0[i], c4[i], rc.x);
                 dp4a_uu(a1[i], c4[i], rc.y);
-                dp4a_uu(a2v[i], c4[i], rc.z);
             }
         }
     }
     const float fsi = *fsit;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-        r.o[i] = fmaf((float)(a0[i] + (a1[i] << 8) + (a2v[i] << 16)), fsi, r.o[i]);
+        r.o[i] = fmaf((float)(a0[i] + (a1[i] << 8)), fsi, r.o[i]); // sum <= 15 * 2^15 * 32 < 2^24: exact
     __syncwarp();
 }
 
