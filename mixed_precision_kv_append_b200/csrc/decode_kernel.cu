@@ -189,13 +189,122 @@ __device__ __forceinline__ void key_word2(uint32_t wa, uint32_t wb, const uint4 
     }
 }
 
+// Scores (log2 units) of the 32 tokens of a group: token j of block A is token j, token j
+// of block B is token 16 + j; blkA and blkB point at the blocks' key regions (codes, then
+// the per-channel scales in block A and zeros in block B).  Returns the score of token
+// `lane`.  scr: the warp's scratch (digit records).
+//
+// The factors a_c = q_c s_c of the group are rounded to 22-bit fixed point I_c = round(a_c
+// 2^F), F = 21 - E (E = exponent of max |a|; one less when the rounding of the largest
+// could reach 2^22; capped so that 2^F and 2^-F stay normal), with one FMA against
+// 1.5 * 2^23; the low three bytes of the float become three digits (the top one re-centred
+// to a signed byte).  A lane then sums code * digit with dp4a for one channel half of one
+// token of each block, both sharing every digit-record load, and the halves are exchanged.
+// Lane L takes token t = (L & 3) | (L >> 3) << 2 and half hf = (L >> 2) & 1, and loads its
+// two 16-byte chunks in the order (t >> 1) & 1 first: the 8 lanes of a shared-memory phase
+// then touch 8 different 16-byte bank groups.  The record of channel quad q sits at
+// q + q / 8 (16 bytes each), so that the records read together do too.
+template <int BITS, int D>
+__device__ __forceinline__ float group_scores(const uint8_t *blkA, const uint8_t *blkB, uint8_t *scr,
+                                              const float (&qreg)[4], const int lane)
+{
+    using G = Geo<BITS, D>;
+    constexpr int HW = G::WORDSK / 2;        // code words per channel half
+    constexpr int NCH = HW >= 4 ? HW / 4 : 1; // 16-byte chunks per half (8 bytes when HW = 2)
+    constexpr int WPC = HW >= 4 ? 4 : HW;     // words per chunk
+    constexpr int QPW = BITS == 4 ? 2 : 4;    // channel quads per code word
+    const bool ownq = lane < G::NQ;
+    const int hf = (lane >> 2) & 1, t = (lane & 3) | ((lane >> 3) << 2);
+    const int c0 = NCH == 2 ? (t >> 1) & 1 : 0;
+    const uint8_t *krA = blkA + t * G::ROWK + hf * (G::ROWK / 2);
+    const uint8_t *krB = blkB + t * G::ROWK + hf * (G::ROWK / 2);
+    uint32_t cwA[HW], cwB[HW]; // chunk by chunk in load order, loaded before the digit build
+#pragma unroll
+    for (int j = 0; j < NCH; ++j) {
+        const int c = j == 0 ? c0 : 1 - c0;
+        if (HW >= 4) {
+            const uint4 ca = *reinterpret_cast<const uint4 *>(krA + 16 * c);
+            const uint4 cb = *reinterpret_cast<const uint4 *>(krB + 16 * c);
+            cwA[4 * j] = ca.x, cwA[4 * j + 1] = ca.y, cwA[4 * j + 2] = ca.z, cwA[4 * j + 3] = ca.w;
+            cwB[4 * j] = cb.x, cwB[4 * j + 1] = cb.y, cwB[4 * j + 2] = cb.z, cwB[4 * j + 3] = cb.w;
+        } else {
+            const uint2 ca = *reinterpret_cast<const uint2 *>(krA);
+            const uint2 cb = *reinterpret_cast<const uint2 *>(krB);
+            cwA[0] = ca.x, cwA[1] = ca.y;
+            cwB[0] = cb.x, cwB[1] = cb.y;
+        }
+    }
+    // factors a_c = q_c s_c of the lane's quad and the zero term sum_c q_c z_c
+    float av[4], zs = 0.f;
+    {
+        uint2 sr = make_uint2(0u, 0u), zr = make_uint2(0u, 0u);
+        if (ownq) {
+            sr = *reinterpret_cast<const uint2 *>(blkA + G::KCODES + 8 * lane); // scales
+            zr = *reinterpret_cast<const uint2 *>(blkB + G::KCODES + 8 * lane); // zeros
+        }
+        const float2 s01 = __half22float2(*reinterpret_cast<const __half2 *>(&sr.x));
+        const float2 s23 = __half22float2(*reinterpret_cast<const __half2 *>(&sr.y));
+        const float2 z01 = __half22float2(*reinterpret_cast<const __half2 *>(&zr.x));
+        const float2 z23 = __half22float2(*reinterpret_cast<const __half2 *>(&zr.y));
+        av[0] = qreg[0] * s01.x;
+        av[1] = qreg[1] * s01.y;
+        av[2] = qreg[2] * s23.x;
+        av[3] = qreg[3] * s23.y;
+        zs = fmaf(qreg[0], z01.x, fmaf(qreg[1], z01.y, fmaf(qreg[2], z23.x, qreg[3] * z23.y)));
+    }
+    const float amax = warp_max_abs(fmaxf(fmaxf(fabsf(av[0]), fabsf(av[1])), fmaxf(fabsf(av[2]), fabsf(av[3]))));
+    zs = warp_sum(zs);
+    const uint32_t ab = __float_as_uint(amax);
+    int F = 21 - ((int)(ab >> 23) - 127) - ((ab & 0x7FFFFFu) >= 0x7FFFFEu ? 1 : 0);
+    F = F > 126 ? 126 : F;
+    const float fs = __int_as_float((F + 127) << 23), fsi = __int_as_float((127 - F) << 23);
+    if (ownq) {
+        // low 23 bits of y = I + 2^22: bytes b0, b1 and b2 < 128
+        const uint32_t y0 = __float_as_uint(fmaf(av[0], fs, 12582912.f));
+        const uint32_t y1 = __float_as_uint(fmaf(av[1], fs, 12582912.f));
+        const uint32_t y2 = __float_as_uint(fmaf(av[2], fs, 12582912.f));
+        const uint32_t y3 = __float_as_uint(fmaf(av[3], fs, 12582912.f));
+        const uint32_t t01 = __byte_perm(y0, y1, 0x5140), t23 = __byte_perm(y2, y3, 0x5140);
+        const uint32_t u01 = __byte_perm(y0, y1, 0x0062), u23 = __byte_perm(y2, y3, 0x0062);
+        const uint32_t d0 = __byte_perm(t01, t23, 0x5410), d1 = __byte_perm(t01, t23, 0x7632);
+        // top digit b2 - 64 as a signed byte: flip bit 6, copy the new bit 6 into bit 7
+        const uint32_t x2 = __byte_perm(u01, u23, 0x5410) ^ 0x40404040u;
+        const uint32_t d2 = x2 | ((x2 & 0x40404040u) << 1);
+        reinterpret_cast<uint4 *>(scr)[lane + (lane >> 3)] = make_uint4(d0, d1, d2, 0u);
+    }
+    __syncwarp();
+    const uint4 *rec = reinterpret_cast<const uint4 *>(scr);
+    KeyAcc accA = {{0u, 0u}, {0u, 0u}, {0, 0}}, accB = {{0u, 0u}, {0u, 0u}, {0, 0}};
+#pragma unroll
+    for (int j = 0; j < NCH; ++j) {
+        const int c = j == 0 ? c0 : 1 - c0;
+#pragma unroll
+        for (int i = 0; i < WPC; ++i) {
+            const int q = hf * (G::NQ / 2) + QPW * (WPC * c + i); // first quad of the word (never
+            key_word2<BITS>(cwA[WPC * j + i], cwB[WPC * j + i], rec + q + (q >> 3), accA, accB); // across 8)
+        }
+    }
+    // per token and half: A01 = sum of d0 terms + 256 * sum of d1 terms (< 2^30), A2 = sum of
+    // d2 terms; both exact in 32-bit integers
+    const uint32_t a01A = accA.a0[0] + accA.a0[1] + ((accA.a1[0] + accA.a1[1]) << 8);
+    const uint32_t a01B = accB.a0[0] + accB.a0[1] + ((accB.a1[0] + accB.a1[1]) << 8);
+    const int a2A = accA.a2[0] + accA.a2[1], a2B = accB.a2[0] + accB.a2[1];
+    // lane L ^ 4 holds the other half: half 0 keeps token t, half 1 token 16 + t
+    const uint32_t a01 = (hf ? a01B : a01A) + __shfl_xor_sync(0xFFFFFFFFu, hf ? a01A : a01B, 4);
+    const int a2 = (hf ? a2B : a2A) + __shfl_xor_sync(0xFFFFFFFFu, hf ? a2A : a2B, 4);
+    // sum_c code_c I_c = A01 + 65536 A2; one rounding when they are added
+    const float s = fmaf(fmaf((float)a2, 65536.f, (float)a01), fsi, zs);
+    // token L's score to lane L (held by the lane with t = L % 16, hf = L / 16)
+    return __shfl_sync(0xFFFFFFFFu, s, (lane & 3) | (((lane & 15) >> 2) << 3) | ((lane >> 4) << 2));
+}
+
 struct Smem {
     uint8_t *ring;     // [kWarps][spw][STAGE] stage slots (kGPS groups each), a private slice per warp
     uint64_t *full;    // [kWarps][spw] completion barriers of the slots
     float *scores;     // [nbuf][kWarps][capw * 32] scores of a warp's groups, by row parity
     float *tscores;    // [2][32] tail scores, by row parity
     uint8_t *scr;      // [kWarps][SCR] per-warp scratch, used in turn as: key digit records
-                       // [D/4][16 B] during a K stage, the fixed-point weight transpose
+                       // [D/4 + D/32][16 B] (padded) during a K stage, the fixed-point weight transpose
                        // [D/32][40 words] (overwritten in place by the value digit records)
                        // and 2^-F during a V stage, the warp's partial o and l [D + 1] at
                        // the end of a V pass
@@ -223,7 +332,7 @@ __host__ __device__ constexpr int imax(int a, int b) { return a > b ? a : b; }
 // Bytes of a warp's scratch: the largest of its three uses.
 template <int D> __host__ __device__ constexpr int scratch_bytes()
 {
-    return align16(imax((D / 4) * 16, imax((D + 1) * 4, (D / 32) * 40 * 4 + 4)));
+    return align16(imax((D / 4 + D / 32) * 16, imax((D + 2) * 4, (D / 32) * 40 * 4 + 4)));
 }
 
 // nbuf: score buffers (2 when a cluster reads more than one row, so that the next row's
@@ -289,7 +398,7 @@ template <int BITS, int D> bool layout_ok(int spw, int capw, int nbuf)
         prev = o;
     }
     return (Geo<BITS, D>::GSLOT % 128) == 0 && L.total >= prev && (spw & (spw - 1)) == 0 &&
-           scratch_bytes<D>() >= (D / 4) * 16 && scratch_bytes<D>() >= (D + 1) * 4 &&
+           scratch_bytes<D>() >= (D / 4 + D / 32) * 16 && scratch_bytes<D>() >= (D + 1) * 4 &&
            scratch_bytes<D>() >= (D / 32) * 40 * 4 + 4 && (2 * capw * 4) % 8 == 0;
 }
 
@@ -492,10 +601,12 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
 #pragma unroll
         for (int j = 0; j < kGPS; ++j) {
             const uint32_t tm = j < ng ? __ballot_sync(0xFFFFFFFFu, sc[j * 32 + lane] >= thr2) : 0u;
-            uint32_t qm = 0; // bit q: token quad q has a hot token
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                qm |= ((tm >> (4 * q)) & 0xFu) ? 1u << q : 0u;
+            // bit q of qm: token quad q has a hot token (bit 4q of x, then gathered to bit q)
+            uint32_t x = tm | (tm >> 1);
+            x = (x | (x >> 2)) & 0x11111111u;
+            x = (x | (x >> 3)) & 0x03030303u;
+            x = (x | (x >> 6)) & 0x000F000Fu;
+            const uint32_t qm = (x | (x >> 12)) & 0xFFu;
             mask[j] = tm == 0xFFFFFFFFu ? 0xFFFFFFFFu : qm;
             bytes += tm == 0xFFFFFFFFu ? 2 * G::LOB : (uint32_t)__popc(qm) * D;
         }
@@ -616,7 +727,6 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     // ---------------------------------------------------------------- compute
     constexpr int SCR = scratch_bytes<D>();
     uint8_t *scr = sm.scr + warp * SCR;
-    const uint4 *rec = reinterpret_cast<const uint4 *>(scr); // K stage: digit records, one per quad
     int prc_n = 0;
     bool timed_out = false; // after one bounded wait gives up, later waits are skipped
     auto wait_stage = [&](int n) {
@@ -664,89 +774,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
                 stg = ring + (n & smask) * G::STAGE;
             }
             const uint8_t *st = stg + (k % kGPS) * G::GSLOT;
-            // the lane's code words (two tokens, one channel half), loaded before the digit
-            // build so that their latency overlaps it
-            const int hf = lane >> 4;
-            constexpr int HW = G::WORDSK / 2; // code words per channel half
-            const uint8_t *krA = st + (lane & 15) * G::ROWK + hf * (G::ROWK / 2);
-            const uint8_t *krB = krA + G::KB;
-            uint32_t cwA[HW], cwB[HW];
-#pragma unroll
-            for (int w = 0; w < HW; w += (HW % 4 == 0 ? 4 : 2)) {
-                if (HW % 4 == 0) {
-                    const uint4 ca = *reinterpret_cast<const uint4 *>(krA + 4 * w);
-                    const uint4 cb = *reinterpret_cast<const uint4 *>(krB + 4 * w);
-                    cwA[w] = ca.x, cwA[w + 1] = ca.y, cwA[w + 2] = ca.z, cwA[w + 3] = ca.w;
-                    cwB[w] = cb.x, cwB[w + 1] = cb.y, cwB[w + 2] = cb.z, cwB[w + 3] = cb.w;
-                } else {
-                    const uint2 ca = *reinterpret_cast<const uint2 *>(krA + 4 * w);
-                    const uint2 cb = *reinterpret_cast<const uint2 *>(krB + 4 * w);
-                    cwA[w] = ca.x, cwA[w + 1] = ca.y;
-                    cwB[w] = cb.x, cwB[w + 1] = cb.y;
-                }
-            }
-            // factors a_c = q_c s_c of the lane's quad and the zero term sum_c q_c z_c
-            float av[4], zs = 0.f;
-            {
-                uint2 sr = make_uint2(0u, 0u), zr = make_uint2(0u, 0u);
-                if (ownq) {
-                    sr = *reinterpret_cast<const uint2 *>(st + G::KCODES + 8 * lane);          // scales (even block)
-                    zr = *reinterpret_cast<const uint2 *>(st + G::KB + G::KCODES + 8 * lane); // zeros (odd block)
-                }
-                const float2 s01 = __half22float2(*reinterpret_cast<const __half2 *>(&sr.x));
-                const float2 s23 = __half22float2(*reinterpret_cast<const __half2 *>(&sr.y));
-                const float2 z01 = __half22float2(*reinterpret_cast<const __half2 *>(&zr.x));
-                const float2 z23 = __half22float2(*reinterpret_cast<const __half2 *>(&zr.y));
-                av[0] = qreg[0] * s01.x;
-                av[1] = qreg[1] * s01.y;
-                av[2] = qreg[2] * s23.x;
-                av[3] = qreg[3] * s23.y;
-                zs = fmaf(qreg[0], z01.x, fmaf(qreg[1], z01.y, fmaf(qreg[2], z23.x, qreg[3] * z23.y)));
-            }
-            const float amax = warp_max_abs(fmaxf(fmaxf(fabsf(av[0]), fabsf(av[1])), fmaxf(fabsf(av[2]), fabsf(av[3]))));
-            zs = warp_sum(zs);
-            // I_c = round(a_c 2^F), F = 21 - E (E = exponent of max |a|), so |I_c| < 2^22
-            // (one less when the rounding of the largest could reach 2^22); F is capped so
-            // that 2^F and 2^-F stay normal.
-            const uint32_t ab = __float_as_uint(amax);
-            int F = 21 - ((int)(ab >> 23) - 127) - ((ab & 0x7FFFFFu) >= 0x7FFFFEu ? 1 : 0);
-            F = F > 126 ? 126 : F;
-            const float fs = __int_as_float((F + 127) << 23), fsi = __int_as_float((127 - F) << 23);
-            if (ownq) {
-                // low 23 bits of y = I + 2^22: bytes b0, b1 and b2 < 128
-                const uint32_t y0 = __float_as_uint(fmaf(av[0], fs, 12582912.f));
-                const uint32_t y1 = __float_as_uint(fmaf(av[1], fs, 12582912.f));
-                const uint32_t y2 = __float_as_uint(fmaf(av[2], fs, 12582912.f));
-                const uint32_t y3 = __float_as_uint(fmaf(av[3], fs, 12582912.f));
-                const uint32_t t01 = __byte_perm(y0, y1, 0x5140), t23 = __byte_perm(y2, y3, 0x5140);
-                const uint32_t u01 = __byte_perm(y0, y1, 0x0062), u23 = __byte_perm(y2, y3, 0x0062);
-                const uint32_t d0 = __byte_perm(t01, t23, 0x5410), d1 = __byte_perm(t01, t23, 0x7632);
-                // top digit b2 - 64 as a signed byte: flip bit 6, copy the new bit 6 into bit 7
-                const uint32_t x2 = __byte_perm(u01, u23, 0x5410) ^ 0x40404040u;
-                const uint32_t d2 = x2 | ((x2 & 0x40404040u) << 1);
-                reinterpret_cast<uint4 *>(scr)[lane] = make_uint4(d0, d1, d2, 0u);
-            }
-            __syncwarp();
-            // Lane L sums channel half hf = L / 16 of tokens tA = L % 16 (block 0) and
-            // tB = tA + 16 (block 1); both share every digit-record load.  The halves are
-            // then exchanged so that lane L ends with the whole dot product of token L.
-            constexpr int QPW = BITS == 4 ? 2 : 4; // quads per code word
-            const uint4 *rh = rec + hf * (G::NQ / 2);
-            KeyAcc accA = {{0u, 0u}, {0u, 0u}, {0, 0}}, accB = {{0u, 0u}, {0u, 0u}, {0, 0}};
-#pragma unroll
-            for (int w = 0; w < HW; ++w)
-                key_word2<BITS>(cwA[w], cwB[w], rh + QPW * w, accA, accB);
-            // per token and half: A01 = sum of d0 terms + 256 * sum of d1 terms (< 2^30),
-            // A2 = sum of d2 terms; both exact in 32-bit integers
-            const uint32_t a01A = accA.a0[0] + accA.a0[1] + ((accA.a1[0] + accA.a1[1]) << 8);
-            const uint32_t a01B = accB.a0[0] + accB.a0[1] + ((accB.a1[0] + accB.a1[1]) << 8);
-            const int a2A = accA.a2[0] + accA.a2[1], a2B = accB.a2[0] + accB.a2[1];
-            // lane L keeps token L: half 0 keeps A and sends B, half 1 keeps B and sends A
-            const uint32_t a01 = (hf ? a01B : a01A) + __shfl_xor_sync(0xFFFFFFFFu, hf ? a01A : a01B, 16);
-            const int a2 = (hf ? a2B : a2A) + __shfl_xor_sync(0xFFFFFFFFu, hf ? a2A : a2B, 16);
-            // sum_c code_c I_c = A01 + 65536 A2 (A01 < 2^31); one rounding when they are added
-            const float dot = fmaf((float)a2, 65536.f, (float)a01);
-            const float s2 = fmaf(dot, fsi, zs);
+            const float s2 = group_scores<BITS, D>(st, st + G::KB, scr, qreg, lane);
             sc[k * 32 + lane] = s2;
             mx = fmaxf(mx, s2);
             __syncwarp();
@@ -1150,8 +1178,6 @@ __device__ __forceinline__ void run1_group(const uint8_t *st, const uint8_t *lo,
                                            const int lane, Run1<D> &r)
 {
     using G = Geo<BITS, D>;
-    const uint4 *rec = reinterpret_cast<const uint4 *>(scr);
-    const bool ownq = lane < G::NQ;
     constexpr int NCG = G::NCG;
     constexpr int YS = 40;
     const int pt8 = lane / NCG, pg = lane % NCG;
@@ -1161,74 +1187,7 @@ __device__ __forceinline__ void run1_group(const uint8_t *st, const uint8_t *lo,
     const int vb0 = G::NQ == 32 ? 0 : lane / G::NQ;
     uint32_t *ybuf = reinterpret_cast<uint32_t *>(scr);
     float *fsit = reinterpret_cast<float *>(ybuf + NCG * YS);
-    // ---- keys: the exact integer dot products of decode_kernel's key pass
-    const int hf = lane >> 4;
-    constexpr int HW = G::WORDSK / 2;
-    const uint8_t *krA = st + (lane & 15) * G::ROWK + hf * (G::ROWK / 2);
-    const uint8_t *krB = krA + G::HM;
-    uint32_t cwA[HW], cwB[HW];
-#pragma unroll
-    for (int w = 0; w < HW; w += (HW % 4 == 0 ? 4 : 2)) {
-        if (HW % 4 == 0) {
-            const uint4 ca = *reinterpret_cast<const uint4 *>(krA + 4 * w);
-            const uint4 cb = *reinterpret_cast<const uint4 *>(krB + 4 * w);
-            cwA[w] = ca.x, cwA[w + 1] = ca.y, cwA[w + 2] = ca.z, cwA[w + 3] = ca.w;
-            cwB[w] = cb.x, cwB[w + 1] = cb.y, cwB[w + 2] = cb.z, cwB[w + 3] = cb.w;
-        } else {
-            const uint2 ca = *reinterpret_cast<const uint2 *>(krA + 4 * w);
-            const uint2 cb = *reinterpret_cast<const uint2 *>(krB + 4 * w);
-            cwA[w] = ca.x, cwA[w + 1] = ca.y;
-            cwB[w] = cb.x, cwB[w + 1] = cb.y;
-        }
-    }
-    float av[4], zs = 0.f;
-    {
-        uint2 sr = make_uint2(0u, 0u), zr = make_uint2(0u, 0u);
-        if (ownq) {
-            sr = *reinterpret_cast<const uint2 *>(st + G::KCODES + 8 * lane);          // scales (even block)
-            zr = *reinterpret_cast<const uint2 *>(st + G::HM + G::KCODES + 8 * lane); // zeros (odd block)
-        }
-        const float2 s01 = __half22float2(*reinterpret_cast<const __half2 *>(&sr.x));
-        const float2 s23 = __half22float2(*reinterpret_cast<const __half2 *>(&sr.y));
-        const float2 z01 = __half22float2(*reinterpret_cast<const __half2 *>(&zr.x));
-        const float2 z23 = __half22float2(*reinterpret_cast<const __half2 *>(&zr.y));
-        av[0] = qreg[0] * s01.x;
-        av[1] = qreg[1] * s01.y;
-        av[2] = qreg[2] * s23.x;
-        av[3] = qreg[3] * s23.y;
-        zs = fmaf(qreg[0], z01.x, fmaf(qreg[1], z01.y, fmaf(qreg[2], z23.x, qreg[3] * z23.y)));
-    }
-    const float amax = warp_max_abs(fmaxf(fmaxf(fabsf(av[0]), fabsf(av[1])), fmaxf(fabsf(av[2]), fabsf(av[3]))));
-    zs = warp_sum(zs);
-    const uint32_t ab = __float_as_uint(amax);
-    int F = 21 - ((int)(ab >> 23) - 127) - ((ab & 0x7FFFFFu) >= 0x7FFFFEu ? 1 : 0);
-    F = F > 126 ? 126 : F;
-    const float fs = __int_as_float((F + 127) << 23), fsk = __int_as_float((127 - F) << 23);
-    if (ownq) {
-        const uint32_t y0 = __float_as_uint(fmaf(av[0], fs, 12582912.f));
-        const uint32_t y1 = __float_as_uint(fmaf(av[1], fs, 12582912.f));
-        const uint32_t y2 = __float_as_uint(fmaf(av[2], fs, 12582912.f));
-        const uint32_t y3 = __float_as_uint(fmaf(av[3], fs, 12582912.f));
-        const uint32_t t01 = __byte_perm(y0, y1, 0x5140), t23 = __byte_perm(y2, y3, 0x5140);
-        const uint32_t u01 = __byte_perm(y0, y1, 0x0062), u23 = __byte_perm(y2, y3, 0x0062);
-        const uint32_t d0 = __byte_perm(t01, t23, 0x5410), d1 = __byte_perm(t01, t23, 0x7632);
-        const uint32_t x2 = __byte_perm(u01, u23, 0x5410) ^ 0x40404040u;
-        const uint32_t d2 = x2 | ((x2 & 0x40404040u) << 1);
-        reinterpret_cast<uint4 *>(scr)[lane] = make_uint4(d0, d1, d2, 0u);
-    }
-    __syncwarp();
-    constexpr int QPW = BITS == 4 ? 2 : 4;
-    const uint4 *rh = rec + hf * (G::NQ / 2);
-    KeyAcc accA = {{0u, 0u}, {0u, 0u}, {0, 0}}, accB = {{0u, 0u}, {0u, 0u}, {0, 0}};
-#pragma unroll
-    for (int w = 0; w < HW; ++w)
-        key_word2<BITS>(cwA[w], cwB[w], rh + QPW * w, accA, accB);
-    const uint32_t a01A = accA.a0[0] + accA.a0[1] + ((accA.a1[0] + accA.a1[1]) << 8);
-    const uint32_t a01B = accB.a0[0] + accB.a0[1] + ((accB.a1[0] + accB.a1[1]) << 8);
-    const int a2A = accA.a2[0] + accA.a2[1], a2B = accB.a2[0] + accB.a2[1];
-    const uint32_t a01 = (hf ? a01B : a01A) + __shfl_xor_sync(0xFFFFFFFFu, hf ? a01A : a01B, 16);
-    const int a2 = (hf ? a2B : a2A) + __shfl_xor_sync(0xFFFFFFFFu, hf ? a2A : a2B, 16);
-    const float s2l = fmaf(fmaf((float)a2, 65536.f, (float)a01), fsk, zs); // score of token `lane`
+    const float s2l = group_scores<BITS, D>(st, st + G::HM, scr, qreg, lane); // score of token `lane`
     // ---- running maximum (warp-uniform): rescale the warp's sums when it grows
     const float mg = warp_max_f(s2l);
     if (mg > r.m) {
@@ -1717,8 +1676,7 @@ template <int BITS, int D, typename DT>
 int launch_t(const DecodeArgs &a, const DecodeShape &shp, cudaStream_t s)
 {
     if (shp.onepass)
-        return launch_shape(shp.min_ctas == 5 ? decode_kernel_1p<BITS, D, DT, 5> : decode_kernel_1p<BITS, D, DT, 4>, shp,
-                            s, a, shp.stages_log2);
+        return launch_shape(decode_kernel_1p<BITS, D, DT, 4>, shp, s, a, shp.stages_log2);
     auto kern = shp.min_ctas == 5 ? decode_kernel<BITS, D, DT, 5> : decode_kernel<BITS, D, DT, 4>;
     return launch_shape(kern, shp, s, a, shp.stages_log2, shp.score_bufs);
 }
@@ -1793,7 +1751,9 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
     const char *env_c = getenv("LOOPKV_DECODE_CLUSTER");
     const char *env_s = getenv("LOOPKV_DECODE_STAGES");
     const char *env_o = getenv("LOOPKV_DECODE_CTAS_PER_SM");
-    for (int want_ctas = 4; want_ctas <= 5; ++want_ctas) { // builds for 4 and 5 CTAs per SM
+    // two-phase builds for 4 and 5 CTAs per SM; the single-pass kernel for 4 (its 96-register
+    // build measured 5% slower on the same grid)
+    for (int want_ctas = 4; want_ctas <= (onepass ? 4 : 5); ++want_ctas) {
         if (env_o && atoi(env_o) != want_ctas)
             continue;
         for (int C = 1; C <= 16; C = C < 8 ? C + 1 : 2 * C) { // 1..8, 16
@@ -1812,8 +1772,7 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
                 const int smem = kernel_smem<BITS, D>(onepass, spw, capw, nbuf);
                 if (smem <= 0 || smem > 227 * 1024)
                     continue;
-                int ncl = onepass ? (want_ctas == 5 ? max_active_clusters(decode_kernel_1p<BITS, D, DT, 5>, C, smem)
-                                                    : max_active_clusters(decode_kernel_1p<BITS, D, DT, 4>, C, smem))
+                int ncl = onepass ? max_active_clusters(decode_kernel_1p<BITS, D, DT, 4>, C, smem)
                           : want_ctas == 5 ? max_active_clusters(decode_kernel<BITS, D, DT, 5>, C, smem)
                                            : max_active_clusters(decode_kernel<BITS, D, DT, 4>, C, smem);
                 if (ncl <= 0)
