@@ -335,8 +335,9 @@ template <int D> __host__ __device__ constexpr int scratch_bytes()
     return align16(imax((D / 4 + D / 32) * 16, imax((D + 2) * 4, (D / 32) * 40 * 4 + 4)));
 }
 
-// nbuf: score buffers (2 when a cluster reads more than one row, so that the next row's
-// keys can be scored while the current row's values are read).
+// nbuf: score buffers (2: the next row's keys are scored while the current row's values are
+// read; 1: a cluster's rows run one after another, for long rows whose scores fill the
+// shared memory).
 template <int BITS, int D> __host__ __device__ constexpr SmemLayout smem_layout(int spw, int capw, int nbuf)
 {
     SmemLayout L{};
@@ -405,11 +406,15 @@ template <int BITS, int D> bool layout_ok(int spw, int capw, int nbuf)
 // Groups of a row owned by warp w of the CTA: local groups w, w + kWarps, ...
 __device__ __forceinline__ int owned(int nmy, int w) { return nmy > w ? (nmy - w + kWarps - 1) / kWarps : 0; }
 
-// Segment sig of a warp's stage sequence K(0), K(1), V(0), K(2), V(1), ..., V(n-1):
-// returns whether it is a V segment and its row index.
-__device__ __forceinline__ void segment(int sig, int nrows, bool &is_v, int &ri)
+// Segment sig of a warp's stage sequence: returns whether it is a V segment and its row
+// index.  Overlapped order (two score buffers) K(0), K(1), V(0), K(2), V(1), ..., V(n-1);
+// sequential order (one score buffer) K(0), V(0), K(1), V(1), ...
+__device__ __forceinline__ void segment(int sig, int nrows, bool seq, bool &is_v, int &ri)
 {
-    if (sig == 0) {
+    if (seq) {
+        is_v = sig & 1;
+        ri = sig >> 1;
+    } else if (sig == 0) {
         is_v = false;
         ri = 0;
     } else if (sig == 2 * nrows - 1) {
@@ -464,6 +469,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     Smem sm = carve<BITS, D>(smem_raw, spw, capw, nbuf);
     const bool all_hot = (BITS == 4) && !(a.tau > 0.f);
     const bool decide = (BITS == 4) && (a.tau > 0.f); // lo planes depend on the row max
+    const bool seq = nbuf == 1; // one score buffer: rows one after another (see the main loop)
     // byte distance between consecutive block ids in the pools (one block = H heads)
     const uint32_t bstride = (uint32_t)a.H * G::HM, lstride = (uint32_t)a.H * G::LOB;
 
@@ -576,7 +582,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         __syncwarp();
     };
     auto load_segment = [&]() {
-        segment(iss_sig, nrows, seg_v, seg_ri);
+        segment(iss_sig, nrows, seq, seg_v, seg_ri);
         const int32_t *st = irow_of(seg_ri);
         seg_n = st[IR_N];
         seg_len = (seg_n + kGPS - 1) / kGPS;
@@ -702,7 +708,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
                 break;
             bool nv;
             int nri;
-            segment(nsig, nrows, nv, nri);
+            segment(nsig, nrows, seq, nv, nri);
             if (!nv && nri > setup_upto)
                 break;
             iss_sig = nsig;
@@ -1057,29 +1063,39 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         return a.tau_mode == LOOPKV_TAU_ABS_PROB ? m + log2f(a.tau * l) : m + log2f(a.tau);
     };
 
-    // Iteration i scores row i and reads the values of row i - 1; each phase has a single
-    // call site (keeps the kernel's code small).  Barrier i publishes the maxima of row i
-    // and the partials of row i - 1.
+    // Overlapped order: iteration i scores row i and reads the values of row i - 1; barrier
+    // i (arrived after the iteration) publishes the maxima of row i and the partials of row
+    // i - 1.  Sequential order (one score buffer): iteration i scores row i, passes barrier
+    // i (maxima of row i, partials of row i - 1), merges row i - 1 and reads the values of
+    // row i.  Each phase has a single call site (keeps the kernel's code small).
     float m_prev = 0.f;
     for (int i = 0; i <= nrows; ++i) {
         if (i < nrows)
             consume_k(i);
-        if (i > 0) {
-            cluster_wait(); // barrier i - 1: maxima of row i - 1, partials of row i - 2
-            if (i >= 2)
-                merge(i - 2, m_prev);
-            float m2, l2;
-            cluster_row_stats(sm.stat + ((i - 1) % 3) * kWarps * 2, C, lane, m2, l2);
-            const float thr2 = row_threshold(m2, l2);
-            release_row(i - 1, thr2);
-            consume_v(i - 1, m2, thr2);
-            m_prev = m2;
+        if (seq)
+            cluster_arrive(); // barrier i
+        if (seq || i > 0) {
+            cluster_wait(); // barrier i (sequential) or i - 1
+            const int mr = seq ? i - 1 : i - 2, vr = seq ? i : i - 1;
+            if (mr >= 0)
+                merge(mr, m_prev);
+            if (vr < nrows) {
+                float m2, l2;
+                cluster_row_stats(sm.stat + (vr % 3) * kWarps * 2, C, lane, m2, l2);
+                const float thr2 = row_threshold(m2, l2);
+                release_row(vr, thr2);
+                consume_v(vr, m2, thr2);
+                m_prev = m2;
+            }
         }
-        cluster_arrive(); // barrier i
+        if (!seq)
+            cluster_arrive(); // barrier i
     }
-    cluster_wait(); // partials of the last row
-    if (nrows > 0)
-        merge(nrows - 1, m_prev);
+    if (!seq) {
+        cluster_wait(); // partials of the last row
+        if (nrows > 0)
+            merge(nrows - 1, m_prev);
+    }
     cluster_arrive(); // remote reads done
     cluster_wait();
 }
@@ -1711,10 +1727,12 @@ template <typename K> int max_active_clusters(K kern, int C, int smem)
 // Launch shape.  Model: a cluster of C CTAs serves ceil(rows / clusters) rows one after
 // another; a CTA's share of one row costs (groups / C + kRowFixed) group-times, and an SM
 // running n CTAs gives each 1 / max(n, kSaturate) of its throughput.  Time is then
-// rounds * (G / C + kRowFixed) * max(n, kSaturate) with n the CTAs on the busiest SM.
-// Among equal times the deeper ring (more bytes in flight) wins.
+// rounds * (G / C + kRowFixed) * max(n, kSaturate) with n the CTAs on the busiest SM; rows
+// that do not overlap (one score buffer, several rounds) cost kSeqRow more each.  Among
+// equal times the deeper ring (more bytes in flight) wins.
 constexpr double kRowFixed = 6.0;  // per-CTA cost of a row outside its groups (setup, merge, bubble)
 constexpr double kSaturate = 3.5;  // CTAs per SM that keep its issue slots busy
+constexpr double kSeqRow = 4.0;    // extra per-row cost when rows do not overlap (one score buffer)
 
 // Overlap with the previous launch of the stream (programmatic dependent launch): measured
 // faster with clusters of up to 4 CTAs and slower with larger ones; LOOPKV_DECODE_PDL=0/1
@@ -1751,6 +1769,7 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
     const char *env_c = getenv("LOOPKV_DECODE_CLUSTER");
     const char *env_s = getenv("LOOPKV_DECODE_STAGES");
     const char *env_o = getenv("LOOPKV_DECODE_CTAS_PER_SM");
+    const char *env_b = getenv("LOOPKV_DECODE_SCORE_BUFS");
     // two-phase builds for 4 and 5 CTAs per SM; the single-pass kernel for 4 (its 96-register
     // build measured 5% slower on the same grid)
     for (int want_ctas = 4; want_ctas <= (onepass ? 4 : 5); ++want_ctas) {
@@ -1779,11 +1798,13 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
                     continue;
                 if (ncl > rows)
                     ncl = rows;
-                if (!onepass && nbuf == 1 && ncl < rows)
-                    continue; // a cluster would read several rows: it needs two score buffers
+                if (!onepass && env_b && atoi(env_b) != nbuf)
+                    continue;
                 const int rounds = (rows + ncl - 1) / ncl;
                 const int per_sm = (ncl * C + sm_count - 1) / sm_count;
-                const double t = rounds * ((double)max_groups / C + kRowFixed) * std::max((double)per_sm, kSaturate) *
+                // one score buffer with several rows per cluster: rows run one after another
+                const double row_cost = kRowFixed + (!onepass && nbuf == 1 && rounds > 1 ? kSeqRow : 0.0);
+                const double t = rounds * ((double)max_groups / C + row_cost) * std::max((double)per_sm, kSaturate) *
                                  (1.0 - 0.01 * spw);
                 if (t < best_t * (1.0 - 1e-9)) {
                     best_t = t;
@@ -1799,7 +1820,8 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
                     best.pdl = pdl_default(C);
                     best.onepass = onepass;
                 }
-                break;
+                if (onepass)
+                    break; // no score buffers
             }
         }
     }
