@@ -237,6 +237,22 @@ def test_full_size_sampled_rows(name, B, T, modes, tau, steps):
             m.check_bytes(lp, 0, reqs=[0, B - 1], heads=[0, 7])
 
 
+@pytest.mark.parametrize("score_bufs", ["1", "2"])
+def test_two_phase_score_buffer_orders(monkeypatch, score_bufs):
+    """The decide path (4-bit, tau > 0) with one score buffer (a cluster's rows in sequence)
+    and with two (the next row's keys overlapping the current row's values), forced through
+    the launch-shape override on a batch with more rows than clusters."""
+    monkeypatch.setenv("LOOPKV_DECODE_SCORE_BUFS", score_bufs)
+    base = synth.workload("mixed_8k")
+    w = synth.Workload("mixed_8k", 1, 4, 16, 128, 32, [8192] * 32, torch.bfloat16, [0, 1, 2, 0], 0.01, seed=2)
+    m = Model(w, max_blocks=base.max_blocks)
+    m.ingest()
+    rng = np.random.default_rng(1)
+    for lp in (0, 2, 3):  # 4-bit, share of a 4-bit source, final loop
+        rows = [(int(rng.integers(32)), int(rng.integers(16))) for _ in range(6)] + [(31, 15), (0, 0)]
+        m.check_cell(lp, 0, _q(w, 0, 0, lp), rows=rows, where=f"score buffers {score_bufs}")
+
+
 def test_graph_replay_matches_eager():
     modes = [L.CELL_4B, L.CELL_SHARE, L.CELL_2B, L.CELL_4B]  # loop 0: [4b, share], loop 1: [2b, 4b]
     w = synth.Workload("graph", 2, 2, 4, 128, 3, [33, 64, 200], torch.bfloat16, modes, 0.01, append_steps=40,
