@@ -1,5 +1,10 @@
 // decode_kernel.cu -- fused, plan-driven decode attention over the LoopKV cache.
 //
+// Two kernels.  decode_kernel (below) serves reads whose refine set depends on the row
+// maximum (4-bit sources, tau > 0) and takes the exact maximum in two phases;
+// decode_kernel_1p (further down) serves reads whose refine set is fixed in advance
+// (2-bit sources, tau <= 0) in a single pass with a running maximum.
+//
 // One launch per cell (LoopKV paper, §3.4 "One launch per cell").  The grid is a set
 // of persistent thread-block clusters of C CTAs; cluster c serves the (request, head)
 // rows c, c + NC, c + 2NC, ... one after another.  Inside a row, CTA k of the cluster
@@ -23,10 +28,11 @@
 //      are folded into the weight and a running sum.
 //   4. Merge: since all CTAs used the same m, their partial sums add directly; the CTAs
 //      reduce them through distributed shared memory and write out = o / l.
-// Rows are software-pipelined: while the cluster barrier that publishes row r's maxima
-// completes, the warp already streams and scores the keys of row r+1, so the memory pipe
-// never drains at a row boundary.  One cluster barrier per row carries both the
-// per-warp maxima of row r and the partial outputs of row r-1.
+// With two score buffers rows are software-pipelined: while the cluster barrier that
+// publishes row r's maxima completes, the warp already streams and scores the keys of row
+// r+1, so the memory pipe never drains at a row boundary, and one cluster barrier per row
+// carries both the per-warp maxima of row r and the partial outputs of row r-1.  Long
+// rows, whose scores fill the shared memory, take one score buffer and run in sequence.
 //
 // Keys: the dot product of a 32-token group is computed exactly in integers.  The
 // group's per-channel factor a_c = q_c * s_c is rounded to a 22-bit fixed-point integer
@@ -35,6 +41,8 @@
 // signed byte) with byte permutes.  The 4-bit (or 2-bit) codes are unpacked four at a
 // time into bytes with one AND, and dp4a accumulates code * digit in int32 with no
 // rounding.
+// The key loads are laid out so that the lanes of a shared-memory phase hit distinct
+// banks (group_scores).
 // Values: a value-plane word holds 4 tokens x 4 channels (token in the byte).  The hi and
 // lo words merge into 4-bit codes (lo bits of cold tokens masked off), one AND unpacks the
 // codes of one channel for 4 tokens, and dp4a against the two 8-bit digits of the tokens'
