@@ -234,7 +234,10 @@ int loopkv_reset_request(loopkv_cache *cache, int req, void *stream);
  * over its own tail; exact row max m; refine set S = history tokens of a 4-bit
  * source whose weight passes tau; values decoded as z + s*(4h+l) for tokens in S,
  * z + s*(4h+1.5) for the other 4-bit tokens, z + s*code for 2-bit cells, raw for the
- * tail; out = sum_t exp(s_t - m) v_t / sum_t exp(s_t - m).
+ * tail; out = sum_t exp(s_t - m) v_t / sum_t exp(s_t - m).  When S does not depend on
+ * m (2-bit source, or tau <= 0) the launch accumulates with a running maximum instead;
+ * the result is the same up to fp32 rounding.  The call allocates nothing and keeps no
+ * state between launches, so decodes of different cells may run on different streams.
  */
 int loopkv_decode(const loopkv_plan *plan, int loop, int layer, const void *q,
                   const loopkv_cache *cache, float *out, int B, void *stream);
@@ -259,7 +262,9 @@ int loopkv_status(loopkv_cache *cache, void *stream, int *device_status);
 int loopkv_cell_view_get(const loopkv_cache *cache, int loop, int layer, loopkv_cell_view *out);
 
 /* Decode launch shape chosen for a batch of B requests (cluster size, CTAs, shared
- * memory per CTA), for reporting.  Queries the occupancy of the current device. */
+ * memory per CTA) when the source cell is 4-bit, for reporting: the single-pass reader
+ * when the plan's tau <= 0 (every token refined), else the exact-maximum reader.
+ * Queries the occupancy of the current device (LOOPKV_ERR_NO_DEVICE without one). */
 int loopkv_decode_shape(const loopkv_plan *plan, int B, int *cluster_size, int *ctas, int *smem_bytes);
 
 const char *loopkv_strerror(int code);
