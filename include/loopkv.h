@@ -236,8 +236,10 @@ int loopkv_reset_request(loopkv_cache *cache, int req, void *stream);
  * z + s*(4h+1.5) for the other 4-bit tokens, z + s*code for 2-bit cells, raw for the
  * tail; out = sum_t exp(s_t - m) v_t / sum_t exp(s_t - m).  When S does not depend on
  * m (2-bit source, or tau <= 0) the launch accumulates with a running maximum instead;
- * the result is the same up to fp32 rounding.  The call allocates nothing and keeps no
- * state between launches, so decodes of different cells may run on different streams.
+ * the result is the same up to fp32 rounding.  A decode uses no device scratch, so
+ * decodes of different cells may run on different streams.  The first call for a batch
+ * size queries the device occupancy to pick the launch shape (cached in the cache
+ * object); make it before capturing a stream.
  */
 int loopkv_decode(const loopkv_plan *plan, int loop, int layer, const void *q,
                   const loopkv_cache *cache, float *out, int B, void *stream);
