@@ -493,3 +493,53 @@ int orc_decode_row(int D, int bits, int n_hist, const double *q, const uint8_t *
     free(r);
     return ORC_OK;
 }
+
+/*
+ * Refine set of the streaming reader (LoopKV §3.3 "Read-time V precision", §3.4 launch
+ * grid): instead of the row's exact maximum, the reader tests each token against a
+ * maximum that starts at a seed m0 (the published sink maximum; when it does not arrive
+ * in time the seed is chosen so that every token is hot).  The pages leave open whether
+ * that maximum also grows with the scores the reader has already computed; both
+ * readings are provided:
+ *   running = 1: the history is read in 32-token groups in the order order[0..ng-1]; a
+ *                group's scores are known before its values are read, so the running
+ *                maximum takes the group's largest score before its tokens are tested;
+ *   running = 0: every token is tested against the seed alone (m0 = -infinity then
+ *                marks every token hot, the fallback of §3.4).
+ * Token t is hot iff exp(s_t - m) >= tau for the maximum m it is tested against.  As
+ * long as m0 does not exceed the exact row maximum, neither maximum does, and the set
+ * contains the exact one (a superset).
+ *   s[n_hist]            scores in natural-log units (q.k / sqrt(D))
+ *   order[ng]            each group index 0..n_hist/32-1 exactly once
+ *   s_bits[n_hist/32]    output, bit (t % 32) of word t/32 set iff t is hot
+ * Returns ORC_BADARG on a malformed order.
+ */
+int orc_stream_refine(int n_hist, const double *s, const int *order, int ng, double m0, int running,
+                      double tau, uint32_t *s_bits)
+{
+    if (n_hist < 0 || n_hist % ORC_GROUP || ng != n_hist / ORC_GROUP)
+        return ORC_BADARG;
+    unsigned char *seen = (unsigned char *)calloc((size_t)(ng > 0 ? ng : 1), 1);
+    for (int i = 0; i < ng; ++i) {
+        if (order[i] < 0 || order[i] >= ng || seen[order[i]]) {
+            free(seen);
+            return ORC_BADARG;
+        }
+        seen[order[i]] = 1;
+    }
+    free(seen);
+    double m_run = m0;
+    for (int i = 0; i < ng; ++i) {
+        const int g = order[i];
+        if (running)
+            for (int j = 0; j < ORC_GROUP; ++j)
+                if (s[g * ORC_GROUP + j] > m_run)
+                    m_run = s[g * ORC_GROUP + j];
+        uint32_t w = 0;
+        for (int j = 0; j < ORC_GROUP; ++j)
+            if (exp(s[g * ORC_GROUP + j] - m_run) >= tau)
+                w |= 1u << j;
+        s_bits[g] = w;
+    }
+    return ORC_OK;
+}

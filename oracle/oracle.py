@@ -70,6 +70,9 @@ def lib():
                                          _u8p, _u16p, _u16p, ctypes.c_int, _f64p, _f64p, ctypes.c_double,
                                          ctypes.c_int, _u32p, _f64p, _f64p, _f64p, _u32p, _f64p]
             L.orc_decode_row.restype = ctypes.c_int
+            L.orc_stream_refine.argtypes = [ctypes.c_int, _f64p, ctypes.POINTER(ctypes.c_int), ctypes.c_int,
+                                            ctypes.c_double, ctypes.c_int, ctypes.c_double, _u32p]
+            L.orc_stream_refine.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -254,3 +257,17 @@ def dequant_v(hist: HeadHistory, hot: np.ndarray | None) -> np.ndarray:
     if hot is None:
         hot = np.ones(hist.T, bool)
     return np.where(hot[:, None], z + s * code, z + s * cold)
+
+
+def stream_refine(scores, order, m0: float, tau: float, running: bool = True) -> np.ndarray:
+    """Refine set of the streaming reader (seeded maximum, growing with the scores read when
+    `running`; see orc_stream_refine): scores [n_hist] in natural-log units, order = group
+    reading order.  Returns the bitmap [n_hist / 32] (uint32)."""
+    s = np.ascontiguousarray(scores, np.float64)
+    o = np.ascontiguousarray(order, np.int32)
+    bits = np.zeros(max(s.size // GROUP, 1), np.uint32)
+    st = lib().orc_stream_refine(int(s.size), _p(s, _f64p), o.ctypes.data_as(ctypes.POINTER(ctypes.c_int)),
+                                 int(o.size), float(m0), int(bool(running)), float(tau), _p(bits, _u32p))
+    if st != OK:
+        raise ValueError(f"oracle stream_refine status {st}")
+    return bits[: s.size // GROUP]
