@@ -214,6 +214,30 @@ int loopkv_append(loopkv_cache *cache, int loop, int layer, const void *k, const
                   const int32_t *req_ids, int B, void *stream);
 
 /*
+ * loopkv_append for callers that cannot allocate device memory: engines that hand all
+ * device memory to their own arena up front (so no further allocation can succeed), or
+ * code on a decode loop that cannot take the device-wide synchronisation an allocation may
+ * cause.  The LoopKV paper has no counterpart; this is an interface convenience.
+ *
+ * Same arguments, results and device-side errors as loopkv_append.  The request ids go to
+ * the device through a fixed array inside the library (LOOPKV_NOALLOC_MAX_IDS int32, 16 KiB,
+ * which every GPU that loads the library keeps until the process exits) instead of the
+ * cache's staging words, and the call allocates nothing: no cudaMalloc, no cudaFree, no
+ * allocating library routine.
+ *   - B > LOOPKV_NOALLOC_MAX_IDS (or > max_batch) returns LOOPKV_ERR_SHAPE before any
+ *     device work.
+ *   - The first call on a device looks up the array's device address with the device
+ *     current (cudaGetSymbolAddress) and keeps it; make that first call before any stream
+ *     capture.  A failed look-up returns LOOPKV_ERR_CUDA.
+ *   - Every call shares the one array and leaves its ids there; each call writes all B ids
+ *     it reads, so nothing has to start at zero.  Calls whose copies and kernels overlap on
+ *     the GPU (different streams, no ordering between them) race on the array: order them.
+ */
+#define LOOPKV_NOALLOC_MAX_IDS 4096
+int loopkv_append_noalloc(loopkv_cache *cache, int loop, int layer, const void *k, const void *v,
+                          const int32_t *req_ids, int B, void *stream);
+
+/*
  * Window exit: quantize every tail that holds 32 tokens into two new 16-token blocks
  * of its cell (K per channel over the 32 tokens, V per token over 32 channels, fp16
  * scale/zero, V split into hi/lo planes) and empty it; a share cell only empties its

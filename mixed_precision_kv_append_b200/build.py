@@ -12,7 +12,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libloopkv.so")
 OBJDIR = os.path.join(ROOT, "_build")
-SOURCES = ["runtime.cu", "quant_kernels.cu", "decode_kernel.cu", "plan_search.cu"]
+SOURCES = ["runtime.cu", "quant_kernels.cu", "decode_kernel.cu", "plan_search.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]
 

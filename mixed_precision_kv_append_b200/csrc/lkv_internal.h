@@ -83,4 +83,11 @@ int launch_ingest(const DevState &st, int cell, int mode, int H, int D, int dtyp
 int launch_reset(const DevState &st, const uint8_t *cell_modes_dev, int n_cells, int max_batch, int max_blocks,
                  int req, cudaStream_t s);
 
+// What an entry point defined outside runtime.cu needs to know about a cache.
+struct CacheInfo {
+    DevState st;
+    int n_loops, n_layers, n_heads, head_dim, in_dtype, max_batch;
+};
+int cache_info(const loopkv_cache *cache, CacheInfo *out);
+
 }  // namespace lkv

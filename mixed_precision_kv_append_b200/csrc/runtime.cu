@@ -171,6 +171,21 @@ int check_device()
 
 }  // namespace
 
+int lkv::cache_info(const loopkv_cache *cache, lkv::CacheInfo *out)
+{
+    if (!cache || !out)
+        return LOOPKV_ERR_INVALID_ARG;
+    const loopkv_config &c = cache->plan.cfg;
+    out->st = cache->st;
+    out->n_loops = c.n_loops;
+    out->n_layers = c.n_layers;
+    out->n_heads = c.n_heads;
+    out->head_dim = c.head_dim;
+    out->in_dtype = c.in_dtype;
+    out->max_batch = c.max_batch;
+    return LOOPKV_OK;
+}
+
 extern "C" {
 
 int loopkv_version(void) { return 100; }

@@ -33,8 +33,9 @@ EXPORTS = [
     "loopkv_plan_create", "loopkv_plan_free", "loopkv_plan_bytes", "loopkv_required_bytes", "loopkv_alloc",
     "loopkv_free", "loopkv_ingest", "loopkv_append", "loopkv_flush", "loopkv_reset_request", "loopkv_decode",
     "loopkv_decode_debug", "loopkv_status", "loopkv_cell_view_get", "loopkv_decode_shape", "loopkv_strerror",
-    "loopkv_version", "loopkv_plan_search",
+    "loopkv_version", "loopkv_plan_search", "loopkv_append_noalloc",
 ]
+NOALLOC_MAX_IDS = 4096
 
 
 class LoopKVError(RuntimeError):
@@ -91,6 +92,7 @@ def lib() -> ctypes.CDLL:
         L.loopkv_free.restype = None
         L.loopkv_ingest.argtypes = [vp, i, i, i, vp, vp, i, vp]
         L.loopkv_append.argtypes = [vp, i, i, vp, vp, ctypes.POINTER(ctypes.c_int32), i, vp]
+        L.loopkv_append_noalloc.argtypes = [vp, i, i, vp, vp, ctypes.POINTER(ctypes.c_int32), i, vp]
         L.loopkv_flush.argtypes = [vp, vp]
         L.loopkv_reset_request.argtypes = [vp, i, vp]
         L.loopkv_decode.argtypes = [vp, i, i, vp, vp, vp, i, vp]
@@ -197,6 +199,18 @@ def loopkv_append(cache, loop: int, layer: int, k: torch.Tensor, v: torch.Tensor
     if req_ids is not None:
         ids = (ctypes.c_int32 * B)(*[int(r) for r in req_ids])
     _check(lib().loopkv_append(cache, loop, layer, _ptr(k), _ptr(v), ids, B, _stream(stream)), "loopkv_append")
+
+
+def loopkv_append_noalloc(cache, loop: int, layer: int, k: torch.Tensor, v: torch.Tensor, req_ids=None,
+                          stream=None):
+    """loopkv_append with the request ids staged in the library's fixed device array (the call
+    allocates nothing)."""
+    ids = None
+    B = int(k.shape[0])
+    if req_ids is not None:
+        ids = (ctypes.c_int32 * B)(*[int(r) for r in req_ids])
+    _check(lib().loopkv_append_noalloc(cache, loop, layer, _ptr(k), _ptr(v), ids, B, _stream(stream)),
+           "loopkv_append_noalloc")
 
 
 def loopkv_flush(cache, stream=None):
