@@ -6,11 +6,14 @@ full tails at the start of the step] and one fused decode launch, replayed as on
 graph (the pages replay a whole decode step as one graph).  Inputs are resident in HBM;
 the per-step KV working set (16 GB and up) is far larger than L2, so no flush is needed.
 
-Prints one JSON line.  `value` = algorithmic KV bytes read per step / step time (GB/s);
-`e2e` = the same through the public API with the step's queries copied from pinned host
-memory and the outputs copied back inside the timed region.
+Prints one JSON line.  `value` = algorithmic KV bytes read per step / step time (GB/s) of the
+headline workload (default long_16k, the largest single-GPU configuration, with appends);
+`e2e` = the same through the public API with the step's inputs (queries, and the new keys and
+values of an appending workload) copied from pinned host memory and the outputs copied back
+inside the timed region; `workloads` = the other workloads measured the same way.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--config kivi4_8k] [--impl ours|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config long_16k] [--workloads kivi4_8k,mixed_8k]
+                  [--impl ours|reference]
 """
 from __future__ import annotations
 
@@ -224,7 +227,10 @@ class Runner:
         return total, (hot_tokens / all_tokens if all_tokens else 0.0)
 
 
-def _time_graph(runner: Runner, steps: int, e2e: bool, host_q=None, host_out=None):
+def _time_graph(runner: Runner, steps: int, e2e: bool, host=None):
+    """Device time of `steps` graph replays on the runner's stream (CUDA events on that stream).
+    With e2e, every step first copies its inputs from pinned host memory (queries, and the new
+    keys and values of an appending workload) and ends with a copy of all outputs to the host."""
     s = runner.stream
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
@@ -232,17 +238,20 @@ def _time_graph(runner: Runner, steps: int, e2e: bool, host_q=None, host_out=Non
         ev0.record(s)
         for _ in range(steps):
             if e2e:
-                runner.q.copy_(host_q, non_blocking=True)
+                for dev_t, host_t in host["in"]:
+                    dev_t.copy_(host_t, non_blocking=True)
             runner.graph.replay()
             if e2e:
-                host_out.copy_(runner.out, non_blocking=True)
+                host["out"].copy_(runner.out, non_blocking=True)
         ev1.record(s)
     ev1.synchronize()
     return ev0.elapsed_time(ev1) / 1e3  # seconds
 
 
-def _workload(args):
-    w = synth.workload(args.config, seed=args.seed)
+def _workload(name, args):
+    w = synth.workload(name, seed=args.seed)
+    if w.append_steps:  # room for every appended token of this run (warm-up, timing, e2e, setup)
+        w.append_steps = max(w.append_steps, 2 * (args.steps + args.warmup) + 8)
     if args.layers and args.layers < w.n_layers:
         n = args.layers
         w.modes = [w.modes[lp * w.n_layers + la] for lp in range(w.n_loops) for la in range(n)]
@@ -251,14 +260,11 @@ def _workload(args):
     return w
 
 
-def run_ours(args, rank, world, device):
-    w = _workload(args)
+def measure(w, args, rank, world, device, e2e: bool):
+    """One workload: build the cache, capture a step, time it.  Returns (result dict, runner)."""
     runner = Runner(w, device)
     algo_bytes, hot = runner.hot_fraction_and_bytes()
     runner.capture()
-    host_q = torch.empty(runner.q.shape, dtype=runner.q.dtype, pin_memory=True)
-    host_q.copy_(runner.q)
-    host_out = torch.empty(runner.out.shape, dtype=torch.float32, pin_memory=True)
     for _ in range(args.warmup):
         runner.graph.replay()
     torch.cuda.synchronize(device)
@@ -268,32 +274,61 @@ def run_ours(args, rank, world, device):
     with ClockSampler(device.index if device.index is not None else 0) as clk:
         t = _time_graph(runner, args.steps, False)
     torch.cuda.synchronize(device)
-    for _ in range(2):
-        runner.graph.replay()
-    if world > 1:
-        dist.barrier()
-    t_e2e = _time_graph(runner, args.steps, True, host_q, host_out)
+    t_e2e, h2d = None, 0
+    if e2e:
+        ins = [runner.q] + ([runner.knew, runner.vnew] if w.append_steps else [])
+        host = {"in": [], "out": torch.empty(runner.out.shape, dtype=torch.float32, pin_memory=True)}
+        for dev_t in ins:
+            h = torch.empty(dev_t.shape, dtype=dev_t.dtype, pin_memory=True)
+            h.copy_(dev_t)
+            host["in"].append((dev_t, h))
+            h2d += dev_t.numel() * dev_t.element_size()
+        for _ in range(2):
+            runner.graph.replay()
+        if world > 1:
+            dist.barrier()
+        t_e2e = _time_graph(runner, args.steps, True, host)
     runner.cache.check("timed steps")
-    t, t_e2e = max_over_ranks([t, t_e2e], device)
+    t, t_e2e = max_over_ranks([t, t_e2e if t_e2e is not None else 0.0], device)
     peak, peak_kind = _peaks()
     ms = t / args.steps * 1e3
     gbs = algo_bytes * world * args.steps / t / 1e9
-    gbs_e2e = algo_bytes * world * args.steps / t_e2e / 1e9
+    # per decode launch: algorithmic bytes of one launch / (step time / decode launches); the
+    # step's flush and append launches are counted in the time, so this is a lower bound
     n_decode = len(runner.order)
-    per_launch_s = t / args.steps / n_decode
-    per_launch_bytes = algo_bytes / n_decode
-    achieved = per_launch_bytes / per_launch_s / 1e9 if not w.append_steps else gbs / world
+    achieved = (algo_bytes / n_decode) / (t / args.steps / n_decode) / 1e9
     shape = runner.plan.decode_shape(w.B)
+    res = {
+        "value": round(gbs, 2), "ms_per_step": round(ms, 4), "steps_per_s": round(1e3 / ms, 2),
+        "pct_hbm_peak": round(100.0 * gbs / world / peak, 2), "hot_fraction": round(hot, 4),
+        "frac": round(achieved / peak, 4), "traffic": _profiled_traffic(w.name) if not args.layers else None,
+        "algorithmic_bytes_per_step": int(algo_bytes), "cluster": shape["cluster"], "ctas_per_launch": shape["ctas"],
+        "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "clocks": clk.summary(),
+        "launches_per_step": runner.launches_per_step,
+    }
+    if e2e:
+        res["e2e"] = {"value": round(algo_bytes * world * args.steps / t_e2e / 1e9, 2), "unit": "GB/s",
+                      "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(runner.out.numel() * 4),
+                      "ms_per_step": round(t_e2e / args.steps * 1e3, 4)}
+    return res, runner
+
+
+def run_ours(args, rank, world, device):
+    w = _workload(args.config, args)
+    head, runner = measure(w, args, rank, world, device, e2e=True)
+    algo_bytes = head["algorithmic_bytes_per_step"]
+    del runner
+    torch.cuda.empty_cache()
     result = {
         "metric": METRIC,
-        "value": round(gbs, 2),
+        "value": head["value"],
         "unit": "GB/s",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(ms, 4),
-        "steps_per_s": round(1e3 / ms, 2),
-        "pct_hbm_peak": round(100.0 * gbs / world / peak, 2),
+        "ms_per_step": head["ms_per_step"],
+        "steps_per_s": head["steps_per_s"],
+        "pct_hbm_peak": head["pct_hbm_peak"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -302,69 +337,119 @@ def run_ours(args, rank, world, device):
         "config": {"workload": w.name, "layers": w.n_layers, "loops": w.n_loops, "heads": w.H, "head_dim": w.D,
                    "batch_per_gpu": w.B, "global_batch": w.B * world, "context": max(w.lengths),
                    "tau": w.tau, "cells_4b_2b_share": [w.modes.count(0), w.modes.count(1), w.modes.count(2)],
-                   "append": bool(w.append_steps), "hot_fraction": round(hot, 4),
-                   "algorithmic_bytes_per_step": int(algo_bytes), "cluster": shape["cluster"],
-                   "ctas_per_launch": shape["ctas"], "l2": "per-step working set >> 126 MB L2 (no flush needed)",
+                   "append": bool(w.append_steps), "hot_fraction": head["hot_fraction"],
+                   "algorithmic_bytes_per_step": algo_bytes, "cluster": head["cluster"],
+                   "ctas_per_launch": head["ctas_per_launch"],
+                   "l2": "per-step working set >> 126 MB L2 (no flush needed)",
                    "parallelism": f"dp{world} (request-sharded replicas)"},
-        "e2e": {"value": round(gbs_e2e, 2), "unit": "GB/s",
-                "h2d_bytes_per_step": int(runner.q.numel() * runner.q.element_size()),
-                "d2h_bytes_per_step": int(runner.out.numel() * 4),
-                "ms_per_step": round(t_e2e / args.steps * 1e3, 4)},
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4),
-                     "traffic": _profiled_traffic(w.name) if not args.layers else None,
-                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"},
-        "gpu_launches": runner.launches_per_step * args.steps * 2,
-        "clocks": clk.summary(),
+        "e2e": head["e2e"],
+        "roofline": {"bound": "hbm", "achieved": head["achieved"], "peak": head["peak"], "unit": "GB/s",
+                     "frac": head["frac"], "traffic": head["traffic"],
+                     "peak_source": f"{head['peak_kind']} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"},
+        "gpu_launches": head["launches_per_step"] * args.steps * 2,
+        "clocks": head["clocks"],
     }
+    if args.workloads:
+        result["workloads"] = {}
+        for name in [n for n in args.workloads.split(",") if n and n != args.config]:
+            wl, r = measure(_workload(name, args), args, rank, world, device, e2e=False)
+            del r
+            torch.cuda.empty_cache()
+            result["workloads"][name] = {k: wl[k] for k in ("value", "ms_per_step", "steps_per_s", "hot_fraction",
+                                                            "frac", "traffic", "algorithmic_bytes_per_step",
+                                                            "cluster", "ctas_per_launch", "clocks")}
     if rank == 0 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds)
+        result["cpu_baseline"] = cpu_baseline(w, algo_bytes, budget_s=args.cpu_seconds)
     return result
 
 
 # ------------------------------------------------------------------- CPU oracle timing
 
-def cpu_baseline(w: synth.Workload, budget_s: float = 15.0, rows_max: int | None = None):
-    """Time the CPU oracle's decode (single thread) on whole rows of cell (0, 0) at the
-    workload's context, and express it in the benchmark's unit."""
+def _cpu_rows(w: synth.Workload, n_rows: int):
+    """Rows (request, head) of the workload at its context for the CPU oracle, drawn from the
+    cells of layer 0 in loop order: (query, quantized history of the cell read, bytes the GPU
+    path counts for the row).  Share cells read the final loop's history."""
     import numpy as np
 
     from oracle import oracle as O
 
-    bits = 4 if w.modes[0] == 0 else 2
-    T = w.lengths[0] // 32 * 32
-    ks, vs = synth.layer_history(w, 0, 0, T=T, device="cpu")
-    K, V = ks[0].float().numpy(), vs[0].float().numpy()
+    rows = []
+    req = 0
+    T = w.lengths[req] // 32 * 32
+    ks, vs = synth.layer_history(w, 0, req, T=T, device="cpu")
     qs, _, _ = synth.step_tokens(w, 0, 0, device="cpu")
-    q = qs[0].float().numpy()
-    per_tok = (160.0 if bits == 4 else 96.0) * (w.D / 128.0)
-    rows, secs = 0, 0.0
+    cells = list(range(w.n_loops))
+    hists = {}
     h = 0
-    while (rows < rows_max) if rows_max is not None else (secs < budget_s):
-        hist = O.HeadHistory(K[:, h % w.H], V[:, h % w.H], bits)
-        t0 = time.perf_counter()
-        O.decode_row(q[0, h % w.H].astype(np.float64), hist, np.zeros((0, w.D)), np.zeros((0, w.D)), w.tau,
-                     w.tau_mode)
-        secs += time.perf_counter() - t0
-        rows += 1
+    while len(rows) < n_rows:
+        lp = cells[(len(rows) // w.H) % len(cells)]
+        mode = w.modes[lp * w.n_layers]
+        src = w.n_loops - 1 if mode == synth.CELL_SHARE else lp
+        bits = 4 if w.modes[src * w.n_layers] == synth.CELL_4B else 2
+        if (src, h % w.H) not in hists:
+            hists[(src, h % w.H)] = O.HeadHistory(ks[src][:, h % w.H].float().numpy(),
+                                                  vs[src][:, h % w.H].float().numpy(), bits)
+        hh = hists[(src, h % w.H)]
+        per_tok = (128.0 if bits == 4 else 96.0) * (w.D / 128.0)  # + lo bytes of hot tokens, added below
+        rows.append((qs[lp][req, h % w.H].float().numpy().astype(np.float64), hh, per_tok, bits))
         h += 1
-    gbs = rows * T * per_tok / secs / 1e9
-    return {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{rows} rows (request, head) of cell (loop 1, layer 1) at {T} tokens, decode only, "
-                      f"{secs:.1f} s single-threaded fp64; bytes counted as the GPU path's algorithmic bytes"}
+    return rows
+
+
+def _time_oracle(w, rows, threads: int):
+    """Decode the rows with the oracle on `threads` host threads (the oracle is C; its calls
+    run in parallel).  Returns (seconds, algorithmic bytes of the rows)."""
+    import numpy as np
+    from concurrent.futures import ThreadPoolExecutor
+
+    from oracle import oracle as O
+
+    empty = np.zeros((0, w.D))
+
+    def one(r):
+        q, hh, per_tok, bits = r
+        res = O.decode_row(q, hh, empty, empty, w.tau, w.tau_mode)
+        hot = int(sum(bin(int(x)).count("1") for x in res["s_bits"])) if bits == 4 else 0
+        return hh.T * per_tok + hot * (w.D / 4.0)
+
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        nbytes = sum(ex.map(one, rows))
+    return time.perf_counter() - t0, nbytes
+
+
+def cpu_baseline(w: synth.Workload, step_bytes: float, budget_s: float = 15.0):
+    """The CPU oracle's decode on the host cores, on a bounded sample of the workload's rows,
+    in the benchmark's unit; steps/s extrapolated linearly in bytes to a whole step."""
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    probe = _cpu_rows(w, cores)
+    t1, _ = _time_oracle(w, probe, cores)  # one row per thread: sizes the sample to the budget
+    n = max(cores, int(budget_s / max(t1, 1e-3)) * cores)
+    rows = _cpu_rows(w, n)
+    secs, nbytes = _time_oracle(w, rows, cores)
+    gbs = nbytes / secs / 1e9
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "extrapolated_steps_per_s": round(nbytes / secs / step_bytes, 6),
+            "sample": f"{n} rows (request 0, every head) of the layer-0 cells in loop order at {w.lengths[0] // 32 * 32} "
+                      f"tokens, decode only, fp64 oracle on {cores} host threads, {secs:.1f} s; bytes counted as "
+                      f"the GPU path's algorithmic bytes; steps/s extrapolated linearly in bytes"}
 
 
 def run_reference(args, rank, world):
     """The oracle as the reference arm: K steps of a bounded sample on the host cores."""
-    w = _workload(args)
+    w = _workload(args.config, args)
     if rank != 0:
         return None
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    rows = _cpu_rows(w, cores)
     for _ in range(args.warmup):
-        cpu_baseline(w, budget_s=0.0, rows_max=1)
-    t0 = time.perf_counter()
-    vals = [cpu_baseline(w, budget_s=0.0, rows_max=2) for _ in range(args.steps)]
-    wall = time.perf_counter() - t0
-    value = statistics.mean(v["value"] for v in vals)
+        _time_oracle(w, rows[:1], 1)
+    secs = nbytes = 0.0
+    for _ in range(args.steps):
+        t, b = _time_oracle(w, rows, cores)
+        secs += t
+        nbytes += b
+    value = nbytes / secs / 1e9
     return {
         "impl": "reference",
         "metric": METRIC,
@@ -373,15 +458,16 @@ def run_reference(args, rank, world):
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(wall / args.steps * 1e3, 2),
+        "ms_per_step": round(secs / args.steps * 1e3, 2),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded Ouro-shaped Q/K/V)",
         "config": {"workload": w.name, "context": max(w.lengths), "tau": w.tau},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": "each step: 2 rows (request, head) of cell (loop 1, layer 1), decode only"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {len(rows)} rows (request 0, every head) of the layer-0 cells, "
+                                   f"decode only, on {cores} host threads"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -391,10 +477,13 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--config", default="kivi4_8k", choices=synth.WORKLOADS[1:])
+    ap.add_argument("--config", default="long_16k", choices=synth.WORKLOADS[1:])
+    ap.add_argument("--workloads", default="kivi4_8k,mixed_8k",
+                    help="further workloads measured after the headline one and reported under 'workloads' "
+                         "(comma-separated; empty for none)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=0, help="keep only the first N layers (small profiling cases)")
     args = ap.parse_args()

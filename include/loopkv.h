@@ -125,10 +125,10 @@ typedef struct {
 
 /* ---- plan ---------------------------------------------------------------- */
 /*
- * Build a plan: one storage option per cell (LoopKV paper §3, "the planner ...
- * assigns each cell one storage option"; the offline knapsack itself is not part of
- * this library).  modes[n_loops * n_layers] is loop-major: cell (loop, layer) at
- * loop * n_layers + layer.  Cells of the final loop must be 4B or 2B; a share cell
+ * Build a plan: one storage option per cell, as the paper's offline planner produces it
+ * (LoopKV paper §3; loopkv_plan_search below is one such planner).  modes[n_loops *
+ * n_layers] is loop-major: cell (loop, layer) at loop * n_layers + layer.  Cells of the
+ * final loop must be 4B or 2B; a share cell
  * reads cell (n_loops - 1, layer).  tau >= 0; tau = 0 reads every lo plane, tau > 1
  * none.  Returns LOOPKV_ERR_PLAN / LOOPKV_ERR_INVALID_ARG / LOOPKV_ERR_SHAPE.
  */
@@ -241,9 +241,9 @@ int loopkv_append_noalloc(loopkv_cache *cache, int loop, int layer, const void *
  * Window exit: quantize every tail that holds 32 tokens into two new 16-token blocks
  * of its cell (K per channel over the 32 tokens, V per token over 32 channels, fp16
  * scale/zero, V split into hi/lo planes) and empty it; a share cell only empties its
- * tail (LoopKV paper §3.2, §3.4 "Window-exit quantization ... runs just before the
- * replay").  Blocks come from the device free list, so the call needs no host
- * round trip and can sit inside a captured graph.
+ * tail (LoopKV paper §3.2; §3.4 "Layout", where pages are quantized as they leave the
+ * window, ahead of the step's graph).  Blocks come from the device free list, so the call
+ * needs no host round trip and can sit inside a captured graph.
  */
 int loopkv_flush(loopkv_cache *cache, void *stream);
 
@@ -263,7 +263,13 @@ int loopkv_reset_request(loopkv_cache *cache, int req, void *stream);
  * the result is the same up to fp32 rounding.  A decode uses no device scratch, so
  * decodes of different cells may run on different streams.  The first call for a batch
  * size queries the device occupancy to pick the launch shape (cached in the cache
- * object); make it before capturing a stream.
+ * object); make it before capturing a stream.  Calls on one cache may come from several
+ * host threads (the host bookkeeping is locked).
+ * A decode may start while the previous kernel on its stream is finishing (programmatic
+ * dependent launch); it reads q and the tails, and writes out, only after that kernel has
+ * completed.  It reads lengths, block tables and pools earlier, so a decode that directly
+ * follows a loopkv_flush, loopkv_ingest or loopkv_reset_request on the same stream is
+ * launched without the overlap.
  */
 int loopkv_decode(const loopkv_plan *plan, int loop, int layer, const void *q,
                   const loopkv_cache *cache, float *out, int B, void *stream);
@@ -283,6 +289,23 @@ int loopkv_decode_debug(const loopkv_plan *plan, int loop, int layer, const void
  * of LOOPKV_DEV_*) and clear it.  Returns the first matching LOOPKV_ERR_* code, or
  * LOOPKV_OK when the word is zero. */
 int loopkv_status(loopkv_cache *cache, void *stream, int *device_status);
+
+/*
+ * Bounded device waits and a fault-injection hook for testing them.  Every wait of a decode
+ * kernel on data it has requested (a pipeline stage's bytes) gives up after wait_limit_ns
+ * (default 500 ms): the kernel then records LOOPKV_DEV_TIMEOUT, issues no further copies,
+ * waits (again bounded) for the copies it already issued, and returns, so the stream and
+ * the context stay usable; loopkv_status reports LOOPKV_ERR_TIMEOUT.  The outputs of a
+ * decode that timed out are meaningless.
+ * inject: LOOPKV_INJECT_NONE, or LOOPKV_INJECT_STALLED_STAGE: in later decodes one warp of
+ * the first CTA arms its first stage for bytes that it never requests, so that wait runs
+ * out (the LoopKV paper's reader gives up on a late publisher, §3.4; this makes the give-up
+ * path testable without any fault).  Applies to decodes launched after the call.
+ * Returns LOOPKV_ERR_INVALID_ARG for a zero limit or an unknown inject value.
+ */
+#define LOOPKV_INJECT_NONE 0
+#define LOOPKV_INJECT_STALLED_STAGE 1
+int loopkv_set_wait_policy(loopkv_cache *cache, uint64_t wait_limit_ns, int inject);
 
 /* Device addresses of cell (loop, layer). */
 int loopkv_cell_view_get(const loopkv_cache *cache, int loop, int layer, loopkv_cell_view *out);

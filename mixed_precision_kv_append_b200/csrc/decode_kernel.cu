@@ -130,119 +130,54 @@ __device__ __forceinline__ float warp_max_abs(float v)
 }
 
 
-// Accumulate one key word: quads `rec[0..]` hold the digits of the word's channels.
-// 4-bit word: low nibbles = quad 2w, high nibbles = quad 2w+1; 2-bit word: quad 4w+i at
-// bit 2i of every byte.
-struct KeyAcc {
-    uint32_t a0[2], a1[2];
-    int a2[2];
-};
-
-template <int BITS>
-__device__ __forceinline__ void key_word(uint32_t w, const uint4 *rec, KeyAcc &acc)
+// d += A (16 x 32, u8) * B (32 x 8, s8) with s32 accumulation: one warp-level tensor-core
+// product.  Fragments (per lane, groupID g = lane / 4, t = lane % 4): a0 = row g, k 4t..4t+3;
+// a1 = row g + 8, same k; a2 = row g, k 16 + 4t..; a3 = row g + 8, k 16 + 4t..; b0 = k 4t..4t+3
+// of column g; b1 = k 16 + 4t.. of column g; d0, d1 = row g, columns 2t, 2t + 1; d2, d3 = row
+// g + 8.  Element i of a register is its byte i.
+__device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1)
 {
-    if (BITS == 4) {
-        const uint32_t u0 = w & 0x0F0F0F0Fu, u1 = (w >> 4) & 0x0F0F0F0Fu;
-        const uint4 r0 = rec[0], r1 = rec[1];
-        dp4a_uu(acc.a0[0], u0, r0.x);
-        dp4a_uu(acc.a1[0], u0, r0.y);
-        dp4a_us(acc.a2[0], u0, r0.z);
-        dp4a_uu(acc.a0[1], u1, r1.x);
-        dp4a_uu(acc.a1[1], u1, r1.y);
-        dp4a_us(acc.a2[1], u1, r1.z);
-    } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t u = (w >> (2 * i)) & 0x03030303u;
-            const uint4 r = rec[i];
-            dp4a_uu(acc.a0[i & 1], u, r.x);
-            dp4a_uu(acc.a1[i & 1], u, r.y);
-            dp4a_us(acc.a2[i & 1], u, r.z);
-        }
-    }
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// One code word of two tokens against the same digit records.
-template <int BITS>
-__device__ __forceinline__ void key_word2(uint32_t wa, uint32_t wb, const uint4 *rec, KeyAcc &a, KeyAcc &b)
-{
-    if (BITS == 4) {
-        const uint32_t ua0 = wa & 0x0F0F0F0Fu, ua1 = (wa >> 4) & 0x0F0F0F0Fu;
-        const uint32_t ub0 = wb & 0x0F0F0F0Fu, ub1 = (wb >> 4) & 0x0F0F0F0Fu;
-        const uint4 r0 = rec[0], r1 = rec[1];
-        dp4a_uu(a.a0[0], ua0, r0.x);
-        dp4a_uu(b.a0[0], ub0, r0.x);
-        dp4a_uu(a.a1[0], ua0, r0.y);
-        dp4a_uu(b.a1[0], ub0, r0.y);
-        dp4a_us(a.a2[0], ua0, r0.z);
-        dp4a_us(b.a2[0], ub0, r0.z);
-        dp4a_uu(a.a0[1], ua1, r1.x);
-        dp4a_uu(b.a0[1], ub1, r1.x);
-        dp4a_uu(a.a1[1], ua1, r1.y);
-        dp4a_uu(b.a1[1], ub1, r1.y);
-        dp4a_us(a.a2[1], ua1, r1.z);
-        dp4a_us(b.a2[1], ub1, r1.z);
-    } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t ua = (wa >> (2 * i)) & 0x03030303u, ub = (wb >> (2 * i)) & 0x03030303u;
-            const uint4 r = rec[i];
-            dp4a_uu(a.a0[i & 1], ua, r.x);
-            dp4a_uu(b.a0[i & 1], ub, r.x);
-            dp4a_uu(a.a1[i & 1], ua, r.y);
-            dp4a_uu(b.a1[i & 1], ub, r.y);
-            dp4a_us(a.a2[i & 1], ua, r.z);
-            dp4a_us(b.a2[i & 1], ub, r.z);
-        }
-    }
-}
+// Bytes of the per-warp digit table of group_scores: 4 rows (one per digit) of D bytes, each
+// padded by 16 so that the B-fragment loads of two digit rows fall in different banks.
+template <int D> __host__ __device__ constexpr int digit_table_bytes() { return 4 * (D + 16); }
 
-// Scores (log2 units) of the 32 tokens of a group: token j of block A is token j, token j
-// of block B is token 16 + j; blkA and blkB point at the blocks' key regions (codes, then
-// the per-channel scales in block A and zeros in block B).  Returns the score of token
-// `lane`.  scr: the warp's scratch (digit records).
+// Scores (log2 units) of the 32 tokens of a group, exact up to one fp32 rounding of each
+// partial sum: token j of block A is token j, token j of block B is token 16 + j; blkA and
+// blkB point at the blocks' key regions (codes, then the per-channel scales in block A and
+// zeros in block B).  Returns the score of token `lane`.  qreg: the query of the lane's channel
+// quad as read (bf16 widens exactly); qscale = log2(e) / sqrt(D).  scr: the warp's scratch.
 //
-// The factors a_c = q_c s_c of the group are rounded to 22-bit fixed point I_c = round(a_c
-// 2^F), F = 21 - E (E = exponent of max |a|; one less when the rounding of the largest
-// could reach 2^22; capped so that 2^F and 2^-F stay normal), with one FMA against
-// 1.5 * 2^23; the low three bytes of the float become three digits (the top one re-centred
-// to a signed byte).  A lane then sums code * digit with dp4a for one channel half of one
-// token of each block, both sharing every digit-record load, and the halves are exchanged.
-// Lane L takes token t = (L & 3) | (L >> 3) << 2 and half hf = (L >> 2) & 1, and loads its
-// two 16-byte chunks in the order (t >> 1) & 1 first: the 8 lanes of a shared-memory phase
-// then touch 8 different 16-byte bank groups.  The record of channel quad q sits at
-// q + q / 8 (16 bytes each), so that the records read together do too.
+// The group's score is a dense integer contraction.  The factors a_c = q_c s_c are products of
+// an 8-bit and an 11-bit significand, exact in fp32; they are rounded to 30-bit fixed point
+// I_c = round(a_c 2^F), F = 29 - E (E = exponent of max |a|), which is exact for every channel
+// within 2^11 of the largest, and I_c is split into four signed base-256 digits (balanced:
+// I = d0 + 2^8 d1 + 2^16 d2 + 2^24 d3, each in [-128, 127]).  The codes of 32 tokens x D channels
+// times the D x 4 digit matrix is then a [32 x D] x [D x 4] integer product, which the tensor
+// cores take as m16n8k32 tiles (u8 codes, s8 digits, digits in columns 0..3 of the 8): tokens
+// are the 16 rows of a tile (one tile per block), channels the k dimension.  Since the sum runs
+// over channels in any order, each lane takes one 4-byte code word per k half as it lies in the
+// row: 4-bit codes unpack with one mask into the low nibbles (channels 8W..8W+3 of word W) and
+// one into the high nibbles (16 x channels 8W+4..8W+7, accumulated apart and divided by 16
+// exactly); 2-bit codes unpack field by field (channels 16W+4i..16W+4i+3).  The B fragment of a
+// lane is the digits of exactly the channels its A words hold, loaded from a table that the
+// factor lanes fill.  Per token, sum_c I_c code_c = P0 + 2^8 P1 + 2^16 P2 + 2^24 P3 with P_k the
+// exact int32 column sums; the pairs (P0, P1) and (P2, P3) combine exactly in int32 and meet in
+// fp32, scaled by 2^-F, with the zero term sum_c q_c z_c.
 template <int BITS, int D>
 __device__ __forceinline__ float group_scores(const uint8_t *blkA, const uint8_t *blkB, uint8_t *scr,
-                                              const float (&qreg)[4], const int lane)
+                                              const float (&qreg)[4], const float qscale, const int lane)
 {
     using G = Geo<BITS, D>;
-    constexpr int HW = G::WORDSK / 2;        // code words per channel half
-    constexpr int NCH = HW >= 4 ? HW / 4 : 1; // 16-byte chunks per half (8 bytes when HW = 2)
-    constexpr int WPC = HW >= 4 ? 4 : HW;     // words per chunk
-    constexpr int QPW = BITS == 4 ? 2 : 4;    // channel quads per code word
+    constexpr int DROW = D + 16;
     const bool ownq = lane < G::NQ;
-    const int hf = (lane >> 2) & 1, t = (lane & 3) | ((lane >> 3) << 2);
-    const int c0 = NCH == 2 ? (t >> 1) & 1 : 0;
-    const uint8_t *krA = blkA + t * G::ROWK + hf * (G::ROWK / 2);
-    const uint8_t *krB = blkB + t * G::ROWK + hf * (G::ROWK / 2);
-    uint32_t cwA[HW], cwB[HW]; // chunk by chunk in load order, loaded before the digit build
-#pragma unroll
-    for (int j = 0; j < NCH; ++j) {
-        const int c = j == 0 ? c0 : 1 - c0;
-        if (HW >= 4) {
-            const uint4 ca = *reinterpret_cast<const uint4 *>(krA + 16 * c);
-            const uint4 cb = *reinterpret_cast<const uint4 *>(krB + 16 * c);
-            cwA[4 * j] = ca.x, cwA[4 * j + 1] = ca.y, cwA[4 * j + 2] = ca.z, cwA[4 * j + 3] = ca.w;
-            cwB[4 * j] = cb.x, cwB[4 * j + 1] = cb.y, cwB[4 * j + 2] = cb.z, cwB[4 * j + 3] = cb.w;
-        } else {
-            const uint2 ca = *reinterpret_cast<const uint2 *>(krA);
-            const uint2 cb = *reinterpret_cast<const uint2 *>(krB);
-            cwA[0] = ca.x, cwA[1] = ca.y;
-            cwB[0] = cb.x, cwB[1] = cb.y;
-        }
-    }
-    // factors a_c = q_c s_c of the lane's quad and the zero term sum_c q_c z_c
+    // factors a_c = q_c s_c of the lane's quad (exact) and the zero term sum_c q_c z_c
     float av[4], zs = 0.f;
     {
         uint2 sr = make_uint2(0u, 0u), zr = make_uint2(0u, 0u);
@@ -262,49 +197,139 @@ __device__ __forceinline__ float group_scores(const uint8_t *blkA, const uint8_t
     }
     const float amax = warp_max_abs(fmaxf(fmaxf(fabsf(av[0]), fabsf(av[1])), fmaxf(fabsf(av[2]), fabsf(av[3]))));
     zs = warp_sum(zs);
-    const uint32_t ab = __float_as_uint(amax);
-    int F = 21 - ((int)(ab >> 23) - 127) - ((ab & 0x7FFFFFu) >= 0x7FFFFEu ? 1 : 0);
+    // F = 29 - E keeps |I| < 2^30 (capped so that 2^F and 2^-F stay normal)
+    int F = 29 - ((int)(__float_as_uint(amax) >> 23) - 127);
     F = F > 126 ? 126 : F;
-    const float fs = __int_as_float((F + 127) << 23), fsi = __int_as_float((127 - F) << 23);
+    const float fs = __int_as_float((F + 127) << 23);
     if (ownq) {
-        // low 23 bits of y = I + 2^22: bytes b0, b1 and b2 < 128
-        const uint32_t y0 = __float_as_uint(fmaf(av[0], fs, 12582912.f));
-        const uint32_t y1 = __float_as_uint(fmaf(av[1], fs, 12582912.f));
-        const uint32_t y2 = __float_as_uint(fmaf(av[2], fs, 12582912.f));
-        const uint32_t y3 = __float_as_uint(fmaf(av[3], fs, 12582912.f));
-        const uint32_t t01 = __byte_perm(y0, y1, 0x5140), t23 = __byte_perm(y2, y3, 0x5140);
-        const uint32_t u01 = __byte_perm(y0, y1, 0x0062), u23 = __byte_perm(y2, y3, 0x0062);
-        const uint32_t d0 = __byte_perm(t01, t23, 0x5410), d1 = __byte_perm(t01, t23, 0x7632);
-        // top digit b2 - 64 as a signed byte: flip bit 6, copy the new bit 6 into bit 7
-        const uint32_t x2 = __byte_perm(u01, u23, 0x5410) ^ 0x40404040u;
-        const uint32_t d2 = x2 | ((x2 & 0x40404040u) << 1);
-        reinterpret_cast<uint4 *>(scr)[lane + (lane >> 3)] = make_uint4(d0, d1, d2, 0u);
-    }
-    __syncwarp();
-    const uint4 *rec = reinterpret_cast<const uint4 *>(scr);
-    KeyAcc accA = {{0u, 0u}, {0u, 0u}, {0, 0}}, accB = {{0u, 0u}, {0u, 0u}, {0, 0}};
+        int I[4];
 #pragma unroll
-    for (int j = 0; j < NCH; ++j) {
-        const int c = j == 0 ? c0 : 1 - c0;
+        for (int i = 0; i < 4; ++i)
+            I[i] = __float2int_rn(av[i] * fs);
+        // byte k of I + (0x80 in each byte below k) is digit k as a signed byte
+        uint32_t *tab = reinterpret_cast<uint32_t *>(scr) + lane;
+        tab[0] = __byte_perm(__byte_perm(I[0], I[1], 0x0040), __byte_perm(I[2], I[3], 0x0040), 0x5410);
 #pragma unroll
-        for (int i = 0; i < WPC; ++i) {
-            const int q = hf * (G::NQ / 2) + QPW * (WPC * c + i); // first quad of the word (never
-            key_word2<BITS>(cwA[WPC * j + i], cwB[WPC * j + i], rec + q + (q >> 3), accA, accB); // across 8)
+        for (int k = 1; k < 4; ++k) {
+            const int off = (int)(0x808080u >> (8 * (3 - k)));
+            const uint32_t sel = (uint32_t)(((4 + k) << 4) | k);
+            tab[k * DROW / 4] = __byte_perm(__byte_perm(I[0] + off, I[1] + off, sel),
+                                            __byte_perm(I[2] + off, I[3] + off, sel), 0x5410);
         }
     }
-    // per token and half: A01 = sum of d0 terms + 256 * sum of d1 terms (< 2^30), A2 = sum of
-    // d2 terms; both exact in 32-bit integers
-    const uint32_t a01A = accA.a0[0] + accA.a0[1] + ((accA.a1[0] + accA.a1[1]) << 8);
-    const uint32_t a01B = accB.a0[0] + accB.a0[1] + ((accB.a1[0] + accB.a1[1]) << 8);
-    const int a2A = accA.a2[0] + accA.a2[1], a2B = accB.a2[0] + accB.a2[1];
-    // lane L ^ 4 holds the other half: half 0 keeps token t, half 1 token 16 + t
-    const uint32_t a01 = (hf ? a01B : a01A) + __shfl_xor_sync(0xFFFFFFFFu, hf ? a01A : a01B, 4);
-    const int a2 = (hf ? a2B : a2A) + __shfl_xor_sync(0xFFFFFFFFu, hf ? a2A : a2B, 4);
-    // sum_c code_c I_c = A01 + 65536 A2; one rounding when they are added
-    const float s = fmaf(fmaf((float)a2, 65536.f, (float)a01), fsi, zs);
-    // token L's score to lane L (held by the lane with t = L % 16, hf = L / 16)
-    return __shfl_sync(0xFFFFFFFFu, s, (lane & 3) | (((lane & 15) >> 2) << 3) | ((lane >> 4) << 2));
+    __syncwarp();
+    const int g = lane >> 2, t = lane & 3;
+    constexpr int NB = D / 16; // digit words (channel quads) of a lane's B fragment
+    uint32_t b[NB];
+    if (g < 4) {
+        const uint8_t *row = scr + g * DROW + t * (4 * NB);
+#pragma unroll
+        for (int j = 0; j < NB / 4; ++j) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(row + 16 * j);
+            b[4 * j] = v.x, b[4 * j + 1] = v.y, b[4 * j + 2] = v.z, b[4 * j + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < NB; ++j)
+            b[j] = 0u;
+    }
+    constexpr uint32_t M2 = 0x03030303u, M4 = 0x0F0F0F0Fu, H4 = 0xF0F0F0F0u;
+    float sv[2][2]; // scores of tokens g, g + 8 of each block (valid in lanes with t = 0)
+    const float k1 = qscale * __int_as_float((127 - F) << 23), zq = zs * qscale;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+        const uint8_t *rows = (mt ? blkB : blkA);
+        int c[4] = {0, 0, 0, 0};
+        if (BITS == 4) {
+            int ch[4] = {0, 0, 0, 0};
+            if (D == 128) { // words 4t..4t+3: quads 8t + 2w (low nibbles) and 8t + 2w + 1 (high)
+                const uint4 r0 = *reinterpret_cast<const uint4 *>(rows + g * G::ROWK + 16 * t);
+                const uint4 r1 = *reinterpret_cast<const uint4 *>(rows + (g + 8) * G::ROWK + 16 * t);
+                mma_u8s8(c, r0.x & M4, r1.x & M4, r0.y & M4, r1.y & M4, b[0], b[2]);
+                mma_u8s8(c, r0.z & M4, r1.z & M4, r0.w & M4, r1.w & M4, b[4], b[6]);
+                mma_u8s8(ch, r0.x & H4, r1.x & H4, r0.y & H4, r1.y & H4, b[1], b[3]);
+                mma_u8s8(ch, r0.z & H4, r1.z & H4, r0.w & H4, r1.w & H4, b[5], b[7]);
+            } else { // D = 64: words 2t, 2t+1: quads 4t, 4t+2 (low), 4t+1, 4t+3 (high)
+                const uint2 r0 = *reinterpret_cast<const uint2 *>(rows + g * G::ROWK + 8 * t);
+                const uint2 r1 = *reinterpret_cast<const uint2 *>(rows + (g + 8) * G::ROWK + 8 * t);
+                mma_u8s8(c, r0.x & M4, r1.x & M4, r0.y & M4, r1.y & M4, b[0], b[2]);
+                mma_u8s8(ch, r0.x & H4, r1.x & H4, r0.y & H4, r1.y & H4, b[1], b[3]);
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+                c[r] += ch[r] >> 4; // a multiple of 16: exact
+        } else if (D == 128) { // words 2t, 2t+1: field i is quad 8t + i, resp. 8t + 4 + i
+            const uint2 r0 = *reinterpret_cast<const uint2 *>(rows + g * G::ROWK + 8 * t);
+            const uint2 r1 = *reinterpret_cast<const uint2 *>(rows + (g + 8) * G::ROWK + 8 * t);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                mma_u8s8(c, (r0.x >> (2 * i)) & M2, (r1.x >> (2 * i)) & M2, (r0.y >> (2 * i)) & M2,
+                         (r1.y >> (2 * i)) & M2, b[i], b[4 + i]);
+        } else { // D = 64, 2-bit: word t, field i is quad 4t + i
+            const uint32_t r0 = *reinterpret_cast<const uint32_t *>(rows + g * G::ROWK + 4 * t);
+            const uint32_t r1 = *reinterpret_cast<const uint32_t *>(rows + (g + 8) * G::ROWK + 4 * t);
+#pragma unroll
+            for (int i = 0; i < 4; i += 2)
+                mma_u8s8(c, (r0 >> (2 * i)) & M2, (r1 >> (2 * i)) & M2, (r0 >> (2 * i + 2)) & M2,
+                         (r1 >> (2 * i + 2)) & M2, b[i], b[i + 1]);
+        }
+        // lane t = 0 holds digits 0, 1 of tokens g, g + 8; lane t = 1 digits 2, 3 (|P_k| < 2^18)
+        const float e0 = (float)(c[0] + (c[1] << 8)), e1 = (float)(c[2] + (c[3] << 8));
+        const float h0 = __shfl_down_sync(0xFFFFFFFFu, e0, 1), h1 = __shfl_down_sync(0xFFFFFFFFu, e1, 1);
+        sv[mt][0] = fmaf(h0, k1 * 65536.f, fmaf(e0, k1, zq));
+        sv[mt][1] = fmaf(h1, k1 * 65536.f, fmaf(e1, k1, zq));
+    }
+    // token L sits in lane 4 (L % 8): block L / 16, row half (L / 8) % 2
+    const int src = (lane & 7) << 2, j = lane >> 3;
+    const float v0 = __shfl_sync(0xFFFFFFFFu, sv[0][0], src), v1 = __shfl_sync(0xFFFFFFFFu, sv[0][1], src);
+    const float v2 = __shfl_sync(0xFFFFFFFFu, sv[1][0], src), v3 = __shfl_sync(0xFFFFFFFFu, sv[1][1], src);
+    return j == 0 ? v0 : (j == 1 ? v1 : (j == 2 ? v2 : v3));
 }
+
+// Value sums of one 32-token group for a lane's channel quad (channels 0..3 of the quad).  A
+// plane word holds 4 tokens x 4 channels (token in the byte).  E packs the codes of channels 0
+// and 2 of each token into one byte (c0 + 16 c2), O those of channels 1 and 3; dp4a of E and of
+// E with its low nibbles masked (16 c2) against a weight digit gives sum c0 d + 16 sum c2 d and
+// 16 sum c2 d, from which both sums follow exactly, so no nibble is shifted down.  Two weight
+// digits (d0, d1: the token weights' 15-bit fixed point) per word.
+struct VSums {
+    uint32_t a0[4] = {0u, 0u, 0u, 0u}, a1[4] = {0u, 0u, 0u, 0u}; // E, E & 0xF0.., O, O & 0xF0..
+
+    // 4-bit: hi word hw (2-bit fields h) and lo word lw (fields l, zero for cold tokens) give
+    // codes 4h + l; 2-bit: hw holds the codes themselves.
+    template <int BITS> __device__ __forceinline__ void add(uint32_t hw, uint32_t lw, uint32_t d0, uint32_t d1)
+    {
+        uint32_t E, O;
+        if (BITS == 4) {
+            E = ((hw << 2) & 0xCCCCCCCCu) | (lw & 0x33333333u);
+            O = (hw & 0xCCCCCCCCu) | ((lw >> 2) & 0x33333333u);
+        } else {
+            E = hw & 0x33333333u;
+            O = (hw >> 2) & 0x33333333u;
+        }
+        const uint32_t EH = E & 0xF0F0F0F0u, OH = O & 0xF0F0F0F0u;
+        dp4a_uu(a0[0], E, d0);
+        dp4a_uu(a1[0], E, d1);
+        dp4a_uu(a0[1], EH, d0);
+        dp4a_uu(a1[1], EH, d1);
+        dp4a_uu(a0[2], O, d0);
+        dp4a_uu(a1[2], O, d1);
+        dp4a_uu(a0[3], OH, d0);
+        dp4a_uu(a1[3], OH, d1);
+    }
+
+    // o[i] += (sum over tokens of code_i * weight) * fsi.  Per channel sum_t code I < 15 * 2^15 * 32
+    // < 2^24, exact in fp32; the sums of E bytes stay below 2^30.
+    __device__ __forceinline__ void finish(float fsi, float (&o)[4]) const
+    {
+        const uint32_t vE = a0[0] + (a1[0] << 8), vEH = a0[1] + (a1[1] << 8);
+        const uint32_t vO = a0[2] + (a1[2] << 8), vOH = a0[3] + (a1[3] << 8);
+        o[0] = fmaf((float)(vE - vEH), fsi, o[0]);
+        o[1] = fmaf((float)(vO - vOH), fsi, o[1]);
+        o[2] = fmaf((float)(vEH >> 4), fsi, o[2]);
+        o[3] = fmaf((float)(vOH >> 4), fsi, o[3]);
+    }
+};
 
 struct Smem {
     uint8_t *ring;     // [kWarps][spw][STAGE] stage slots (kGPS groups each), a private slice per warp
@@ -340,7 +365,7 @@ __host__ __device__ constexpr int imax(int a, int b) { return a > b ? a : b; }
 // Bytes of a warp's scratch: the largest of its three uses.
 template <int D> __host__ __device__ constexpr int scratch_bytes()
 {
-    return align16(imax((D / 4 + D / 32) * 16, imax((D + 2) * 4, (D / 32) * 40 * 4 + 4)));
+    return align16(imax(digit_table_bytes<D>(), imax((D + 2) * 4, (D / 32) * 40 * 4 + 4)));
 }
 
 // nbuf: score buffers (2: the next row's keys are scored while the current row's values are
@@ -407,7 +432,7 @@ template <int BITS, int D> bool layout_ok(int spw, int capw, int nbuf)
         prev = o;
     }
     return (Geo<BITS, D>::GSLOT % 128) == 0 && L.total >= prev && (spw & (spw - 1)) == 0 &&
-           scratch_bytes<D>() >= (D / 4 + D / 32) * 16 && scratch_bytes<D>() >= (D + 1) * 4 &&
+           scratch_bytes<D>() >= digit_table_bytes<D>() && scratch_bytes<D>() >= (D + 1) * 4 &&
            scratch_bytes<D>() >= (D / 32) * 40 * 4 + 4 && (2 * capw * 4) % 8 == 0;
 }
 
@@ -541,20 +566,23 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     const uint8_t *seg_lo = nullptr;  // lo pool + head offset of the segment's row
     const int2 *seg_ids = nullptr;
     int setup_upto = -1;           // rows 0..setup_upto have their parameters and ids in place
+    // After one bounded wait gives up, later waits are skipped, nothing new is issued, and the
+    // stages from drain_from on are waited for (bounded) before the CTA exits.
+    bool timed_out = false;
+    int drain_from = 0;
 
     // Row parameters, validation and the warp's block ids of row ri.
     auto setup_row = [&](int ri) {
         const int row = row_of(ri);
         const int b = row / a.H, h = row - b * a.H;
-        int hist = a.hist_len[b], tail = a.tail_len[b];
+        // history length and block ids come from flush / ingest / reset launches, which the
+        // host never overlaps with a decode; the tail length (appends) is read after the grid
+        // dependency wait (read_tail)
+        int hist = a.hist_len[b];
         bool bad = false;
         if (hist < 0 || hist > a.max_blocks * 16 || (hist & 31)) {
             bad = true;
             hist = 0;
-        }
-        if (tail < 0 || tail > 32) {
-            bad = true;
-            tail = 0;
         }
         const int ngroups = hist >> 5;
         int nmy = ngroups > (int)crank ? (ngroups - (int)crank + (int)C - 1) / (int)C : 0;
@@ -582,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             st[IR_B] = b;
             st[IR_H] = h;
             st[IR_N] = n;
-            st[IR_TAIL] = (crank == C - 1) ? tail : 0;
+            st[IR_TAIL] = (crank == C - 1 && warp == kWarps - 1) ? -1 : 0; // -1: tail owner, length not read
             st[IR_VFIRST] = 0;
             st[IR_VISSUED] = 0;
             st[IR_THR] = __float_as_int(NAN);
@@ -603,6 +631,12 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     // tokens per word, so a 4-token quad with a hot token is copied whole (D bytes); a
     // group whose 32 tokens are all hot copies both blocks' planes.
     auto issue_lo = [&](int ri, int k2, int n, float thr2) {
+        if (timed_out) { // no new copies after a give-up; the arrival keeps the stage's phase complete
+            if (lane == 0)
+                mbar_arrive(&full[n & smask]);
+            __syncwarp();
+            return;
+        }
         const int32_t *st_row = irow_of(ri);
         const int ng = min(kGPS, st_row[IR_N] - kGPS * k2);
         uint8_t *stg = ring + (n & smask) * G::STAGE + 2 * G::VB;
@@ -657,6 +691,8 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         if (!seg_v) {
             if (lane == 0) {
                 mbar_arrive_expect_tx(fb, (uint32_t)ng * 2 * G::KB);
+                if (a.inject == LOOPKV_INJECT_STALLED_STAGE && n == 0 && warp == 0 && blockIdx.x == 0)
+                    return; // test hook: the stage's bytes never arrive, so its wait runs out
                 for (int j = 0; j < ng; ++j) {
                     const int2 id = ids[j];
                     bulk_g2s(stg + j * G::GSLOT, seg_src + (uint64_t)(uint32_t)id.x * bstride, G::KB, fb);
@@ -702,6 +738,8 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     // of a row waits until the row is set up (the compute side sets up row r + 1 when it
     // starts scoring row r, see consume_k).
     auto pump = [&](int limit) {
+        if (timed_out)
+            return; // after a give-up nothing new is issued
         for (;;) {
             if (iss_k < seg_len) {
                 if (iss_n >= limit)
@@ -742,10 +780,11 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     constexpr int SCR = scratch_bytes<D>();
     uint8_t *scr = sm.scr + warp * SCR;
     int prc_n = 0;
-    bool timed_out = false; // after one bounded wait gives up, later waits are skipped
     auto wait_stage = [&](int n) {
-        if (!timed_out)
-            timed_out = !mbar_wait(&full[n & smask], (n >> spw_log2) & 1, a.status);
+        if (!timed_out && !mbar_wait(&full[n & smask], (n >> spw_log2) & 1, a.status, a.wait_ns)) {
+            timed_out = true;
+            drain_from = n;
+        }
     };
 
     // K pass of the warp's groups of row ri; per-warp (max, sum) into stat.
@@ -757,16 +796,29 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             setup_row(r);
             setup_upto = r;
         }
-        const int32_t *srow = irow_of(ri);
-        const int row = srow[IR_ROW], nown = srow[IR_N], tail = srow[IR_TAIL];
+        int32_t *srow = irow_of(ri);
+        const int row = srow[IR_ROW], nown = srow[IR_N];
         float *sc = scores_of(ri);
         if (ri == 0) {
-            // Prefetch the first stages (pools, block tables and lengths come from earlier
-            // flush / append / ingest launches, which let dependents start only when they
-            // complete), then wait for the previous grid of the stream: q, and the outputs
-            // this grid writes, may be shared with it.
+            // Prefetch the first stages, then wait for the previous grid of the stream: it may
+            // have written q or the tails (an append), and it may read the outputs this grid
+            // writes.  Lengths, block tables and pools were written by flush / ingest / reset
+            // launches that the host does not let a decode overlap.
             pump(prc_n + spw);
             asm volatile("griddepcontrol.wait;" ::: "memory");
+        }
+        int tail = srow[IR_TAIL];
+        if (tail < 0) { // the tail owner reads the tail length
+            tail = a.tail_len[srow[IR_B]];
+            if (tail < 0 || tail > 32) {
+                if (lane == 0)
+                    atomicOr(a.status, LOOPKV_DEV_STATE);
+                tail = 0;
+            }
+            __syncwarp();
+            if (lane == 0)
+                srow[IR_TAIL] = tail;
+            __syncwarp();
         }
         // lane owns the channel quad 4*lane .. 4*lane+3 (lanes >= D/4 own none)
         const bool ownq = lane < G::NQ;
@@ -775,7 +827,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             const DT *qrow = reinterpret_cast<const DT *>(a.q) + (int64_t)row * D + 4 * lane;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                qreg[i] = ownq ? to_f32(qrow[i]) * a.qscale : 0.f;
+                qreg[i] = ownq ? to_f32(qrow[i]) : 0.f;
         }
         float mx = -INFINITY;
         const uint8_t *stg = ring;
@@ -788,7 +840,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
                 stg = ring + (n & smask) * G::STAGE;
             }
             const uint8_t *st = stg + (k % kGPS) * G::GSLOT;
-            const float s2 = group_scores<BITS, D>(st, st + G::KB, scr, qreg, lane);
+            const float s2 = group_scores<BITS, D>(st, st + G::KB, scr, qreg, a.qscale, lane);
             sc[k * 32 + lane] = s2;
             mx = fmaxf(mx, s2);
             __syncwarp();
@@ -808,6 +860,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
                 for (int i = 0; i < 4; ++i)
                     s2 = fmaf(__shfl_sync(0xFFFFFFFFu, qreg[i], q4), kv[i], s2);
             }
+            s2 *= a.qscale;
             if (lane < tail) {
                 tsc[lane] = s2;
                 mx = fmaxf(mx, s2);
@@ -918,25 +971,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             }
             __syncwarp();
             // ---- accumulate: channel quad vk, dp4a over the tokens of each token quad
-            uint32_t a0[4] = {0u, 0u, 0u, 0u}, a1[4] = {0u, 0u, 0u, 0u};
-            // codes of channel 4vk+i of the quad's 4 tokens, one per byte, into the sums
-            auto acc_quad = [&](const uint32_t (&c4)[4], const uint4 &rc) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    dp4a_uu(a0[i], c4[i], rc.x);
-                    dp4a_uu(a1[i], c4[i], rc.y);
-                }
-            };
-            // 4-bit codes 4h + l from a hi and a lo word: nibble 0 of each byte is channel 0
-            // (E) or 1 (O), nibble 1 channel 2 (E) or 3 (O)
-            auto merged = [](uint32_t hw, uint32_t lw, uint32_t (&c4)[4]) {
-                const uint32_t E = ((hw << 2) & 0xCCCCCCCCu) | (lw & 0x33333333u);
-                const uint32_t O = (hw & 0xCCCCCCCCu) | ((lw >> 2) & 0x33333333u);
-                c4[0] = E & 0x0F0F0F0Fu;
-                c4[1] = O & 0x0F0F0F0Fu;
-                c4[2] = (E >> 4) & 0x0F0F0F0Fu;
-                c4[3] = (O >> 4) & 0x0F0F0F0Fu;
-            };
+            VSums acc;
 #pragma unroll
             for (int bb = 0; bb < BPL; ++bb) {
                 const int blk = vb0 + bb;
@@ -944,37 +979,19 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
                 const uint32_t hwv[4] = {h4.x, h4.y, h4.z, h4.w};
                 const uint8_t *lop = st + 2 * G::VB + blk * G::LOB + 4 * vk;
                 const uint4 *rq = reinterpret_cast<const uint4 *>(ybuf + vg * YS) + 4 * blk;
-                if (BITS == 2) { // own 2-bit codes: channel i of every byte at bit 2i
 #pragma unroll
-                    for (int tau = 0; tau < 4; ++tau) {
-                        const uint32_t hw = hwv[tau];
-                        const uint32_t c4[4] = {hw & 0x03030303u, (hw >> 2) & 0x03030303u, (hw >> 4) & 0x03030303u,
-                                                (hw >> 6) & 0x03030303u};
-                        acc_quad(c4, rq[tau]);
+                for (int tau = 0; tau < 4; ++tau) {
+                    const uint4 rc = rq[tau];
+                    uint32_t lw = 0u;
+                    if (BITS == 4) { // lo words exist for quads with a hot token; keep the hot tokens' bits
+                        lw = *reinterpret_cast<const uint32_t *>(lop + tau * D);
+                        if (!all_hot)
+                            lw &= rc.z;
                     }
-                } else if (all_hot) { // every lo word was copied
-#pragma unroll
-                    for (int tau = 0; tau < 4; ++tau) {
-                        uint32_t c4[4];
-                        merged(hwv[tau], *reinterpret_cast<const uint32_t *>(lop + tau * D), c4);
-                        acc_quad(c4, rq[tau]);
-                    }
-                } else { // lo words exist for quads with a hot token; keep the hot tokens' bits
-#pragma unroll
-                    for (int tau = 0; tau < 4; ++tau) {
-                        const uint4 rc = rq[tau];
-                        const uint32_t lw = rc.z ? *reinterpret_cast<const uint32_t *>(lop + tau * D) & rc.z : 0u;
-                        uint32_t c4[4];
-                        merged(hwv[tau], lw, c4);
-                        acc_quad(c4, rc);
-                    }
+                    acc.add<BITS>(hwv[tau], lw, rc.x, rc.y);
                 }
             }
-            // sum_t code * I <= 15 * 2^15 * 32 < 2^24: exact in 32 bits and in fp32
-            const float fsi = *fsit;
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                facc[i] = fmaf((float)(a0[i] + (a1[i] << 8)), fsi, facc[i]);
+            acc.finish(*fsit, facc);
             __syncwarp();
         }
         // zero terms: lane ends with the warp's sum of zl[lane % NCG] (reduce-scatter over
@@ -1104,6 +1121,9 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         if (nrows > 0)
             merge(nrows - 1, m_prev);
     }
+    if (timed_out) // copies issued before the give-up must land before the shared memory is freed
+        for (int n = drain_from; n < iss_n; ++n)
+            mbar_wait(&full[n & smask], (n >> spw_log2) & 1, a.status, a.wait_ns);
     cluster_arrive(); // remote reads done
     cluster_wait();
 }
@@ -1199,7 +1219,7 @@ template <int D> __device__ __forceinline__ void run1_init(Run1<D> &r)
 // (4-bit source) or plain 2-bit codes.  scr: the warp's scratch.
 template <int BITS, int D>
 __device__ __forceinline__ void run1_group(const uint8_t *st, const uint8_t *lo, uint8_t *scr, const float (&qreg)[4],
-                                           const int lane, Run1<D> &r)
+                                           const float qscale, const int lane, Run1<D> &r)
 {
     using G = Geo<BITS, D>;
     constexpr int NCG = G::NCG;
@@ -1211,7 +1231,7 @@ __device__ __forceinline__ void run1_group(const uint8_t *st, const uint8_t *lo,
     const int vb0 = G::NQ == 32 ? 0 : lane / G::NQ;
     uint32_t *ybuf = reinterpret_cast<uint32_t *>(scr);
     float *fsit = reinterpret_cast<float *>(ybuf + NCG * YS);
-    const float s2l = group_scores<BITS, D>(st, st + G::HM, scr, qreg, lane); // score of token `lane`
+    const float s2l = group_scores<BITS, D>(st, st + G::HM, scr, qreg, qscale, lane); // score of token `lane`
     // ---- running maximum (warp-uniform): rescale the warp's sums when it grows
     const float mg = warp_max_f(s2l);
     if (mg > r.m) {
@@ -1259,7 +1279,7 @@ __device__ __forceinline__ void run1_group(const uint8_t *st, const uint8_t *lo,
             make_uint2(__byte_perm(t01, t23, 0x5410), __byte_perm(t01, t23, 0x7632));
     }
     __syncwarp();
-    uint32_t a0[4] = {0u, 0u, 0u, 0u}, a1[4] = {0u, 0u, 0u, 0u};
+    VSums acc;
 #pragma unroll
     for (int bb = 0; bb < BPL; ++bb) {
         const int blk = vb0 + bb;
@@ -1270,33 +1290,11 @@ __device__ __forceinline__ void run1_group(const uint8_t *st, const uint8_t *lo,
 #pragma unroll
         for (int tau = 0; tau < 4; ++tau) {
             const uint2 rc = *reinterpret_cast<const uint2 *>(rq + 4 * tau);
-            const uint32_t hw = hwv[tau];
-            uint32_t c4[4];
-            if (BITS == 2) { // own 2-bit codes: channel i of every byte at bit 2i
-                c4[0] = hw & 0x03030303u;
-                c4[1] = (hw >> 2) & 0x03030303u;
-                c4[2] = (hw >> 4) & 0x03030303u;
-                c4[3] = (hw >> 6) & 0x03030303u;
-            } else { // 4h + l
-                const uint32_t lw = *reinterpret_cast<const uint32_t *>(lop + tau * D);
-                const uint32_t E = ((hw << 2) & 0xCCCCCCCCu) | (lw & 0x33333333u);
-                const uint32_t O = (hw & 0xCCCCCCCCu) | ((lw >> 2) & 0x33333333u);
-                c4[0] = E & 0x0F0F0F0Fu;
-                c4[1] = O & 0x0F0F0F0Fu;
-                c4[2] = (E >> 4) & 0x0F0F0F0Fu;
-                c4[3] = (O >> 4) & 0x0F0F0F0Fu;
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                dp4a_uu(a0[i], c4[i], rc.x);
-                dp4a_uu(a1[i], c4[i], rc.y);
-            }
+            const uint32_t lw = BITS == 4 ? *reinterpret_cast<const uint32_t *>(lop + tau * D) : 0u;
+            acc.add<BITS>(hwv[tau], lw, rc.x, rc.y);
         }
     }
-    const float fsi = *fsit;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        r.o[i] = fmaf((float)(a0[i] + (a1[i] << 8)), fsi, r.o[i]); // sum <= 15 * 2^15 * 32 < 2^24: exact
+    acc.finish(*fsit, r.o);
     __syncwarp();
 }
 
@@ -1342,8 +1340,8 @@ template <int BITS, int D> __device__ __forceinline__ void run1_finish(Run1<D> &
 // Tail tokens t < tail (exact; lane = tail token) folded into the warp's partial red:
 // keys kt [32][D] and values vt0 [32][D]; rescales red when a tail score raises r.m.
 template <int D, typename DT>
-__device__ __forceinline__ void run1_tail(Run1<D> &r, float *red, const int lane, const float (&qreg)[4], const DT *kt,
-                                          const DT *vt0, const int tail)
+__device__ __forceinline__ void run1_tail(Run1<D> &r, float *red, const int lane, const float (&qreg)[4],
+                                          const float qscale, const DT *kt, const DT *vt0, const int tail)
 {
     constexpr int NQ = D / 4;
     float s2 = 0.f;
@@ -1357,6 +1355,7 @@ __device__ __forceinline__ void run1_tail(Run1<D> &r, float *red, const int lane
         for (int i = 0; i < 4; ++i)
             s2 = fmaf(__shfl_sync(0xFFFFFFFFu, qreg[i], q4), kv[i], s2);
     }
+    s2 *= qscale;
     const float mt = warp_max_f(lane < tail ? s2 : -INFINITY);
     if (mt > r.m) { // rescale the warp's partial in the scratch
         const float f = ex2(r.m - mt);
@@ -1444,19 +1443,17 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
     // ---------------------------------------------------------------- issuing
     int iss_n = 0, iss_row = -1, iss_k = 0, seg_n = 0, setup_upto = -1;
     const uint8_t *seg_src = nullptr, *seg_lo = nullptr;
+    bool timed_out = false; // as in decode_kernel: no waits or copies after a give-up, then a drain
+    int drain_from = 0;
     // row parameters, validation and the warp's block ids of row ri (as in decode_kernel)
     auto setup_row = [&](int ri) {
         const int row = row_of(ri);
         const int b = row / a.H, h = row - b * a.H;
-        int hist = a.hist_len[b], tail = a.tail_len[b];
+        int hist = a.hist_len[b]; // the tail length is read after the grid dependency wait
         bool bad = false;
         if (hist < 0 || hist > a.max_blocks * 16 || (hist & 31)) {
             bad = true;
             hist = 0;
-        }
-        if (tail < 0 || tail > 32) {
-            bad = true;
-            tail = 0;
         }
         const int ngroups = hist >> 5;
         int nmy = ngroups > (int)crank ? (ngroups - (int)crank + (int)C - 1) / (int)C : 0;
@@ -1482,7 +1479,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
             irow[IR_B] = b;
             irow[IR_H] = h;
             irow[IR_N] = n;
-            irow[IR_TAIL] = (crank == C - 1) ? tail : 0;
+            irow[IR_TAIL] = (crank == C - 1 && warp == kWarps - 1) ? -1 : 0; // -1: tail owner
         }
         __syncwarp();
         setup_upto = ri;
@@ -1494,6 +1491,8 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
         uint64_t *fb = &full[n & smask];
         if (lane == 0) {
             mbar_arrive_expect_tx(fb, 2 * G::HM + 2 * G::LOB);
+            if (a.inject == LOOPKV_INJECT_STALLED_STAGE && n == 0 && warp == 0 && blockIdx.x == 0)
+                return; // test hook: the stage's bytes never arrive, so its wait runs out
             bulk_g2s(st, seg_src + (uint64_t)(uint32_t)id.x * bstride, G::HM, fb);
             bulk_g2s(st + G::HM, seg_src + (uint64_t)(uint32_t)id.y * bstride, G::HM, fb);
             if (BITS == 4) {
@@ -1504,6 +1503,8 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
     };
     // issue every stage numbered below `limit`; a row's stages follow once it is set up
     auto pump = [&](int limit) {
+        if (timed_out)
+            return;
         for (;;) {
             if (iss_k < seg_n) {
                 if (iss_n >= limit)
@@ -1527,10 +1528,11 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
 
     // ---------------------------------------------------------------- compute
     int prc_n = 0;
-    bool timed_out = false;
     auto wait_stage = [&](int n) {
-        if (!timed_out)
-            timed_out = !mbar_wait(&full[n & smask], (n >> spw_log2) & 1, a.status);
+        if (!timed_out && !mbar_wait(&full[n & smask], (n >> spw_log2) & 1, a.status, a.wait_ns)) {
+            timed_out = true;
+            drain_from = n;
+        }
     };
     const bool ownq = lane < G::NQ;
 
@@ -1539,7 +1541,8 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
     auto row_pass = [&](int ri) {
         if (ri == 0)
             setup_row(0);
-        const int row = irow[IR_ROW], nown = irow[IR_N], tail = irow[IR_TAIL], rb = irow[IR_B], rh = irow[IR_H];
+        const int row = irow[IR_ROW], nown = irow[IR_N], rb = irow[IR_B], rh = irow[IR_H];
+        int tail = irow[IR_TAIL];
         // the slot takes row ri + 1 once row ri's stages are all issued (after the pump of
         // group nown - spw, or at once when the warp has no group)
         const int k_setup = nown > spw ? nown - spw : 0;
@@ -1549,12 +1552,20 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
             pump(prc_n + spw);
             asm volatile("griddepcontrol.wait;" ::: "memory");
         }
+        if (tail < 0) { // the tail owner reads the tail length (an append may have written it)
+            tail = a.tail_len[rb];
+            if (tail < 0 || tail > 32) {
+                if (lane == 0)
+                    atomicOr(a.status, LOOPKV_DEV_STATE);
+                tail = 0;
+            }
+        }
         float qreg[4];
         {
             const DT *qrow = reinterpret_cast<const DT *>(a.q) + (int64_t)row * D + 4 * lane;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                qreg[i] = ownq ? to_f32(qrow[i]) * a.qscale : 0.f;
+                qreg[i] = ownq ? to_f32(qrow[i]) : 0.f;
         }
         Run1<D> run;
         run1_init(run);
@@ -1568,7 +1579,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
             }
             wait_stage(n);
             const uint8_t *st = ring + (n & smask) * G1::STAGE;
-            run1_group<BITS, D>(st, st + G1::LOFF, scr, qreg, lane, run);
+            run1_group<BITS, D>(st, st + G1::LOFF, scr, qreg, a.qscale, lane, run);
             if (a.s_bitmap && lane == 0) // refine set: every token (4-bit, tau <= 0) or none (2-bit)
                 a.s_bitmap[(int64_t)row * a.bitmap_words + (int)crank + (warp + k * kWarps) * (int)C] =
                     BITS == 4 ? 0xFFFFFFFFu : 0u;
@@ -1578,7 +1589,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
         if (tail > 0 && warp == kWarps - 1) {
             const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)rb * 2 * a.H + rh) * 32 * D;
             const DT *vt0 = reinterpret_cast<const DT *>(a.tail) + ((int64_t)(rb * 2 + 1) * a.H + rh) * 32 * D;
-            run1_tail<D, DT>(run, red, lane, qreg, kt, vt0, tail);
+            run1_tail<D, DT>(run, red, lane, qreg, a.qscale, kt, vt0, tail);
         }
         if (lane == 0)
             red[D + 1] = run.m;
@@ -1662,6 +1673,9 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
             cluster_arrive();       // barrier i
         }
     }
+    if (timed_out) // copies issued before the give-up must land before the shared memory is freed
+        for (int n = drain_from; n < iss_n; ++n)
+            mbar_wait(&full[n & smask], (n >> spw_log2) & 1, a.status, a.wait_ns);
     cluster_arrive(); // the remote reads of the last merge are done
     cluster_wait();
 }
@@ -1669,7 +1683,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
 // Launch `kern` with the shape's grid, cluster and shared memory (and programmatic
 // stream serialization when the shape asks for it).
 template <typename K, typename... Args>
-int launch_shape(K kern, const DecodeShape &shp, cudaStream_t s, Args... args)
+int launch_shape(K kern, const DecodeShape &shp, bool pdl, cudaStream_t s, Args... args)
 {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, shp.smem);
     if (e == cudaSuccess)
@@ -1691,18 +1705,18 @@ int launch_shape(K kern, const DecodeShape &shp, cudaStream_t s, Args... args)
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization; // see griddepcontrol in the kernels
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = shp.pdl ? 2 : 1;
+    cfg.numAttrs = (shp.pdl && pdl) ? 2 : 1;
     e = cudaLaunchKernelEx(&cfg, kern, args...);
     return e == cudaSuccess ? LOOPKV_OK : LOOPKV_ERR_CUDA;
 }
 
 template <int BITS, int D, typename DT>
-int launch_t(const DecodeArgs &a, const DecodeShape &shp, cudaStream_t s)
+int launch_t(const DecodeArgs &a, const DecodeShape &shp, bool pdl, cudaStream_t s)
 {
     if (shp.onepass)
-        return launch_shape(decode_kernel_1p<BITS, D, DT, 4>, shp, s, a, shp.stages_log2);
+        return launch_shape(decode_kernel_1p<BITS, D, DT, 4>, shp, pdl, s, a, shp.stages_log2);
     auto kern = shp.min_ctas == 5 ? decode_kernel<BITS, D, DT, 5> : decode_kernel<BITS, D, DT, 4>;
-    return launch_shape(kern, shp, s, a, shp.stages_log2, shp.score_bufs);
+    return launch_shape(kern, shp, pdl, s, a, shp.stages_log2, shp.score_bufs);
 }
 
 // Clusters of size C that can be resident at once for this kernel and shared memory.
@@ -1852,19 +1866,19 @@ DecodeShape decode_shape(int bits, int D, int dtype, int rows, int max_blocks, b
     return bf ? shape_t<2, 64, __nv_bfloat16>(rows, mb, onepass) : shape_t<2, 64, float>(rows, mb, onepass);
 }
 
-int launch_decode(const DecodeArgs &a, int bits, int D, int dtype, const DecodeShape &shp, cudaStream_t s)
+int launch_decode(const DecodeArgs &a, int bits, int D, int dtype, const DecodeShape &shp, bool pdl, cudaStream_t s)
 {
     if (shp.cluster <= 0 || shp.clusters <= 0)
         return LOOPKV_ERR_CUDA;
     const bool bf = dtype == LOOPKV_DTYPE_BF16;
     if (bits == 4) {
         if (D == 128)
-            return bf ? launch_t<4, 128, __nv_bfloat16>(a, shp, s) : launch_t<4, 128, float>(a, shp, s);
-        return bf ? launch_t<4, 64, __nv_bfloat16>(a, shp, s) : launch_t<4, 64, float>(a, shp, s);
+            return bf ? launch_t<4, 128, __nv_bfloat16>(a, shp, pdl, s) : launch_t<4, 128, float>(a, shp, pdl, s);
+        return bf ? launch_t<4, 64, __nv_bfloat16>(a, shp, pdl, s) : launch_t<4, 64, float>(a, shp, pdl, s);
     }
     if (D == 128)
-        return bf ? launch_t<2, 128, __nv_bfloat16>(a, shp, s) : launch_t<2, 128, float>(a, shp, s);
-    return bf ? launch_t<2, 64, __nv_bfloat16>(a, shp, s) : launch_t<2, 64, float>(a, shp, s);
+        return bf ? launch_t<2, 128, __nv_bfloat16>(a, shp, pdl, s) : launch_t<2, 128, float>(a, shp, pdl, s);
+    return bf ? launch_t<2, 64, __nv_bfloat16>(a, shp, pdl, s) : launch_t<2, 64, float>(a, shp, pdl, s);
 }
 
 }  // namespace lkv

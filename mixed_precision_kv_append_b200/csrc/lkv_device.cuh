@@ -10,10 +10,11 @@
 
 namespace lkv {
 
-// Bounded waits: a wait that has not completed after this many nanoseconds records
-// LOOPKV_DEV_TIMEOUT and lets the thread go on, so that every thread still reaches
-// the cluster barriers and the kernel ends.
-constexpr unsigned long long kWaitLimitNs = 500ull * 1000ull * 1000ull;
+// Bounded waits: a wait that has not completed after its limit (a launch argument,
+// 500 ms unless the cache's wait policy says otherwise) records LOOPKV_DEV_TIMEOUT and
+// lets the thread go on, so that every thread still reaches the cluster barriers and the
+// kernel ends.
+constexpr unsigned long long kDefaultWaitNs = 500ull * 1000ull * 1000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
@@ -72,8 +73,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity, ui
     return ok != 0;
 }
 
-// Wait for phase `parity` of an mbarrier, giving up after kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *status)
+// Wait for phase `parity` of an mbarrier, giving up after limit_ns nanoseconds.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *status,
+                                          unsigned long long limit_ns)
 {
     if (mbar_try_wait(bar, parity))
         return true;
@@ -81,7 +83,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity))
             return true;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > limit_ns) {
             atomicOr(status, LOOPKV_DEV_TIMEOUT);
             return false;
         }

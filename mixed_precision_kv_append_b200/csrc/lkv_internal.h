@@ -51,6 +51,8 @@ struct DecodeArgs {
     float qscale;               // log2(e) / sqrt(D)
     float tau;
     int tau_mode;
+    unsigned long long wait_ns; // limit of every bounded wait, in nanoseconds
+    int inject;                 // LOOPKV_INJECT_*: LOOPKV_INJECT_NONE in normal operation
 };
 
 struct DecodeShape {
@@ -68,7 +70,11 @@ struct DecodeShape {
 };
 
 // Launchers (defined in the .cu files).  Return LOOPKV_OK or an error code.
-int launch_decode(const DecodeArgs &a, int bits, int D, int dtype, const DecodeShape &shp, cudaStream_t s);
+// pdl: launch with programmatic stream serialization (see launch_shape in decode_kernel.cu); the
+// caller passes false when the previous launch on the stream may have written lengths, block
+// tables or pools, which the kernel reads before its grid dependency wait.
+int launch_decode(const DecodeArgs &a, int bits, int D, int dtype, const DecodeShape &shp, bool pdl,
+                  cudaStream_t s);
 // onepass: the rows' refine set does not depend on the row maximum (2-bit source, or a
 // 4-bit source read with tau <= 0), so the single-pass kernel may read them.
 DecodeShape decode_shape(int bits, int D, int dtype, int rows, int max_blocks, bool onepass);

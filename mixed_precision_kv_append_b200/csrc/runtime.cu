@@ -7,10 +7,12 @@
 #include <cstdlib>
 #include <cstring>
 #include <map>
+#include <mutex>
 #include <new>
 #include <tuple>
 #include <vector>
 
+#include "lkv_device.cuh"
 #include "lkv_internal.h"
 
 struct loopkv_plan {
@@ -29,11 +31,36 @@ struct loopkv_plan {
 
 struct loopkv_cache {
     loopkv_plan plan;
-    // decode launch shapes by (storage bits, batch, single-pass), computed once (occupancy
-    // queries must not run while a stream is being captured)
+    // Host bookkeeping shared by calls from several host threads, under `mu`:
+    //   shapes: decode launch shapes by (storage bits, batch, single-pass), computed once
+    //           (occupancy queries must not run while a stream is being captured);
+    //   state_written: per stream, whether the last call of this library on it launched a
+    //           kernel that writes lengths, block tables or pools (flush, ingest, reset).  A
+    //           decode reads those before its grid dependency wait, so a decode right after
+    //           such a launch does not overlap it (no programmatic dependent launch).
+    std::mutex mu;
     std::map<std::tuple<int, int, bool>, lkv::DecodeShape> shapes;
-    const lkv::DecodeShape &shape(int bits, int B, bool onepass)
+    std::map<void *, bool> state_written;
+    unsigned long long wait_ns = lkv::kDefaultWaitNs;
+    int inject = LOOPKV_INJECT_NONE;
+    void mark_state_written(void *stream)
     {
+        std::lock_guard<std::mutex> lock(mu);
+        state_written[stream] = true;
+    }
+    // Whether a decode on `stream` may overlap the previous launch; clears the mark.
+    bool decode_may_overlap(void *stream)
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = state_written.find(stream);
+        const bool written = it != state_written.end() && it->second;
+        if (written)
+            it->second = false;
+        return !written;
+    }
+    lkv::DecodeShape shape(int bits, int B, bool onepass)
+    {
+        std::lock_guard<std::mutex> lock(mu);
         auto key = std::make_tuple(bits, B, onepass);
         auto it = shapes.find(key);
         if (it == shapes.end())
@@ -395,6 +422,7 @@ int loopkv_ingest(loopkv_cache *cache, int loop, int layer, int req, const void 
     if (T / LKV_GROUP * 2 > p.cfg.max_blocks_per_seq)
         return LOOPKV_ERR_SHAPE;
     const int cell = p.cell(loop, layer);
+    cache->mark_state_written(stream);
     return lkv::launch_ingest(cache->st, cell, p.modes[cell], p.cfg.n_heads, p.cfg.head_dim, p.cfg.in_dtype,
                               p.cfg.max_batch, p.cfg.max_blocks_per_seq, req, k, v, T,
                               static_cast<cudaStream_t>(stream));
@@ -431,6 +459,7 @@ int loopkv_flush(loopkv_cache *cache, void *stream)
     if (!cache)
         return LOOPKV_ERR_INVALID_ARG;
     const loopkv_plan &p = cache->plan;
+    cache->mark_state_written(stream);
     return lkv::launch_flush(cache->st, cache->modes_dev, p.n_cells(), p.cfg.n_heads, p.cfg.head_dim, p.cfg.in_dtype,
                              p.cfg.max_batch, p.cfg.max_blocks_per_seq, static_cast<cudaStream_t>(stream));
 }
@@ -442,6 +471,7 @@ int loopkv_reset_request(loopkv_cache *cache, int req, void *stream)
     const loopkv_plan &p = cache->plan;
     if (req < 0 || req >= p.cfg.max_batch)
         return LOOPKV_ERR_INVALID_ARG;
+    cache->mark_state_written(stream);
     return lkv::launch_reset(cache->st, cache->modes_dev, p.n_cells(), p.cfg.max_batch, p.cfg.max_blocks_per_seq, req,
                              static_cast<cudaStream_t>(stream));
 }
@@ -451,7 +481,7 @@ int loopkv_decode_debug(const loopkv_plan *plan, int loop, int layer, const void
 {
     if (!plan || !ccache || !q || !out)
         return LOOPKV_ERR_INVALID_ARG;
-    loopkv_cache *cache = const_cast<loopkv_cache *>(ccache); // only the launch-shape memo changes
+    loopkv_cache *cache = const_cast<loopkv_cache *>(ccache); // only the host bookkeeping changes
     int rc = check_cell(plan, loop, layer);
     if (rc)
         return rc;
@@ -486,9 +516,15 @@ int loopkv_decode_debug(const loopkv_plan *plan, int loop, int layer, const void
     a.qscale = (float)(1.4426950408889634 / std::sqrt((double)D));
     a.tau = plan->tau;
     a.tau_mode = plan->tau_mode;
-    const lkv::DecodeShape &shp = cache->shape(bits, B, single_pass(bits, plan->tau));
+    const lkv::DecodeShape shp = cache->shape(bits, B, single_pass(bits, plan->tau));
     a.cap_groups = shp.cap;
-    return lkv::launch_decode(a, bits, D, cp.cfg.in_dtype, shp, static_cast<cudaStream_t>(stream));
+    {
+        std::lock_guard<std::mutex> lock(cache->mu);
+        a.wait_ns = cache->wait_ns;
+        a.inject = cache->inject;
+    }
+    const bool overlap = cache->decode_may_overlap(stream);
+    return lkv::launch_decode(a, bits, D, cp.cfg.in_dtype, shp, overlap, static_cast<cudaStream_t>(stream));
 }
 
 int loopkv_decode(const loopkv_plan *plan, int loop, int layer, const void *q, const loopkv_cache *cache, float *out,
@@ -526,6 +562,16 @@ int loopkv_status(loopkv_cache *cache, void *stream, int *device_status)
         return LOOPKV_ERR_STATE;
     if (w & LOOPKV_DEV_EMPTY_ROW)
         return LOOPKV_ERR_EMPTY_ROW;
+    return LOOPKV_OK;
+}
+
+int loopkv_set_wait_policy(loopkv_cache *cache, uint64_t wait_limit_ns, int inject)
+{
+    if (!cache || wait_limit_ns == 0 || (inject != LOOPKV_INJECT_NONE && inject != LOOPKV_INJECT_STALLED_STAGE))
+        return LOOPKV_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(cache->mu);
+    cache->wait_ns = wait_limit_ns;
+    cache->inject = inject;
     return LOOPKV_OK;
 }
 

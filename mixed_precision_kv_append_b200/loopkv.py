@@ -33,8 +33,9 @@ EXPORTS = [
     "loopkv_plan_create", "loopkv_plan_free", "loopkv_plan_bytes", "loopkv_required_bytes", "loopkv_alloc",
     "loopkv_free", "loopkv_ingest", "loopkv_append", "loopkv_flush", "loopkv_reset_request", "loopkv_decode",
     "loopkv_decode_debug", "loopkv_status", "loopkv_cell_view_get", "loopkv_decode_shape", "loopkv_strerror",
-    "loopkv_version", "loopkv_plan_search", "loopkv_append_noalloc",
+    "loopkv_version", "loopkv_plan_search", "loopkv_append_noalloc", "loopkv_set_wait_policy",
 ]
+INJECT_NONE, INJECT_STALLED_STAGE = 0, 1
 NOALLOC_MAX_IDS = 4096
 
 
@@ -98,6 +99,7 @@ def lib() -> ctypes.CDLL:
         L.loopkv_decode.argtypes = [vp, i, i, vp, vp, vp, i, vp]
         L.loopkv_decode_debug.argtypes = [vp, i, i, vp, vp, vp, i, vp, vp, vp, vp]
         L.loopkv_status.argtypes = [vp, vp, ip]
+        L.loopkv_set_wait_policy.argtypes = [vp, ctypes.c_uint64, i]
         L.loopkv_cell_view_get.argtypes = [vp, i, i, ctypes.POINTER(CellView)]
         L.loopkv_decode_shape.argtypes = [vp, i, ip, ip, ip]
         L.loopkv_strerror.argtypes = [i]
@@ -235,6 +237,10 @@ def loopkv_status(cache, stream=None) -> tuple[int, int]:
     bits = ctypes.c_int()
     rc = lib().loopkv_status(cache, _stream(stream), ctypes.byref(bits))
     return rc, bits.value
+
+
+def loopkv_set_wait_policy(cache, wait_limit_ns: int, inject: int = INJECT_NONE):
+    _check(lib().loopkv_set_wait_policy(cache, int(wait_limit_ns), int(inject)), "loopkv_set_wait_policy")
 
 
 def loopkv_cell_view_get(cache, loop: int, layer: int) -> CellView:

@@ -371,3 +371,85 @@ def test_decode_shape_reports_cluster_launch():
     shp = p.decode_shape(8)
     assert shp["cluster"] in (1, 2, 3, 4, 5, 6, 7, 8, 16) and shp["ctas"] % shp["cluster"] == 0
     assert shp["ctas"] >= 148 and 0 < shp["smem"] <= 227 * 1024
+
+
+@pytest.mark.parametrize("modes,tau", [([L.CELL_4B, L.CELL_4B], 0.01), ([L.CELL_2B, L.CELL_4B], 0.0)])
+def test_bounded_wait_gives_up_and_recovers(modes, tau):
+    """A stage armed for bytes that are never requested (the injection hook) makes its wait run
+    out after the short limit: the decode reports LOOPKV_ERR_TIMEOUT, the stream completes, and
+    the next decode with the normal policy matches the oracle.  Both kernels: the exact-maximum
+    reader (4-bit, tau > 0) and the single-pass reader (2-bit / tau = 0)."""
+    w = synth.Workload("timeout", 1, 2, 4, 128, 3, [512, 96, 1000], torch.bfloat16, modes, tau, seed=23)
+    m = Model(w)
+    m.ingest()
+    q = _q(w, 0, 0, 0)
+    L.loopkv_set_wait_policy(m.cache.handle, 200_000, L.INJECT_STALLED_STAGE)
+    m.cache.decode(0, 0, q)
+    torch.cuda.synchronize()
+    rc, bits = m.cache.status()
+    assert rc == -7 and bits & L.DEV_TIMEOUT
+    L.loopkv_set_wait_policy(m.cache.handle, 500_000_000, L.INJECT_NONE)
+    m.check_cell(0, 0, q, where="after a timed-out decode")
+    assert m.cache.status() == (0, 0)
+    with pytest.raises(L.LoopKVError):
+        L.loopkv_set_wait_policy(m.cache.handle, 0, L.INJECT_NONE)
+
+
+@pytest.mark.parametrize("graph", [False, True])
+def test_flush_then_decode_without_append(graph):
+    """A decode launched right after a flush on the same stream (no append between) reads the
+    lengths and block tables the flush wrote, in eager mode and inside a captured graph."""
+    modes = [L.CELL_4B, L.CELL_SHARE, L.CELL_2B, L.CELL_4B]  # loop 0: [4b, share], loop 1: [2b, 4b]
+    w = synth.Workload("flushdec", 2, 2, 4, 128, 3, [20, 64, 95], torch.bfloat16, modes, 0.01, append_steps=40,
+                       seed=29)
+    m = Model(w)
+    m.ingest()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    outs = {}
+    qs = {(lp, la): _q(w, 5, la, lp) for lp in range(2) for la in range(2)}
+    for step in range(36):  # every tail fills up at least once
+        _, ks, vs = synth.step_tokens(w, step, 0, device="cuda")
+        with torch.cuda.stream(s):
+            m.cache.flush(stream=s)
+            for la in range(2):
+                for lp in range(2):
+                    m.cache.append(lp, la, ks[lp].contiguous(), vs[lp].contiguous(), stream=s)
+        s.synchronize()
+        for la in range(2):
+            for lp in range(2):
+                c = m.cell(lp, la)
+                for req in range(w.B):
+                    K, V = m.tokens[(c, req)]
+                    m.tokens[(c, req)] = (np.concatenate([K, f32(ks[lp][req:req + 1])]),
+                                          np.concatenate([V, f32(vs[lp][req:req + 1])]))
+    m._hist_cache.clear()
+    for la in range(2):  # launch shapes fixed before any capture
+        for lp in range(2):
+            outs[(lp, la)] = m.cache.decode(lp, la, qs[(lp, la)])
+    torch.cuda.synchronize()
+
+    def step(stream):
+        m.cache.flush(stream=stream)
+        for la in range(2):
+            for lp in range(2):
+                L.loopkv_decode(m.plan.handle, lp, la, qs[(lp, la)], m.cache.handle, outs[(lp, la)], stream=stream)
+
+    with torch.cuda.stream(s):
+        if graph:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                step(s)
+            g.replay()
+        else:
+            step(s)
+    s.synchronize()
+    m.cache.check("flush then decode")
+    for la in range(2):
+        for lp in range(2):
+            hist, tail = m.cache.lengths(lp, la)
+            assert all(int(tail[r]) < 32 for r in range(w.B))
+            ref = outs[(lp, la)].clone()
+            again = m.cache.decode(lp, la, qs[(lp, la)])
+            assert torch.equal(ref, again)
+            m.check_cell(lp, la, qs[(lp, la)], where=f"flush then decode graph={graph}")
