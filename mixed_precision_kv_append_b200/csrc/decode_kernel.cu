@@ -56,6 +56,7 @@
 #include "lkv_internal.h"
 
 #include <algorithm>
+#include <cstdio>
 #include <cstdlib>
 
 namespace lkv {
@@ -206,8 +207,14 @@ __device__ __forceinline__ float group_scores(const uint8_t *blkA, const uint8_t
 #pragma unroll
         for (int i = 0; i < 4; ++i)
             I[i] = __float2int_rn(av[i] * fs);
-        // byte k of I + (0x80 in each byte below k) is digit k as a signed byte
-        uint32_t *tab = reinterpret_cast<uint32_t *>(scr) + lane;
+        // byte k of I + (0x80 in each byte below k) is digit k as a signed byte.  Quad L goes to
+        // word NB t + pos(j) of each row (t = L / NB, j = L % NB), ordered so that the two words
+        // of every B fragment are adjacent in the lane's loaded registers (see the mma calls)
+        constexpr int NBW = D / 16;
+        const int jq = lane % NBW;
+        const int pos = NBW == 8 ? (BITS == 4 ? (jq & 1) * 4 + (jq >> 1) : (jq & 3) * 2 + (jq >> 2))
+                                 : (BITS == 4 ? (jq & 1) * 2 + (jq >> 1) : jq);
+        uint32_t *tab = reinterpret_cast<uint32_t *>(scr) + (lane - jq) + pos;
         tab[0] = __byte_perm(__byte_perm(I[0], I[1], 0x0040), __byte_perm(I[2], I[3], 0x0040), 0x5410);
 #pragma unroll
         for (int k = 1; k < 4; ++k) {
@@ -245,15 +252,17 @@ __device__ __forceinline__ float group_scores(const uint8_t *blkA, const uint8_t
             if (D == 128) { // words 4t..4t+3: quads 8t + 2w (low nibbles) and 8t + 2w + 1 (high)
                 const uint4 r0 = *reinterpret_cast<const uint4 *>(rows + g * G::ROWK + 16 * t);
                 const uint4 r1 = *reinterpret_cast<const uint4 *>(rows + (g + 8) * G::ROWK + 16 * t);
-                mma_u8s8(c, r0.x & M4, r1.x & M4, r0.y & M4, r1.y & M4, b[0], b[2]);
-                mma_u8s8(c, r0.z & M4, r1.z & M4, r0.w & M4, r1.w & M4, b[4], b[6]);
-                mma_u8s8(ch, r0.x & H4, r1.x & H4, r0.y & H4, r1.y & H4, b[1], b[3]);
-                mma_u8s8(ch, r0.z & H4, r1.z & H4, r0.w & H4, r1.w & H4, b[5], b[7]);
+                // b = digits of quads 8t + {0, 2, 4, 6, 1, 3, 5, 7}
+                mma_u8s8(c, r0.x & M4, r1.x & M4, r0.y & M4, r1.y & M4, b[0], b[1]);
+                mma_u8s8(c, r0.z & M4, r1.z & M4, r0.w & M4, r1.w & M4, b[2], b[3]);
+                mma_u8s8(ch, r0.x & H4, r1.x & H4, r0.y & H4, r1.y & H4, b[4], b[5]);
+                mma_u8s8(ch, r0.z & H4, r1.z & H4, r0.w & H4, r1.w & H4, b[6], b[7]);
             } else { // D = 64: words 2t, 2t+1: quads 4t, 4t+2 (low), 4t+1, 4t+3 (high)
                 const uint2 r0 = *reinterpret_cast<const uint2 *>(rows + g * G::ROWK + 8 * t);
                 const uint2 r1 = *reinterpret_cast<const uint2 *>(rows + (g + 8) * G::ROWK + 8 * t);
-                mma_u8s8(c, r0.x & M4, r1.x & M4, r0.y & M4, r1.y & M4, b[0], b[2]);
-                mma_u8s8(ch, r0.x & H4, r1.x & H4, r0.y & H4, r1.y & H4, b[1], b[3]);
+                // b = digits of quads 4t + {0, 2, 1, 3}
+                mma_u8s8(c, r0.x & M4, r1.x & M4, r0.y & M4, r1.y & M4, b[0], b[1]);
+                mma_u8s8(ch, r0.x & H4, r1.x & H4, r0.y & H4, r1.y & H4, b[2], b[3]);
             }
 #pragma unroll
             for (int r = 0; r < 4; ++r)
@@ -262,9 +271,9 @@ __device__ __forceinline__ float group_scores(const uint8_t *blkA, const uint8_t
             const uint2 r0 = *reinterpret_cast<const uint2 *>(rows + g * G::ROWK + 8 * t);
             const uint2 r1 = *reinterpret_cast<const uint2 *>(rows + (g + 8) * G::ROWK + 8 * t);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < 4; ++i) // b = digits of quads 8t + {0, 4, 1, 5, 2, 6, 3, 7}
                 mma_u8s8(c, (r0.x >> (2 * i)) & M2, (r1.x >> (2 * i)) & M2, (r0.y >> (2 * i)) & M2,
-                         (r1.y >> (2 * i)) & M2, b[i], b[4 + i]);
+                         (r1.y >> (2 * i)) & M2, b[2 * i], b[2 * i + 1]);
         } else { // D = 64, 2-bit: word t, field i is quad 4t + i
             const uint32_t r0 = *reinterpret_cast<const uint32_t *>(rows + g * G::ROWK + 4 * t);
             const uint32_t r1 = *reinterpret_cast<const uint32_t *>(rows + (g + 8) * G::ROWK + 4 * t);
@@ -500,8 +509,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
 
     const int capw = (a.cap_groups + kWarps - 1) / kWarps;
     Smem sm = carve<BITS, D>(smem_raw, spw, capw, nbuf);
-    const bool all_hot = (BITS == 4) && !(a.tau > 0.f);
-    const bool decide = (BITS == 4) && (a.tau > 0.f); // lo planes depend on the row max
+    static_assert(BITS == 4, "the exact-maximum reader serves 4-bit sources read with tau > 0");
     const bool seq = nbuf == 1; // one score buffer: rows one after another (see the main loop)
     // byte distance between consecutive block ids in the pools (one block = H heads)
     const uint32_t bstride = (uint32_t)a.H * G::HM, lstride = (uint32_t)a.H * G::LOB;
@@ -701,22 +709,6 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             }
             return;
         }
-        if (!decide) { // the whole V stage now: hi parts, and lo planes of every token (4-bit)
-            if (lane == 0) {
-                mbar_arrive_expect_tx(fb, (uint32_t)ng * (2 * G::VB + 2 * G::LOB));
-                for (int j = 0; j < ng; ++j) {
-                    const int2 id = ids[j];
-                    uint8_t *st = stg + j * G::GSLOT;
-                    bulk_g2s(st, seg_src + (uint64_t)(uint32_t)id.x * bstride, G::VB, fb);
-                    bulk_g2s(st + G::VB, seg_src + (uint64_t)(uint32_t)id.y * bstride, G::VB, fb);
-                    if (BITS == 4) {
-                        bulk_g2s(st + 2 * G::VB, seg_lo + (uint64_t)(uint32_t)id.x * lstride, G::LOB, fb);
-                        bulk_g2s(st + 2 * G::VB + G::LOB, seg_lo + (uint64_t)(uint32_t)id.y * lstride, G::LOB, fb);
-                    }
-                }
-            }
-            return;
-        }
         int32_t *st_row = irow_of(seg_ri);
         if (lane == 0) {
             if (k2 == 0)
@@ -764,16 +756,14 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     };
     // the threshold of row ri is known: finish the V stages issued without their lo part
     auto release_row = [&](int ri, float thr2) {
-        if (decide) {
-            int32_t *st_row = irow_of(ri);
-            const int vfirst = st_row[IR_VFIRST], vissued = st_row[IR_VISSUED];
-            __syncwarp();
-            if (lane == 0)
-                st_row[IR_THR] = __float_as_int(thr2);
-            __syncwarp();
-            for (int k2 = 0; k2 < vissued; ++k2)
-                issue_lo(ri, k2, vfirst + k2, thr2);
-        }
+        int32_t *st_row = irow_of(ri);
+        const int vfirst = st_row[IR_VFIRST], vissued = st_row[IR_VISSUED];
+        __syncwarp();
+        if (lane == 0)
+            st_row[IR_THR] = __float_as_int(thr2);
+        __syncwarp();
+        for (int k2 = 0; k2 < vissued; ++k2)
+            issue_lo(ri, k2, vfirst + k2, thr2);
     };
 
     // ---------------------------------------------------------------- compute
@@ -926,7 +916,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             }
             const float s2l = sc[k * 32 + lane];
             const float wl = ex2(s2l - m2);
-            const bool hotl = all_hot || (BITS == 4 && s2l >= thr2);
+            const bool hotl = s2l >= thr2;
             const uint32_t hm = __ballot_sync(0xFFFFFFFFu, hotl);
             if (a.s_bitmap && lane == 0) // refine set of the debug entry point, one bit per token
                 a.s_bitmap[(int64_t)srow[IR_ROW] * a.bitmap_words + (int)crank + (warp + k * kWarps) * (int)C] = hm;
@@ -943,7 +933,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
 #pragma unroll
                 for (int g = 0; g < NCG; ++g) {
                     const float2 m = __half22float2(*reinterpret_cast<const __half2 *>(vm + 64 * g));
-                    zl[g] = fmaf(wl, (BITS == 4 && !hotl) ? fmaf(1.5f, m.x, m.y) : m.y, zl[g]);
+                    zl[g] = fmaf(wl, hotl ? m.y : fmaf(1.5f, m.x, m.y), zl[g]);
                     W[g] = wl * m.x;
                     wmax = fmaxf(wmax, W[g]);
                 }
@@ -982,12 +972,8 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
 #pragma unroll
                 for (int tau = 0; tau < 4; ++tau) {
                     const uint4 rc = rq[tau];
-                    uint32_t lw = 0u;
-                    if (BITS == 4) { // lo words exist for quads with a hot token; keep the hot tokens' bits
-                        lw = *reinterpret_cast<const uint32_t *>(lop + tau * D);
-                        if (!all_hot)
-                            lw &= rc.z;
-                    }
+                    // lo words exist for quads with a hot token; keep the hot tokens' bits
+                    const uint32_t lw = *reinterpret_cast<const uint32_t *>(lop + tau * D) & rc.z;
                     acc.add<BITS>(hwv[tau], lw, rc.x, rc.y);
                 }
             }
@@ -1083,8 +1069,6 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     };
 
     auto row_threshold = [&](float m, float l) {
-        if (!decide)
-            return -INFINITY;
         return a.tau_mode == LOOPKV_TAU_ABS_PROB ? m + log2f(a.tau * l) : m + log2f(a.tau);
     };
 
@@ -1713,10 +1697,15 @@ int launch_shape(K kern, const DecodeShape &shp, bool pdl, cudaStream_t s, Args.
 template <int BITS, int D, typename DT>
 int launch_t(const DecodeArgs &a, const DecodeShape &shp, bool pdl, cudaStream_t s)
 {
-    if (shp.onepass)
-        return launch_shape(decode_kernel_1p<BITS, D, DT, 4>, shp, pdl, s, a, shp.stages_log2);
-    auto kern = shp.min_ctas == 5 ? decode_kernel<BITS, D, DT, 5> : decode_kernel<BITS, D, DT, 4>;
-    return launch_shape(kern, shp, pdl, s, a, shp.stages_log2, shp.score_bufs);
+    if constexpr (BITS == 4) {
+        if (!shp.onepass) {
+            auto kern = shp.min_ctas == 5 ? decode_kernel<BITS, D, DT, 5> : decode_kernel<BITS, D, DT, 4>;
+            return launch_shape(kern, shp, pdl, s, a, shp.stages_log2, shp.score_bufs);
+        }
+    }
+    if (!shp.onepass)
+        return LOOPKV_ERR_CUDA; // 2-bit sources have no refine set: always the single-pass reader
+    return launch_shape(decode_kernel_1p<BITS, D, DT, 4>, shp, pdl, s, a, shp.stages_log2);
 }
 
 // Clusters of size C that can be resident at once for this kernel and shared memory.
@@ -1756,15 +1745,26 @@ constexpr double kRowFixed = 6.0;  // per-CTA cost of a row outside its groups (
 constexpr double kSaturate = 3.5;  // CTAs per SM that keep its issue slots busy
 constexpr double kSeqRow = 4.0;    // extra per-row cost when rows do not overlap (one score buffer)
 
-// Overlap with the previous launch of the stream (programmatic dependent launch): measured
-// faster with clusters of up to 4 CTAs and slower with larger ones; LOOPKV_DECODE_PDL=0/1
-// overrides.
-inline int pdl_default(int C)
+// Overlap with the previous launch of the stream (programmatic dependent launch): on B200
+// measured faster for the single-pass reader with clusters of up to 4 CTAs (+9% on the 8K
+// KIVI-4 workload) and slower for the exact-maximum reader (-9% on the mixed 8K workload).
+inline int pdl_default(int C, bool onepass) { return onepass && C <= 4; }
+
+// Debug override of the launch-shape model, for measurements only: LOOPKV_DECODE_SHAPE =
+// "cluster,stages,ctas_per_sm,score_buffers,pdl", each field 0 (or absent) for the model's
+// choice; pdl 1 = on, 2 = off.  Read when a cache first computes the shape of a batch size.
+struct ShapeOverride {
+    int cluster = 0, stages = 0, ctas = 0, bufs = 0, pdl = 0;
+};
+inline ShapeOverride shape_override()
 {
-    const char *env = getenv("LOOPKV_DECODE_PDL");
-    if (env)
-        return atoi(env) != 0;
-    return C <= 4;
+    ShapeOverride o;
+    if (const char *env = getenv("LOOPKV_DECODE_SHAPE")) {
+        int v[5] = {0, 0, 0, 0, 0};
+        sscanf(env, "%d,%d,%d,%d,%d", &v[0], &v[1], &v[2], &v[3], &v[4]);
+        o.cluster = v[0], o.stages = v[1], o.ctas = v[2], o.bufs = v[3], o.pdl = v[4];
+    }
+    return o;
 }
 
 // Shared memory of a kernel with `spw` ring slots per warp.
@@ -1788,17 +1788,16 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
             sm_count = 148;
     }
     const int smem_per_sm = 228 * 1024;
-    const char *env_c = getenv("LOOPKV_DECODE_CLUSTER");
-    const char *env_s = getenv("LOOPKV_DECODE_STAGES");
-    const char *env_o = getenv("LOOPKV_DECODE_CTAS_PER_SM");
-    const char *env_b = getenv("LOOPKV_DECODE_SCORE_BUFS");
+    const ShapeOverride ov = shape_override();
+    if (BITS == 2)
+        onepass = true;
     // two-phase builds for 4 and 5 CTAs per SM; the single-pass kernel for 4 (its 96-register
     // build measured 5% slower on the same grid)
     for (int want_ctas = 4; want_ctas <= (onepass ? 4 : 5); ++want_ctas) {
-        if (env_o && atoi(env_o) != want_ctas)
+        if (ov.ctas && ov.ctas != want_ctas)
             continue;
         for (int C = 1; C <= 16; C = C < 8 ? C + 1 : 2 * C) { // 1..8, 16
-            if (env_c && atoi(env_c) != C)
+            if (ov.cluster && ov.cluster != C)
                 continue;
             const int cap = (max_groups + C - 1) / C;
             const int capw = (cap + kWarps - 1) / kWarps;
@@ -1808,19 +1807,22 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
                 int spw = 8;
                 while (spw > 2 && kernel_smem<BITS, D>(onepass, spw, capw, nbuf) > budget)
                     spw >>= 1;
-                if (env_s)
-                    spw = atoi(env_s);
+                if (ov.stages)
+                    spw = ov.stages;
                 const int smem = kernel_smem<BITS, D>(onepass, spw, capw, nbuf);
                 if (smem <= 0 || smem > 227 * 1024)
                     continue;
-                int ncl = onepass ? max_active_clusters(decode_kernel_1p<BITS, D, DT, 4>, C, smem)
-                          : want_ctas == 5 ? max_active_clusters(decode_kernel<BITS, D, DT, 5>, C, smem)
-                                           : max_active_clusters(decode_kernel<BITS, D, DT, 4>, C, smem);
+                int ncl = 0;
+                if (onepass)
+                    ncl = max_active_clusters(decode_kernel_1p<BITS, D, DT, 4>, C, smem);
+                else if constexpr (BITS == 4)
+                    ncl = want_ctas == 5 ? max_active_clusters(decode_kernel<BITS, D, DT, 5>, C, smem)
+                                         : max_active_clusters(decode_kernel<BITS, D, DT, 4>, C, smem);
                 if (ncl <= 0)
                     continue;
                 if (ncl > rows)
                     ncl = rows;
-                if (!onepass && env_b && atoi(env_b) != nbuf)
+                if (!onepass && ov.bufs && ov.bufs != nbuf)
                     continue;
                 const int rounds = (rows + ncl - 1) / ncl;
                 const int per_sm = (ncl * C + sm_count - 1) / sm_count;
@@ -1839,7 +1841,7 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
                     best.threads = kThreads;
                     best.cap = cap;
                     best.min_ctas = want_ctas;
-                    best.pdl = pdl_default(C);
+                    best.pdl = ov.pdl ? ov.pdl == 1 : pdl_default(C, onepass);
                     best.onepass = onepass;
                 }
                 if (onepass)

@@ -88,16 +88,8 @@ int head_main_bytes(int bits, int D) { return bits == 4 ? LKV_HEAD_MAIN_4B(D) : 
 
 // Whether a read's refine set is fixed before any score is known: a 2-bit source has no lo
 // plane (S empty), a 4-bit source read with tau <= 0 refines every token.  Such reads go to
-// the single-pass kernel (running maximum); LOOPKV_DECODE_ONEPASS=0 keeps them on the
-// two-phase one.
-bool single_pass(int bits, float tau)
-{
-    static const bool allowed = [] {
-        const char *env = getenv("LOOPKV_DECODE_ONEPASS");
-        return !env || atoi(env) != 0;
-    }();
-    return allowed && (bits == 2 || !(tau > 0.f));
-}
+// the single-pass kernel (running maximum), the others to the exact-maximum kernel.
+bool single_pass(int bits, float tau) { return bits == 2 || !(tau > 0.f); }
 
 int check_config(const loopkv_config *c)
 {

@@ -242,9 +242,16 @@ def test_two_phase_score_buffer_orders(monkeypatch, score_bufs):
     """The decide path (4-bit, tau > 0) with one score buffer (a cluster's rows in sequence)
     and with two (the next row's keys overlapping the current row's values), forced through
     the launch-shape override on a batch with more rows than clusters."""
-    monkeypatch.setenv("LOOPKV_DECODE_SCORE_BUFS", score_bufs)
     base = synth.workload("mixed_8k")
     w = synth.Workload("mixed_8k", 1, 4, 16, 128, 32, [8192] * 32, torch.bfloat16, [0, 1, 2, 0], 0.01, seed=2)
+    shapes = {}
+    for nb in ("1", "2"):  # the override takes effect: two score buffers take more shared memory
+        monkeypatch.setenv("LOOPKV_DECODE_SHAPE", f"0,0,0,{nb},0")
+        shapes[nb] = L.Plan(1, 4, 16, 128, 32, base.max_blocks, [0, 1, 2, 0], 0.01).decode_shape(32)
+    assert shapes["2"]["smem"] > shapes["1"]["smem"]
+    monkeypatch.setenv("LOOPKV_DECODE_SHAPE", f"0,0,0,{score_bufs},0")
+    # more rows (32 requests x 16 heads) than clusters: every cluster reads several rows in order
+    assert 32 * 16 > shapes[score_bufs]["ctas"] // shapes[score_bufs]["cluster"]
     m = Model(w, max_blocks=base.max_blocks)
     m.ingest()
     rng = np.random.default_rng(1)
