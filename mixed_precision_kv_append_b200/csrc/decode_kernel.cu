@@ -340,6 +340,19 @@ struct VSums {
     }
 };
 
+// q . k of one unquantized (near) token, in log2 units: the lane holds channels 4 lane ..
+// 4 lane + 3 of the exact query; krow: the token's D keys.  Warp-uniform result.
+template <int D, typename DT>
+__device__ __forceinline__ float near_score(const DT *krow, const float (&qreg)[4], const float qscale, const int lane)
+{
+    float s = 0.f;
+    if (lane < D / 4) {
+        const DT *k4 = krow + 4 * lane;
+        s = fmaf(qreg[0], to_f32(k4[0]), fmaf(qreg[1], to_f32(k4[1]), fmaf(qreg[2], to_f32(k4[2]), qreg[3] * to_f32(k4[3]))));
+    }
+    return warp_sum(s) * qscale;
+}
+
 struct Smem {
     uint8_t *ring;     // [kWarps][spw][STAGE] stage slots (kGPS groups each), a private slice per warp
     uint64_t *full;    // [kWarps][spw] completion barriers of the slots
@@ -389,7 +402,7 @@ template <int BITS, int D> __host__ __device__ constexpr SmemLayout smem_layout(
     L.scores = o;
     o = align16(o + nbuf * kWarps * capw * 32 * 4);
     L.tscores = o;
-    o = align16(o + 2 * 32 * 4);
+    o = align16(o + 2 * LKV_TAIL_TOKENS * 4);
     L.scr = o;
     o = align16(o + kWarps * scratch_bytes<D>());
     L.stat = o;
@@ -618,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             st[IR_B] = b;
             st[IR_H] = h;
             st[IR_N] = n;
-            st[IR_TAIL] = (crank == C - 1 && warp == kWarps - 1) ? -1 : 0; // -1: tail owner, length not read
+            st[IR_TAIL] = -1; // tail length not read yet (read after the grid dependency wait)
             st[IR_VFIRST] = 0;
             st[IR_VISSUED] = 0;
             st[IR_THR] = __float_as_int(NAN);
@@ -798,10 +811,10 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             asm volatile("griddepcontrol.wait;" ::: "memory");
         }
         int tail = srow[IR_TAIL];
-        if (tail < 0) { // the tail owner reads the tail length
+        if (tail < 0) { // the tail length (an append may just have written it)
             tail = a.tail_len[srow[IR_B]];
-            if (tail < 0 || tail > 32) {
-                if (lane == 0)
+            if (tail < 0 || tail > LKV_TAIL_TOKENS) {
+                if (lane == 0 && warp == 0)
                     atomicOr(a.status, LOOPKV_DEV_STATE);
                 tail = 0;
             }
@@ -835,34 +848,28 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             mx = fmaxf(mx, s2);
             __syncwarp();
         }
-        float *tsc = sm.tscores + (ri & 1) * 32;
-        if (tail > 0 && warp == kWarps - 1) { // tail keys, exact; lane = tail token
-            const int b = srow[IR_B], h = srow[IR_H];
-            const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)b * 2 * a.H + h) * 32 * D;
-            float s2 = 0.f;
-            for (int q4 = 0; q4 < G::NQ; ++q4) {
-                float kv[4] = {0.f, 0.f, 0.f, 0.f};
-                if (lane < tail)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        kv[i] = to_f32(kt[(int64_t)lane * D + 4 * q4 + i]);
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    s2 = fmaf(__shfl_sync(0xFFFFFFFFu, qreg[i], q4), kv[i], s2);
-            }
-            s2 *= a.qscale;
-            if (lane < tail) {
-                tsc[lane] = s2;
+        // tail tokens (exact keys), dealt over every warp of the cluster: token j to warp
+        // j mod (C * kWarps) of the cluster, so that no warp carries the whole tail
+        float *tsc = sm.tscores + (ri & 1) * LKV_TAIL_TOKENS;
+        const int wg = (int)crank * kWarps + warp, nw = (int)C * kWarps;
+        if (tail > wg) {
+            const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)srow[IR_B] * 2 * a.H + srow[IR_H]) *
+                                                                      LKV_TAIL_TOKENS * D;
+            for (int j = wg; j < tail; j += nw) {
+                const float s2 = near_score<D, DT>(kt + (int64_t)j * D, qreg, a.qscale, lane);
+                if (lane == 0)
+                    tsc[j] = s2;
                 mx = fmaxf(mx, s2);
             }
+            __syncwarp();
         }
         mx = warp_max(mx);
         float ls = 0.f;
         if (a.tau_mode == LOOPKV_TAU_ABS_PROB && mx != -INFINITY) {
             for (int k = 0; k < nown; ++k)
                 ls += exp2f(sc[k * 32 + lane] - mx);
-            if (tail > 0 && warp == kWarps - 1 && lane < tail)
-                ls += exp2f(tsc[lane] - mx);
+            for (int j = wg + lane * nw; j < tail; j += 32 * nw)
+                ls += exp2f(tsc[j] - mx);
             ls = warp_sum(ls);
         }
         if (lane == 0) {
@@ -1011,12 +1018,13 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         if (lane == 0)
             red[D] = lsum;
         __syncwarp();
-        if (tail > 0 && warp == kWarps - 1) { // tail values, exact
+        const int wg = (int)crank * kWarps + warp, nw = (int)C * kWarps;
+        if (tail > wg) { // this warp's tail tokens (see consume_k), exact values
             const int b = srow[IR_B], h = srow[IR_H];
-            const float *tsc = sm.tscores + (ri & 1) * 32;
-            const DT *vt0 = reinterpret_cast<const DT *>(a.tail) + ((int64_t)(b * 2 + 1) * a.H + h) * 32 * D;
+            const float *tsc = sm.tscores + (ri & 1) * LKV_TAIL_TOKENS;
+            const DT *vt0 = reinterpret_cast<const DT *>(a.tail) + ((int64_t)(b * 2 + 1) * a.H + h) * LKV_TAIL_TOKENS * D;
             float tl = 0.f;
-            for (int t = 0; t < tail; ++t) {
+            for (int t = wg; t < tail; t += nw) {
                 const float w = exp2f(tsc[t] - m2);
                 tl += w;
                 const DT *vt = vt0 + (int64_t)t * D;
@@ -1321,45 +1329,31 @@ template <int BITS, int D> __device__ __forceinline__ void run1_finish(Run1<D> &
     __syncwarp();
 }
 
-// Tail tokens t < tail (exact; lane = tail token) folded into the warp's partial red:
-// keys kt [32][D] and values vt0 [32][D]; rescales red when a tail score raises r.m.
+// Tail tokens j0, j0 + stride, ... < n (exact keys kt [*][D], values vt0 [*][D]) folded into the
+// warp's partial red (o[D], l relative to 2^r.m), raising r.m (and rescaling red) when a
+// tail score exceeds it.
 template <int D, typename DT>
 __device__ __forceinline__ void run1_tail(Run1<D> &r, float *red, const int lane, const float (&qreg)[4],
-                                          const float qscale, const DT *kt, const DT *vt0, const int tail)
+                                          const float qscale, const DT *kt, const DT *vt0, const int j0,
+                                          const int stride, const int n)
 {
-    constexpr int NQ = D / 4;
-    float s2 = 0.f;
-    for (int q4 = 0; q4 < NQ; ++q4) {
-        float kv[4] = {0.f, 0.f, 0.f, 0.f};
-        if (lane < tail)
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                kv[i] = to_f32(kt[(int64_t)lane * D + 4 * q4 + i]);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            s2 = fmaf(__shfl_sync(0xFFFFFFFFu, qreg[i], q4), kv[i], s2);
-    }
-    s2 *= qscale;
-    const float mt = warp_max_f(lane < tail ? s2 : -INFINITY);
-    if (mt > r.m) { // rescale the warp's partial in the scratch
-        const float f = ex2(r.m - mt);
-        for (int c = lane; c <= D; c += 32)
-            red[c] *= f;
-        r.m = mt;
-    }
-    __syncwarp();
-    float tl = 0.f;
-    for (int t = 0; t < tail; ++t) {
-        const float w = ex2(__shfl_sync(0xFFFFFFFFu, s2, t) - r.m);
-        tl += w;
-        const DT *vt = vt0 + (int64_t)t * D;
+    for (int j = j0; j < n; j += stride) {
+        const float s2 = near_score<D, DT>(kt + (int64_t)j * D, qreg, qscale, lane);
+        if (s2 > r.m) { // warp-uniform
+            const float f = ex2(r.m - s2);
+            for (int c = lane; c <= D; c += 32)
+                red[c] *= f;
+            r.m = s2;
+        }
+        const float w = ex2(s2 - r.m);
+        const DT *vt = vt0 + (int64_t)j * D;
 #pragma unroll
         for (int c4 = 0; c4 < D / 32; ++c4)
             red[lane + 32 * c4] = fmaf(w, to_f32(vt[lane + 32 * c4]), red[lane + 32 * c4]);
+        if (lane == 0)
+            red[D] += w;
     }
     __syncwarp();
-    if (lane == 0)
-        red[D] += tl;
 }
 
 template <int BITS, int D, typename DT, int MINCTA>
@@ -1463,7 +1457,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
             irow[IR_B] = b;
             irow[IR_H] = h;
             irow[IR_N] = n;
-            irow[IR_TAIL] = (crank == C - 1 && warp == kWarps - 1) ? -1 : 0; // -1: tail owner
+            irow[IR_TAIL] = -1; // tail length read after the grid dependency wait
         }
         __syncwarp();
         setup_upto = ri;
@@ -1536,10 +1530,10 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
             pump(prc_n + spw);
             asm volatile("griddepcontrol.wait;" ::: "memory");
         }
-        if (tail < 0) { // the tail owner reads the tail length (an append may have written it)
+        if (tail < 0) { // the tail length (an append may have written it)
             tail = a.tail_len[rb];
-            if (tail < 0 || tail > 32) {
-                if (lane == 0)
+            if (tail < 0 || tail > LKV_TAIL_TOKENS) {
+                if (lane == 0 && warp == 0)
                     atomicOr(a.status, LOOPKV_DEV_STATE);
                 tail = 0;
             }
@@ -1570,10 +1564,12 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
         }
         float *red = reinterpret_cast<float *>(scr);
         run1_finish<BITS, D>(run, red, lane);
-        if (tail > 0 && warp == kWarps - 1) {
-            const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)rb * 2 * a.H + rh) * 32 * D;
-            const DT *vt0 = reinterpret_cast<const DT *>(a.tail) + ((int64_t)(rb * 2 + 1) * a.H + rh) * 32 * D;
-            run1_tail<D, DT>(run, red, lane, qreg, a.qscale, kt, vt0, tail);
+        const int wg = (int)crank * kWarps + warp; // tail token j to warp j mod (C * kWarps) of the cluster
+        if (tail > wg) {
+            const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)rb * 2 * a.H + rh) * LKV_TAIL_TOKENS * D;
+            const DT *vt0 =
+                reinterpret_cast<const DT *>(a.tail) + ((int64_t)(rb * 2 + 1) * a.H + rh) * LKV_TAIL_TOKENS * D;
+            run1_tail<D, DT>(run, red, lane, qreg, a.qscale, kt, vt0, wg, (int)C * kWarps, tail);
         }
         if (lane == 0)
             red[D + 1] = run.m;
