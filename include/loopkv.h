@@ -49,7 +49,7 @@ extern "C" {
 #define LOOPKV_ERR_RANGE (-6)          /* fp16 zero point or scale overflows */
 #define LOOPKV_ERR_TIMEOUT (-7)        /* a bounded device wait gave up */
 #define LOOPKV_ERR_CUDA (-8)           /* a CUDA runtime call failed */
-#define LOOPKV_ERR_TAIL_FULL (-9)      /* append to a 32-token tail not yet flushed */
+#define LOOPKV_ERR_TAIL_FULL (-9)      /* append to a full window (W + 32 tokens) not yet flushed */
 #define LOOPKV_ERR_STATE (-10)         /* ingest into a non-empty (cell, request), bad block id */
 #define LOOPKV_ERR_EMPTY_ROW (-11)     /* decode of a row with no token at all */
 #define LOOPKV_ERR_NO_DEVICE (-12)     /* no CUDA device of compute capability 10.x */
@@ -90,6 +90,17 @@ typedef struct {
     int max_batch;          /* request slots per cell */
     int max_blocks_per_seq; /* capacity of a cell's history in 16-token blocks (even) */
     int in_dtype;           /* loopkv_dtype */
+    /* Unquantized near region of every (cell, request) (LoopKV paper §2.3 and §3.4: the
+     * attention sink and the recent window stay BF16, and a 32-token page is quantized when
+     * it leaves the window).  sink_tokens: the first tokens of a sequence, never quantized
+     * (0..64, a multiple of 32; the paper uses 32).  window_tokens: W, multiple of 32, 0..512
+     * (the paper uses 256).  The window holds the most recent W to W + 31 tokens after a
+     * flush; loopkv_flush quantizes its oldest page once it holds W + 32.  The history (the
+     * quantized pages) lies between sink and window in sequence order.  Both 0 (the zero
+     * default of older callers): no sink, and a tail of up to 32 tokens quantized as soon as
+     * it is full. */
+    int sink_tokens;
+    int window_tokens;
 } loopkv_config;
 
 typedef struct loopkv_plan loopkv_plan;   /* opaque: config + per-cell modes + tau */
@@ -118,8 +129,13 @@ typedef struct {
     const uint8_t *lo_pool;     /* device: block b, head h at (b*H + h)*head_lo_bytes */
     const int32_t *block_table; /* device [max_batch][max_blocks_per_seq] of src_cell */
     const int32_t *hist_len;    /* device [max_batch] history tokens of src_cell */
-    const int32_t *tail_len;    /* device [max_batch] tail tokens of this cell */
-    const void *tail;           /* device [max_batch][2 (K,V)][H][32][D] in in_dtype */
+    const int32_t *tail_len;    /* device [max_batch] unquantized (near) tokens of this cell:
+                                 * sink fill + window length */
+    const int32_t *win_start;   /* device [max_batch] ring slot of the oldest window token */
+    const void *tail;           /* device [max_batch][2 (K,V)][H][near_cap][D] in in_dtype: near
+                                 * token slots; slots 0..sink-1 the sink, then the window ring of
+                                 * window_tokens + 32 slots (see loopkv_config) */
+    int near_cap;               /* sink_tokens + window_tokens + 32 */
     int64_t pool_blocks;        /* capacity of the pool in blocks */
 } loopkv_cell_view;
 
@@ -195,20 +211,23 @@ void loopkv_free(loopkv_cache *cache);
 /*
  * Bulk history of one request in one cell (prefill).  k, v: device [T][H][D] in
  * in_dtype.  The (cell, request) must be empty (else LOOPKV_DEV_STATE and nothing is
- * written).  The first 32*floor(T/32) tokens are quantized into 16-token blocks by
- * the same kernel as loopkv_flush; the remaining T mod 32 go to the tail.  A share
- * cell stores only its tail; its history is the final loop's (LoopKV paper §3.2),
- * which must be ingested with the same T before decoding.
+ * written).  The first min(T, sink) tokens fill the sink; of the remaining R, the first
+ * 32 * floor((R - W) / 32) (none if R < W) are quantized into 16-token blocks by the same
+ * kernel as loopkv_flush, and the last go to the window (W to W + 31 of them, or all R
+ * when R < W); with sink = W = 0 that is T mod 32 tokens.  A share cell stores only its
+ * sink and window; its history is the final loop's (LoopKV paper §3.2), which must be
+ * ingested with the same T before decoding.
  */
 int loopkv_ingest(loopkv_cache *cache, int loop, int layer, int req, const void *k, const void *v,
                   int T, void *stream);
 
 /*
- * Append one token per request to a cell's unquantized tail (LoopKV paper §3.4:
- * sink and window stay BF16; share cells keep their own, §3.2).  k, v: device
- * [B][H][D] in in_dtype for requests req_ids[0..B-1] (host array) or 0..B-1 when
- * req_ids is NULL.  A tail already holding 32 tokens raises LOOPKV_DEV_TAIL_FULL
- * for that request and drops its token: call loopkv_flush first.
+ * Append one token per request to a cell's unquantized near region (LoopKV paper §3.4:
+ * sink and window stay BF16; share cells keep their own, §3.2): into the sink while it is
+ * not full, else into the window.  k, v: device [B][H][D] in in_dtype for requests
+ * req_ids[0..B-1] (host array) or 0..B-1 when req_ids is NULL.  A window already holding
+ * W + 32 tokens raises LOOPKV_DEV_TAIL_FULL for that request and drops its token: call
+ * loopkv_flush first.
  */
 int loopkv_append(loopkv_cache *cache, int loop, int layer, const void *k, const void *v,
                   const int32_t *req_ids, int B, void *stream);
@@ -238,12 +257,13 @@ int loopkv_append_noalloc(loopkv_cache *cache, int loop, int layer, const void *
                           const int32_t *req_ids, int B, void *stream);
 
 /*
- * Window exit: quantize every tail that holds 32 tokens into two new 16-token blocks
- * of its cell (K per channel over the 32 tokens, V per token over 32 channels, fp16
- * scale/zero, V split into hi/lo planes) and empty it; a share cell only empties its
- * tail (LoopKV paper §3.2; §3.4 "Layout", where pages are quantized as they leave the
- * window, ahead of the step's graph).  Blocks come from the device free list, so the call
- * needs no host round trip and can sit inside a captured graph.
+ * Window exit: in every (cell, request) whose window holds W + 32 tokens, quantize its
+ * oldest 32 into two new 16-token blocks of the cell (K per channel over the 32 tokens, V
+ * per token over 32 channels, fp16 scale/zero, V split into hi/lo planes) and drop them
+ * from the window; a share cell only drops them (LoopKV paper §3.2; §3.4 "Layout", where
+ * pages are quantized as they leave the window, ahead of the step's graph).  Blocks come
+ * from the device free list, so the call needs no host round trip and can sit inside a
+ * captured graph.
  */
 int loopkv_flush(loopkv_cache *cache, void *stream);
 
@@ -255,10 +275,10 @@ int loopkv_reset_request(loopkv_cache *cache, int req, void *stream);
  * launch per cell").  q: device [B][H][D] in in_dtype for request slots 0..B-1;
  * out: device [B][H][D] fp32.  Per (request, head) row: scores over the full keys of
  * the history the cell reads (own pages, or the final loop's for a share cell) and
- * over its own tail; exact row max m; refine set S = history tokens of a 4-bit
+ * over its own sink and window; exact row max m; refine set S = history tokens of a 4-bit
  * source whose weight passes tau; values decoded as z + s*(4h+l) for tokens in S,
  * z + s*(4h+1.5) for the other 4-bit tokens, z + s*code for 2-bit cells, raw for the
- * tail; out = sum_t exp(s_t - m) v_t / sum_t exp(s_t - m).  When S does not depend on
+ * sink and window; out = sum_t exp(s_t - m) v_t / sum_t exp(s_t - m).  When S does not depend on
  * m (2-bit source, or tau <= 0) the launch accumulates with a running maximum instead;
  * the result is the same up to fp32 rounding.  A decode uses no device scratch, so
  * decodes of different cells may run on different streams.  The first call for a batch

@@ -353,6 +353,14 @@ __device__ __forceinline__ float near_score(const DT *krow, const float (&qreg)[
     return warp_sum(s) * qscale;
 }
 
+// Slot of near token j (0 .. near tokens - 1) in a (cell, request)'s near region: the sink
+// slots first, then the window ring from its oldest token (ws).  The order of the tokens
+// does not matter to attention, only that each is read once.
+__device__ __forceinline__ int near_slot(const DecodeArgs &a, int j, int ws)
+{
+    return j < a.sink ? j : a.sink + (ws + (j - a.sink)) % a.wring;
+}
+
 struct Smem {
     uint8_t *ring;     // [kWarps][spw][STAGE] stage slots (kGPS groups each), a private slice per warp
     uint64_t *full;    // [kWarps][spw] completion barriers of the slots
@@ -371,7 +379,7 @@ struct Smem {
 };
 
 // Fields of a row slot (Smem::irow).
-enum { IR_ROW = 0, IR_B, IR_H, IR_N, IR_TAIL, IR_VFIRST, IR_VISSUED, IR_THR, IR_N_FIELDS = 12 };
+enum { IR_ROW = 0, IR_B, IR_H, IR_N, IR_TAIL, IR_VFIRST, IR_VISSUED, IR_THR, IR_WS, IR_N_FIELDS = 12 };
 
 // Byte offsets of the shared-memory regions; every region starts on a 16-byte boundary
 // (digit records, weights and stage data are read with 16-byte vector loads).
@@ -393,7 +401,8 @@ template <int D> __host__ __device__ constexpr int scratch_bytes()
 // nbuf: score buffers (2: the next row's keys are scored while the current row's values are
 // read; 1: a cluster's rows run one after another, for long rows whose scores fill the
 // shared memory).
-template <int BITS, int D> __host__ __device__ constexpr SmemLayout smem_layout(int spw, int capw, int nbuf)
+template <int BITS, int D>
+__host__ __device__ constexpr SmemLayout smem_layout(int spw, int capw, int nbuf, int near_cap)
 {
     SmemLayout L{};
     int o = kWarps * spw * Geo<BITS, D>::STAGE; // ring, 128-byte aligned slots
@@ -402,7 +411,7 @@ template <int BITS, int D> __host__ __device__ constexpr SmemLayout smem_layout(
     L.scores = o;
     o = align16(o + nbuf * kWarps * capw * 32 * 4);
     L.tscores = o;
-    o = align16(o + 2 * LKV_TAIL_TOKENS * 4);
+    o = align16(o + 2 * near_cap * 4);
     L.scr = o;
     o = align16(o + kWarps * scratch_bytes<D>());
     L.stat = o;
@@ -419,14 +428,14 @@ template <int BITS, int D> __host__ __device__ constexpr SmemLayout smem_layout(
     return L;
 }
 
-template <int BITS, int D> __host__ __device__ constexpr int smem_bytes(int spw, int capw, int nbuf)
+template <int BITS, int D> __host__ __device__ constexpr int smem_bytes(int spw, int capw, int nbuf, int near_cap)
 {
-    return smem_layout<BITS, D>(spw, capw, nbuf).total;
+    return smem_layout<BITS, D>(spw, capw, nbuf, near_cap).total;
 }
 
-template <int BITS, int D> __device__ Smem carve(uint8_t *base, int spw, int capw, int nbuf)
+template <int BITS, int D> __device__ Smem carve(uint8_t *base, int spw, int capw, int nbuf, int near_cap)
 {
-    const SmemLayout L = smem_layout<BITS, D>(spw, capw, nbuf);
+    const SmemLayout L = smem_layout<BITS, D>(spw, capw, nbuf, near_cap);
     Smem s;
     s.ring = base;
     s.full = reinterpret_cast<uint64_t *>(base + L.full);
@@ -443,9 +452,9 @@ template <int BITS, int D> __device__ Smem carve(uint8_t *base, int spw, int cap
 
 // Host check of a layout: every region 16-byte aligned, in order, inside the allocation;
 // the per-warp id lists 8-byte aligned (read as pairs).
-template <int BITS, int D> bool layout_ok(int spw, int capw, int nbuf)
+template <int BITS, int D> bool layout_ok(int spw, int capw, int nbuf, int near_cap)
 {
-    const SmemLayout L = smem_layout<BITS, D>(spw, capw, nbuf);
+    const SmemLayout L = smem_layout<BITS, D>(spw, capw, nbuf, near_cap);
     const int offs[] = {L.full, L.scores, L.tscores, L.scr, L.stat, L.part, L.ids, L.irow, L.order};
     int prev = kWarps * spw * Geo<BITS, D>::STAGE;
     for (int o : offs) {
@@ -521,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     const int cid = blockIdx.x / (int)C, ncl = gridDim.x / (int)C;
 
     const int capw = (a.cap_groups + kWarps - 1) / kWarps;
-    Smem sm = carve<BITS, D>(smem_raw, spw, capw, nbuf);
+    Smem sm = carve<BITS, D>(smem_raw, spw, capw, nbuf, a.near_cap);
     static_assert(BITS == 4, "the exact-maximum reader serves 4-bit sources read with tau > 0");
     const bool seq = nbuf == 1; // one score buffer: rows one after another (see the main loop)
     // byte distance between consecutive block ids in the pools (one block = H heads)
@@ -811,16 +820,20 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             asm volatile("griddepcontrol.wait;" ::: "memory");
         }
         int tail = srow[IR_TAIL];
-        if (tail < 0) { // the tail length (an append may just have written it)
+        if (tail < 0) { // near tokens and ring start (an append may just have written them)
             tail = a.tail_len[srow[IR_B]];
-            if (tail < 0 || tail > LKV_TAIL_TOKENS) {
+            int ws = a.win_start[srow[IR_B]];
+            if (tail < 0 || tail > a.sink + a.wring || ws < 0 || ws >= a.wring) {
                 if (lane == 0 && warp == 0)
                     atomicOr(a.status, LOOPKV_DEV_STATE);
                 tail = 0;
+                ws = 0;
             }
             __syncwarp();
-            if (lane == 0)
+            if (lane == 0) {
                 srow[IR_TAIL] = tail;
+                srow[IR_WS] = ws;
+            }
             __syncwarp();
         }
         // lane owns the channel quad 4*lane .. 4*lane+3 (lanes >= D/4 own none)
@@ -850,13 +863,14 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         }
         // tail tokens (exact keys), dealt over every warp of the cluster: token j to warp
         // j mod (C * kWarps) of the cluster, so that no warp carries the whole tail
-        float *tsc = sm.tscores + (ri & 1) * LKV_TAIL_TOKENS;
+        float *tsc = sm.tscores + (ri & 1) * a.near_cap;
         const int wg = (int)crank * kWarps + warp, nw = (int)C * kWarps;
         if (tail > wg) {
             const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)srow[IR_B] * 2 * a.H + srow[IR_H]) *
-                                                                      LKV_TAIL_TOKENS * D;
+                                                                      a.near_cap * D;
+            const int ws = srow[IR_WS];
             for (int j = wg; j < tail; j += nw) {
-                const float s2 = near_score<D, DT>(kt + (int64_t)j * D, qreg, a.qscale, lane);
+                const float s2 = near_score<D, DT>(kt + (int64_t)near_slot(a, j, ws) * D, qreg, a.qscale, lane);
                 if (lane == 0)
                     tsc[j] = s2;
                 mx = fmaxf(mx, s2);
@@ -1021,13 +1035,14 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         const int wg = (int)crank * kWarps + warp, nw = (int)C * kWarps;
         if (tail > wg) { // this warp's tail tokens (see consume_k), exact values
             const int b = srow[IR_B], h = srow[IR_H];
-            const float *tsc = sm.tscores + (ri & 1) * LKV_TAIL_TOKENS;
-            const DT *vt0 = reinterpret_cast<const DT *>(a.tail) + ((int64_t)(b * 2 + 1) * a.H + h) * LKV_TAIL_TOKENS * D;
+            const float *tsc = sm.tscores + (ri & 1) * a.near_cap;
+            const DT *vt0 = reinterpret_cast<const DT *>(a.tail) + ((int64_t)(b * 2 + 1) * a.H + h) * a.near_cap * D;
+            const int ws = srow[IR_WS];
             float tl = 0.f;
             for (int t = wg; t < tail; t += nw) {
                 const float w = exp2f(tsc[t] - m2);
                 tl += w;
-                const DT *vt = vt0 + (int64_t)t * D;
+                const DT *vt = vt0 + (int64_t)near_slot(a, t, ws) * D;
 #pragma unroll
                 for (int c4 = 0; c4 < D / 32; ++c4)
                     red[lane + 32 * c4] = fmaf(w, to_f32(vt[lane + 32 * c4]), red[lane + 32 * c4]);
@@ -1334,11 +1349,12 @@ template <int BITS, int D> __device__ __forceinline__ void run1_finish(Run1<D> &
 // tail score exceeds it.
 template <int D, typename DT>
 __device__ __forceinline__ void run1_tail(Run1<D> &r, float *red, const int lane, const float (&qreg)[4],
-                                          const float qscale, const DT *kt, const DT *vt0, const int j0,
-                                          const int stride, const int n)
+                                          const DecodeArgs &a, const DT *kt, const DT *vt0, const int ws,
+                                          const int j0, const int stride, const int n)
 {
     for (int j = j0; j < n; j += stride) {
-        const float s2 = near_score<D, DT>(kt + (int64_t)j * D, qreg, qscale, lane);
+        const int slot = near_slot(a, j, ws);
+        const float s2 = near_score<D, DT>(kt + (int64_t)slot * D, qreg, a.qscale, lane);
         if (s2 > r.m) { // warp-uniform
             const float f = ex2(r.m - s2);
             for (int c = lane; c <= D; c += 32)
@@ -1346,7 +1362,7 @@ __device__ __forceinline__ void run1_tail(Run1<D> &r, float *red, const int lane
             r.m = s2;
         }
         const float w = ex2(s2 - r.m);
-        const DT *vt = vt0 + (int64_t)j * D;
+        const DT *vt = vt0 + (int64_t)slot * D;
 #pragma unroll
         for (int c4 = 0; c4 < D / 32; ++c4)
             red[lane + 32 * c4] = fmaf(w, to_f32(vt[lane + 32 * c4]), red[lane + 32 * c4]);
@@ -1530,12 +1546,15 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
             pump(prc_n + spw);
             asm volatile("griddepcontrol.wait;" ::: "memory");
         }
-        if (tail < 0) { // the tail length (an append may have written it)
+        int ws = 0;
+        if (tail < 0) { // near tokens and ring start (an append may have written them)
             tail = a.tail_len[rb];
-            if (tail < 0 || tail > LKV_TAIL_TOKENS) {
+            ws = a.win_start[rb];
+            if (tail < 0 || tail > a.sink + a.wring || ws < 0 || ws >= a.wring) {
                 if (lane == 0 && warp == 0)
                     atomicOr(a.status, LOOPKV_DEV_STATE);
                 tail = 0;
+                ws = 0;
             }
         }
         float qreg[4];
@@ -1566,10 +1585,10 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
         run1_finish<BITS, D>(run, red, lane);
         const int wg = (int)crank * kWarps + warp; // tail token j to warp j mod (C * kWarps) of the cluster
         if (tail > wg) {
-            const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)rb * 2 * a.H + rh) * LKV_TAIL_TOKENS * D;
+            const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)rb * 2 * a.H + rh) * a.near_cap * D;
             const DT *vt0 =
-                reinterpret_cast<const DT *>(a.tail) + ((int64_t)(rb * 2 + 1) * a.H + rh) * LKV_TAIL_TOKENS * D;
-            run1_tail<D, DT>(run, red, lane, qreg, a.qscale, kt, vt0, wg, (int)C * kWarps, tail);
+                reinterpret_cast<const DT *>(a.tail) + ((int64_t)(rb * 2 + 1) * a.H + rh) * a.near_cap * D;
+            run1_tail<D, DT>(run, red, lane, qreg, a, kt, vt0, ws, wg, (int)C * kWarps, tail);
         }
         if (lane == 0)
             red[D + 1] = run.m;
@@ -1764,14 +1783,14 @@ inline ShapeOverride shape_override()
 }
 
 // Shared memory of a kernel with `spw` ring slots per warp.
-template <int BITS, int D> int kernel_smem(bool onepass, int spw, int capw, int nbuf)
+template <int BITS, int D> int kernel_smem(bool onepass, int spw, int capw, int nbuf, int near_cap)
 {
     if (onepass)
         return layout1_ok<BITS, D>(spw, capw) ? smem_layout1<BITS, D>(spw, capw).total : -1;
-    return layout_ok<BITS, D>(spw, capw, nbuf) ? smem_bytes<BITS, D>(spw, capw, nbuf) : -1;
+    return layout_ok<BITS, D>(spw, capw, nbuf, near_cap) ? smem_bytes<BITS, D>(spw, capw, nbuf, near_cap) : -1;
 }
 
-template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_blocks, bool onepass)
+template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_blocks, int near_cap, bool onepass)
 {
     DecodeShape best = {};
     double best_t = 1e300;
@@ -1801,11 +1820,11 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
             for (int nbuf = 1; nbuf <= 2; ++nbuf) {
                 // slots per warp (a power of two): fill the shared memory of `want_ctas` CTAs per SM
                 int spw = 8;
-                while (spw > 2 && kernel_smem<BITS, D>(onepass, spw, capw, nbuf) > budget)
+                while (spw > 2 && kernel_smem<BITS, D>(onepass, spw, capw, nbuf, near_cap) > budget)
                     spw >>= 1;
                 if (ov.stages)
                     spw = ov.stages;
-                const int smem = kernel_smem<BITS, D>(onepass, spw, capw, nbuf);
+                const int smem = kernel_smem<BITS, D>(onepass, spw, capw, nbuf, near_cap);
                 if (smem <= 0 || smem > 227 * 1024)
                     continue;
                 int ncl = 0;
@@ -1850,18 +1869,18 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
 
 }  // namespace
 
-DecodeShape decode_shape(int bits, int D, int dtype, int rows, int max_blocks, bool onepass)
+DecodeShape decode_shape(int bits, int D, int dtype, int rows, int max_blocks, int near_cap, bool onepass)
 {
     const bool bf = dtype == LOOPKV_DTYPE_BF16;
     const int mb = max_blocks;
     if (bits == 4) {
         if (D == 128)
-            return bf ? shape_t<4, 128, __nv_bfloat16>(rows, mb, onepass) : shape_t<4, 128, float>(rows, mb, onepass);
-        return bf ? shape_t<4, 64, __nv_bfloat16>(rows, mb, onepass) : shape_t<4, 64, float>(rows, mb, onepass);
+            return bf ? shape_t<4, 128, __nv_bfloat16>(rows, mb, near_cap, onepass) : shape_t<4, 128, float>(rows, mb, near_cap, onepass);
+        return bf ? shape_t<4, 64, __nv_bfloat16>(rows, mb, near_cap, onepass) : shape_t<4, 64, float>(rows, mb, near_cap, onepass);
     }
     if (D == 128)
-        return bf ? shape_t<2, 128, __nv_bfloat16>(rows, mb, onepass) : shape_t<2, 128, float>(rows, mb, onepass);
-    return bf ? shape_t<2, 64, __nv_bfloat16>(rows, mb, onepass) : shape_t<2, 64, float>(rows, mb, onepass);
+        return bf ? shape_t<2, 128, __nv_bfloat16>(rows, mb, near_cap, onepass) : shape_t<2, 128, float>(rows, mb, near_cap, onepass);
+    return bf ? shape_t<2, 64, __nv_bfloat16>(rows, mb, near_cap, onepass) : shape_t<2, 64, float>(rows, mb, near_cap, onepass);
 }
 
 int launch_decode(const DecodeArgs &a, int bits, int D, int dtype, const DecodeShape &shp, bool pdl, cudaStream_t s)

@@ -15,14 +15,17 @@ struct DevState {
     uint32_t *status;     // [1] LOOPKV_DEV_* bits
     int32_t *ctrl;        // [8] per-call control words (ingest admission flag)
     int32_t *hist_len;    // [n_cells][max_batch]
-    int32_t *tail_len;    // [n_cells][max_batch]
+    int32_t *tail_len;    // [n_cells][max_batch] near tokens (sink fill + window length)
+    int32_t *win_start;   // [n_cells][max_batch] window ring slot of the oldest window token
     int32_t *block_table; // [n_cells][max_batch][max_blocks]
     int32_t *free4;       // free stack of the 4-bit pool, ids [0, n4)
     int32_t *top4;        // number of free ids in free4
     int32_t *free2;
     int32_t *top2;
     int64_t n4, n2;       // pool capacities in blocks
-    uint8_t *tail;        // [n_cells][max_batch][2][H][32][D] elements of in_dtype
+    uint8_t *tail;        // [n_cells][max_batch][2][H][near_cap][D] elements of in_dtype
+    int sink, wring;      // sink slots, window ring slots (window_tokens + 32)
+    int near_cap;         // sink + wring
     uint8_t *main4;       // [n4][H][LKV_HEAD_MAIN_4B(D)]
     uint8_t *lo4;         // [n4][H][LKV_HEAD_LO_4B(D)]
     uint8_t *main2;       // [n2][H][LKV_HEAD_MAIN_2B(D)]
@@ -36,8 +39,9 @@ struct DecodeArgs {
     const uint8_t *lo;          // lo pool (4-bit sources)
     const int32_t *block_table; // source cell [max_batch][max_blocks]
     const int32_t *hist_len;    // source cell [max_batch]
-    const int32_t *tail_len;    // own cell [max_batch]
-    const uint8_t *tail;        // own cell [max_batch][2][H][32][D]
+    const int32_t *tail_len;    // own cell [max_batch] near tokens
+    const int32_t *win_start;   // own cell [max_batch] ring slot of the oldest window token
+    const uint8_t *tail;        // own cell [max_batch][2][H][near_cap][D]
     uint32_t *status;
     uint32_t *s_bitmap;         // optional [B][H][bitmap_words]
     float *row_max;             // optional [B][H]
@@ -51,6 +55,7 @@ struct DecodeArgs {
     float qscale;               // log2(e) / sqrt(D)
     float tau;
     int tau_mode;
+    int sink, wring, near_cap;  // near region geometry (see DevState)
     unsigned long long wait_ns; // limit of every bounded wait, in nanoseconds
     int inject;                 // LOOPKV_INJECT_*: LOOPKV_INJECT_NONE in normal operation
 };
@@ -77,7 +82,7 @@ int launch_decode(const DecodeArgs &a, int bits, int D, int dtype, const DecodeS
                   cudaStream_t s);
 // onepass: the rows' refine set does not depend on the row maximum (2-bit source, or a
 // 4-bit source read with tau <= 0), so the single-pass kernel may read them.
-DecodeShape decode_shape(int bits, int D, int dtype, int rows, int max_blocks, bool onepass);
+DecodeShape decode_shape(int bits, int D, int dtype, int rows, int max_blocks, int near_cap, bool onepass);
 
 int launch_init_state(const DevState &st, cudaStream_t s);
 int launch_append(const DevState &st, int cell, int H, int D, int dtype, int max_batch, const void *k,

@@ -248,6 +248,13 @@ __device__ void quant_into_blocks(const DevState &st, int bits, int H, int h, co
     }
 }
 
+// Slot of near token j (arrival order among the tokens held) of a (cell, request): the
+// sink slots first, then the window ring of st.wring slots from its oldest token.
+__device__ __forceinline__ int near_slot(const DevState &st, int j, int win_start)
+{
+    return j < st.sink ? j : st.sink + (win_start + (j - st.sink)) % st.wring;
+}
+
 __global__ void init_state_kernel(DevState st)
 {
     int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -277,7 +284,7 @@ __global__ void append_kernel(DevState st, int cell, int H, int D, int max_batch
             atomicOr(st.status, LOOPKV_DEV_STATE);
         } else {
             pos = st.tail_len[(int64_t)cell * max_batch + req];
-            if (pos >= LKV_TAIL_TOKENS || pos < 0) {
+            if (pos >= st.sink + st.wring || pos < 0) { // window full: flush first
                 atomicOr(st.status, LOOPKV_DEV_TAIL_FULL);
                 pos = -1;
             }
@@ -288,19 +295,22 @@ __global__ void append_kernel(DevState st, int cell, int H, int D, int max_batch
     const int pos = s_pos;
     if (pos < 0)
         return;
-    DT *tail = reinterpret_cast<DT *>(st.tail) + ((int64_t)cell * max_batch + req) * 2 * H * 32 * D;
+    const int slot = near_slot(st, pos, st.win_start[(int64_t)cell * max_batch + req]);
+    const int NC = st.near_cap;
+    DT *tail = reinterpret_cast<DT *>(st.tail) + ((int64_t)cell * max_batch + req) * 2 * H * NC * D;
     const int64_t HD = (int64_t)H * D;
     for (int64_t e = threadIdx.x; e < HD; e += blockDim.x) {
         int h = (int)(e / D), c = (int)(e % D);
-        tail[((int64_t)h * 32 + pos) * D + c] = k[(int64_t)bi * HD + e];
-        tail[((int64_t)(H + h) * 32 + pos) * D + c] = v[(int64_t)bi * HD + e];
+        tail[((int64_t)h * NC + slot) * D + c] = k[(int64_t)bi * HD + e];
+        tail[((int64_t)(H + h) * NC + slot) * D + c] = v[(int64_t)bi * HD + e];
     }
     __syncthreads();
     if (threadIdx.x == 0)
         st.tail_len[(int64_t)cell * max_batch + req] = pos + 1;
 }
 
-// One CTA per (cell, request): a tail holding 32 tokens becomes two new blocks.
+// One CTA per (cell, request): the oldest 32 tokens of a window holding W + 32 become two
+// new blocks (the window ring's oldest page, contiguous in the ring).
 template <int D, typename DT>
 __global__ void __launch_bounds__(kQThreads) flush_kernel(DevState st, const uint8_t *modes, int H, int max_batch,
                                                           int max_blocks)
@@ -311,10 +321,11 @@ __global__ void __launch_bounds__(kQThreads) flush_kernel(DevState st, const uin
     const int cell = blockIdx.x / max_batch, req = blockIdx.x % max_batch;
     int32_t *tl = st.tail_len + (int64_t)cell * max_batch + req;
     int32_t *hl = st.hist_len + (int64_t)cell * max_batch + req;
+    int32_t *ws = st.win_start + (int64_t)cell * max_batch + req;
     const int mode = modes[cell];
     if (threadIdx.x == 0) {
         int go = 0;
-        if (*tl == LKV_TAIL_TOKENS) {
+        if (*tl == st.sink + st.wring) {
             int nb = *hl / LKV_BLOCK_TOKENS;
             if (nb + 2 > max_blocks) {
                 atomicOr(st.status, LOOPKV_DEV_STATE);
@@ -340,26 +351,27 @@ __global__ void __launch_bounds__(kQThreads) flush_kernel(DevState st, const uin
         return;
     if (go == 1) {
         const int bits = mode == LOOPKV_CELL_4B ? 4 : 2;
-        const DT *tail = reinterpret_cast<const DT *>(st.tail) + ((int64_t)cell * max_batch + req) * 2 * H * 32 * D;
+        const int NC = st.near_cap, slot0 = st.sink + *ws;
+        const DT *tail = reinterpret_cast<const DT *>(st.tail) + ((int64_t)cell * max_batch + req) * 2 * H * NC * D;
         for (int h = 0; h < H; ++h)
-            quant_into_blocks<D, DT>(st, bits, H, h, s_ids, tail + (int64_t)h * 32 * D,
-                                     tail + (int64_t)(H + h) * 32 * D, D, kc_smem);
+            quant_into_blocks<D, DT>(st, bits, H, h, s_ids, tail + ((int64_t)h * NC + slot0) * D,
+                                     tail + ((int64_t)(H + h) * NC + slot0) * D, D, kc_smem);
     }
     __syncthreads();
     if (threadIdx.x == 0) {
         *hl = *hl + LKV_GROUP;
-        *tl = 0;
+        *tl = *tl - LKV_GROUP;
+        *ws = (*ws + LKV_GROUP) % st.wring;
     }
 }
 
 // Ingest, step 1 (one thread): admit the (cell, request) if empty, take its blocks,
 // set its lengths.  ctrl[0] = 1 admits the following ingest kernels.
 __global__ void ingest_prep_kernel(DevState st, int cell, int mode, int D, int max_batch, int max_blocks, int req,
-                                   int T)
+                                   int T, int ngroups)
 {
     int32_t *tl = st.tail_len + (int64_t)cell * max_batch + req;
     int32_t *hl = st.hist_len + (int64_t)cell * max_batch + req;
-    const int ngroups = T / LKV_GROUP;
     st.ctrl[0] = 0;
     if (*tl != 0 || *hl != 0 || 2 * ngroups > max_blocks) {
         atomicOr(st.status, LOOPKV_DEV_STATE);
@@ -379,7 +391,8 @@ __global__ void ingest_prep_kernel(DevState st, int cell, int mode, int D, int m
             bt[i] = p.free_ids[old - 1 - i];
     }
     *hl = ngroups * LKV_GROUP;
-    *tl = T % LKV_GROUP;
+    *tl = T - ngroups * LKV_GROUP; // sink fill + window length
+    st.win_start[(int64_t)cell * max_batch + req] = 0;
     st.ctrl[0] = 1;
 }
 
@@ -387,7 +400,7 @@ __global__ void ingest_prep_kernel(DevState st, int cell, int mode, int D, int m
 template <int D, typename DT>
 __global__ void __launch_bounds__(kQThreads) ingest_quant_kernel(DevState st, int cell, int mode, int H,
                                                                  int max_batch, int max_blocks, int req,
-                                                                 const DT *k, const DT *v)
+                                                                 const DT *k, const DT *v, int t0)
 {
     __shared__ __align__(16) uint8_t kc_smem[32 * D];
     if (st.ctrl[0] != 1)
@@ -396,27 +409,30 @@ __global__ void __launch_bounds__(kQThreads) ingest_quant_kernel(DevState st, in
     const int32_t *bt = st.block_table + ((int64_t)cell * max_batch + req) * max_blocks;
     int32_t ids[2] = {bt[2 * g], bt[2 * g + 1]};
     const int64_t tok = (int64_t)H * D;
-    const int64_t off = (int64_t)g * LKV_GROUP * tok + (int64_t)h * D;
+    const int64_t off = ((int64_t)t0 + (int64_t)g * LKV_GROUP) * tok + (int64_t)h * D; // pages start after the sink
     quant_into_blocks<D, DT>(st, mode == LOOPKV_CELL_4B ? 4 : 2, H, h, ids, k + off, v + off, tok, kc_smem);
 }
 
-// Ingest, step 3: the last T mod 32 tokens go to the tail.
+// Ingest, step 3: the unquantized tokens go to the near region: the first sf (sink) to
+// slots 0..sf-1, the last nw (window) to the ring from its slot 0.
 template <typename DT>
 __global__ void ingest_tail_kernel(DevState st, int cell, int H, int D, int max_batch, int req, const DT *k,
-                                   const DT *v, int T)
+                                   const DT *v, int T, int sf, int nw)
 {
     if (st.ctrl[0] != 1)
         return;
-    const int n = T % LKV_GROUP, t0 = T - n;
-    DT *tail = reinterpret_cast<DT *>(st.tail) + ((int64_t)cell * max_batch + req) * 2 * H * 32 * D;
+    const int NC = st.near_cap;
+    DT *tail = reinterpret_cast<DT *>(st.tail) + ((int64_t)cell * max_batch + req) * 2 * H * NC * D;
     const int64_t HD = (int64_t)H * D;
-    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < (int64_t)n * HD;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < (int64_t)(sf + nw) * HD;
          e += (int64_t)gridDim.x * blockDim.x) {
-        int t = (int)(e / HD);
-        int64_t r = e % HD;
-        int h = (int)(r / D), c = (int)(r % D);
-        tail[((int64_t)h * 32 + t) * D + c] = k[(int64_t)(t0 + t) * HD + r];
-        tail[((int64_t)(H + h) * 32 + t) * D + c] = v[(int64_t)(t0 + t) * HD + r];
+        const int j = (int)(e / HD); // near token j: sink token j, or window token j - sf
+        const int64_t r = e % HD;
+        const int h = (int)(r / D), c = (int)(r % D);
+        const int t = j < sf ? j : T - nw + (j - sf);
+        const int slot = j < sf ? j : st.sink + (j - sf);
+        tail[((int64_t)h * NC + slot) * D + c] = k[(int64_t)t * HD + r];
+        tail[((int64_t)(H + h) * NC + slot) * D + c] = v[(int64_t)t * HD + r];
     }
 }
 
@@ -444,6 +460,7 @@ __global__ void reset_kernel(DevState st, const uint8_t *modes, int n_cells, int
     }
     *hl = 0;
     *tl = 0;
+    st.win_start[(int64_t)cell * max_batch + req] = 0;
 }
 
 }  // namespace
@@ -495,13 +512,19 @@ template <int D, typename DT>
 static void ingest_dispatch(const DevState &st, int cell, int mode, int H, int max_batch, int max_blocks, int req,
                             const void *k, const void *v, int T, cudaStream_t s)
 {
-    const int ngroups = T / LKV_GROUP;
-    ingest_prep_kernel<<<1, 1, 0, s>>>(st, cell, mode, D, max_batch, max_blocks, req, T);
+    // sink sf = min(T, sink); of the rest R, 32 * floor((R - W) / 32) pages (none if R < W),
+    // then the window
+    const int W = st.wring - LKV_GROUP;
+    const int sf = T < st.sink ? T : st.sink, R = T - sf;
+    const int ngroups = R >= W ? (R - W) / LKV_GROUP : 0;
+    const int nw = R - ngroups * LKV_GROUP;
+    ingest_prep_kernel<<<1, 1, 0, s>>>(st, cell, mode, D, max_batch, max_blocks, req, T, ngroups);
     if (mode != LOOPKV_CELL_SHARE && ngroups > 0)
         ingest_quant_kernel<D, DT><<<dim3(ngroups, H), kQThreads, 0, s>>>(st, cell, mode, H, max_batch, max_blocks,
-                                                                         req, (const DT *)k, (const DT *)v);
-    if (T % LKV_GROUP)
-        ingest_tail_kernel<DT><<<64, 256, 0, s>>>(st, cell, H, D, max_batch, req, (const DT *)k, (const DT *)v, T);
+                                                                         req, (const DT *)k, (const DT *)v, sf);
+    if (sf + nw > 0)
+        ingest_tail_kernel<DT><<<64, 256, 0, s>>>(st, cell, H, D, max_batch, req, (const DT *)k, (const DT *)v, T,
+                                                  sf, nw);
 }
 
 int launch_ingest(const DevState &st, int cell, int mode, int H, int D, int dtype, int max_batch, int max_blocks,

@@ -29,6 +29,9 @@ struct loopkv_plan {
     }
 };
 
+// Unquantized slots per (cell, request): the sink, then a window ring of window + 32.
+static int near_cap(const loopkv_config &c) { return c.sink_tokens + c.window_tokens + 32; }
+
 struct loopkv_cache {
     loopkv_plan plan;
     // Host bookkeeping shared by calls from several host threads, under `mu`:
@@ -64,8 +67,8 @@ struct loopkv_cache {
         auto key = std::make_tuple(bits, B, onepass);
         auto it = shapes.find(key);
         if (it == shapes.end())
-            it = shapes.emplace(key, lkv::decode_shape(bits, plan.cfg.head_dim, plan.cfg.in_dtype,
-                                                       B * plan.cfg.n_heads, plan.cfg.max_blocks_per_seq, onepass))
+            it = shapes.emplace(key, lkv::decode_shape(bits, plan.cfg.head_dim, plan.cfg.in_dtype, B * plan.cfg.n_heads,
+                                                       plan.cfg.max_blocks_per_seq, near_cap(plan.cfg), onepass))
                      .first;
         return it->second;
     }
@@ -105,11 +108,15 @@ int check_config(const loopkv_config *c)
         return LOOPKV_ERR_INVALID_ARG;
     if ((int64_t)c->n_heads * c->max_batch > 65535)
         return LOOPKV_ERR_SHAPE;
+    if (c->sink_tokens < 0 || c->sink_tokens > 64 || c->sink_tokens % 32 || c->window_tokens < 0 ||
+        c->window_tokens > 512 || c->window_tokens % 32)
+        return LOOPKV_ERR_SHAPE;
     return LOOPKV_OK;
 }
 
 struct Layout {
-    size_t status, ctrl, reqs, hist, tail_len, table, free4, top4, free2, top2, tail, main4, lo4, main2, modes, end;
+    size_t status, ctrl, reqs, hist, tail_len, win_start, table, free4, top4, free2, top2, tail, main4, lo4, main2, modes,
+        end;
     int64_t n4, n2;
 };
 
@@ -130,6 +137,8 @@ Layout layout(const loopkv_plan &p, int64_t n4, int64_t n2)
     o = align_up(o + 4 * cells * c.max_batch);
     L.tail_len = o;
     o = align_up(o + 4 * cells * c.max_batch);
+    L.win_start = o;
+    o = align_up(o + 4 * cells * c.max_batch);
     L.table = o;
     o = align_up(o + 4 * cells * c.max_batch * (int64_t)c.max_blocks_per_seq);
     L.modes = o;
@@ -143,7 +152,7 @@ Layout layout(const loopkv_plan &p, int64_t n4, int64_t n2)
     L.top2 = o;
     o = align_up(o + 4);
     L.tail = o;
-    o = align_up(o + (size_t)cells * c.max_batch * 2 * c.n_heads * 32 * c.head_dim * dtype_size(c.in_dtype));
+    o = align_up(o + (size_t)cells * c.max_batch * 2 * c.n_heads * near_cap(c) * c.head_dim * dtype_size(c.in_dtype));
     L.main4 = o;
     o = align_up(o + (size_t)n4 * c.n_heads * LKV_HEAD_MAIN_4B(c.head_dim));
     L.lo4 = o;
@@ -369,6 +378,10 @@ int loopkv_alloc(const loopkv_plan *plan, void *dev_buf, size_t dev_bytes, void 
     st.ctrl = reinterpret_cast<int32_t *>(b + L.ctrl);
     st.hist_len = reinterpret_cast<int32_t *>(b + L.hist);
     st.tail_len = reinterpret_cast<int32_t *>(b + L.tail_len);
+    st.win_start = reinterpret_cast<int32_t *>(b + L.win_start);
+    st.sink = plan->cfg.sink_tokens;
+    st.wring = plan->cfg.window_tokens + 32;
+    st.near_cap = near_cap(plan->cfg);
     st.block_table = reinterpret_cast<int32_t *>(b + L.table);
     st.free4 = reinterpret_cast<int32_t *>(b + L.free4);
     st.top4 = reinterpret_cast<int32_t *>(b + L.top4);
@@ -495,7 +508,11 @@ int loopkv_decode_debug(const loopkv_plan *plan, int loop, int layer, const void
     a.block_table = cache->st.block_table + (int64_t)src * cp.cfg.max_batch * MB;
     a.hist_len = cache->st.hist_len + (int64_t)src * cp.cfg.max_batch;
     a.tail_len = cache->st.tail_len + (int64_t)cell * cp.cfg.max_batch;
-    a.tail = cache->st.tail + (size_t)cell * cp.cfg.max_batch * 2 * H * 32 * D * cache->esz;
+    a.win_start = cache->st.win_start + (int64_t)cell * cp.cfg.max_batch;
+    a.tail = cache->st.tail + (size_t)cell * cp.cfg.max_batch * 2 * H * cache->st.near_cap * D * cache->esz;
+    a.sink = cache->st.sink;
+    a.wring = cache->st.wring;
+    a.near_cap = cache->st.near_cap;
     a.status = cache->st.status;
     a.s_bitmap = s_bitmap;
     a.row_max = row_max;
@@ -588,7 +605,9 @@ int loopkv_cell_view_get(const loopkv_cache *cache, int loop, int layer, loopkv_
     out->block_table = cache->st.block_table + (int64_t)src * p.cfg.max_batch * MB;
     out->hist_len = cache->st.hist_len + (int64_t)src * p.cfg.max_batch;
     out->tail_len = cache->st.tail_len + (int64_t)cell * p.cfg.max_batch;
-    out->tail = cache->st.tail + (size_t)cell * p.cfg.max_batch * 2 * H * 32 * D * cache->esz;
+    out->win_start = cache->st.win_start + (int64_t)cell * p.cfg.max_batch;
+    out->tail = cache->st.tail + (size_t)cell * p.cfg.max_batch * 2 * H * cache->st.near_cap * D * cache->esz;
+    out->near_cap = cache->st.near_cap;
     out->pool_blocks = bits == 4 ? cache->st.n4 : cache->st.n2;
     return LOOPKV_OK;
 }
@@ -601,7 +620,7 @@ int loopkv_decode_shape(const loopkv_plan *plan, int B, int *cluster_size, int *
         return LOOPKV_ERR_NO_DEVICE; // the shape comes from an occupancy query of the device
     // the shape of a 4-bit source cell (the larger pipeline stage) under the plan's tau
     lkv::DecodeShape shp = lkv::decode_shape(4, plan->cfg.head_dim, plan->cfg.in_dtype, B * plan->cfg.n_heads,
-                                             plan->cfg.max_blocks_per_seq, single_pass(4, plan->tau));
+                                             plan->cfg.max_blocks_per_seq, near_cap(plan->cfg), single_pass(4, plan->tau));
     if (cluster_size)
         *cluster_size = shp.cluster;
     if (ctas)

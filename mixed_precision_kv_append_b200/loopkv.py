@@ -49,7 +49,7 @@ class LoopKVError(RuntimeError):
 class Config(ctypes.Structure):
     _fields_ = [("n_layers", ctypes.c_int), ("n_loops", ctypes.c_int), ("n_heads", ctypes.c_int),
                 ("head_dim", ctypes.c_int), ("max_batch", ctypes.c_int), ("max_blocks_per_seq", ctypes.c_int),
-                ("in_dtype", ctypes.c_int)]
+                ("in_dtype", ctypes.c_int), ("sink_tokens", ctypes.c_int), ("window_tokens", ctypes.c_int)]
 
 
 class ByteReport(ctypes.Structure):
@@ -67,8 +67,8 @@ class CellView(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int), ("src_cell", ctypes.c_int), ("src_mode", ctypes.c_int),
                 ("head_main_bytes", ctypes.c_int), ("head_lo_bytes", ctypes.c_int),
                 ("main_pool", ctypes.c_void_p), ("lo_pool", ctypes.c_void_p), ("block_table", ctypes.c_void_p),
-                ("hist_len", ctypes.c_void_p), ("tail_len", ctypes.c_void_p), ("tail", ctypes.c_void_p),
-                ("pool_blocks", ctypes.c_int64)]
+                ("hist_len", ctypes.c_void_p), ("tail_len", ctypes.c_void_p), ("win_start", ctypes.c_void_p),
+                ("tail", ctypes.c_void_p), ("near_cap", ctypes.c_int), ("pool_blocks", ctypes.c_int64)]
 
 
 _lib = None
@@ -266,9 +266,10 @@ class Plan:
     """A plan: config + one storage mode per (loop, layer) cell + tau (host object)."""
 
     def __init__(self, n_layers, n_loops, n_heads, head_dim, max_batch, max_blocks_per_seq, modes, tau,
-                 tau_mode=TAU_REL_MAX, in_dtype=torch.bfloat16):
+                 tau_mode=TAU_REL_MAX, in_dtype=torch.bfloat16, sink_tokens=0, window_tokens=0):
         self.cfg = Config(n_layers, n_loops, n_heads, head_dim, max_batch, max_blocks_per_seq,
-                          _dtype_code(in_dtype))
+                          _dtype_code(in_dtype), sink_tokens, window_tokens)
+        self.sink, self.window = sink_tokens, window_tokens
         self.in_dtype = in_dtype
         self.modes = [int(m) for m in modes]
         self.tau = float(tau)
@@ -358,7 +359,8 @@ class Cache:
         return self.buf[off: off + nbytes]
 
     def lengths(self, loop, layer) -> tuple[torch.Tensor, torch.Tensor]:
-        """(history lengths of the source cell, tail lengths of this cell), [max_batch] int32 on host."""
+        """(history lengths of the source cell, near (sink + window) token counts of this cell),
+        [max_batch] int32 on host."""
         v = self.cell_view(loop, layer)
         mb = self.plan.cfg.max_batch
         h = self._slice(v.hist_len, 4 * mb).view(torch.int32).cpu()
@@ -390,13 +392,25 @@ class Cache:
         return main, lo
 
     def tail(self, loop, layer, req) -> torch.Tensor:
-        """Unquantized tail of this cell for `req`: [2][H][32][D] in the input dtype (device view)."""
+        """Unquantized near slots of this cell for `req`: [2][H][near_cap][D] in the input dtype
+        (device view): the sink slots, then the window ring."""
         v = self.cell_view(loop, layer)
         c = self.plan.cfg
         esz = 2 if self.plan.in_dtype == torch.bfloat16 else 4
-        per = 2 * c.n_heads * 32 * c.head_dim * esz
+        per = 2 * c.n_heads * v.near_cap * c.head_dim * esz
         t = self._slice(v.tail + req * per, per)
-        return t.view(self.plan.in_dtype).view(2, c.n_heads, 32, c.head_dim)
+        return t.view(self.plan.in_dtype).view(2, c.n_heads, v.near_cap, c.head_dim)
+
+    def near_tokens(self, loop, layer, req) -> torch.Tensor:
+        """The near tokens of this cell for `req` in arrival order: [2][H][n][D] (a copy): sink first,
+        then the window from its oldest token."""
+        v = self.cell_view(loop, layer)
+        mb = self.plan.cfg.max_batch
+        n = int(self._slice(v.tail_len, 4 * mb).view(torch.int32)[req])
+        ws = int(self._slice(v.win_start, 4 * mb).view(torch.int32)[req])
+        S, WR = self.plan.sink, self.plan.window + 32
+        slots = [j if j < S else S + (ws + j - S) % WR for j in range(n)]
+        return self.tail(loop, layer, req)[:, :, slots].clone()
 
     def close(self):
         if self.handle:

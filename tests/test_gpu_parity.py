@@ -19,19 +19,21 @@ pytestmark = pytest.mark.gpu
 BITS = {L.CELL_4B: 4, L.CELL_2B: 2}
 
 
-def _plan(n_layers, n_loops, H, D, B, max_blocks, modes, tau, tau_mode=L.TAU_REL_MAX, dtype=torch.bfloat16):
-    return L.Plan(n_layers, n_loops, H, D, B, max_blocks, modes, tau, tau_mode, dtype)
+def _plan(n_layers, n_loops, H, D, B, max_blocks, modes, tau, tau_mode=L.TAU_REL_MAX, dtype=torch.bfloat16, sink=0,
+          window=0):
+    return L.Plan(n_layers, n_loops, H, D, B, max_blocks, modes, tau, tau_mode, dtype, sink, window)
 
 
 class Model:
     """A small cache plus the raw token history of every (cell, request), as the oracle sees it."""
 
-    def __init__(self, w: synth.Workload, max_blocks=None, tau=None, tau_mode=None):
+    def __init__(self, w: synth.Workload, max_blocks=None, tau=None, tau_mode=None, sink=0, window=0):
         self.w = w
         self.tau = w.tau if tau is None else tau
         self.tau_mode = w.tau_mode if tau_mode is None else tau_mode
+        self.sink = sink
         self.plan = _plan(w.n_layers, w.n_loops, w.H, w.D, w.B, max_blocks or w.max_blocks, w.modes, self.tau,
-                          self.tau_mode, w.dtype)
+                          self.tau_mode, w.dtype, sink, window)
         self.cache = L.Cache(self.plan)
         self.tokens = {}  # (cell, req) -> (K [n, H, D] float32, V)
         self._hist_cache = {}
@@ -71,12 +73,21 @@ class Model:
         self._hist_cache.clear()
 
     def head_history(self, cell, req, h, n_hist):
+        """Quantized history of a head: the n_hist tokens after the sink."""
         key = (cell, req, h, n_hist)
         if key not in self._hist_cache:
             K, V = self.tokens[(cell, req)]
-            self._hist_cache[key] = O.HeadHistory(K[:n_hist, h], V[:n_hist, h], BITS[self.w.modes[cell]]) \
+            S = self.sink
+            self._hist_cache[key] = O.HeadHistory(K[S:S + n_hist, h], V[S:S + n_hist, h], BITS[self.w.modes[cell]]) \
                 if n_hist else None
         return self._hist_cache[key]
+
+    def raw_tokens(self, K, V, n_hist, n_near):
+        """The unquantized tokens of a sequence: the sink, then the window after the history."""
+        if n_hist == 0:
+            return K[:n_near], V[:n_near]
+        S = self.sink
+        return np.concatenate([K[:S], K[S + n_hist:]]), np.concatenate([V[:S], V[S + n_hist:]])
 
     def check_cell(self, loop, layer, q, rows=None, where=""):
         """Decode cell (loop, layer) on the GPU and compare the given (req, head) rows."""
@@ -95,8 +106,9 @@ class Model:
             n_own = K.shape[0]
             assert n_own == n_hist + n_tail, (n_own, n_hist, n_tail)
             hh = self.head_history(s, req, h, n_hist)
+            Kr, Vr = self.raw_tokens(K, V, n_hist, n_tail)
             err, nt = check_row(out[req, h], bm[req, h], rm[req, h], rs[req, h], qn[req, h].astype(np.float64),
-                                hh, K[n_hist:, h], V[n_hist:, h], self.tau, self.tau_mode,
+                                hh, Kr[:, h], Vr[:, h], self.tau, self.tau_mode,
                                 where=f"{where} cell ({loop},{layer}) req {req} head {h}")
             worst, ties = max(worst, err), ties + nt
         return worst, ties
@@ -460,3 +472,59 @@ def test_flush_then_decode_without_append(graph):
             again = m.cache.decode(lp, la, qs[(lp, la)])
             assert torch.equal(ref, again)
             m.check_cell(lp, la, qs[(lp, la)], where=f"flush then decode graph={graph}")
+
+
+@pytest.mark.parametrize("sink,window", [(32, 64), (32, 256), (0, 96)])
+def test_sink_window_sequence(sink, window):
+    """Sink and window stay unquantized (LoopKV §2.3, §3.4): requests whose tokens are all in the
+    sink, that have a window but no history, and that have history between sink and window;
+    appends fill the window ring and each flush quantizes its oldest page.  Packed pages are
+    bit-exact with the oracle's quantization of the tokens after the sink, decodes match."""
+    modes = [L.CELL_4B, L.CELL_SHARE, L.CELL_2B, L.CELL_4B]  # loop 0: [4b, share], loop 1: [2b, 4b]
+    w = synth.Workload("sinkwin", 2, 2, 4, 128, 3, [20, sink + window + 4, 600], torch.bfloat16, modes, 0.02,
+                       append_steps=80, seed=31)
+    m = Model(w, sink=sink, window=window)
+    m.ingest()
+    for lp in range(2):
+        for la in range(2):
+            m.check_cell(lp, la, _q(w, 0, la, lp), where=f"ingest s={sink} w={window}")
+    for step in range(80):
+        m.append_step(step)
+        if step % 17 == 0 or step in (31, 32, 33, 79):
+            for la in range(2):
+                for lp in range(2):
+                    m.check_cell(lp, la, _q(w, step, la, lp), where=f"s={sink} w={window} step {step}")
+    m.cache.check("sink/window sequence")
+    for la in range(2):
+        for lp in range(2):
+            c = m.cell(lp, la)
+            if modes[c] != L.CELL_SHARE:
+                m.check_bytes(lp, la)
+            hist, near = m.cache.lengths(lp, la)
+            for req in range(w.B):
+                n = w.lengths[req] + 80
+                h, nn = int(hist[req]), int(near[req])
+                assert h + nn == n and h % 32 == 0
+                if h:
+                    assert sink + window <= nn <= sink + window + 32  # a full window is flushed at the next step
+                # the near slots hold exactly the sink and the window, in arrival order
+                K, _ = m.tokens[(c, req)]
+                Kr, _ = m.raw_tokens(K, K, h, nn)
+                got = f32(m.cache.near_tokens(lp, la, req)[0]).transpose(1, 0, 2)
+                assert np.array_equal(got, Kr.astype(np.float32)), (lp, la, req)
+
+
+def test_sink_window_ouro_shape():
+    """The paper's geometry (32-token sink, 256-token window) at Ouro-1.4B head shape, 8K
+    context, sampled rows of a 4-bit, a share and a 2-bit cell, tau = 0.01."""
+    w = synth.Workload("sinkwin_8k", 1, 4, 16, 128, 4, [8192, 8000, 5000, 300], torch.bfloat16, [0, 1, 2, 0], 0.01,
+                       append_steps=40, seed=37)
+    m = Model(w, sink=32, window=256)
+    m.ingest()
+    for s in range(40):
+        m.append_step(s)
+    rng = np.random.default_rng(3)
+    for lp in range(4):
+        rows = [(int(rng.integers(4)), int(rng.integers(16))) for _ in range(6)] + [(3, 15), (0, 0)]
+        m.check_cell(lp, 0, _q(w, 40, 0, lp), rows=rows, where="sink/window 8K")
+    m.check_bytes(0, 0, reqs=[0, 2], heads=[0, 9])
