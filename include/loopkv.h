@@ -74,8 +74,18 @@ typedef enum {
 
 /* Which weight the threshold tau is compared with (LoopKV paper, §3.3). */
 typedef enum {
-    LOOPKV_TAU_REL_MAX = 0, /* hot iff exp(s_t - m) >= tau, m = exact row max (default) */
-    LOOPKV_TAU_ABS_PROB = 1 /* hot iff exp(s_t - m) / sum_u exp(s_u - m) >= tau */
+    LOOPKV_TAU_REL_MAX = 0,  /* hot iff exp(s_t - m) >= tau, m = exact row max (default) */
+    LOOPKV_TAU_ABS_PROB = 1, /* hot iff exp(s_t - m) / sum_u exp(s_u - m) >= tau */
+    /* The paper's streaming rule (§3.3: the reader tests tokens against a running maximum
+     * that starts at a seed, the sink maximum).  Each reading warp takes its 32-token groups
+     * in order; the running maximum starts at the row's largest sink score (minus infinity
+     * without a sink) and takes each group's largest score before that group's tokens are
+     * tested: hot iff exp(s_t - m_run) >= tau.  A superset of the REL_MAX set; which tokens
+     * it adds depends on the split of the row over the reading warps (group g of the row is
+     * read by CTA g mod C of the cluster, as its local group g / C, and local group i by warp
+     * i mod 4 in increasing i; C from loopkv_decode_shape).  The seed travels with the row
+     * statistics the cluster exchanges anyway, so no reader waits for it. */
+    LOOPKV_TAU_STREAM = 2
 } loopkv_tau_mode;
 
 /* Element type of q, k, v inputs and of the unquantized tail. */

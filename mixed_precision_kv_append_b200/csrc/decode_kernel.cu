@@ -371,7 +371,7 @@ struct Smem {
                        // [D/32][40 words] (overwritten in place by the value digit records)
                        // and 2^-F during a V stage, the warp's partial o and l [D + 1] at
                        // the end of a V pass
-    float *stat;       // [3][kWarps][2] per-warp (max, sum exp(s - max)), by row index mod 3
+    float *stat;       // [3][kWarps][4] per-warp (max, sum exp(s - max), sink max, -), by row index mod 3
     float *part;       // [2][D + 1] CTA partial o and l of a row, by row parity
     int32_t *ids;      // [3][kWarps][2 * capw] block ids of a warp's groups, by row index mod 3
     int32_t *irow;     // [3][kWarps][IR_N] row parameters and issuer state, by row index mod 3
@@ -379,7 +379,7 @@ struct Smem {
 };
 
 // Fields of a row slot (Smem::irow).
-enum { IR_ROW = 0, IR_B, IR_H, IR_N, IR_TAIL, IR_VFIRST, IR_VISSUED, IR_THR, IR_WS, IR_N_FIELDS = 12 };
+enum { IR_ROW = 0, IR_B, IR_H, IR_N, IR_TAIL, IR_VFIRST, IR_VISSUED, IR_THR, IR_WS, IR_RUN, IR_N_FIELDS = 12 };
 
 // Byte offsets of the shared-memory regions; every region starts on a 16-byte boundary
 // (digit records, weights and stage data are read with 16-byte vector loads).
@@ -415,7 +415,7 @@ __host__ __device__ constexpr SmemLayout smem_layout(int spw, int capw, int nbuf
     L.scr = o;
     o = align16(o + kWarps * scratch_bytes<D>());
     L.stat = o;
-    o = align16(o + 3 * kWarps * 2 * 4);
+    o = align16(o + 3 * kWarps * 4 * 4);
     L.part = o;
     o = align16(o + 2 * (D + 1) * 4);
     L.ids = o;
@@ -491,15 +491,18 @@ __device__ __forceinline__ void segment(int sig, int nrows, bool seq, bool &is_v
     }
 }
 
-// Row max m (log2 units) and, for the normalised rule, l = sum_t 2^(s_t - m), from the
-// per-warp pairs of every CTA of the cluster.  Lane j < C * kWarps fetches pair j; the
-// warp reductions give every lane the same m and l.
-__device__ __forceinline__ void cluster_row_stats(const float *stat, uint32_t C, int lane, float &m, float &l)
+// Row max m (log2 units), for the normalised rule l = sum_t 2^(s_t - m), and the largest
+// sink score m0 (the streaming rule's seed), from the per-warp records of every CTA of the
+// cluster.  Lane j < C * kWarps fetches record j; the warp reductions give every lane the
+// same values.
+__device__ __forceinline__ void cluster_row_stats(const float *stat, uint32_t C, int lane, float &m, float &l,
+                                                  float &m0)
 {
-    float mw = -INFINITY, lw = 0.f;
+    float mw = -INFINITY, lw = 0.f, sw = -INFINITY;
     for (int j = lane; j < (int)C * kWarps; j += 32) {
-        const float mj = ld_dsmem_f32(stat + 2 * (j % kWarps), (uint32_t)(j / kWarps));
-        const float lj = ld_dsmem_f32(stat + 2 * (j % kWarps) + 1, (uint32_t)(j / kWarps));
+        const float mj = ld_dsmem_f32(stat + 4 * (j % kWarps), (uint32_t)(j / kWarps));
+        const float lj = ld_dsmem_f32(stat + 4 * (j % kWarps) + 1, (uint32_t)(j / kWarps));
+        sw = fmaxf(sw, ld_dsmem_f32(stat + 4 * (j % kWarps) + 2, (uint32_t)(j / kWarps)));
         if (mj == -INFINITY)
             continue;
         if (mw == -INFINITY) {
@@ -512,6 +515,7 @@ __device__ __forceinline__ void cluster_row_stats(const float *stat, uint32_t C,
         }
     }
     m = warp_max(mw);
+    m0 = warp_max(sw);
     l = 0.f;
     if (m == -INFINITY)
         return;
@@ -532,6 +536,10 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     const int capw = (a.cap_groups + kWarps - 1) / kWarps;
     Smem sm = carve<BITS, D>(smem_raw, spw, capw, nbuf, a.near_cap);
     static_assert(BITS == 4, "the exact-maximum reader serves 4-bit sources read with tau > 0");
+    // streaming refine rule (LOOPKV_TAU_STREAM): per warp, tokens are tested against a running
+    // maximum seeded with the row's largest sink score, in the warp's group order
+    const bool stream = a.tau_mode == LOOPKV_TAU_STREAM;
+    const float ltau = log2f(a.tau);
     const bool seq = nbuf == 1; // one score buffer: rows one after another (see the main loop)
     // byte distance between consecutive block ids in the pools (one block = H heads)
     const uint32_t bstride = (uint32_t)a.H * G::HM, lstride = (uint32_t)a.H * G::LOB;
@@ -667,7 +675,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             __syncwarp();
             return;
         }
-        const int32_t *st_row = irow_of(ri);
+        int32_t *st_row = irow_of(ri);
         const int ng = min(kGPS, st_row[IR_N] - kGPS * k2);
         uint8_t *stg = ring + (n & smask) * G::STAGE + 2 * G::VB;
         uint64_t *fb = &full[n & smask];
@@ -676,9 +684,17 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         const float *sc = scores_of(ri) + kGPS * k2 * 32;
         uint32_t mask[kGPS];
         uint32_t bytes = 0;
+        // streaming rule: the row's running maximum (seeded, then raised by each group's largest
+        // score in reading order before its tokens are tested), as consume_v recomputes it
+        float run = stream ? __int_as_float(st_row[IR_RUN]) : 0.f;
 #pragma unroll
         for (int j = 0; j < kGPS; ++j) {
-            const uint32_t tm = j < ng ? __ballot_sync(0xFFFFFFFFu, sc[j * 32 + lane] >= thr2) : 0u;
+            float thr_j = thr2;
+            if (stream) {
+                run = fmaxf(run, warp_max_f(j < ng ? sc[j * 32 + lane] : -INFINITY));
+                thr_j = run + ltau;
+            }
+            const uint32_t tm = j < ng ? __ballot_sync(0xFFFFFFFFu, sc[j * 32 + lane] >= thr_j) : 0u;
             // bit q of qm: token quad q has a hot token (bit 4q of x, then gathered to bit q)
             uint32_t x = tm | (tm >> 1);
             x = (x | (x >> 2)) & 0x11111111u;
@@ -688,8 +704,12 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             mask[j] = tm == 0xFFFFFFFFu ? 0xFFFFFFFFu : qm;
             bytes += tm == 0xFFFFFFFFu ? 2 * G::LOB : (uint32_t)__popc(qm) * D;
         }
-        if (lane == 0)
+        __syncwarp();
+        if (lane == 0) {
+            if (stream)
+                st_row[IR_RUN] = __float_as_int(run);
             mbar_arrive_expect_tx(fb, bytes);
+        }
         __syncwarp();
 #pragma unroll
         for (int j = 0; j < kGPS; ++j) {
@@ -781,8 +801,10 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         int32_t *st_row = irow_of(ri);
         const int vfirst = st_row[IR_VFIRST], vissued = st_row[IR_VISSUED];
         __syncwarp();
-        if (lane == 0)
-            st_row[IR_THR] = __float_as_int(thr2);
+        if (lane == 0) {
+            st_row[IR_THR] = __float_as_int(thr2); // streaming rule: thr2 is the seed
+            st_row[IR_RUN] = __float_as_int(thr2);
+        }
         __syncwarp();
         for (int k2 = 0; k2 < vissued; ++k2)
             issue_lo(ri, k2, vfirst + k2, thr2);
@@ -865,6 +887,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         // j mod (C * kWarps) of the cluster, so that no warp carries the whole tail
         float *tsc = sm.tscores + (ri & 1) * a.near_cap;
         const int wg = (int)crank * kWarps + warp, nw = (int)C * kWarps;
+        float smx = -INFINITY; // largest sink score of this warp's near tokens
         if (tail > wg) {
             const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)srow[IR_B] * 2 * a.H + srow[IR_H]) *
                                                                       a.near_cap * D;
@@ -874,6 +897,8 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
                 if (lane == 0)
                     tsc[j] = s2;
                 mx = fmaxf(mx, s2);
+                if (j < a.sink)
+                    smx = fmaxf(smx, s2);
             }
             __syncwarp();
         }
@@ -887,9 +912,10 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             ls = warp_sum(ls);
         }
         if (lane == 0) {
-            float *stw = sm.stat + (ri % 3) * kWarps * 2;
-            stw[2 * warp] = mx;
-            stw[2 * warp + 1] = ls;
+            float *stw = sm.stat + (ri % 3) * kWarps * 4;
+            stw[4 * warp] = mx;
+            stw[4 * warp + 1] = ls;
+            stw[4 * warp + 2] = smx;
         }
     };
 
@@ -926,6 +952,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         for (int g = 0; g < NCG; ++g)
             zl[g] = 0.f;
         float lsum = 0.f;
+        float run_v = thr2; // streaming rule: running maximum from the seed
         const uint8_t *stg = ring;
         for (int k = 0; k < nown; ++k) {
             const bool first = k % kGPS == 0; // first group of a stage
@@ -937,7 +964,12 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             }
             const float s2l = sc[k * 32 + lane];
             const float wl = ex2(s2l - m2);
-            const bool hotl = s2l >= thr2;
+            float thr_k = thr2;
+            if (stream) { // the same running maximum as issue_lo computed for this group
+                run_v = fmaxf(run_v, warp_max_f(s2l));
+                thr_k = run_v + ltau;
+            }
+            const bool hotl = s2l >= thr_k;
             const uint32_t hm = __ballot_sync(0xFFFFFFFFu, hotl);
             if (a.s_bitmap && lane == 0) // refine set of the debug entry point, one bit per token
                 a.s_bitmap[(int64_t)srow[IR_ROW] * a.bitmap_words + (int)crank + (warp + k * kWarps) * (int)C] = hm;
@@ -1091,8 +1123,11 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         }
     };
 
-    auto row_threshold = [&](float m, float l) {
-        return a.tau_mode == LOOPKV_TAU_ABS_PROB ? m + log2f(a.tau * l) : m + log2f(a.tau);
+    // exact rules: the row threshold; streaming rule: the seed (the largest sink score)
+    auto row_threshold = [&](float m, float l, float m0) {
+        if (stream)
+            return m0;
+        return a.tau_mode == LOOPKV_TAU_ABS_PROB ? m + log2f(a.tau * l) : m + ltau;
     };
 
     // Overlapped order: iteration i scores row i and reads the values of row i - 1; barrier
@@ -1112,9 +1147,9 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             if (mr >= 0)
                 merge(mr, m_prev);
             if (vr < nrows) {
-                float m2, l2;
-                cluster_row_stats(sm.stat + (vr % 3) * kWarps * 2, C, lane, m2, l2);
-                const float thr2 = row_threshold(m2, l2);
+                float m2, l2, m0;
+                cluster_row_stats(sm.stat + (vr % 3) * kWarps * 4, C, lane, m2, l2, m0);
+                const float thr2 = row_threshold(m2, l2, m0);
                 release_row(vr, thr2);
                 consume_v(vr, m2, thr2);
                 m_prev = m2;

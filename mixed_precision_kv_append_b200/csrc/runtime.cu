@@ -264,7 +264,7 @@ int loopkv_plan_create(const loopkv_config *cfg, const uint8_t *modes, float tau
         return rc;
     if (!(tau >= 0.f) || std::isinf(tau))
         return LOOPKV_ERR_INVALID_ARG;
-    if (tau_mode != LOOPKV_TAU_REL_MAX && tau_mode != LOOPKV_TAU_ABS_PROB)
+    if (tau_mode != LOOPKV_TAU_REL_MAX && tau_mode != LOOPKV_TAU_ABS_PROB && tau_mode != LOOPKV_TAU_STREAM)
         return LOOPKV_ERR_INVALID_ARG;
     const int n = cfg->n_loops * cfg->n_layers;
     for (int c = 0; c < n; ++c) {

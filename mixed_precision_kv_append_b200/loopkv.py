@@ -24,7 +24,7 @@ ERRORS = {
     -13: "INFEASIBLE",
 }
 CELL_4B, CELL_2B, CELL_SHARE = 0, 1, 2
-TAU_REL_MAX, TAU_ABS_PROB = 0, 1
+TAU_REL_MAX, TAU_ABS_PROB, TAU_STREAM = 0, 1, 2
 DTYPE_BF16, DTYPE_F32 = 0, 1
 DEV_NONFINITE, DEV_RANGE, DEV_POOL_EXHAUSTED, DEV_TAIL_FULL, DEV_STATE, DEV_TIMEOUT, DEV_EMPTY_ROW = (
     0x01, 0x02, 0x04, 0x08, 0x10, 0x20, 0x40)

@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 import torch
 
-from lkv_helpers import bits_of, check_row, f32
+from lkv_helpers import bits_of, check_row, f32, words_from_bits
 from mixed_precision_kv_append_b200 import loopkv as L
 from mixed_precision_kv_append_b200 import synth
 from oracle import oracle as O
@@ -258,10 +258,10 @@ def test_two_phase_score_buffer_orders(monkeypatch, score_bufs):
     w = synth.Workload("mixed_8k", 1, 4, 16, 128, 32, [8192] * 32, torch.bfloat16, [0, 1, 2, 0], 0.01, seed=2)
     shapes = {}
     for nb in ("1", "2"):  # the override takes effect: two score buffers take more shared memory
-        monkeypatch.setenv("LOOPKV_DECODE_SHAPE", f"0,0,0,{nb},0")
+        monkeypatch.setenv("LOOPKV_DECODE_SHAPE", f"4,0,0,{nb},0")  # clusters of 4 in both
         shapes[nb] = L.Plan(1, 4, 16, 128, 32, base.max_blocks, [0, 1, 2, 0], 0.01).decode_shape(32)
     assert shapes["2"]["smem"] > shapes["1"]["smem"]
-    monkeypatch.setenv("LOOPKV_DECODE_SHAPE", f"0,0,0,{score_bufs},0")
+    monkeypatch.setenv("LOOPKV_DECODE_SHAPE", f"4,0,0,{score_bufs},0")
     # more rows (32 requests x 16 heads) than clusters: every cluster reads several rows in order
     assert 32 * 16 > shapes[score_bufs]["ctas"] // shapes[score_bufs]["cluster"]
     m = Model(w, max_blocks=base.max_blocks)
@@ -528,3 +528,77 @@ def test_sink_window_ouro_shape():
         rows = [(int(rng.integers(4)), int(rng.integers(16))) for _ in range(6)] + [(3, 15), (0, 0)]
         m.check_cell(lp, 0, _q(w, 40, 0, lp), rows=rows, where="sink/window 8K")
     m.check_bytes(0, 0, reqs=[0, 2], heads=[0, 9])
+
+
+def _stream_expected(scores, m0, C, tau, n_hist):
+    """The streaming refine set as the kernel reads a row (LOOPKV_TAU_STREAM): group g to CTA
+    g mod C as its local group g // C, local group i to warp i mod 4 in increasing i; per warp,
+    the oracle's streaming rule over its groups in that order, seeded with m0."""
+    ng = n_hist // 32
+    bits = np.zeros(n_hist, bool)
+    for c in range(C):
+        for wp in range(4):
+            groups = [c + i * C for i in range(wp, (ng + C - 1) // C + 4, 4) if c + i * C < ng]
+            if not groups:
+                continue
+            sub = np.concatenate([scores[32 * g:32 * g + 32] for g in groups])
+            words = O.stream_refine(sub, list(range(len(groups))), m0, tau, running=True)
+            for k, g in enumerate(groups):
+                bits[32 * g:32 * g + 32] = bits_of(words[k:k + 1], 32)
+    return bits
+
+
+@pytest.mark.parametrize("tau", [0.05, 0.01])
+def test_streaming_refine_rule(tau):
+    """LOOPKV_TAU_STREAM (the paper's running maximum seeded with the sink maximum): the GPU's set
+    equals the oracle's streaming rule in the order the kernel reads (ties within 1e-6 of tau
+    aside), contains the exact set, and the output matches the oracle on the GPU's set."""
+    modes = [L.CELL_4B, L.CELL_SHARE, L.CELL_2B, L.CELL_4B]
+    w = synth.Workload("stream", 2, 2, 4, 128, 4, [2000, 700, 130, 1500], torch.bfloat16, modes, tau, seed=41,
+                       tau_mode=L.TAU_STREAM)
+    m = Model(w, sink=32, window=64)
+    m.ingest()
+    C = m.plan.decode_shape(w.B)["cluster"]
+    for lp, la in [(0, 0), (0, 1), (1, 1)]:  # 4-bit cells and the share cell of a 4-bit source
+        assert BITS[w.modes[m.src(lp, la)]] == 4
+        if True:
+            q = _q(w, 0, la, lp)
+            out, bm, _, _ = m.cache.decode_debug(lp, la, q)
+            m.cache.check("stream decode")
+            out, bm, qn = f32(out), bm.cpu().numpy().view(np.uint32), f32(q)
+            hist, near = m.cache.lengths(lp, la)
+            c, src = m.cell(lp, la), m.src(lp, la)
+            for req in range(w.B):
+                n_hist, n_near = int(hist[req]), int(near[req])
+                K, V = m.tokens[(c, req)]
+                Kr, Vr = m.raw_tokens(K, V, n_hist, n_near)
+                for h in range(w.H):
+                    qq = qn[req, h].astype(np.float64)
+                    hh = m.head_history(src, req, h, n_hist)
+                    got = bits_of(bm[req, h], n_hist)
+                    if n_hist == 0:
+                        continue
+                    g = np.arange(n_hist) // 32
+                    kq = O.f16_bits_to_f64(hh.kz)[g] + O.f16_bits_to_f64(hh.ks)[g] * hh.kc.astype(np.float64)
+                    s = kq @ qq / np.sqrt(w.D)
+                    m0 = float((Kr[:32, h].astype(np.float64) @ qq).max() / np.sqrt(w.D))
+                    want = _stream_expected(s, m0, C, tau, n_hist)
+                    exact = O.decode_row(qq, hh, Kr[:, h], Vr[:, h], tau)
+                    ex_bits = bits_of(exact["s_bits"], n_hist)
+                    assert not (ex_bits & ~got).any(), "streaming set must contain the exact set"
+                    diff = np.flatnonzero(want != got)
+                    if diff.size:  # only ties: recompute the running maximum each differing token saw
+                        run = np.full(n_hist, -np.inf)
+                        for c2 in range(C):
+                            for wp in range(4):
+                                mr = m0
+                                for i in range(wp, n_hist // 32, 4):
+                                    gg = c2 + i * C
+                                    if gg >= n_hist // 32:
+                                        break
+                                    mr = max(mr, s[32 * gg:32 * gg + 32].max())
+                                    run[32 * gg:32 * gg + 32] = mr
+                        far = diff[np.abs(np.exp(s[diff] - run[diff]) - tau) > 1e-6]
+                        assert far.size == 0, f"streaming set differs at {far[:8]}"
+                    ref = O.decode_row(qq, hh, Kr[:, h], Vr[:, h], tau, s_force=words_from_bits(got))
+                    assert np.abs(out[req, h] - ref["o"]).max() <= 2e-3
