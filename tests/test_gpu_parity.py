@@ -602,3 +602,74 @@ def test_streaming_refine_rule(tau):
                         assert far.size == 0, f"streaming set differs at {far[:8]}"
                     ref = O.decode_row(qq, hh, Kr[:, h], Vr[:, h], tau, s_force=words_from_bits(got))
                     assert np.abs(out[req, h] - ref["o"]).max() <= 2e-3
+
+
+def _exact_scores(K, q):
+    """Oracle quantization of keys K [T, D] and the exact scores (natural log) of query q."""
+    hh = O.HeadHistory(K, np.zeros_like(K), 4)
+    g = np.arange(K.shape[0]) // 32
+    kq = O.f16_bits_to_f64(hh.kz)[g] + O.f16_bits_to_f64(hh.ks)[g] * hh.kc.astype(np.float64)
+    return kq @ q / np.sqrt(K.shape[1])
+
+
+def _threshold_row(rng, d_rel, tau_target, D=128, T=256):
+    """Keys of one row with a cluster of tokens whose scores are spaced by about d_rel (natural
+    log) around m + ln(tau_target), m the row maximum: group 3 holds 32 copies of one key except
+    channel c*, which steps through 16 codes; every other channel of that group is constant
+    (scale 0).  The other groups are random keys with wide (lognormal, sigma 1.5) channel
+    scales, so that the fixed-point factors of those groups are coarse and the row maximum lies
+    there.  Returns bf16 keys [T, D] and query [D] as float32 arrays of bf16 values."""
+    bf = lambda x: torch.tensor(x, dtype=torch.float32).to(torch.bfloat16).float().numpy()  # noqa: E731
+    sc = np.exp(1.5 * rng.standard_normal(D))
+    k = rng.standard_normal((T, D)) * sc
+    cstar = 5
+    u = rng.standard_normal(D) * sc
+    u[cstar] = 0.0
+    q = rng.standard_normal(D)
+    q[cstar] = d_rel * np.sqrt(D)  # one code step (scale ~0.5 below) moves the score by ~d_rel / 2
+    q = bf(q)
+
+    def build(alpha):
+        kk = k.copy()
+        kk[96:128] = alpha * u
+        kk[96:128, cstar] = 1.0 + np.arange(32) * 0.5
+        return bf(kk)
+
+    s = _exact_scores(build(1.0), q)
+    m = np.delete(s, np.arange(96, 128)).max()
+    s0 = _exact_scores(build(0.0), q)[96:128].mean()  # the cluster's score without the base key
+    alpha = (m + np.log(tau_target) - s0) / ((s[96:128].mean() - s0))
+    return build(alpha), q
+
+
+@pytest.mark.parametrize("d_rel", [1e-5, 1e-4, 1e-3])
+@pytest.mark.parametrize("tau_target", [0.01, 0.3])
+def test_refine_set_exact_near_threshold(d_rel, tau_target):
+    """Tokens placed at r = tau * exp(j * d), around the threshold, with wide channel scales: the
+    decide path's refine set may differ from the oracle's only within 1e-6 of tau."""
+    rng = np.random.default_rng(int(d_rel * 1e7) + int(tau_target * 100))
+    K, qv = _threshold_row(rng, d_rel, tau_target)
+    s = _exact_scores(K, qv.astype(np.float64))
+    m = s.max()
+    assert s[96:128].max() < m  # the row maximum lies in another group
+    mid = np.sort(np.unique(s[96:128]))
+    tau = float(np.exp(mid[len(mid) // 2] - m))  # a cluster token exactly at the threshold
+    assert 0.3 * tau_target < tau < 3 * tau_target
+    V = torch.randn((256, 128), generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    k = torch.tensor(K).to(torch.bfloat16)
+    q = torch.tensor(qv).to(torch.bfloat16)
+    plan = _plan(1, 1, 1, 128, 1, 32, [L.CELL_4B], tau)
+    cache = L.Cache(plan)
+    cache.ingest(0, 0, 0, k.view(256, 1, 128).contiguous().cuda(), V.view(256, 1, 128).contiguous().cuda())
+    out, bm, _, _ = cache.decode_debug(0, 0, q.view(1, 1, 128).contiguous().cuda())
+    cache.check("near-threshold decode")
+    got = bits_of(bm.cpu().numpy().view(np.uint32)[0, 0], 256)
+    hh = O.HeadHistory(K, V.float().numpy(), 4)
+    res = O.decode_row(qv.astype(np.float64), hh, np.zeros((0, 128)), np.zeros((0, 128)), tau)
+    want = bits_of(res["s_bits"], 256)
+    r = res["r"][:256]
+    assert (np.abs(r[96:128] / tau - 1) < 20 * d_rel).sum() >= 8  # many tokens close to the threshold
+    diff = np.flatnonzero(got != want)
+    assert np.all(np.abs(r[diff] - tau) <= 1e-6), (diff, r[diff] / tau - 1)
+
+
