@@ -404,14 +404,39 @@ void orc_pack_head_block(int bits, int D, const uint8_t *kcodes, const uint16_t 
  *   r_out[n_hist+n_tail] exp(s_t - m) (history first), may be NULL
  * Returns ORC_BADARG if no token is attended.
  */
+int orc_decode_row_from(int D, int bits, int n_hist, int hist_first, const double *q, const uint8_t *kc,
+                        const uint16_t *ks, const uint16_t *kz, const uint8_t *vc, const uint16_t *vs,
+                        const uint16_t *vz, int n_tail, const double *tk, const double *tv, double tau,
+                        int tau_mode, const uint32_t *s_force, double *o, double *m_out, double *l_out,
+                        uint32_t *s_bits, double *r_out);
+
 int orc_decode_row(int D, int bits, int n_hist, const double *q, const uint8_t *kc,
                    const uint16_t *ks, const uint16_t *kz, const uint8_t *vc,
                    const uint16_t *vs, const uint16_t *vz, int n_tail, const double *tk,
                    const double *tv, double tau, int tau_mode, const uint32_t *s_force,
                    double *o, double *m_out, double *l_out, uint32_t *s_bits, double *r_out)
 {
+    return orc_decode_row_from(D, bits, n_hist, 0, q, kc, ks, kz, vc, vs, vz, n_tail, tk, tv, tau, tau_mode,
+                               s_force, o, m_out, l_out, s_bits, r_out);
+}
+
+/*
+ * orc_decode_row for a layer with a sliding attention window (the Dory model's
+ * sliding-window layers, LoopKV paper §2.1): history tokens t < hist_first lie before the
+ * window and are not attended (weight 0, never in S, r_out 0); the caller passes only the
+ * attended tail tokens.  hist_first = 0 is plain orc_decode_row.  The history is still
+ * quantized in its 32-token groups from token 0, as it is stored.
+ */
+int orc_decode_row_from(int D, int bits, int n_hist, int hist_first, const double *q, const uint8_t *kc,
+                        const uint16_t *ks, const uint16_t *kz, const uint8_t *vc, const uint16_t *vs,
+                        const uint16_t *vz, int n_tail, const double *tk, const double *tv, double tau,
+                        int tau_mode, const uint32_t *s_force, double *o, double *m_out, double *l_out,
+                        uint32_t *s_bits, double *r_out)
+{
     int n = n_hist + n_tail, G = D / ORC_GROUP;
-    if (n <= 0 || n_hist % ORC_GROUP || (bits != 4 && bits != 2))
+    if (hist_first < 0 || hist_first > n_hist)
+        return ORC_BADARG;
+    if (n - hist_first <= 0 || n_hist % ORC_GROUP || (bits != 4 && bits != 2))
         return ORC_BADARG;
     double *s = (double *)malloc(sizeof(double) * (size_t)n);
     double *r = (double *)malloc(sizeof(double) * (size_t)n);
@@ -433,21 +458,21 @@ int orc_decode_row(int D, int bits, int n_hist, const double *q, const uint8_t *
         }
         s[t] = acc * inv_sqrt_d;
     }
-    /* 2. exact row maximum and weights r_t = exp(s_t - m) */
-    double m = s[0];
-    for (int t = 1; t < n; ++t)
+    /* 2. exact row maximum over the attended tokens and weights r_t = exp(s_t - m) */
+    double m = s[hist_first];
+    for (int t = hist_first + 1; t < n; ++t)
         if (s[t] > m)
             m = s[t];
     double l = 0.0;
     for (int t = 0; t < n; ++t) {
-        r[t] = exp(s[t] - m);
+        r[t] = t < hist_first ? 0.0 : exp(s[t] - m);
         l += r[t];
     }
     /* 3. refine set S (history tokens of a 4-bit cell only) */
     int W = n_hist / ORC_GROUP;
     for (int w = 0; w < W; ++w)
         s_bits[w] = 0;
-    for (int t = 0; t < n_hist; ++t) {
+    for (int t = hist_first; t < n_hist; ++t) {
         int hot;
         if (s_force)
             hot = (s_force[t / 32] >> (t % 32)) & 1;
@@ -463,7 +488,7 @@ int orc_decode_row(int D, int bits, int n_hist, const double *q, const uint8_t *
     /* 4. output: hot -> z + s*q, cold -> z + s*(4h + 1.5), 2-bit -> z + s*code, tail raw */
     for (int c = 0; c < D; ++c) {
         double acc = 0.0;
-        for (int t = 0; t < n; ++t) {
+        for (int t = hist_first; t < n; ++t) {
             double vv;
             if (t < n_hist) {
                 int j = c / ORC_GROUP;

@@ -70,6 +70,11 @@ def lib():
                                          _u8p, _u16p, _u16p, ctypes.c_int, _f64p, _f64p, ctypes.c_double,
                                          ctypes.c_int, _u32p, _f64p, _f64p, _f64p, _u32p, _f64p]
             L.orc_decode_row.restype = ctypes.c_int
+            L.orc_decode_row_from.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _f64p, _u8p,
+                                              _u16p, _u16p, _u8p, _u16p, _u16p, ctypes.c_int, _f64p, _f64p,
+                                              ctypes.c_double, ctypes.c_int, _u32p, _f64p, _f64p, _f64p, _u32p,
+                                              _f64p]
+            L.orc_decode_row_from.restype = ctypes.c_int
             L.orc_stream_refine.argtypes = [ctypes.c_int, _f64p, ctypes.POINTER(ctypes.c_int), ctypes.c_int,
                                             ctypes.c_double, ctypes.c_int, ctypes.c_double, _u32p]
             L.orc_stream_refine.restype = ctypes.c_int
@@ -198,11 +203,13 @@ class HeadHistory:
 # ------------------------------------------------------------------------ decode
 
 def decode_row(q, hist: HeadHistory | None, tail_k, tail_v, tau: float, tau_mode: int = TAU_REL_MAX,
-               s_force: np.ndarray | None = None, bits: int | None = None, D: int | None = None):
+               s_force: np.ndarray | None = None, bits: int | None = None, D: int | None = None,
+               hist_first: int = 0):
     """Attention for one (request, head) row in fp64.
 
     q: [D]; hist: quantized history of the cell that is read (own or final loop's);
-    tail_k/tail_v: [n_tail][D] raw tail.  Returns dict(o, m, l, s_bits, r).
+    tail_k/tail_v: [n_tail][D] raw tail; hist_first: history tokens before it are outside a
+    sliding attention window (not attended).  Returns dict(o, m, l, s_bits, r).
     """
     q = np.ascontiguousarray(q, np.float64)
     D = q.size
@@ -230,10 +237,11 @@ def decode_row(q, hist: HeadHistory | None, tail_k, tail_v, tau: float, tau_mode
     if tk.size == 0:
         tk = np.zeros((1, D))
         tv = np.zeros((1, D))
-    st = lib().orc_decode_row(D, bits, n_hist, _p(q, _f64p), _p(kc, _u8p), _p(ks, _u16p), _p(kz, _u16p),
-                              _p(vc, _u8p), _p(vs, _u16p), _p(vz, _u16p), n_tail, _p(tk, _f64p), _p(tv, _f64p),
-                              float(tau), int(tau_mode), _p(sf, _u32p) if sf is not None else None,
-                              _p(o, _f64p), ctypes.byref(m), ctypes.byref(l_), _p(s_bits, _u32p), _p(r, _f64p))
+    st = lib().orc_decode_row_from(D, bits, n_hist, int(hist_first), _p(q, _f64p), _p(kc, _u8p), _p(ks, _u16p),
+                                   _p(kz, _u16p), _p(vc, _u8p), _p(vs, _u16p), _p(vz, _u16p), n_tail,
+                                   _p(tk, _f64p), _p(tv, _f64p), float(tau), int(tau_mode),
+                                   _p(sf, _u32p) if sf is not None else None, _p(o, _f64p), ctypes.byref(m),
+                                   ctypes.byref(l_), _p(s_bits, _u32p), _p(r, _f64p))
     if st != OK:
         raise ValueError(f"oracle decode_row status {st}")
     return dict(o=o, m=m.value, l=l_.value, s_bits=s_bits[: n_hist // 32], r=r[: n_hist + n_tail])
