@@ -152,6 +152,8 @@ class Runner:
         self.dev = device
         self.plan = L.Plan(w.n_layers, w.n_loops, w.H, w.D, w.B, w.max_blocks, w.modes, w.tau, w.tau_mode,
                            w.dtype)
+        for layer, win in w.layer_windows.items():  # sliding-window layers
+            self.plan.set_window(layer, win)
         self.cache = L.Cache(self.plan, device=device)
         for layer in range(w.n_layers):
             for req in range(w.B):
@@ -213,7 +215,10 @@ class Runner:
                 hist, tail = self.cache.lengths(lp, layer)
                 v = self.cache.cell_view(lp, layer)
                 per_tok = v.head_main_bytes / 16.0
-                nh = int(hist[: w.B].sum())
+                win = w.layer_windows.get(layer, 0)
+                # history tokens read: all, or those inside a sliding window (from its first group)
+                nh = sum(int(hist[r]) - (min(max(int(hist[r]) + int(tail[r]) - win, 0), int(hist[r])) // 32) * 32
+                         if win else int(hist[r]) for r in range(w.B))
                 hot = 0
                 if v.head_lo_bytes:
                     bits = bm.view(torch.int32).cpu()
@@ -256,6 +261,7 @@ def _workload(name, args):
         n = args.layers
         w.modes = [w.modes[lp * w.n_layers + la] for lp in range(w.n_loops) for la in range(n)]
         w.n_layers = n
+        w.layer_windows = {la: win for la, win in w.layer_windows.items() if la < n}
         w.name = f"{w.name}[{n} layer{'s' if n > 1 else ''}]"
     return w
 

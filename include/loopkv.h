@@ -163,6 +163,19 @@ int loopkv_plan_create(const loopkv_config *cfg, const uint8_t *modes, float tau
 void loopkv_plan_free(loopkv_plan *plan);
 
 /*
+ * Sliding-window attention for one layer (the Dory model's recurrent block mixes
+ * full-attention and sliding-window layers, LoopKV paper §2.1): every cell of `layer`
+ * attends only to the last window_tokens positions of its sequence (sink, history pages
+ * and window in sequence order); 0 restores full attention (the default).  The refine set,
+ * row maximum and output then run over those tokens only, and a decode reads only the
+ * history pages that reach into the window.  Storage is unchanged (older pages are kept).
+ * Applies to decodes made with this plan after the call.  Such decodes are launched
+ * without programmatic dependent launch.  Returns LOOPKV_ERR_INVALID_ARG for a bad layer or a
+ * negative window.
+ */
+int loopkv_plan_set_window(loopkv_plan *plan, int layer, int window_tokens);
+
+/*
  * Byte accounting of a plan (LoopKV paper §2.2 and §3.3: KiB stored and read per
  * token).  hot_fraction: host [n_loops * n_layers] fraction of history tokens read
  * with their lo plane per reading cell, or NULL for 1.0 (every lo plane read).

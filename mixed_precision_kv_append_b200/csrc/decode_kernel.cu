@@ -379,7 +379,33 @@ struct Smem {
 };
 
 // Fields of a row slot (Smem::irow).
-enum { IR_ROW = 0, IR_B, IR_H, IR_N, IR_TAIL, IR_VFIRST, IR_VISSUED, IR_THR, IR_WS, IR_RUN, IR_N_FIELDS = 12 };
+enum {
+    IR_ROW = 0, IR_B, IR_H, IR_N, IR_TAIL, IR_VFIRST, IR_VISSUED, IR_THR, IR_WS, IR_RUN,
+    IR_G0,   // first history group inside the attention window
+    IR_M0,   // tokens of group IR_G0 before the window
+    IR_HIST, // history tokens of the row
+    IR_N_FIELDS = 16
+};
+
+// First history token inside a sliding attention window of `win` tokens (0: full attention)
+// for a row of `hist` history and `nnear` near tokens: positions are the sink (0 .. sink-1),
+// the history (sink .. sink+hist-1), then the window; the last `win` positions are attended.
+__host__ __device__ __forceinline__ int window_first(int win, int sink, int hist, int nnear)
+{
+    if (win <= 0)
+        return 0;
+    int h0 = hist + nnear - win - sink;
+    return h0 < 0 ? 0 : (h0 > hist ? hist : h0);
+}
+
+// Whether near token j (sink first, then the window) is inside the attention window.
+__device__ __forceinline__ bool near_attended(const DecodeArgs &a, int j, int hist, int nnear)
+{
+    if (a.attn_window <= 0)
+        return true;
+    const int pos = j < a.sink ? j : hist + j;
+    return pos >= hist + nnear - a.attn_window;
+}
 
 // Byte offsets of the shared-memory regions; every region starts on a 16-byte boundary
 // (digit records, weights and stage data are read with 16-byte vector loads).
@@ -622,7 +648,15 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             bad = true;
             hist = 0;
         }
-        const int ngroups = hist >> 5;
+        // sliding attention window: only the groups from the window's first token on (the
+        // host launches windowed reads without overlap, so the near count is final here)
+        int h0 = 0;
+        if (a.attn_window > 0) {
+            const int nn = a.tail_len[b];
+            h0 = window_first(a.attn_window, a.sink, hist, nn < 0 ? 0 : nn);
+        }
+        const int g0 = h0 >> 5;
+        const int ngroups = (hist >> 5) - g0;
         int nmy = ngroups > (int)crank ? (ngroups - (int)crank + (int)C - 1) / (int)C : 0;
         if (nmy > a.cap_groups) {
             bad = true;
@@ -634,7 +668,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         const int32_t *bt = a.block_table + (int64_t)b * a.max_blocks;
         int32_t *ids = ids_of(ri);
         for (int k = lane; k < 2 * n; k += 32) {
-            const int g = (int)crank + (warp + (k >> 1) * kWarps) * (int)C;
+            const int g = g0 + (int)crank + (warp + (k >> 1) * kWarps) * (int)C;
             int id = bt[2 * g + (k & 1)];
             if (id < 0 || id >= a.pool_blocks) {
                 atomicOr(a.status, LOOPKV_DEV_STATE);
@@ -652,6 +686,9 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             st[IR_VFIRST] = 0;
             st[IR_VISSUED] = 0;
             st[IR_THR] = __float_as_int(NAN);
+            st[IR_G0] = g0;
+            st[IR_M0] = h0 & 31;
+            st[IR_HIST] = hist;
         }
         __syncwarp();
     };
@@ -878,7 +915,9 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
                 stg = ring + (n & smask) * G::STAGE;
             }
             const uint8_t *st = stg + (k % kGPS) * G::GSLOT;
-            const float s2 = group_scores<BITS, D>(st, st + G::KB, scr, qreg, a.qscale, lane);
+            float s2 = group_scores<BITS, D>(st, st + G::KB, scr, qreg, a.qscale, lane);
+            if (k == 0 && crank == 0 && warp == 0 && lane < srow[IR_M0])
+                s2 = -INFINITY; // before the attention window
             sc[k * 32 + lane] = s2;
             mx = fmaxf(mx, s2);
             __syncwarp();
@@ -891,9 +930,11 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         if (tail > wg) {
             const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)srow[IR_B] * 2 * a.H + srow[IR_H]) *
                                                                       a.near_cap * D;
-            const int ws = srow[IR_WS];
+            const int ws = srow[IR_WS], hist = srow[IR_HIST];
             for (int j = wg; j < tail; j += nw) {
-                const float s2 = near_score<D, DT>(kt + (int64_t)near_slot(a, j, ws) * D, qreg, a.qscale, lane);
+                const float s2 = near_attended(a, j, hist, tail)
+                                     ? near_score<D, DT>(kt + (int64_t)near_slot(a, j, ws) * D, qreg, a.qscale, lane)
+                                     : -INFINITY;
                 if (lane == 0)
                     tsc[j] = s2;
                 mx = fmaxf(mx, s2);
@@ -972,7 +1013,8 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             const bool hotl = s2l >= thr_k;
             const uint32_t hm = __ballot_sync(0xFFFFFFFFu, hotl);
             if (a.s_bitmap && lane == 0) // refine set of the debug entry point, one bit per token
-                a.s_bitmap[(int64_t)srow[IR_ROW] * a.bitmap_words + (int)crank + (warp + k * kWarps) * (int)C] = hm;
+                a.s_bitmap[(int64_t)srow[IR_ROW] * a.bitmap_words + srow[IR_G0] + (int)crank +
+                           (warp + k * kWarps) * (int)C] = hm;
             lsum += wl;
             if (first) {
                 wait_stage(n);
@@ -1196,6 +1238,7 @@ struct SmemLayout1 {
 // (word D + 1).  CTA partials (o[D], l, m) by row parity (see the barrier note in the
 // kernel).
 constexpr int kFields1 = 8;
+constexpr int I1_G0 = 5, I1_M0 = 6, I1_HIST = 7; // fields after IR_ROW .. IR_TAIL (see decode_kernel)
 
 template <int BITS, int D> __host__ __device__ constexpr SmemLayout1 smem_layout1(int spw, int capw)
 {
@@ -1261,7 +1304,7 @@ template <int D> __device__ __forceinline__ void run1_init(Run1<D> &r)
 // (4-bit source) or plain 2-bit codes.  scr: the warp's scratch.
 template <int BITS, int D>
 __device__ __forceinline__ void run1_group(const uint8_t *st, const uint8_t *lo, uint8_t *scr, const float (&qreg)[4],
-                                           const float qscale, const int lane, Run1<D> &r)
+                                           const float qscale, const int lane, Run1<D> &r, const int masked = 0)
 {
     using G = Geo<BITS, D>;
     constexpr int NCG = G::NCG;
@@ -1273,7 +1316,9 @@ __device__ __forceinline__ void run1_group(const uint8_t *st, const uint8_t *lo,
     const int vb0 = G::NQ == 32 ? 0 : lane / G::NQ;
     uint32_t *ybuf = reinterpret_cast<uint32_t *>(scr);
     float *fsit = reinterpret_cast<float *>(ybuf + NCG * YS);
-    const float s2l = group_scores<BITS, D>(st, st + G::HM, scr, qreg, qscale, lane); // score of token `lane`
+    float s2l = group_scores<BITS, D>(st, st + G::HM, scr, qreg, qscale, lane); // score of token `lane`
+    if (lane < masked)
+        s2l = -INFINITY; // before a sliding attention window
     // ---- running maximum (warp-uniform): rescale the warp's sums when it grows
     const float mg = warp_max_f(s2l);
     if (mg > r.m) {
@@ -1385,9 +1430,11 @@ template <int BITS, int D> __device__ __forceinline__ void run1_finish(Run1<D> &
 template <int D, typename DT>
 __device__ __forceinline__ void run1_tail(Run1<D> &r, float *red, const int lane, const float (&qreg)[4],
                                           const DecodeArgs &a, const DT *kt, const DT *vt0, const int ws,
-                                          const int j0, const int stride, const int n)
+                                          const int hist, const int j0, const int stride, const int n)
 {
     for (int j = j0; j < n; j += stride) {
+        if (!near_attended(a, j, hist, n))
+            continue;
         const int slot = near_slot(a, j, ws);
         const float s2 = near_score<D, DT>(kt + (int64_t)slot * D, qreg, a.qscale, lane);
         if (s2 > r.m) { // warp-uniform
@@ -1484,7 +1531,13 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
             bad = true;
             hist = 0;
         }
-        const int ngroups = hist >> 5;
+        int h0 = 0; // sliding attention window (see decode_kernel's setup_row)
+        if (a.attn_window > 0) {
+            const int nn = a.tail_len[b];
+            h0 = window_first(a.attn_window, a.sink, hist, nn < 0 ? 0 : nn);
+        }
+        const int g0 = h0 >> 5;
+        const int ngroups = (hist >> 5) - g0;
         int nmy = ngroups > (int)crank ? (ngroups - (int)crank + (int)C - 1) / (int)C : 0;
         if (nmy > a.cap_groups) {
             bad = true;
@@ -1495,7 +1548,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
         const int n = owned(nmy, warp);
         const int32_t *bt = a.block_table + (int64_t)b * a.max_blocks;
         for (int k = lane; k < 2 * n; k += 32) {
-            const int g = (int)crank + (warp + (k >> 1) * kWarps) * (int)C;
+            const int g = g0 + (int)crank + (warp + (k >> 1) * kWarps) * (int)C;
             int id = bt[2 * g + (k & 1)];
             if (id < 0 || id >= a.pool_blocks) {
                 atomicOr(a.status, LOOPKV_DEV_STATE);
@@ -1509,6 +1562,9 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
             irow[IR_H] = h;
             irow[IR_N] = n;
             irow[IR_TAIL] = -1; // tail length read after the grid dependency wait
+            irow[I1_G0] = g0;
+            irow[I1_M0] = h0 & 31;
+            irow[I1_HIST] = hist;
         }
         __syncwarp();
         setup_upto = ri;
@@ -1571,6 +1627,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
         if (ri == 0)
             setup_row(0);
         const int row = irow[IR_ROW], nown = irow[IR_N], rb = irow[IR_B], rh = irow[IR_H];
+        const int rg0 = irow[I1_G0], rm0 = (crank == 0 && warp == 0) ? irow[I1_M0] : 0, rhist = irow[I1_HIST];
         int tail = irow[IR_TAIL];
         // the slot takes row ri + 1 once row ri's stages are all issued (after the pump of
         // group nown - spw, or at once when the warp has no group)
@@ -1611,10 +1668,11 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
             }
             wait_stage(n);
             const uint8_t *st = ring + (n & smask) * G1::STAGE;
-            run1_group<BITS, D>(st, st + G1::LOFF, scr, qreg, a.qscale, lane, run);
-            if (a.s_bitmap && lane == 0) // refine set: every token (4-bit, tau <= 0) or none (2-bit)
-                a.s_bitmap[(int64_t)row * a.bitmap_words + (int)crank + (warp + k * kWarps) * (int)C] =
-                    BITS == 4 ? 0xFFFFFFFFu : 0u;
+            const int masked = k == 0 ? rm0 : 0; // tokens of the first group before a sliding window
+            run1_group<BITS, D>(st, st + G1::LOFF, scr, qreg, a.qscale, lane, run, masked);
+            if (a.s_bitmap && lane == 0) // refine set: every attended token (4-bit, tau <= 0) or none (2-bit)
+                a.s_bitmap[(int64_t)row * a.bitmap_words + rg0 + (int)crank + (warp + k * kWarps) * (int)C] =
+                    BITS == 4 ? ~((1u << masked) - 1u) : 0u;
         }
         float *red = reinterpret_cast<float *>(scr);
         run1_finish<BITS, D>(run, red, lane);
@@ -1623,7 +1681,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
             const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)rb * 2 * a.H + rh) * a.near_cap * D;
             const DT *vt0 =
                 reinterpret_cast<const DT *>(a.tail) + ((int64_t)(rb * 2 + 1) * a.H + rh) * a.near_cap * D;
-            run1_tail<D, DT>(run, red, lane, qreg, a, kt, vt0, ws, wg, (int)C * kWarps, tail);
+            run1_tail<D, DT>(run, red, lane, qreg, a, kt, vt0, ws, rhist, wg, (int)C * kWarps, tail);
         }
         if (lane == 0)
             red[D + 1] = run.m;

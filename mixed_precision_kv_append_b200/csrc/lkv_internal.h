@@ -56,6 +56,7 @@ struct DecodeArgs {
     float tau;
     int tau_mode;
     int sink, wring, near_cap;  // near region geometry (see DevState)
+    int attn_window;            // sliding attention window of the cell's layer in tokens, 0 = full
     unsigned long long wait_ns; // limit of every bounded wait, in nanoseconds
     int inject;                 // LOOPKV_INJECT_*: LOOPKV_INJECT_NONE in normal operation
 };

@@ -18,6 +18,7 @@
 struct loopkv_plan {
     loopkv_config cfg;
     std::vector<uint8_t> modes;
+    std::vector<int> layer_window; // sliding attention window per layer in tokens, 0 = full
     float tau;
     int tau_mode;
     int n_cells() const { return cfg.n_loops * cfg.n_layers; }
@@ -278,6 +279,7 @@ int loopkv_plan_create(const loopkv_config *cfg, const uint8_t *modes, float tau
         return LOOPKV_ERR_INVALID_ARG;
     p->cfg = *cfg;
     p->modes.assign(modes, modes + n);
+    p->layer_window.assign(cfg->n_layers, 0);
     p->tau = tau;
     p->tau_mode = tau_mode;
     *out = p;
@@ -285,6 +287,14 @@ int loopkv_plan_create(const loopkv_config *cfg, const uint8_t *modes, float tau
 }
 
 void loopkv_plan_free(loopkv_plan *plan) { delete plan; }
+
+int loopkv_plan_set_window(loopkv_plan *plan, int layer, int window_tokens)
+{
+    if (!plan || layer < 0 || layer >= plan->cfg.n_layers || window_tokens < 0)
+        return LOOPKV_ERR_INVALID_ARG;
+    plan->layer_window[layer] = window_tokens;
+    return LOOPKV_OK;
+}
 
 int loopkv_plan_bytes(const loopkv_plan *plan, const float *hot_fraction, loopkv_byte_report *out)
 {
@@ -525,6 +535,7 @@ int loopkv_decode_debug(const loopkv_plan *plan, int loop, int layer, const void
     a.qscale = (float)(1.4426950408889634 / std::sqrt((double)D));
     a.tau = plan->tau;
     a.tau_mode = plan->tau_mode;
+    a.attn_window = plan->layer_window[layer];
     const lkv::DecodeShape shp = cache->shape(bits, B, single_pass(bits, plan->tau));
     a.cap_groups = shp.cap;
     {
@@ -532,7 +543,8 @@ int loopkv_decode_debug(const loopkv_plan *plan, int loop, int layer, const void
         a.wait_ns = cache->wait_ns;
         a.inject = cache->inject;
     }
-    const bool overlap = cache->decode_may_overlap(stream);
+    // a windowed read sets up its rows from the near counts, which appends write: no overlap
+    const bool overlap = cache->decode_may_overlap(stream) && a.attn_window == 0;
     return lkv::launch_decode(a, bits, D, cp.cfg.in_dtype, shp, overlap, static_cast<cudaStream_t>(stream));
 }
 

@@ -34,6 +34,7 @@ EXPORTS = [
     "loopkv_free", "loopkv_ingest", "loopkv_append", "loopkv_flush", "loopkv_reset_request", "loopkv_decode",
     "loopkv_decode_debug", "loopkv_status", "loopkv_cell_view_get", "loopkv_decode_shape", "loopkv_strerror",
     "loopkv_version", "loopkv_plan_search", "loopkv_append_noalloc", "loopkv_set_wait_policy",
+    "loopkv_plan_set_window",
 ]
 INJECT_NONE, INJECT_STALLED_STAGE = 0, 1
 NOALLOC_MAX_IDS = 4096
@@ -86,6 +87,7 @@ def lib() -> ctypes.CDLL:
                                          ctypes.POINTER(vp)]
         L.loopkv_plan_free.argtypes = [vp]
         L.loopkv_plan_free.restype = None
+        L.loopkv_plan_set_window.argtypes = [vp, i, i]
         L.loopkv_plan_bytes.argtypes = [vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ByteReport)]
         L.loopkv_required_bytes.argtypes = [vp, ctypes.POINTER(ctypes.c_size_t)]
         L.loopkv_alloc.argtypes = [vp, vp, ctypes.c_size_t, vp, ctypes.POINTER(vp)]
@@ -288,6 +290,12 @@ class Plan:
 
     def required_bytes(self) -> int:
         return loopkv_required_bytes(self.handle)
+
+    def set_window(self, layer: int, window_tokens: int):
+        """Sliding attention window of a layer (0 = full attention)."""
+        _check(lib().loopkv_plan_set_window(self.handle, layer, window_tokens), "loopkv_plan_set_window")
+        self.windows = getattr(self, "windows", {})
+        self.windows[layer] = window_tokens
 
     def decode_shape(self, B) -> dict:
         return loopkv_decode_shape(self.handle, B)

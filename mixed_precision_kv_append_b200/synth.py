@@ -44,6 +44,7 @@ class Workload:
     tau_mode: int = 0      # 0 = relative to the row max, 1 = normalised weight
     append_steps: int = 0  # decode steps that append one token per request per cell
     seed: int = 0
+    layer_windows: dict = dataclasses.field(default_factory=dict)  # layer -> sliding window (tokens)
 
     @property
     def n_cells(self):
@@ -100,11 +101,20 @@ def workload(name: str, seed: int = 0) -> Workload:
         B = 32 * 8192 // T
         modes = seeded_plan(48, 4, [0, 1, 2], 0.35, 0.25, seed)
         return Workload(name, 48, 4, 16, 128, B, [T] * B, torch.bfloat16, modes, 0.01, seed=seed)
+    if name == "dory_16k":
+        # Dory-4B-shaped recurrent block (LoopKV §2.1: 20 recurrent attention layers, 5 with full
+        # attention and 15 with a sliding window).  The pages give neither the loop count, the
+        # head shape nor the window size: 4 loops, 16 x 128 heads and a 4096-token window are
+        # assumptions of this workload; every fourth layer attends fully
+        modes = seeded_plan(20, 4, [1, 2], 0.35, 0.25, seed)
+        windows = {la: 4096 for la in range(20) if la % 4 != 0}
+        return Workload("dory_16k", 20, 4, 16, 128, 16, [16384] * 16, torch.bfloat16, modes, 0.01, seed=seed,
+                        layer_windows=windows)
     raise KeyError(name)
 
 
 WORKLOADS = ["tiny", "kivi4_8k", "mixed_8k", "long_16k", "ragged_2p6b", "ouro2p6b_8k", "ouro2p6b_16k",
-             "ouro2p6b_32k"]
+             "ouro2p6b_32k", "dory_16k"]
 
 
 def _gen(seed: int, device) -> torch.Generator:

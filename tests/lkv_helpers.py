@@ -33,9 +33,10 @@ def oracle_packed(hist: O.HeadHistory):
 
 def check_row(gpu_out: np.ndarray, gpu_bits: np.ndarray, gpu_m: float | None, gpu_l: float | None,
               q: np.ndarray, hist: O.HeadHistory | None, tail_k: np.ndarray, tail_v: np.ndarray,
-              tau: float, tau_mode: int, where: str = ""):
-    """Compare one (request, head) row.  Returns (max abs error, n S mismatches inside the tie band)."""
-    res = O.decode_row(q, hist, tail_k, tail_v, tau, tau_mode)
+              tau: float, tau_mode: int, where: str = "", hist_first: int = 0):
+    """Compare one (request, head) row; history tokens before hist_first are outside a sliding
+    attention window.  Returns (max abs error, n S mismatches inside the tie band)."""
+    res = O.decode_row(q, hist, tail_k, tail_v, tau, tau_mode, hist_first=hist_first)
     n_hist = 0 if hist is None else hist.T
     ref_bits = bits_of(res["s_bits"], n_hist)
     got_bits = bits_of(gpu_bits, n_hist) if n_hist else np.zeros(0, bool)
@@ -47,7 +48,8 @@ def check_row(gpu_out: np.ndarray, gpu_bits: np.ndarray, gpu_m: float | None, gp
         assert far.size == 0, (
             f"{where}: refine set differs outside the tie band at tokens {far[:8]} "
             f"(oracle weight {qty[far[:8]]}, tau {tau})")
-        res = O.decode_row(q, hist, tail_k, tail_v, tau, tau_mode, s_force=words_from_bits(got_bits))
+        res = O.decode_row(q, hist, tail_k, tail_v, tau, tau_mode, s_force=words_from_bits(got_bits),
+                           hist_first=hist_first)
     err = float(np.max(np.abs(gpu_out.astype(np.float64) - res["o"])))
     assert err <= OUT_ATOL, f"{where}: max abs output error {err}"
     if gpu_m is not None:

@@ -107,9 +107,17 @@ class Model:
             assert n_own == n_hist + n_tail, (n_own, n_hist, n_tail)
             hh = self.head_history(s, req, h, n_hist)
             Kr, Vr = self.raw_tokens(K, V, n_hist, n_tail)
+            win = getattr(self.plan, "windows", {}).get(layer, 0)
+            h0 = 0
+            if win:  # sliding window: the last `win` positions (sink, history, window in order)
+                n = n_hist + n_tail
+                h0 = min(max(n - win - self.sink, 0), n_hist)
+                pos = np.array([j if j < self.sink else n_hist + j for j in range(n_tail)])
+                keep = pos >= n - win
+                Kr, Vr = Kr[keep], Vr[keep]
             err, nt = check_row(out[req, h], bm[req, h], rm[req, h], rs[req, h], qn[req, h].astype(np.float64),
                                 hh, Kr[:, h], Vr[:, h], self.tau, self.tau_mode,
-                                where=f"{where} cell ({loop},{layer}) req {req} head {h}")
+                                where=f"{where} cell ({loop},{layer}) req {req} head {h}", hist_first=h0)
             worst, ties = max(worst, err), ties + nt
         return worst, ties
 
@@ -673,3 +681,24 @@ def test_refine_set_exact_near_threshold(d_rel, tau_target):
     assert np.all(np.abs(r[diff] - tau) <= 1e-6), (diff, r[diff] / tau - 1)
 
 
+
+
+@pytest.mark.parametrize("win", [40, 100, 333, 5000])
+@pytest.mark.parametrize("tau", [0.02, 0.0])
+@pytest.mark.parametrize("sink,window", [(32, 64), (0, 0)])
+def test_sliding_window_layer(win, tau, sink, window):
+    """A layer whose cells attend only to their last `win` positions (Dory's sliding-window
+    layers, LoopKV §2.1) next to a full-attention layer: windows that start inside a history
+    group, inside the near region, and beyond the sequence; both readers (tau > 0 and tau = 0)."""
+    modes = [L.CELL_4B, L.CELL_SHARE, L.CELL_2B, L.CELL_4B]  # loop 0: [4b, share], loop 1: [2b, 4b]
+    w = synth.Workload("slide", 2, 2, 4, 128, 3, [20, 150, 700], torch.bfloat16, modes, tau, append_steps=40, seed=43)
+    m = Model(w, sink=sink, window=window)
+    m.plan.set_window(1, win)
+    m.ingest()
+    for step in range(40):
+        m.append_step(step)
+        if step in (0, 13, 39):
+            for la in range(2):
+                for lp in range(2):
+                    m.check_cell(lp, la, _q(w, step, la, lp), where=f"win={win} step {step}")
+    m.cache.check("sliding window")
