@@ -8,9 +8,9 @@
 // One launch per cell (LoopKV paper, §3.4 "One launch per cell").  The grid is a set
 // of persistent thread-block clusters of C CTAs; cluster c serves the (request, head)
 // rows c, c + NC, c + 2NC, ... one after another.  Inside a row, CTA k of the cluster
-// owns the 32-token groups k, k+C, k+2C, ... of the history, and CTA C-1 also the
-// unquantized tail.  Warp w of a CTA owns the CTA's groups w, w+4, ...  For each row a
-// warp:
+// owns the 32-token groups k, k+C, k+2C, ... of the history; the unquantized near tokens
+// (sink and window) are dealt over every warp of the cluster.  Warp w of a CTA owns the
+// CTA's groups w, w+4, ...  For each row a warp:
 //   1. K pass: streams the key codes and the per-channel key scale/zero of its groups
 //      into shared memory with bulk asynchronous copies that it issues itself (one
 //      elected lane, a private mbarrier ring), and computes every score from the full
@@ -34,15 +34,11 @@
 // carries both the per-warp maxima of row r and the partial outputs of row r-1.  Long
 // rows, whose scores fill the shared memory, take one score buffer and run in sequence.
 //
-// Keys: the dot product of a 32-token group is computed exactly in integers.  The
-// group's per-channel factor a_c = q_c * s_c is rounded to a 22-bit fixed-point integer
-// I_c with one FMA against 1.5 * 2^23 (the float's low 23 bits are then I_c + 2^22), and
-// the three bytes of that field become three 8-bit digits (the top one re-centred to a
-// signed byte) with byte permutes.  The 4-bit (or 2-bit) codes are unpacked four at a
-// time into bytes with one AND, and dp4a accumulates code * digit in int32 with no
-// rounding.
-// The key loads are laid out so that the lanes of a shared-memory phase hit distinct
-// banks (group_scores).
+// Keys: the dot products of a 32-token group run in integers on the tensor cores
+// (group_scores): the per-channel factors a_c = q_c * s_c are rounded to 30-bit fixed point
+// and split into four signed byte digits, the [32 tokens x D] code matrix times the [D x 4]
+// digit matrix runs as m16n8k32 u8 x s8 products with exact int32 accumulation, and the
+// digit sums meet in fp32 with the zero term.
 // Values: a value-plane word holds 4 tokens x 4 channels (token in the byte).  The hi and
 // lo words merge into 4-bit codes (lo bits of cold tokens masked off), one AND unpacks the
 // codes of one channel for 4 tokens, and dp4a against the two 8-bit digits of the tokens'
@@ -80,7 +76,6 @@ template <int BITS, int D> struct Geo {
     static constexpr int GSLOT = ((KSTAGE > VSTAGE ? KSTAGE : VSTAGE) + 127) / 128 * 128; // one group
     static constexpr int STAGE = kGPS * GSLOT;
     static constexpr int ROWK = KCODES / 16;  // key bytes per token
-    static constexpr int WORDSK = ROWK / 4;
     static constexpr int NCG = D / 32;        // 32-channel value groups per token
     static constexpr int NQ = D / 4;          // channel quads
 };
@@ -89,12 +84,6 @@ template <int BITS, int D> struct Geo {
 __device__ __forceinline__ void dp4a_uu(uint32_t &acc, uint32_t u, uint32_t d)
 {
     asm("dp4a.u32.u32 %0, %1, %2, %0;" : "+r"(acc) : "r"(u), "r"(d));
-}
-
-// acc += sum of the four unsigned bytes of `u` times the four signed bytes of `d`
-__device__ __forceinline__ void dp4a_us(int &acc, uint32_t u, uint32_t d)
-{
-    asm("dp4a.u32.s32 %0, %1, %2, %0;" : "+r"(acc) : "r"(u), "r"(d));
 }
 
 // 2^x by the hardware approximation (relative error about 2^-22; tiny results flush to 0)
@@ -380,7 +369,7 @@ struct Smem {
 
 // Fields of a row slot (Smem::irow).
 enum {
-    IR_ROW = 0, IR_B, IR_H, IR_N, IR_TAIL, IR_VFIRST, IR_VISSUED, IR_THR, IR_WS, IR_RUN,
+    IR_ROW = 0, IR_B, IR_H, IR_N, IR_TAIL, IR_WS,
     IR_G0,   // first history group inside the attention window
     IR_M0,   // tokens of group IR_G0 before the window
     IR_HIST, // history tokens of the row
@@ -627,7 +616,6 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     int seg_n = 0;                 // groups of the segment's row owned by this warp
     bool seg_v = false;
     const uint8_t *seg_src = nullptr; // main pool + head offset (+ K part) of the segment's row
-    const uint8_t *seg_lo = nullptr;  // lo pool + head offset of the segment's row
     const int2 *seg_ids = nullptr;
     int setup_upto = -1;           // rows 0..setup_upto have their parameters and ids in place
     // After one bounded wait gives up, later waits are skipped, nothing new is issued, and the
@@ -683,9 +671,6 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             st[IR_H] = h;
             st[IR_N] = n;
             st[IR_TAIL] = -1; // tail length not read yet (read after the grid dependency wait)
-            st[IR_VFIRST] = 0;
-            st[IR_VISSUED] = 0;
-            st[IR_THR] = __float_as_int(NAN);
             st[IR_G0] = g0;
             st[IR_M0] = h0 & 31;
             st[IR_HIST] = hist;
@@ -698,74 +683,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         seg_n = st[IR_N];
         seg_len = (seg_n + kGPS - 1) / kGPS;
         seg_src = a.main + (size_t)st[IR_H] * G::HM + (seg_v ? G::KB : 0);
-        seg_lo = a.lo + (size_t)st[IR_H] * G::LOB;
         seg_ids = reinterpret_cast<const int2 *>(ids_of(seg_ri));
-    };
-    // lo planes (4-bit sources, tau > 0) of the hot tokens of V stage k2 of row ri, then
-    // the one arrival that completes the stage's barrier phase.  The lo plane holds 4
-    // tokens per word, so a 4-token quad with a hot token is copied whole (D bytes); a
-    // group whose 32 tokens are all hot copies both blocks' planes.
-    auto issue_lo = [&](int ri, int k2, int n, float thr2) {
-        if (timed_out) { // no new copies after a give-up; the arrival keeps the stage's phase complete
-            if (lane == 0)
-                mbar_arrive(&full[n & smask]);
-            __syncwarp();
-            return;
-        }
-        int32_t *st_row = irow_of(ri);
-        const int ng = min(kGPS, st_row[IR_N] - kGPS * k2);
-        uint8_t *stg = ring + (n & smask) * G::STAGE + 2 * G::VB;
-        uint64_t *fb = &full[n & smask];
-        const uint8_t *lob = a.lo + (size_t)st_row[IR_H] * G::LOB;
-        const int2 *ids = reinterpret_cast<const int2 *>(ids_of(ri)) + kGPS * k2;
-        const float *sc = scores_of(ri) + kGPS * k2 * 32;
-        uint32_t mask[kGPS];
-        uint32_t bytes = 0;
-        // streaming rule: the row's running maximum (seeded, then raised by each group's largest
-        // score in reading order before its tokens are tested), as consume_v recomputes it
-        float run = stream ? __int_as_float(st_row[IR_RUN]) : 0.f;
-#pragma unroll
-        for (int j = 0; j < kGPS; ++j) {
-            float thr_j = thr2;
-            if (stream) {
-                run = fmaxf(run, warp_max_f(j < ng ? sc[j * 32 + lane] : -INFINITY));
-                thr_j = run + ltau;
-            }
-            const uint32_t tm = j < ng ? __ballot_sync(0xFFFFFFFFu, sc[j * 32 + lane] >= thr_j) : 0u;
-            // bit q of qm: token quad q has a hot token (bit 4q of x, then gathered to bit q)
-            uint32_t x = tm | (tm >> 1);
-            x = (x | (x >> 2)) & 0x11111111u;
-            x = (x | (x >> 3)) & 0x03030303u;
-            x = (x | (x >> 6)) & 0x000F000Fu;
-            const uint32_t qm = (x | (x >> 12)) & 0xFFu;
-            mask[j] = tm == 0xFFFFFFFFu ? 0xFFFFFFFFu : qm;
-            bytes += tm == 0xFFFFFFFFu ? 2 * G::LOB : (uint32_t)__popc(qm) * D;
-        }
-        __syncwarp();
-        if (lane == 0) {
-            if (stream)
-                st_row[IR_RUN] = __float_as_int(run);
-            mbar_arrive_expect_tx(fb, bytes);
-        }
-        __syncwarp();
-#pragma unroll
-        for (int j = 0; j < kGPS; ++j) {
-            if (j >= ng)
-                break;
-            const int2 id = ids[j];
-            uint8_t *st = stg + j * G::GSLOT;
-            if (mask[j] == 0xFFFFFFFFu) {
-                if (lane == 0) {
-                    bulk_g2s(st, lob + (uint64_t)(uint32_t)id.x * lstride, G::LOB, fb);
-                    bulk_g2s(st + G::LOB, lob + (uint64_t)(uint32_t)id.y * lstride, G::LOB, fb);
-                }
-            } else if (lane < 8 && ((mask[j] >> lane) & 1u)) { // lane = token quad
-                const int blk = lane >> 2, tau = lane & 3;
-                const uint32_t bid = (uint32_t)(blk ? id.y : id.x);
-                bulk_g2s(st + blk * G::LOB + tau * D, lob + (uint64_t)bid * lstride + tau * D, D, fb);
-            }
-        }
-        __syncwarp();
     };
     // Stage k2 of the current segment: groups kGPS*k2 .. kGPS*k2 + ng - 1 of the row, group
     // j into sub-slot j.
@@ -788,22 +706,14 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             }
             return;
         }
-        int32_t *st_row = irow_of(seg_ri);
-        if (lane == 0) {
-            if (k2 == 0)
-                st_row[IR_VFIRST] = n;
-            st_row[IR_VISSUED] = k2 + 1;
-            mbar_expect_tx(fb, (uint32_t)ng * 2 * G::VB);
+        if (lane == 0) { // V stage: value meta and hi planes (the lo planes of hot tokens: consume_v)
+            mbar_arrive_expect_tx(fb, (uint32_t)ng * 2 * G::VB);
             for (int j = 0; j < ng; ++j) {
                 const int2 id = ids[j];
                 bulk_g2s(stg + j * G::GSLOT, seg_src + (uint64_t)(uint32_t)id.x * bstride, G::VB, fb);
                 bulk_g2s(stg + j * G::GSLOT + G::VB, seg_src + (uint64_t)(uint32_t)id.y * bstride, G::VB, fb);
             }
         }
-        __syncwarp();
-        const float thr2 = __int_as_float(st_row[IR_THR]);
-        if (!isnan(thr2)) // the lo part needs the row threshold
-            issue_lo(seg_ri, k2, n, thr2);
     };
     // Issue every stage numbered below `limit` that the sequence allows.  The K segment
     // of a row waits until the row is set up (the compute side sets up row r + 1 when it
@@ -833,20 +743,6 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             load_segment();
         }
     };
-    // the threshold of row ri is known: finish the V stages issued without their lo part
-    auto release_row = [&](int ri, float thr2) {
-        int32_t *st_row = irow_of(ri);
-        const int vfirst = st_row[IR_VFIRST], vissued = st_row[IR_VISSUED];
-        __syncwarp();
-        if (lane == 0) {
-            st_row[IR_THR] = __float_as_int(thr2); // streaming rule: thr2 is the seed
-            st_row[IR_RUN] = __float_as_int(thr2);
-        }
-        __syncwarp();
-        for (int k2 = 0; k2 < vissued; ++k2)
-            issue_lo(ri, k2, vfirst + k2, thr2);
-    };
-
     // ---------------------------------------------------------------- compute
     constexpr int SCR = scratch_bytes<D>();
     uint8_t *scr = sm.scr + warp * SCR;
@@ -994,6 +890,43 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             zl[g] = 0.f;
         float lsum = 0.f;
         float run_v = thr2; // streaming rule: running maximum from the seed
+        const uint8_t *lob = a.lo + (size_t)srow[IR_H] * G::LOB;
+        const int2 *gids = reinterpret_cast<const int2 *>(ids_of(ri));
+        // Hot tokens of group k (bit t: token t).  The streaming rule's running maximum takes
+        // each group's largest score before the group's tokens are tested, in group order.
+        auto hot_mask = [&](int k) {
+            const float s2 = sc[k * 32 + lane];
+            float thr_k = thr2;
+            if (stream) {
+                run_v = fmaxf(run_v, warp_max_f(s2));
+                thr_k = run_v + ltau;
+            }
+            return __ballot_sync(0xFFFFFFFFu, s2 >= thr_k);
+        };
+        // Lo planes of the hot token quads of group k into the group's slot of ring stage n,
+        // one group ahead of its use.  A quad (4 tokens x D channels x 2 bits = D bytes) with a
+        // hot token is copied whole in 16-byte pieces, each lane its own; then one commit
+        // group per call (empty when nothing is hot).  The slot is free: its previous stage was
+        // consumed before the current one.
+        auto fetch_lo = [&](int k, int n, uint32_t hm) {
+            if (k < nown && hm != 0u) {
+                uint8_t *dst = ring + (n & smask) * G::STAGE + (k % kGPS) * G::GSLOT + 2 * G::VB;
+                const int2 id = gids[k];
+                constexpr int P = D / 16; // 16-byte pieces of a quad
+#pragma unroll
+                for (int j = 0; j < 8 * P / 32; ++j) {
+                    const int idx = lane + 32 * j, q = idx / P, off = (q & 3) * D + 16 * (idx % P);
+                    if ((hm >> (4 * q)) & 0xFu) {
+                        const int blk = q >> 2;
+                        const uint32_t bid = (uint32_t)(blk ? id.y : id.x);
+                        cp_async16(dst + blk * G::LOB + off, lob + (uint64_t)bid * lstride + off);
+                    }
+                }
+            }
+            cp_async_commit();
+        };
+        uint32_t hm_next = nown > 0 ? hot_mask(0) : 0u;
+        fetch_lo(0, prc_n, hm_next); // group 0 lies in the next stage to be consumed
         const uint8_t *stg = ring;
         for (int k = 0; k < nown; ++k) {
             const bool first = k % kGPS == 0; // first group of a stage
@@ -1005,13 +938,12 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             }
             const float s2l = sc[k * 32 + lane];
             const float wl = ex2(s2l - m2);
-            float thr_k = thr2;
-            if (stream) { // the same running maximum as issue_lo computed for this group
-                run_v = fmaxf(run_v, warp_max_f(s2l));
-                thr_k = run_v + ltau;
-            }
-            const bool hotl = s2l >= thr_k;
-            const uint32_t hm = __ballot_sync(0xFFFFFFFFu, hotl);
+            const uint32_t hm = hm_next;
+            const bool hotl = (hm >> lane) & 1u;
+            if (k + 1 < nown)
+                hm_next = hot_mask(k + 1);
+            // group k + 1 lies in the next stage (prc_n) or in this one (prc_n - 1)
+            fetch_lo(k + 1, (k + 1) % kGPS == 0 ? prc_n : prc_n - 1, hm_next);
             if (a.s_bitmap && lane == 0) // refine set of the debug entry point, one bit per token
                 a.s_bitmap[(int64_t)srow[IR_ROW] * a.bitmap_words + srow[IR_G0] + (int)crank +
                            (warp + k * kWarps) * (int)C] = hm;
@@ -1054,7 +986,8 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
                 reinterpret_cast<uint4 *>(ybuf + pg * YS)[pt8] =
                     make_uint4(__byte_perm(t01, t23, 0x5410), __byte_perm(t01, t23, 0x7632), hb, 0u);
             }
-            __syncwarp();
+            cp_async_wait<1>(); // this lane's lo copies of group k (those of group k + 1 may fly)
+            __syncwarp();       // ... and every other lane's
             // ---- accumulate: channel quad vk, dp4a over the tokens of each token quad
             VSums acc;
 #pragma unroll
@@ -1192,7 +1125,6 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
                 float m2, l2, m0;
                 cluster_row_stats(sm.stat + (vr % 3) * kWarps * 4, C, lane, m2, l2, m0);
                 const float thr2 = row_threshold(m2, l2, m0);
-                release_row(vr, thr2);
                 consume_v(vr, m2, thr2);
                 m_prev = m2;
             }
@@ -1208,6 +1140,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     if (timed_out) // copies issued before the give-up must land before the shared memory is freed
         for (int n = drain_from; n < iss_n; ++n)
             mbar_wait(&full[n & smask], (n >> spw_log2) & 1, a.status, a.wait_ns);
+    cp_async_wait<0>(); // the last (possibly empty) lo commit group of this thread
     cluster_arrive(); // remote reads done
     cluster_wait();
 }
@@ -1915,8 +1848,8 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
                 int spw = 8;
                 while (spw > 2 && kernel_smem<BITS, D>(onepass, spw, capw, nbuf, near_cap) > budget)
                     spw >>= 1;
-                if (ov.stages)
-                    spw = ov.stages;
+                if (ov.stages) // at least 2: the two-phase reader fills the next stage's slot early
+                    spw = std::max(ov.stages, 2);
                 const int smem = kernel_smem<BITS, D>(onepass, spw, capw, nbuf, near_cap);
                 if (smem <= 0 || smem > 227 * 1024)
                     continue;

@@ -47,17 +47,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t tx
                  : "memory");
 }
 
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t tx)
-{
-    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(tx)
-                 : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
-{
-    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
 // Test the phase; a thread whose phase is not complete may be suspended in hardware for a
 // system-dependent time (no busy spinning).
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
@@ -99,6 +88,22 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
             smem_u32(dst)),
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
+}
+
+// Asynchronous 16-byte copy global -> shared by the calling thread; completion is tracked per
+// thread by commit groups (cp_async_commit, cp_async_wait).  Both addresses 16-byte aligned.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+// Close the calling thread's group of cp_async16 copies (an empty group is allowed).
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+// Wait until at most N of the calling thread's committed groups are still in flight.
+template <int N> __device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ uint32_t cluster_ctarank()
@@ -160,20 +165,6 @@ __device__ __forceinline__ float warp_max(float v)
     for (int o = 16; o > 0; o >>= 1)
         v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
     return v;
-}
-
-// x * 2^e computed exactly (power-of-two factors kept inside the normal range).
-__device__ __forceinline__ float mul_pow2(float x, int e)
-{
-    while (e > 127) {
-        x *= 1.7014118346046923e38f; // 2^127
-        e -= 127;
-    }
-    while (e < -126) {
-        x *= 1.1754943508222875e-38f; // 2^-126
-        e += 126;
-    }
-    return x * __int_as_float((e + 127) << 23);
 }
 
 template <typename T> __device__ __forceinline__ float to_f32(T v);
