@@ -537,8 +537,11 @@ __device__ __forceinline__ void cluster_row_stats(const float *stat, uint32_t C,
     l = __shfl_sync(0xFFFFFFFFu, warp_sum(mw == -INFINITY ? 0.f : lw * exp2f(mw - m)), 0); // one value for all lanes
 }
 
-// MINCTA: CTAs per SM the registers are budgeted for (4: <= 128 registers, 5: <= 96).
-template <int BITS, int D, typename DT, int MINCTA>
+// MINCTA: CTAs per SM the registers are budgeted for (4: <= 128 registers, 5: <= 96).  GEN:
+// the general build, which also serves the streaming rule, sliding windows, the refine-set
+// bitmap of the debug entry point and the wait test hook; launches that use none of them take
+// the build without (GEN = false), whose per-group path carries no tests for them.
+template <int BITS, int D, typename DT, int MINCTA, bool GEN>
 __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeArgs a, const int spw_log2, const int nbuf)
 {
     using G = Geo<BITS, D>;
@@ -553,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     static_assert(BITS == 4, "the exact-maximum reader serves 4-bit sources read with tau > 0");
     // streaming refine rule (LOOPKV_TAU_STREAM): per warp, tokens are tested against a running
     // maximum seeded with the row's largest sink score, in the warp's group order
-    const bool stream = a.tau_mode == LOOPKV_TAU_STREAM;
+    const bool stream = GEN && a.tau_mode == LOOPKV_TAU_STREAM;
     const float ltau = log2f(a.tau);
     const bool seq = nbuf == 1; // one score buffer: rows one after another (see the main loop)
     // byte distance between consecutive block ids in the pools (one block = H heads)
@@ -639,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         // sliding attention window: only the groups from the window's first token on (the
         // host launches windowed reads without overlap, so the near count is final here)
         int h0 = 0;
-        if (a.attn_window > 0) {
+        if (GEN && a.attn_window > 0) {
             const int nn = a.tail_len[b];
             h0 = window_first(a.attn_window, a.sink, hist, nn < 0 ? 0 : nn);
         }
@@ -696,7 +699,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         if (!seg_v) {
             if (lane == 0) {
                 mbar_arrive_expect_tx(fb, (uint32_t)ng * 2 * G::KB);
-                if (a.inject == LOOPKV_INJECT_STALLED_STAGE && n == 0 && warp == 0 && blockIdx.x == 0)
+                if (GEN && a.inject == LOOPKV_INJECT_STALLED_STAGE && n == 0 && warp == 0 && blockIdx.x == 0)
                     return; // test hook: the stage's bytes never arrive, so its wait runs out
                 for (int j = 0; j < ng; ++j) {
                     const int2 id = ids[j];
@@ -812,7 +815,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             }
             const uint8_t *st = stg + (k % kGPS) * G::GSLOT;
             float s2 = group_scores<BITS, D>(st, st + G::KB, scr, qreg, a.qscale, lane);
-            if (k == 0 && crank == 0 && warp == 0 && lane < srow[IR_M0])
+            if (GEN && k == 0 && crank == 0 && warp == 0 && lane < srow[IR_M0])
                 s2 = -INFINITY; // before the attention window
             sc[k * 32 + lane] = s2;
             mx = fmaxf(mx, s2);
@@ -828,7 +831,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
                                                                       a.near_cap * D;
             const int ws = srow[IR_WS], hist = srow[IR_HIST];
             for (int j = wg; j < tail; j += nw) {
-                const float s2 = near_attended(a, j, hist, tail)
+                const float s2 = (!GEN || near_attended(a, j, hist, tail))
                                      ? near_score<D, DT>(kt + (int64_t)near_slot(a, j, ws) * D, qreg, a.qscale, lane)
                                      : -INFINITY;
                 if (lane == 0)
@@ -944,7 +947,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
                 hm_next = hot_mask(k + 1);
             // group k + 1 lies in the next stage (prc_n) or in this one (prc_n - 1)
             fetch_lo(k + 1, (k + 1) % kGPS == 0 ? prc_n : prc_n - 1, hm_next);
-            if (a.s_bitmap && lane == 0) // refine set of the debug entry point, one bit per token
+            if (GEN && a.s_bitmap && lane == 0) // refine set of the debug entry point, one bit per token
                 a.s_bitmap[(int64_t)srow[IR_ROW] * a.bitmap_words + srow[IR_G0] + (int)crank +
                            (warp + k * kWarps) * (int)C] = hm;
             lsum += wl;
@@ -1387,7 +1390,7 @@ __device__ __forceinline__ void run1_tail(Run1<D> &r, float *red, const int lane
     __syncwarp();
 }
 
-template <int BITS, int D, typename DT, int MINCTA>
+template <int BITS, int D, typename DT, int MINCTA, bool GEN> // GEN: as for decode_kernel
 __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const DecodeArgs a, const int spw_log2)
 {
     using G = Geo<BITS, D>;
@@ -1465,7 +1468,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
             hist = 0;
         }
         int h0 = 0; // sliding attention window (see decode_kernel's setup_row)
-        if (a.attn_window > 0) {
+        if (GEN && a.attn_window > 0) {
             const int nn = a.tail_len[b];
             h0 = window_first(a.attn_window, a.sink, hist, nn < 0 ? 0 : nn);
         }
@@ -1509,7 +1512,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
         uint64_t *fb = &full[n & smask];
         if (lane == 0) {
             mbar_arrive_expect_tx(fb, 2 * G::HM + 2 * G::LOB);
-            if (a.inject == LOOPKV_INJECT_STALLED_STAGE && n == 0 && warp == 0 && blockIdx.x == 0)
+            if (GEN && a.inject == LOOPKV_INJECT_STALLED_STAGE && n == 0 && warp == 0 && blockIdx.x == 0)
                 return; // test hook: the stage's bytes never arrive, so its wait runs out
             bulk_g2s(st, seg_src + (uint64_t)(uint32_t)id.x * bstride, G::HM, fb);
             bulk_g2s(st + G::HM, seg_src + (uint64_t)(uint32_t)id.y * bstride, G::HM, fb);
@@ -1601,9 +1604,9 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
             }
             wait_stage(n);
             const uint8_t *st = ring + (n & smask) * G1::STAGE;
-            const int masked = k == 0 ? rm0 : 0; // tokens of the first group before a sliding window
+            const int masked = GEN && k == 0 ? rm0 : 0; // tokens of the first group before a sliding window
             run1_group<BITS, D>(st, st + G1::LOFF, scr, qreg, a.qscale, lane, run, masked);
-            if (a.s_bitmap && lane == 0) // refine set: every attended token (4-bit, tau <= 0) or none (2-bit)
+            if (GEN && a.s_bitmap && lane == 0) // refine set: every attended token (4-bit, tau <= 0) or none (2-bit)
                 a.s_bitmap[(int64_t)row * a.bitmap_words + rg0 + (int)crank + (warp + k * kWarps) * (int)C] =
                     BITS == 4 ? ~((1u << masked) - 1u) : 0u;
         }
@@ -1738,15 +1741,20 @@ int launch_shape(K kern, const DecodeShape &shp, bool pdl, cudaStream_t s, Args.
 template <int BITS, int D, typename DT>
 int launch_t(const DecodeArgs &a, const DecodeShape &shp, bool pdl, cudaStream_t s)
 {
+    // the general build for the modes that the lean one leaves out
+    const bool gen = a.s_bitmap != nullptr || a.tau_mode == LOOPKV_TAU_STREAM || a.attn_window > 0 ||
+                     a.inject != LOOPKV_INJECT_NONE;
     if constexpr (BITS == 4) {
         if (!shp.onepass) {
-            auto kern = shp.min_ctas == 5 ? decode_kernel<BITS, D, DT, 5> : decode_kernel<BITS, D, DT, 4>;
+            auto kern = shp.min_ctas == 5 ? (gen ? decode_kernel<BITS, D, DT, 5, true> : decode_kernel<BITS, D, DT, 5, false>)
+                                          : (gen ? decode_kernel<BITS, D, DT, 4, true> : decode_kernel<BITS, D, DT, 4, false>);
             return launch_shape(kern, shp, pdl, s, a, shp.stages_log2, shp.score_bufs);
         }
     }
     if (!shp.onepass)
         return LOOPKV_ERR_CUDA; // 2-bit sources have no refine set: always the single-pass reader
-    return launch_shape(decode_kernel_1p<BITS, D, DT, 4>, shp, pdl, s, a, shp.stages_log2);
+    return launch_shape(gen ? decode_kernel_1p<BITS, D, DT, 4, true> : decode_kernel_1p<BITS, D, DT, 4, false>, shp, pdl,
+                        s, a, shp.stages_log2);
 }
 
 // Clusters of size C that can be resident at once for this kernel and shared memory.
@@ -1854,11 +1862,12 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
                 if (smem <= 0 || smem > 227 * 1024)
                     continue;
                 int ncl = 0;
+                // occupancy of the general build (the lean one has the same launch bounds)
                 if (onepass)
-                    ncl = max_active_clusters(decode_kernel_1p<BITS, D, DT, 4>, C, smem);
+                    ncl = max_active_clusters(decode_kernel_1p<BITS, D, DT, 4, true>, C, smem);
                 else if constexpr (BITS == 4)
-                    ncl = want_ctas == 5 ? max_active_clusters(decode_kernel<BITS, D, DT, 5>, C, smem)
-                                         : max_active_clusters(decode_kernel<BITS, D, DT, 4>, C, smem);
+                    ncl = want_ctas == 5 ? max_active_clusters(decode_kernel<BITS, D, DT, 5, true>, C, smem)
+                                         : max_active_clusters(decode_kernel<BITS, D, DT, 4, true>, C, smem);
                 if (ncl <= 0)
                     continue;
                 if (ncl > rows)

@@ -205,8 +205,8 @@ def test_append_flush_sequence():
 
 @pytest.mark.parametrize("lengths", [[4096, 1000, 33], [2048] * 3])
 def test_repeated_single_pass_decode_is_bit_identical(lengths):
-    # 2-bit cells and tau = 0 reads split long rows across CTAs and merge the pieces through
-    # per-row counters that the merging CTA resets: a second launch must repeat the first.
+    # 2-bit cells and tau = 0 reads (single-pass reader, rows split over the CTAs of a cluster
+    # and merged through distributed shared memory): a second launch must repeat the first.
     modes = [L.CELL_2B, L.CELL_4B]
     w = synth.Workload("repeat", 1, 2, 4, 128, 3, lengths, torch.bfloat16, modes, 0.0, seed=11)
     m = Model(w)
@@ -230,6 +230,29 @@ def test_share_cell_with_final_loop_query_is_bit_identical():
     b = m.cache.decode(1, 0, q)
     m.cache.check("share")
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("tau,tau_mode,D,dtype", [(0.01, 0, 128, torch.bfloat16), (0.05, 1, 128, torch.bfloat16),
+                                              (0.0, 0, 128, torch.bfloat16), (0.02, 0, 64, torch.float32)])
+def test_lean_build_matches_general_build(tau, tau_mode, D, dtype):
+    """loopkv_decode without debug outputs runs the lean kernel builds (no refine-set bitmap,
+    streaming rule, sliding window or test hook on their per-group path); they must give the
+    outputs of the general builds, which the other cases check against the oracle, bit for bit."""
+    modes = [L.CELL_4B, L.CELL_SHARE, L.CELL_2B, L.CELL_4B]  # loop 0: [4b, share], loop 1: [2b, 4b]
+    w = synth.Workload("lean", 2, 2, 4, D, 3, [4096, 1000, 33], dtype, modes, tau, tau_mode=tau_mode,
+                       append_steps=5, seed=21)
+    m = Model(w)
+    m.ingest()
+    for step in range(5):
+        m.append_step(step)
+    for la in range(2):
+        for lp in range(2):
+            q = _q(w, 4, la, lp)
+            lean = m.cache.decode(lp, la, q)
+            general, _, _, _ = m.cache.decode_debug(lp, la, q)
+            m.cache.check("lean vs general build")
+            assert torch.equal(lean, general), f"cell ({lp},{la})"
+    m.check_cell(0, 0, _q(w, 4, 0, 0), where="lean")
 
 
 @pytest.mark.parametrize("name,B,T,modes,tau,steps", [
