@@ -151,7 +151,7 @@ class Runner:
         self.w = w
         self.dev = device
         self.plan = L.Plan(w.n_layers, w.n_loops, w.H, w.D, w.B, w.max_blocks, w.modes, w.tau, w.tau_mode,
-                           w.dtype)
+                           w.dtype, w.sink, w.window)
         for layer, win in w.layer_windows.items():  # sliding-window layers
             self.plan.set_window(layer, win)
         self.cache = L.Cache(self.plan, device=device)

@@ -329,17 +329,53 @@ struct VSums {
     }
 };
 
-// q . k of one unquantized (near) token, in log2 units: the lane holds channels 4 lane ..
-// 4 lane + 3 of the exact query; krow: the token's D keys.  Warp-uniform result.
-template <int D, typename DT>
-__device__ __forceinline__ float near_score(const DT *krow, const float (&qreg)[4], const float qscale, const int lane)
+// Four consecutive elements of a near-region row as floats (bf16 widens exactly); p is
+// 8-byte (bf16) or 16-byte (fp32) aligned.
+__device__ __forceinline__ void load4f(const __nv_bfloat16 *p, float (&f)[4])
 {
-    float s = 0.f;
-    if (lane < D / 4) {
-        const DT *k4 = krow + 4 * lane;
-        s = fmaf(qreg[0], to_f32(k4[0]), fmaf(qreg[1], to_f32(k4[1]), fmaf(qreg[2], to_f32(k4[2]), qreg[3] * to_f32(k4[3]))));
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    f[0] = __uint_as_float(u.x << 16);
+    f[1] = __uint_as_float(u.x & 0xFFFF0000u);
+    f[2] = __uint_as_float(u.y << 16);
+    f[3] = __uint_as_float(u.y & 0xFFFF0000u);
+}
+__device__ __forceinline__ void load4f(const float *p, float (&f)[4])
+{
+    const float4 v = *reinterpret_cast<const float4 *>(p);
+    f[0] = v.x, f[1] = v.y, f[2] = v.z, f[3] = v.w;
+}
+
+// Near tokens a warp takes per round of loads.
+constexpr int kNearBatch = 4;
+
+// q . k of up to kNearBatch unquantized (near) tokens, in log2 units: key rows krow[u] (nullptr:
+// no token, score 0); the lane holds channels 4 lane .. 4 lane + 3 of the exact query.  Every
+// load is issued before the first product, so that one memory latency covers the batch.
+// Warp-uniform results.
+template <int D, typename DT>
+__device__ __forceinline__ void near_scores(const DT *const (&krow)[kNearBatch], const float (&qreg)[4],
+                                            const float qscale, const int lane, float (&s)[kNearBatch])
+{
+    float k[kNearBatch][4];
+#pragma unroll
+    for (int u = 0; u < kNearBatch; ++u) {
+        k[u][0] = k[u][1] = k[u][2] = k[u][3] = 0.f;
+        if (lane < D / 4 && krow[u] != nullptr)
+            load4f(krow[u] + 4 * lane, k[u]);
     }
-    return warp_sum(s) * qscale;
+    float p[kNearBatch];
+#pragma unroll
+    for (int u = 0; u < kNearBatch; ++u)
+        p[u] = lane < D / 4 ? fmaf(qreg[0], k[u][0], fmaf(qreg[1], k[u][1], fmaf(qreg[2], k[u][2], qreg[3] * k[u][3])))
+                            : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int u = 0; u < kNearBatch; ++u)
+            p[u] += __shfl_xor_sync(0xFFFFFFFFu, p[u], o);
+#pragma unroll
+    for (int u = 0; u < kNearBatch; ++u)
+        s[u] = p[u] * qscale;
 }
 
 // Slot of near token j (0 .. near tokens - 1) in a (cell, request)'s near region: the sink
@@ -830,15 +866,29 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)srow[IR_B] * 2 * a.H + srow[IR_H]) *
                                                                       a.near_cap * D;
             const int ws = srow[IR_WS], hist = srow[IR_HIST];
-            for (int j = wg; j < tail; j += nw) {
-                const float s2 = (!GEN || near_attended(a, j, hist, tail))
-                                     ? near_score<D, DT>(kt + (int64_t)near_slot(a, j, ws) * D, qreg, a.qscale, lane)
-                                     : -INFINITY;
-                if (lane == 0)
-                    tsc[j] = s2;
-                mx = fmaxf(mx, s2);
-                if (j < a.sink)
-                    smx = fmaxf(smx, s2);
+            for (int j0 = wg; j0 < tail; j0 += kNearBatch * nw) { // a batch of this warp's near tokens
+                const DT *rows[kNearBatch];
+#pragma unroll
+                for (int u = 0; u < kNearBatch; ++u) {
+                    const int j = j0 + u * nw;
+                    rows[u] = j < tail && (!GEN || near_attended(a, j, hist, tail))
+                                  ? kt + (int64_t)near_slot(a, j, ws) * D
+                                  : nullptr;
+                }
+                float sb[kNearBatch];
+                near_scores<D, DT>(rows, qreg, a.qscale, lane, sb);
+#pragma unroll
+                for (int u = 0; u < kNearBatch; ++u) {
+                    const int j = j0 + u * nw;
+                    if (j < tail) {
+                        const float s2 = rows[u] != nullptr ? sb[u] : -INFINITY; // -inf: outside the window
+                        if (lane == 0)
+                            tsc[j] = s2;
+                        mx = fmaxf(mx, s2);
+                        if (j < a.sink)
+                            smx = fmaxf(smx, s2);
+                    }
+                }
             }
             __syncwarp();
         }
@@ -1048,15 +1098,38 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             const float *tsc = sm.tscores + (ri & 1) * a.near_cap;
             const DT *vt0 = reinterpret_cast<const DT *>(a.tail) + ((int64_t)(b * 2 + 1) * a.H + h) * a.near_cap * D;
             const int ws = srow[IR_WS];
-            float tl = 0.f;
-            for (int t = wg; t < tail; t += nw) {
-                const float w = exp2f(tsc[t] - m2);
-                tl += w;
-                const DT *vt = vt0 + (int64_t)near_slot(a, t, ws) * D;
+            float tl = 0.f, acc[D / 32];
 #pragma unroll
-                for (int c4 = 0; c4 < D / 32; ++c4)
-                    red[lane + 32 * c4] = fmaf(w, to_f32(vt[lane + 32 * c4]), red[lane + 32 * c4]);
+            for (int c4 = 0; c4 < D / 32; ++c4)
+                acc[c4] = 0.f;
+            for (int t0 = wg; t0 < tail; t0 += kNearBatch * nw) { // a batch of tokens, loads first
+                float w[kNearBatch], v[kNearBatch][D / 32];
+#pragma unroll
+                for (int u = 0; u < kNearBatch; ++u) {
+                    const int t = t0 + u * nw;
+                    w[u] = 0.f;
+#pragma unroll
+                    for (int c4 = 0; c4 < D / 32; ++c4)
+                        v[u][c4] = 0.f;
+                    if (t < tail) { // tokens outside a sliding window have score -inf: weight 0
+                        const DT *vt = vt0 + (int64_t)near_slot(a, t, ws) * D;
+                        w[u] = exp2f(tsc[t] - m2);
+#pragma unroll
+                        for (int c4 = 0; c4 < D / 32; ++c4)
+                            v[u][c4] = to_f32(vt[lane + 32 * c4]);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < kNearBatch; ++u) {
+                    tl += w[u];
+#pragma unroll
+                    for (int c4 = 0; c4 < D / 32; ++c4)
+                        acc[c4] = fmaf(w[u], v[u][c4], acc[c4]);
+                }
             }
+#pragma unroll
+            for (int c4 = 0; c4 < D / 32; ++c4)
+                red[lane + 32 * c4] += acc[c4];
             __syncwarp();
             if (lane == 0)
                 red[D] += tl;
@@ -1368,24 +1441,39 @@ __device__ __forceinline__ void run1_tail(Run1<D> &r, float *red, const int lane
                                           const DecodeArgs &a, const DT *kt, const DT *vt0, const int ws,
                                           const int hist, const int j0, const int stride, const int n)
 {
-    for (int j = j0; j < n; j += stride) {
-        if (!near_attended(a, j, hist, n))
-            continue;
-        const int slot = near_slot(a, j, ws);
-        const float s2 = near_score<D, DT>(kt + (int64_t)slot * D, qreg, a.qscale, lane);
-        if (s2 > r.m) { // warp-uniform
-            const float f = ex2(r.m - s2);
-            for (int c = lane; c <= D; c += 32)
-                red[c] *= f;
-            r.m = s2;
-        }
-        const float w = ex2(s2 - r.m);
-        const DT *vt = vt0 + (int64_t)slot * D;
+    for (int jb = j0; jb < n; jb += kNearBatch * stride) { // a batch of tokens: keys and values loaded first
+        const DT *krow[kNearBatch];
+        float v[kNearBatch][D / 32];
 #pragma unroll
-        for (int c4 = 0; c4 < D / 32; ++c4)
-            red[lane + 32 * c4] = fmaf(w, to_f32(vt[lane + 32 * c4]), red[lane + 32 * c4]);
-        if (lane == 0)
-            red[D] += w;
+        for (int u = 0; u < kNearBatch; ++u) {
+            const int j = jb + u * stride;
+            const bool att = j < n && near_attended(a, j, hist, n);
+            const int slot = att ? near_slot(a, j, ws) : 0;
+            krow[u] = att ? kt + (int64_t)slot * D : nullptr;
+#pragma unroll
+            for (int c4 = 0; c4 < D / 32; ++c4)
+                v[u][c4] = att ? to_f32(vt0[(int64_t)slot * D + lane + 32 * c4]) : 0.f;
+        }
+        float sb[kNearBatch];
+        near_scores<D, DT>(krow, qreg, a.qscale, lane, sb);
+#pragma unroll
+        for (int u = 0; u < kNearBatch; ++u) {
+            if (krow[u] == nullptr)
+                continue; // warp-uniform
+            const float s2 = sb[u];
+            if (s2 > r.m) { // warp-uniform
+                const float f = ex2(r.m - s2);
+                for (int c = lane; c <= D; c += 32)
+                    red[c] *= f;
+                r.m = s2;
+            }
+            const float w = ex2(s2 - r.m);
+#pragma unroll
+            for (int c4 = 0; c4 < D / 32; ++c4)
+                red[lane + 32 * c4] = fmaf(w, v[u][c4], red[lane + 32 * c4]);
+            if (lane == 0)
+                red[D] += w;
+        }
     }
     __syncwarp();
 }

@@ -45,6 +45,8 @@ class Workload:
     append_steps: int = 0  # decode steps that append one token per request per cell
     seed: int = 0
     layer_windows: dict = dataclasses.field(default_factory=dict)  # layer -> sliding window (tokens)
+    sink: int = 0          # BF16 sink tokens of every (cell, request)
+    window: int = 0        # BF16 recent-window tokens (the near region holds window .. window + 31)
 
     @property
     def n_cells(self):
@@ -101,6 +103,12 @@ def workload(name: str, seed: int = 0) -> Workload:
         B = 32 * 8192 // T
         modes = seeded_plan(48, 4, [0, 1, 2], 0.35, 0.25, seed)
         return Workload(name, 48, 4, 16, 128, B, [T] * B, torch.bfloat16, modes, 0.01, seed=seed)
+    if name == "mixed_8k_sw":
+        # mixed_8k with the paper's BF16 near region: a 32-token sink and a 256-token window
+        # (LoopKV §2.3, §3.4); the history between them is quantized as in mixed_8k
+        w = workload("mixed_8k", seed)
+        w.name, w.sink, w.window = "mixed_8k_sw", 32, 256
+        return w
     if name == "dory_16k":
         # Dory-4B-shaped recurrent block (LoopKV §2.1: 20 recurrent attention layers, 5 with full
         # attention and 15 with a sliding window).  The pages give neither the loop count, the
@@ -114,7 +122,7 @@ def workload(name: str, seed: int = 0) -> Workload:
 
 
 WORKLOADS = ["tiny", "kivi4_8k", "mixed_8k", "long_16k", "ragged_2p6b", "ouro2p6b_8k", "ouro2p6b_16k",
-             "ouro2p6b_32k", "dory_16k"]
+             "ouro2p6b_32k", "dory_16k", "mixed_8k_sw"]
 
 
 def _gen(seed: int, device) -> torch.Generator:
