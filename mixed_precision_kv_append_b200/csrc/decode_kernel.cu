@@ -386,6 +386,21 @@ __device__ __forceinline__ int near_slot(const DecodeArgs &a, int j, int ws)
     return j < a.sink ? j : a.sink + (ws + (j - a.sink)) % a.wring;
 }
 
+// Warm L2 with the rows of near tokens j0, j0 + stride, ... < n of one (cell, request, K or V,
+// head) near region `base` (rows of D elements in near_slot order), a 128-byte line per lane and
+// step: the rows are read after the row's history groups, long after this call.
+template <int D, typename DT>
+__device__ __forceinline__ void prefetch_near(const DecodeArgs &a, const DT *base, const int ws, const int j0,
+                                              const int stride, const int n, const int lane)
+{
+    constexpr int LPR = D * (int)sizeof(DT) / 128; // lines per row
+    const int cnt = n > j0 ? (n - j0 + stride - 1) / stride : 0;
+    for (int i = lane; i < cnt * LPR; i += 32) {
+        const int j = j0 + (i / LPR) * stride;
+        prefetch_l2_keep(reinterpret_cast<const char *>(base + (int64_t)near_slot(a, j, ws) * D) + 128 * (i % LPR));
+    }
+}
+
 struct Smem {
     uint8_t *ring;     // [kWarps][spw][STAGE] stage slots (kGPS groups each), a private slice per warp
     uint64_t *full;    // [kWarps][spw] completion barriers of the slots
@@ -830,6 +845,11 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             }
             __syncwarp();
         }
+        const int wg = (int)crank * kWarps + warp, nw = (int)C * kWarps; // near token j: warp j mod nw
+        if (tail > wg)
+            prefetch_near<D, DT>(a, reinterpret_cast<const DT *>(a.tail) +
+                                        ((int64_t)srow[IR_B] * 2 * a.H + srow[IR_H]) * a.near_cap * D,
+                                 srow[IR_WS], wg, nw, tail, lane);
         // lane owns the channel quad 4*lane .. 4*lane+3 (lanes >= D/4 own none)
         const bool ownq = lane < G::NQ;
         float qreg[4];
@@ -860,7 +880,6 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         // tail tokens (exact keys), dealt over every warp of the cluster: token j to warp
         // j mod (C * kWarps) of the cluster, so that no warp carries the whole tail
         float *tsc = sm.tscores + (ri & 1) * a.near_cap;
-        const int wg = (int)crank * kWarps + warp, nw = (int)C * kWarps;
         float smx = -INFINITY; // largest sink score of this warp's near tokens
         if (tail > wg) {
             const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)srow[IR_B] * 2 * a.H + srow[IR_H]) *
@@ -924,6 +943,10 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     auto consume_v = [&](int ri, float m2, float thr2) {
         const int32_t *srow = irow_of(ri);
         const int nown = srow[IR_N], tail = srow[IR_TAIL];
+        if (tail > (int)crank * kWarps + warp) // this warp's near values, read after its groups
+            prefetch_near<D, DT>(a, reinterpret_cast<const DT *>(a.tail) +
+                                        ((int64_t)(srow[IR_B] * 2 + 1) * a.H + srow[IR_H]) * a.near_cap * D,
+                                 srow[IR_WS], (int)crank * kWarps + warp, (int)C * kWarps, tail, lane);
         const float *sc = scores_of(ri);
         constexpr int NCG = G::NCG;
         constexpr int YS = 40; // word stride of a group's row in the transpose (conflict-free both ways)
@@ -1672,6 +1695,12 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
                 tail = 0;
                 ws = 0;
             }
+        }
+        if (tail > (int)crank * kWarps + warp) { // this warp's near keys and values, read after its groups
+            const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)rb * 2 * a.H + rh) * a.near_cap * D;
+            prefetch_near<D, DT>(a, kt, ws, (int)crank * kWarps + warp, (int)C * kWarps, tail, lane);
+            prefetch_near<D, DT>(a, kt + (int64_t)a.H * a.near_cap * D, ws, (int)crank * kWarps + warp, (int)C * kWarps,
+                                 tail, lane);
         }
         float qreg[4];
         {

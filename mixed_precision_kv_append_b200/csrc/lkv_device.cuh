@@ -90,6 +90,13 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         : "memory");
 }
 
+// Hint: bring the 128-byte line holding p into L2 with high retention priority (no data is
+// returned; p must be a valid global address).
+__device__ __forceinline__ void prefetch_l2_keep(const void *p)
+{
+    asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p));
+}
+
 // Asynchronous 16-byte copy global -> shared by the calling thread; completion is tracked per
 // thread by commit groups (cp_async_commit, cp_async_wait).  Both addresses 16-byte aligned.
 __device__ __forceinline__ void cp_async16(void *dst, const void *src)
