@@ -386,6 +386,23 @@ __device__ __forceinline__ int near_slot(const DecodeArgs &a, int j, int ws)
     return j < a.sink ? j : a.sink + (ws + (j - a.sink)) % a.wring;
 }
 
+// Near rows per chunk of the two-phase reader's ring (one sub-slot: 16 D bytes, 2 KiB at D = 128).
+template <typename DT> __host__ __device__ constexpr int near_chunk_rows() { return 16 / (int)sizeof(DT); }
+
+// Logical near index (sink first, then the window from its oldest token, as near_slot orders
+// them) of physical slot s of a near region holding nnear tokens, or -1 when the slot is empty.
+__device__ __forceinline__ int near_index(const DecodeArgs &a, const int s, const int ws, const int nnear)
+{
+    int j = s;
+    if (s >= a.sink) {
+        int r = s - a.sink - ws;
+        if (r < 0)
+            r += a.wring;
+        j = a.sink + r;
+    }
+    return j < nnear ? j : -1;
+}
+
 // Warm L2 with the rows of near tokens j0, j0 + stride, ... < n of one (cell, request, K or V,
 // head) near region `base` (rows of D elements in near_slot order), a 128-byte line per lane and
 // step: the rows are read after the row's history groups, long after this call.
@@ -424,6 +441,7 @@ enum {
     IR_G0,   // first history group inside the attention window
     IR_M0,   // tokens of group IR_G0 before the window
     IR_HIST, // history tokens of the row
+    IR_NC,   // near-region chunks read by this warp (streamed near regions)
     IR_N_FIELDS = 16
 };
 
@@ -588,13 +606,16 @@ __device__ __forceinline__ void cluster_row_stats(const float *stat, uint32_t C,
     l = __shfl_sync(0xFFFFFFFFu, warp_sum(mw == -INFINITY ? 0.f : lw * exp2f(mw - m)), 0); // one value for all lanes
 }
 
-// MINCTA: CTAs per SM the registers are budgeted for (4: <= 128 registers, 5: <= 96).  GEN:
-// the general build, which also serves the streaming rule, sliding windows, the refine-set
-// bitmap of the debug entry point and the wait test hook; launches that use none of them take
-// the build without (GEN = false), whose per-group path carries no tests for them.
-template <int BITS, int D, typename DT, int MINCTA, bool GEN>
+// MINCTA: CTAs per SM the registers are budgeted for (4: <= 128 registers, 5: <= 96).  VAR: the
+// build.  2 (general) serves everything: the streaming rule, sliding windows, the refine-set bitmap
+// of the debug entry point, the wait test hook and streamed near regions.  Launches that use none
+// of the first four take a lean build, whose per-group path carries no tests for them: 1 when the
+// near region is streamed (a sink or a window), else 0.
+template <int BITS, int D, typename DT, int MINCTA, int VAR>
 __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeArgs a, const int spw_log2, const int nbuf)
 {
+    constexpr bool GEN = VAR == 2;
+    constexpr bool NSC = VAR >= 1; // the streamed near path is compiled in
     using G = Geo<BITS, D>;
     extern __shared__ __align__(128) uint8_t smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -610,6 +631,18 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     const bool stream = GEN && a.tau_mode == LOOPKV_TAU_STREAM;
     const float ltau = log2f(a.tau);
     const bool seq = nbuf == 1; // one score buffer: rows one after another (see the main loop)
+    // A near region beyond a 32-token tail (a sink or a window) streams through the ring in chunks
+    // of NR physical rows, dealt over the cluster's warps like history groups: chunk c to warp
+    // c mod 4C.  Slots without a token are read too and get score -inf.
+    const bool nstream = NSC && a.near_cap > 32;
+    constexpr int NR = near_chunk_rows<DT>();
+    constexpr uint32_t NRB = (uint32_t)(NR * D * sizeof(DT)); // bytes of a chunk
+    static_assert(NR * D * (int)sizeof(DT) <= G::GSLOT, "a near chunk fills at most one sub-slot");
+    // warp rank in the cluster and warps of the cluster, recomputed where used (cheaper than
+    // holding them in registers through the whole kernel)
+    auto wgl = [&]() { return (int)crank * kWarps + warp; };
+    auto nwl = [&]() { return (int)C * kWarps; };
+    bool dep_ok = false; // the previous grid of the stream has finished (near rows are final)
     // byte distance between consecutive block ids in the pools (one block = H heads)
     const uint32_t bstride = (uint32_t)a.H * G::HM, lstride = (uint32_t)a.H * G::LOB;
 
@@ -670,6 +703,8 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     int seg_n = 0;                 // groups of the segment's row owned by this warp
     bool seg_v = false;
     const uint8_t *seg_src = nullptr; // main pool + head offset (+ K part) of the segment's row
+    const uint8_t *seg_near = nullptr; // near region (K or V) of the segment's row
+    int seg_gst = 0, seg_nc = 0;      // group stages, then near chunks of this warp
     const int2 *seg_ids = nullptr;
     int setup_upto = -1;           // rows 0..setup_upto have their parameters and ids in place
     // After one bounded wait gives up, later waits are skipped, nothing new is issued, and the
@@ -728,6 +763,10 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             st[IR_G0] = g0;
             st[IR_M0] = h0 & 31;
             st[IR_HIST] = hist;
+            if (NSC) {
+                const int nch = nstream ? a.near_cap / NR : 0;
+                st[IR_NC] = nch > wgl() ? (nch - wgl() + nwl() - 1) / nwl() : 0;
+            }
         }
         __syncwarp();
     };
@@ -735,17 +774,33 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         segment(iss_sig, nrows, seq, seg_v, seg_ri);
         const int32_t *st = irow_of(seg_ri);
         seg_n = st[IR_N];
-        seg_len = (seg_n + kGPS - 1) / kGPS;
+        seg_gst = (seg_n + kGPS - 1) / kGPS;
+        seg_len = seg_gst;
         seg_src = a.main + (size_t)st[IR_H] * G::HM + (seg_v ? G::KB : 0);
+        if (NSC) {
+            seg_nc = st[IR_NC];
+            seg_len += (seg_nc + kGPS - 1) / kGPS;
+            seg_near = reinterpret_cast<const uint8_t *>(a.tail) +
+                       ((int64_t)(st[IR_B] * 2 + (seg_v ? 1 : 0)) * a.H + st[IR_H]) * a.near_cap * D * sizeof(DT);
+        }
         seg_ids = reinterpret_cast<const int2 *>(ids_of(seg_ri));
     };
     // Stage k2 of the current segment: groups kGPS*k2 .. kGPS*k2 + ng - 1 of the row, group
     // j into sub-slot j.
     auto issue_stage = [&](int n) {
         const int k2 = iss_k;
-        const int ng = min(kGPS, seg_n - kGPS * k2);
         uint8_t *stg = ring + (n & smask) * G::STAGE;
         uint64_t *fb = &full[n & smask];
+        if (NSC && k2 >= seg_gst) { // near stage: this warp's chunks kGPS*(k2 - seg_gst) .. of the row
+            const int c0 = kGPS * (k2 - seg_gst), ncs = min(kGPS, seg_nc - c0);
+            if (lane == 0) {
+                mbar_arrive_expect_tx(fb, (uint32_t)ncs * NRB);
+                for (int j = 0; j < ncs; ++j)
+                    bulk_g2s(stg + j * G::GSLOT, seg_near + (size_t)(wgl() + (c0 + j) * nwl()) * NRB, NRB, fb);
+            }
+            return;
+        }
+        const int ng = min(kGPS, seg_n - kGPS * k2);
         const int2 *ids = seg_ids + kGPS * k2;
         if (!seg_v) {
             if (lane == 0) {
@@ -777,7 +832,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             return; // after a give-up nothing new is issued
         for (;;) {
             if (iss_k < seg_len) {
-                if (iss_n >= limit)
+                if (iss_n >= limit || (NSC && !dep_ok && iss_k >= seg_gst)) // near rows: after the grid dependency
                     break;
                 issue_stage(iss_n);
                 ++iss_k;
@@ -827,6 +882,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             // launches that the host does not let a decode overlap.
             pump(prc_n + spw);
             asm volatile("griddepcontrol.wait;" ::: "memory");
+            dep_ok = true;
         }
         int tail = srow[IR_TAIL];
         if (tail < 0) { // near tokens and ring start (an append may just have written them)
@@ -845,8 +901,8 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
             }
             __syncwarp();
         }
-        const int wg = (int)crank * kWarps + warp, nw = (int)C * kWarps; // near token j: warp j mod nw
-        if (tail > wg)
+        const int wg = wgl(), nw = nwl(); // near token j: warp j mod nw
+        if (!nstream && tail > wg)
             prefetch_near<D, DT>(a, reinterpret_cast<const DT *>(a.tail) +
                                         ((int64_t)srow[IR_B] * 2 * a.H + srow[IR_H]) * a.near_cap * D,
                                  srow[IR_WS], wg, nw, tail, lane);
@@ -879,9 +935,48 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         }
         // tail tokens (exact keys), dealt over every warp of the cluster: token j to warp
         // j mod (C * kWarps) of the cluster, so that no warp carries the whole tail
-        float *tsc = sm.tscores + (ri & 1) * a.near_cap;
+        float *tsc = sm.tscores + (ri & 1) * a.near_cap; // by near index (register path) or slot (chunks)
         float smx = -INFINITY; // largest sink score of this warp's near tokens
-        if (tail > wg) {
+        const int ncw = nstream ? srow[IR_NC] : 0;
+        if (nstream) { // this warp's chunks of the streamed near region
+            const int ws = srow[IR_WS], hist = srow[IR_HIST];
+            for (int c = 0; c < ncw; ++c) {
+                if (c % kGPS == 0) {
+                    const int n = prc_n++;
+                    if (iss_n < n + spw)
+                        pump(n + spw);
+                    wait_stage(n);
+                    stg = ring + (n & smask) * G::STAGE;
+                }
+                const DT *rows = reinterpret_cast<const DT *>(stg + (c % kGPS) * G::GSLOT);
+                float p[NR];
+#pragma unroll
+                for (int r = 0; r < NR; ++r) { // lane: channels 4 lane .. 4 lane + 3 of every row
+                    float k4[4] = {0.f, 0.f, 0.f, 0.f};
+                    if (lane < D / 4)
+                        load4f(rows + r * D + 4 * lane, k4);
+                    p[r] = lane < D / 4 ? fmaf(qreg[0], k4[0], fmaf(qreg[1], k4[1], fmaf(qreg[2], k4[2], qreg[3] * k4[3])))
+                                        : 0.f;
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                    for (int r = 0; r < NR; ++r)
+                        p[r] += __shfl_xor_sync(0xFFFFFFFFu, p[r], o);
+                const int slot0 = (wg + c * nw) * NR;
+#pragma unroll
+                for (int r = 0; r < NR; ++r) {
+                    const int j = near_index(a, slot0 + r, ws, tail);
+                    const float s2 = j >= 0 && (!GEN || near_attended(a, j, hist, tail)) ? p[r] * a.qscale : -INFINITY;
+                    if (lane == 0)
+                        tsc[slot0 + r] = s2;
+                    mx = fmaxf(mx, s2);
+                    if (j >= 0 && j < a.sink)
+                        smx = fmaxf(smx, s2);
+                }
+                __syncwarp();
+            }
+        } else if (tail > wg) {
             const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)srow[IR_B] * 2 * a.H + srow[IR_H]) *
                                                                       a.near_cap * D;
             const int ws = srow[IR_WS], hist = srow[IR_HIST];
@@ -916,8 +1011,12 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         if (a.tau_mode == LOOPKV_TAU_ABS_PROB && mx != -INFINITY) {
             for (int k = 0; k < nown; ++k)
                 ls += exp2f(sc[k * 32 + lane] - mx);
-            for (int j = wg + lane * nw; j < tail; j += 32 * nw)
-                ls += exp2f(tsc[j] - mx);
+            if (nstream)
+                for (int i = lane; i < ncw * NR; i += 32)
+                    ls += exp2f(tsc[(wg + (i / NR) * nw) * NR + i % NR] - mx);
+            else
+                for (int j = wg + lane * nw; j < tail; j += 32 * nw)
+                    ls += exp2f(tsc[j] - mx);
             ls = warp_sum(ls);
         }
         if (lane == 0) {
@@ -943,7 +1042,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     auto consume_v = [&](int ri, float m2, float thr2) {
         const int32_t *srow = irow_of(ri);
         const int nown = srow[IR_N], tail = srow[IR_TAIL];
-        if (tail > (int)crank * kWarps + warp) // this warp's near values, read after its groups
+        if (!nstream && tail > wgl()) // this warp's near values, read after its groups
             prefetch_near<D, DT>(a, reinterpret_cast<const DT *>(a.tail) +
                                         ((int64_t)(srow[IR_B] * 2 + 1) * a.H + srow[IR_H]) * a.near_cap * D,
                                  srow[IR_WS], (int)crank * kWarps + warp, (int)C * kWarps, tail, lane);
@@ -1115,8 +1214,46 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
         if (lane == 0)
             red[D] = lsum;
         __syncwarp();
-        const int wg = (int)crank * kWarps + warp, nw = (int)C * kWarps;
-        if (tail > wg) { // this warp's tail tokens (see consume_k), exact values
+        const int wg = wgl(), nw = nwl();
+        if (nstream) { // this warp's chunks of the streamed near region; scores by slot from the K pass
+            const int ncw = srow[IR_NC];
+            const float *tsc = sm.tscores + (ri & 1) * a.near_cap;
+            float tl = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f}; // lane: channels 4 lane .. 4 lane + 3
+            for (int c = 0; c < ncw; ++c) {
+                if (c % kGPS == 0) {
+                    const int n = prc_n++;
+                    if (iss_n < n + spw)
+                        pump(n + spw);
+                    wait_stage(n);
+                    stg = ring + (n & smask) * G::STAGE;
+                }
+                const DT *rows = reinterpret_cast<const DT *>(stg + (c % kGPS) * G::GSLOT);
+                const int slot0 = (wg + c * nw) * NR;
+#pragma unroll
+                for (int r = 0; r < NR; ++r) {
+                    const float s2 = tsc[slot0 + r];
+                    if (s2 != -INFINITY) { // warp-uniform: empty slots and tokens outside a window are -inf
+                        const float w = exp2f(s2 - m2);
+                        tl += w;
+                        if (lane < D / 4) {
+                            float v4[4];
+                            load4f(rows + r * D + 4 * lane, v4);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                acc[i] = fmaf(w, v4[i], acc[i]);
+                        }
+                    }
+                }
+                __syncwarp();
+            }
+            if (lane < D / 4)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    red[4 * lane + i] += acc[i];
+            __syncwarp();
+            if (lane == 0)
+                red[D] += tl;
+        } else if (tail > wg) { // this warp's tail tokens (see consume_k), exact values
             const int b = srow[IR_B], h = srow[IR_H];
             const float *tsc = sm.tscores + (ri & 1) * a.near_cap;
             const DT *vt0 = reinterpret_cast<const DT *>(a.tail) + ((int64_t)(b * 2 + 1) * a.H + h) * a.near_cap * D;
@@ -1863,8 +2000,12 @@ int launch_t(const DecodeArgs &a, const DecodeShape &shp, bool pdl, cudaStream_t
                      a.inject != LOOPKV_INJECT_NONE;
     if constexpr (BITS == 4) {
         if (!shp.onepass) {
-            auto kern = shp.min_ctas == 5 ? (gen ? decode_kernel<BITS, D, DT, 5, true> : decode_kernel<BITS, D, DT, 5, false>)
-                                          : (gen ? decode_kernel<BITS, D, DT, 4, true> : decode_kernel<BITS, D, DT, 4, false>);
+            const int var = gen ? 2 : (a.near_cap > 32 ? 1 : 0);
+            auto kern = shp.min_ctas == 5
+                            ? (var == 2 ? decode_kernel<BITS, D, DT, 5, 2>
+                                        : var == 1 ? decode_kernel<BITS, D, DT, 5, 1> : decode_kernel<BITS, D, DT, 5, 0>)
+                            : (var == 2 ? decode_kernel<BITS, D, DT, 4, 2>
+                                        : var == 1 ? decode_kernel<BITS, D, DT, 4, 1> : decode_kernel<BITS, D, DT, 4, 0>);
             return launch_shape(kern, shp, pdl, s, a, shp.stages_log2, shp.score_bufs);
         }
     }
@@ -1983,8 +2124,8 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
                 if (onepass)
                     ncl = max_active_clusters(decode_kernel_1p<BITS, D, DT, 4, true>, C, smem);
                 else if constexpr (BITS == 4)
-                    ncl = want_ctas == 5 ? max_active_clusters(decode_kernel<BITS, D, DT, 5, true>, C, smem)
-                                         : max_active_clusters(decode_kernel<BITS, D, DT, 4, true>, C, smem);
+                    ncl = want_ctas == 5 ? max_active_clusters(decode_kernel<BITS, D, DT, 5, 2>, C, smem)
+                                         : max_active_clusters(decode_kernel<BITS, D, DT, 4, 2>, C, smem);
                 if (ncl <= 0)
                     continue;
                 if (ncl > rows)

@@ -232,16 +232,18 @@ def test_share_cell_with_final_loop_query_is_bit_identical():
     assert torch.equal(a, b)
 
 
-@pytest.mark.parametrize("tau,tau_mode,D,dtype", [(0.01, 0, 128, torch.bfloat16), (0.05, 1, 128, torch.bfloat16),
-                                              (0.0, 0, 128, torch.bfloat16), (0.02, 0, 64, torch.float32)])
-def test_lean_build_matches_general_build(tau, tau_mode, D, dtype):
+@pytest.mark.parametrize("tau,tau_mode,D,dtype,sink,window", [
+    (0.01, 0, 128, torch.bfloat16, 0, 0), (0.05, 1, 128, torch.bfloat16, 0, 0), (0.0, 0, 128, torch.bfloat16, 0, 0),
+    (0.02, 0, 64, torch.float32, 0, 0), (0.01, 0, 128, torch.bfloat16, 32, 64), (0.02, 0, 64, torch.float32, 32, 96)])
+def test_lean_build_matches_general_build(tau, tau_mode, D, dtype, sink, window):
     """loopkv_decode without debug outputs runs the lean kernel builds (no refine-set bitmap,
-    streaming rule, sliding window or test hook on their per-group path); they must give the
-    outputs of the general builds, which the other cases check against the oracle, bit for bit."""
+    streaming rule, sliding window or test hook on their per-group path; with a sink or window, the
+    build that streams the near region); they must give the outputs of the general builds, which
+    the other cases check against the oracle, bit for bit."""
     modes = [L.CELL_4B, L.CELL_SHARE, L.CELL_2B, L.CELL_4B]  # loop 0: [4b, share], loop 1: [2b, 4b]
     w = synth.Workload("lean", 2, 2, 4, D, 3, [4096, 1000, 33], dtype, modes, tau, tau_mode=tau_mode,
                        append_steps=5, seed=21)
-    m = Model(w)
+    m = Model(w, sink=sink, window=window)
     m.ingest()
     for step in range(5):
         m.append_step(step)
