@@ -43,7 +43,7 @@ struct loopkv_cache {
     //           decode reads those before its grid dependency wait, so a decode right after
     //           such a launch does not overlap it (no programmatic dependent launch).
     std::mutex mu;
-    std::map<std::tuple<int, int, bool>, lkv::DecodeShape> shapes;
+    std::map<std::tuple<int, int, bool, int>, lkv::DecodeShape> shapes;
     std::map<void *, bool> state_written;
     unsigned long long wait_ns = lkv::kDefaultWaitNs;
     int inject = LOOPKV_INJECT_NONE;
@@ -62,14 +62,20 @@ struct loopkv_cache {
             it->second = false;
         return !written;
     }
-    lkv::DecodeShape shape(int bits, int B, bool onepass)
+    // window: the layer's sliding attention window (0: full attention).  A window bounds the
+    // history groups a row reads to (window + sink) / 32 + 1 (the first may be partly before the
+    // window), so those reads take the shape of that shorter row.
+    lkv::DecodeShape shape(int bits, int B, bool onepass, int window)
     {
+        int mb = plan.cfg.max_blocks_per_seq;
+        if (window > 0)
+            mb = std::min(mb, 2 * ((window + plan.cfg.sink_tokens + 31) / 32 + 1));
         std::lock_guard<std::mutex> lock(mu);
-        auto key = std::make_tuple(bits, B, onepass);
+        auto key = std::make_tuple(bits, B, onepass, mb);
         auto it = shapes.find(key);
         if (it == shapes.end())
             it = shapes.emplace(key, lkv::decode_shape(bits, plan.cfg.head_dim, plan.cfg.in_dtype, B * plan.cfg.n_heads,
-                                                       plan.cfg.max_blocks_per_seq, near_cap(plan.cfg), onepass))
+                                                       mb, near_cap(plan.cfg), onepass))
                      .first;
         return it->second;
     }
@@ -536,7 +542,7 @@ int loopkv_decode_debug(const loopkv_plan *plan, int loop, int layer, const void
     a.tau = plan->tau;
     a.tau_mode = plan->tau_mode;
     a.attn_window = plan->layer_window[layer];
-    const lkv::DecodeShape shp = cache->shape(bits, B, single_pass(bits, plan->tau));
+    const lkv::DecodeShape shp = cache->shape(bits, B, single_pass(bits, plan->tau), a.attn_window);
     a.cap_groups = shp.cap;
     {
         std::lock_guard<std::mutex> lock(cache->mu);
