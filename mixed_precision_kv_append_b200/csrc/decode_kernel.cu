@@ -866,8 +866,8 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel(const DecodeAr
     // K pass of the warp's groups of row ri; per-warp (max, sum) into stat.
     auto consume_k = [&](int ri) {
         // Set up row ri + 1 (and row 0 first).  Its slot (ri + 1) mod 3 last held row
-        // ri - 2, whose values were read and whose lo copies were all issued in the
-        // previous iteration, so nothing reads that slot any more.
+        // ri - 2, whose values and lo planes were read in the previous iteration, so nothing
+        // reads that slot any more.
         for (int r = ri == 0 ? 0 : ri + 1; r <= ri + 1 && r < nrows; ++r) {
             setup_row(r);
             setup_upto = r;
