@@ -1406,8 +1406,18 @@ struct SmemLayout1 {
 // row's stages are all issued.  A warp's maximum sits in its scratch after its partial
 // (word D + 1).  CTA partials (o[D], l, m) by row parity (see the barrier note in the
 // kernel).
-constexpr int kFields1 = 8;
+constexpr int kFields1 = 9;
 constexpr int I1_G0 = 5, I1_M0 = 6, I1_HIST = 7; // fields after IR_ROW .. IR_TAIL (see decode_kernel)
+constexpr int I1_NC = 8;                          // near-region chunks read by this warp (streamed)
+
+// Near rows per chunk of the single-pass reader: a chunk's key rows and value rows share one
+// ring stage.
+template <int BITS, int D, typename DT> __host__ __device__ constexpr int near_chunk_rows1()
+{
+    return 2 * 8 * D * (int)sizeof(DT) <= Geo1<BITS, D>::STAGE   ? 8
+           : 2 * 4 * D * (int)sizeof(DT) <= Geo1<BITS, D>::STAGE ? 4
+                                                                  : 2;
+}
 
 template <int BITS, int D> __host__ __device__ constexpr SmemLayout1 smem_layout1(int spw, int capw)
 {
@@ -1638,9 +1648,70 @@ __device__ __forceinline__ void run1_tail(Run1<D> &r, float *red, const int lane
     __syncwarp();
 }
 
-template <int BITS, int D, typename DT, int MINCTA, bool GEN> // GEN: as for decode_kernel
+// One chunk of NR near rows of a streamed near region (keys at kr, values at vr, physical slots
+// slot0 ..): exact scores, the running-maximum update of the single-pass reader, and the rows'
+// values added to the warp's sums (lane vk < D/4: channels 4 vk .. 4 vk + 3; l in lane 0).  Empty
+// slots and tokens outside a sliding window score -inf and add nothing.
+template <int D, typename DT, int NR, bool GEN>
+__device__ __forceinline__ void run1_near_chunk(Run1<D> &r, const DT *kr, const DT *vr, const float (&qreg)[4],
+                                                const DecodeArgs &a, const int slot0, const int ws, const int nnear,
+                                                const int hist, const int lane)
+{
+    float p[NR];
+#pragma unroll
+    for (int u = 0; u < NR; ++u) {
+        float k4[4] = {0.f, 0.f, 0.f, 0.f};
+        if (lane < D / 4)
+            load4f(kr + u * D + 4 * lane, k4);
+        p[u] = lane < D / 4 ? fmaf(qreg[0], k4[0], fmaf(qreg[1], k4[1], fmaf(qreg[2], k4[2], qreg[3] * k4[3]))) : 0.f;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int u = 0; u < NR; ++u)
+            p[u] += __shfl_xor_sync(0xFFFFFFFFu, p[u], o);
+    float mc = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < NR; ++u) {
+        const int j = near_index(a, slot0 + u, ws, nnear);
+        p[u] = j >= 0 && (!GEN || near_attended(a, j, hist, nnear)) ? p[u] * a.qscale : -INFINITY;
+        mc = fmaxf(mc, p[u]);
+    }
+    if (mc > r.m) { // warp-uniform: rescale the warp's sums to the new maximum
+        const float f = ex2(r.m - mc);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            r.o[i] *= f;
+#pragma unroll
+        for (int g = 0; g < D / 32; ++g)
+            r.z[g] *= f;
+        r.l *= f;
+        r.m = mc;
+    }
+#pragma unroll
+    for (int u = 0; u < NR; ++u) {
+        if (p[u] == -INFINITY)
+            continue; // warp-uniform
+        const float w = ex2(p[u] - r.m);
+        if (lane == 0)
+            r.l += w;
+        if (lane < D / 4) {
+            float v4[4];
+            load4f(vr + u * D + 4 * lane, v4);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                r.o[i] = fmaf(w, v4[i], r.o[i]);
+        }
+    }
+}
+
+template <int BITS, int D, typename DT, int MINCTA, int VAR> // VAR: as for decode_kernel
 __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const DecodeArgs a, const int spw_log2)
 {
+    constexpr bool GEN = VAR == 2;
+    constexpr bool NSC = VAR >= 1; // the streamed near path is compiled in
+    constexpr int NR = near_chunk_rows1<BITS, D, DT>();
+    constexpr uint32_t NRB = (uint32_t)(NR * D * sizeof(DT)); // bytes of a chunk's keys (and of its values)
     using G = Geo<BITS, D>;
     using G1 = Geo1<BITS, D>;
     extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -1702,7 +1773,12 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
 
     // ---------------------------------------------------------------- issuing
     int iss_n = 0, iss_row = -1, iss_k = 0, seg_n = 0, setup_upto = -1;
+    int seg_groups = 0;                       // group stages of the issuing row, then its near chunks
     const uint8_t *seg_src = nullptr, *seg_lo = nullptr;
+    const uint8_t *seg_near = nullptr;        // near region (keys; values follow H rows on) of the row
+    // a near region beyond a 32-token tail streams through the ring (see decode_kernel)
+    const bool nstream = NSC && a.near_cap > 32;
+    bool dep_ok = false;                      // the previous grid of the stream has finished
     bool timed_out = false; // as in decode_kernel: no waits or copies after a give-up, then a drain
     int drain_from = 0;
     // row parameters, validation and the warp's block ids of row ri (as in decode_kernel)
@@ -1749,15 +1825,28 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
             irow[I1_G0] = g0;
             irow[I1_M0] = h0 & 31;
             irow[I1_HIST] = hist;
+            if (NSC) {
+                const int nch = nstream ? a.near_cap / NR : 0, wg = (int)crank * kWarps + warp, nw = (int)C * kWarps;
+                irow[I1_NC] = nch > wg ? (nch - wg + nw - 1) / nw : 0;
+            }
         }
         __syncwarp();
         setup_upto = ri;
     };
     // stage n = the next group of the issuing row: both head regions (+ both lo regions)
     auto issue_stage = [&](int n) {
-        const int2 id = reinterpret_cast<const int2 *>(ids)[iss_k];
         uint8_t *st = ring + (n & smask) * G1::STAGE;
         uint64_t *fb = &full[n & smask];
+        if (NSC && iss_k >= seg_groups) { // near chunk: NR key rows, then the same NR value rows
+            if (lane == 0) {
+                const size_t off = (size_t)((int)crank * kWarps + warp + (iss_k - seg_groups) * (int)C * kWarps) * NRB;
+                mbar_arrive_expect_tx(fb, 2 * NRB);
+                bulk_g2s(st, seg_near + off, NRB, fb);
+                bulk_g2s(st + NRB, seg_near + (size_t)a.H * a.near_cap * D * sizeof(DT) + off, NRB, fb);
+            }
+            return;
+        }
+        const int2 id = reinterpret_cast<const int2 *>(ids)[iss_k];
         if (lane == 0) {
             mbar_arrive_expect_tx(fb, 2 * G::HM + 2 * G::LOB);
             if (GEN && a.inject == LOOPKV_INJECT_STALLED_STAGE && n == 0 && warp == 0 && blockIdx.x == 0)
@@ -1776,7 +1865,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
             return;
         for (;;) {
             if (iss_k < seg_n) {
-                if (iss_n >= limit)
+                if (iss_n >= limit || (NSC && !dep_ok && iss_k >= seg_groups)) // near rows: after the dependency
                     break;
                 issue_stage(iss_n);
                 ++iss_k;
@@ -1789,9 +1878,14 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
                 break;
             iss_row = setup_upto;
             iss_k = 0;
-            seg_n = irow[IR_N];
+            seg_groups = seg_n = irow[IR_N];
             seg_src = a.main + (size_t)irow[IR_H] * G::HM;
             seg_lo = a.lo + (size_t)irow[IR_H] * G::LOB;
+            if (NSC) {
+                seg_n += irow[I1_NC];
+                seg_near = reinterpret_cast<const uint8_t *>(a.tail) +
+                           ((int64_t)irow[IR_B] * 2 * a.H + irow[IR_H]) * a.near_cap * D * sizeof(DT);
+            }
         }
     };
 
@@ -1811,16 +1905,18 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
         if (ri == 0)
             setup_row(0);
         const int row = irow[IR_ROW], nown = irow[IR_N], rb = irow[IR_B], rh = irow[IR_H];
+        const int ncw = NSC ? irow[I1_NC] : 0, nst = nown + ncw; // this warp's stages: groups, near chunks
         const int rg0 = irow[I1_G0], rm0 = (crank == 0 && warp == 0) ? irow[I1_M0] : 0, rhist = irow[I1_HIST];
         int tail = irow[IR_TAIL];
         // the slot takes row ri + 1 once row ri's stages are all issued (after the pump of
-        // group nown - spw, or at once when the warp has no group)
-        const int k_setup = nown > spw ? nown - spw : 0;
-        if (nown == 0 && ri + 1 < nrows)
+        // stage nst - spw, or at once when the warp has no stage)
+        const int k_setup = nst > spw ? nst - spw : 0;
+        if (nst == 0 && ri + 1 < nrows)
             setup_row(ri + 1);
         if (ri == 0) { // prefetch, then wait for the previous grid of the stream (see decode_kernel)
             pump(prc_n + spw);
             asm volatile("griddepcontrol.wait;" ::: "memory");
+            dep_ok = true;
         }
         int ws = 0;
         if (tail < 0) { // near tokens and ring start (an append may have written them)
@@ -1833,7 +1929,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
                 ws = 0;
             }
         }
-        if (tail > (int)crank * kWarps + warp) { // this warp's near keys and values, read after its groups
+        if (!nstream && tail > (int)crank * kWarps + warp) { // this warp's near keys and values, read after its groups
             const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)rb * 2 * a.H + rh) * a.near_cap * D;
             prefetch_near<D, DT>(a, kt, ws, (int)crank * kWarps + warp, (int)C * kWarps, tail, lane);
             prefetch_near<D, DT>(a, kt + (int64_t)a.H * a.near_cap * D, ws, (int)crank * kWarps + warp, (int)C * kWarps,
@@ -1848,7 +1944,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
         }
         Run1<D> run;
         run1_init(run);
-        for (int k = 0; k < nown; ++k) {
+        for (int k = 0; k < nst; ++k) {
             const int n = prc_n++;
             if (iss_n < n + spw)
                 pump(n + spw);
@@ -1858,6 +1954,13 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
             }
             wait_stage(n);
             const uint8_t *st = ring + (n & smask) * G1::STAGE;
+            if (NSC && k >= nown) { // a chunk of the streamed near region
+                const int slot0 = ((int)crank * kWarps + warp + (k - nown) * (int)C * kWarps) * NR;
+                run1_near_chunk<D, DT, NR, GEN>(run, reinterpret_cast<const DT *>(st),
+                                                reinterpret_cast<const DT *>(st + NRB), qreg, a, slot0, ws, tail, rhist,
+                                                lane);
+                continue;
+            }
             const int masked = GEN && k == 0 ? rm0 : 0; // tokens of the first group before a sliding window
             run1_group<BITS, D>(st, st + G1::LOFF, scr, qreg, a.qscale, lane, run, masked);
             if (GEN && a.s_bitmap && lane == 0) // refine set: every attended token (4-bit, tau <= 0) or none (2-bit)
@@ -1867,7 +1970,7 @@ __global__ void __launch_bounds__(kThreads, MINCTA) decode_kernel_1p(const Decod
         float *red = reinterpret_cast<float *>(scr);
         run1_finish<BITS, D>(run, red, lane);
         const int wg = (int)crank * kWarps + warp; // tail token j to warp j mod (C * kWarps) of the cluster
-        if (tail > wg) {
+        if (!nstream && tail > wg) {
             const DT *kt = reinterpret_cast<const DT *>(a.tail) + ((int64_t)rb * 2 * a.H + rh) * a.near_cap * D;
             const DT *vt0 =
                 reinterpret_cast<const DT *>(a.tail) + ((int64_t)(rb * 2 + 1) * a.H + rh) * a.near_cap * D;
@@ -2011,8 +2114,11 @@ int launch_t(const DecodeArgs &a, const DecodeShape &shp, bool pdl, cudaStream_t
     }
     if (!shp.onepass)
         return LOOPKV_ERR_CUDA; // 2-bit sources have no refine set: always the single-pass reader
-    return launch_shape(gen ? decode_kernel_1p<BITS, D, DT, 4, true> : decode_kernel_1p<BITS, D, DT, 4, false>, shp, pdl,
-                        s, a, shp.stages_log2);
+    const int var = gen ? 2 : (a.near_cap > 32 ? 1 : 0);
+    return launch_shape(var == 2   ? decode_kernel_1p<BITS, D, DT, 4, 2>
+                        : var == 1 ? decode_kernel_1p<BITS, D, DT, 4, 1>
+                                   : decode_kernel_1p<BITS, D, DT, 4, 0>,
+                        shp, pdl, s, a, shp.stages_log2);
 }
 
 // Clusters of size C that can be resident at once for this kernel and shared memory.
@@ -2122,7 +2228,7 @@ template <int BITS, int D, typename DT> DecodeShape shape_t(int rows, int max_bl
                 int ncl = 0;
                 // occupancy of the general build (the lean one has the same launch bounds)
                 if (onepass)
-                    ncl = max_active_clusters(decode_kernel_1p<BITS, D, DT, 4, true>, C, smem);
+                    ncl = max_active_clusters(decode_kernel_1p<BITS, D, DT, 4, 2>, C, smem);
                 else if constexpr (BITS == 4)
                     ncl = want_ctas == 5 ? max_active_clusters(decode_kernel<BITS, D, DT, 5, 2>, C, smem)
                                          : max_active_clusters(decode_kernel<BITS, D, DT, 4, 2>, C, smem);
