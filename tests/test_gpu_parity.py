@@ -547,6 +547,25 @@ def test_sink_window_sequence(sink, window):
                 assert np.array_equal(got, Kr.astype(np.float32)), (lp, la, req)
 
 
+@pytest.mark.parametrize("D,dtype", [(128, torch.bfloat16), (64, torch.float32)])
+def test_sink_window_single_pass_all_hot(D, dtype):
+    """tau = 0 on 4-bit cells (every lo plane read: the single-pass reader) with a sink and a window:
+    the near region streams through that reader's ring in chunks of 8 (bf16) or 4 (fp32) rows next
+    to 4-row chunks of the 2-bit cells; outputs, row maxima and sums against the oracle through
+    appends and flushes."""
+    modes = [L.CELL_4B, L.CELL_SHARE, L.CELL_2B, L.CELL_4B]  # loop 0: [4b, share], loop 1: [2b, 4b]
+    w = synth.Workload("sw1p", 2, 2, 4, D, 3, [20, 32 + 64 + 9, 700], dtype, modes, 0.0, append_steps=40, seed=37)
+    m = Model(w, sink=32, window=64)
+    m.ingest()
+    for step in range(40):
+        m.append_step(step)
+        if step in (0, 17, 33, 39):
+            for la in range(2):
+                for lp in range(2):
+                    m.check_cell(lp, la, _q(w, step, la, lp), where=f"1p sink/window step {step}")
+    m.cache.check("single-pass sink/window")
+
+
 def test_sink_window_ouro_shape():
     """The paper's geometry (32-token sink, 256-token window) at Ouro-1.4B head shape, 8K
     context, sampled rows of a 4-bit, a share and a 2-bit cell, tau = 0.01."""
